@@ -1,0 +1,251 @@
+"""Python front of the fp64 CPU oracle for block-compressed attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg use it; the CUDA library never does, and the two
+share no code.  The arithmetic lives in ``lbca_oracle.c`` (fp64, plain loops,
+OpenMP over independent rows); this module only marshals numpy arrays.
+
+Functions and the passages they follow:
+  * ``pool``      -- block pooling + entry finalisation ("mSeek" README,
+                     "How LBCA works" steps 2-3; HCA page, "What is
+                     implemented", Eqs 20-23; CSA page, "Deviations from
+                     paper": RoPE at block-start positions).
+  * ``attend``    -- attention over visible pooled entries + raw window + sink
+                     ("mSeek" README, "How LBCA works" steps 4-5; CSA page,
+                     "What is implemented": Eqs 18-19, Eq 27, -i rotation).
+  * ``forward``   -- prefill: pool, then attend every row.
+  * ``decode``    -- one query per sequence at position len-1 (ragged lens).
+  * ``Stream``    -- the same definition driven token by token, pooling each
+                     block when it completes ("mSeek" README, repository
+                     layout: generation through the LBCA cache).
+  * ``visible_blocks`` -- P(L) of the block-aligned visibility reading.
+  * ``cache_entries`` / ``kv_cache_bytes`` -- analytic cache accounting
+                     ("mSeek" README, "Results").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lbca_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liblbca_oracle.so")
+_lib = None
+
+KEY, VALUE = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (gcc, -O2, OpenMP, no fast-math) in place."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-fno-fast-math", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("shared_kv", ctypes.c_int),
+                ("block_m", ctypes.c_int), ("n_win", ctypes.c_int),
+                ("rope_dims", ctypes.c_int), ("rmsnorm", ctypes.c_int),
+                ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_double),
+                ("softmax_scale", ctypes.c_double)]
+
+
+@dataclass(frozen=True)
+class Config:
+    """Layer shape and method parameters (same meaning as the C struct)."""
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    shared_kv: bool
+    block_m: int
+    n_win: int
+    rope_dims: int = 0
+    rmsnorm: bool = False
+    rope_theta: float = 10000.0
+    rms_eps: float = 1e-6
+    softmax_scale: float = 0.0
+
+    def c(self) -> _Cfg:
+        return _Cfg(self.n_q_heads, self.n_kv_heads, self.head_dim, int(self.shared_kv),
+                    self.block_m, self.n_win, self.rope_dims, int(self.rmsnorm),
+                    float(self.rope_theta), float(self.rms_eps), float(self.softmax_scale))
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lp = ctypes.POINTER(ctypes.c_long)
+        lib.orc_visible_blocks.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int]
+        lib.orc_visible_blocks.restype = ctypes.c_long
+        lib.orc_pool.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int, ctypes.c_long,
+                                 ctypes.c_long, dp, dp, dp, dp, dp]
+        lib.orc_pool.restype = ctypes.c_int
+        lib.orc_attend.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int, lp, dp, dp, dp,
+                                   ctypes.c_long, dp, dp, ctypes.c_long, lp, dp, dp, dp, dp]
+        lib.orc_attend.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _d(a):
+    """fp64 C-contiguous view (or None -> NULL)."""
+    if a is None:
+        return None, None
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def visible_blocks(L: int, m: int, w: int) -> int:
+    """P(L): pooled entries visible to a query that sees L tokens."""
+    return int(_load().orc_visible_blocks(int(L), int(m), int(w)))
+
+
+def pool(cfg: Config, series: int, x, z, b_pos, gamma=None, pos0: int = 0):
+    """Pooled + finalised entries of one series: [B, T//m, G, D] fp64."""
+    x, xp = _d(x)
+    z, zp = _d(z)
+    b_pos, bp = _d(b_pos)
+    gamma, gp = _d(gamma)
+    B, T, G, D = x.shape
+    assert z.shape == x.shape and G == cfg.n_kv_heads and D == cfg.head_dim
+    assert b_pos.shape == (cfg.block_m, G * D)
+    out = np.zeros((B, T // cfg.block_m, G, D))
+    rc = _load().orc_pool(ctypes.byref(cfg.c()), series, B, T, pos0, xp, zp, bp, gp,
+                          out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc:
+        raise ValueError("orc_pool rejected its arguments")
+    return out
+
+
+def attend(cfg: Config, q, qpos, ek, ev, k, v, lens, sink=None, gamma_q=None, gamma_kv=None):
+    """Attention of query rows q [B, nq, Hq, D] at positions qpos [B, nq]."""
+    q, qp = _d(q)
+    B, nq, Hq, D = q.shape
+    qpos = np.ascontiguousarray(qpos, dtype=np.int64).reshape(B, nq)
+    lens = np.ascontiguousarray(lens, dtype=np.int64).reshape(B)
+    k, kp = _d(k)
+    v, vp = _d(v)
+    if ek is None:
+        ek = np.zeros((B, 0, cfg.n_kv_heads, D))
+    ek, ekp = _d(ek)
+    ev, evp = _d(ev)
+    sink, sp = _d(sink)
+    gamma_q, gqp = _d(gamma_q)
+    gamma_kv, gkp = _d(gamma_kv)
+    out = np.zeros((B, nq, Hq, D))
+    lp = ctypes.POINTER(ctypes.c_long)
+    rc = _load().orc_attend(ctypes.byref(cfg.c()), B, nq, qpos.ctypes.data_as(lp), qp, ekp, evp,
+                            ek.shape[1], kp, vp, k.shape[1], lens.ctypes.data_as(lp), sp, gqp, gkp,
+                            out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc:
+        raise ValueError("orc_attend rejected its arguments")
+    return out
+
+
+def forward(cfg: Config, q, k, v, zk, zv, bpos_k, bpos_v=None, sink=None,
+            gamma_q=None, gamma_kv=None, rows=None):
+    """Prefill: outputs [B, len(rows), Hq, D] for query rows (all by default).
+
+    Pools the blocks that any requested row can see, then attends.
+    In the shared form pass k=C, zk=Z and leave v, zv, bpos_v as None.
+    """
+    q = np.asarray(q)
+    B, T = q.shape[:2]
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    need = visible_blocks(int(rows.max()) + 1, cfg.block_m, cfg.n_win) if len(rows) else 0
+    kk = np.asarray(k)[:, :need * cfg.block_m]
+    ek = pool(cfg, KEY, kk, np.asarray(zk)[:, :need * cfg.block_m], bpos_k, gamma_kv)
+    ev = None
+    if not cfg.shared_kv:
+        ev = pool(cfg, VALUE, np.asarray(v)[:, :need * cfg.block_m],
+                  np.asarray(zv)[:, :need * cfg.block_m], bpos_v)
+    qpos = np.broadcast_to(rows, (B, len(rows)))
+    return attend(cfg, q[:, rows], qpos, ek, ev, k, v, np.full(B, T), sink, gamma_q, gamma_kv)
+
+
+def decode(cfg: Config, q, k, v, zk, zv, bpos_k, bpos_v, lens, sink=None,
+           gamma_q=None, gamma_kv=None):
+    """One query per sequence: q [B, Hq, D] at position lens[b]-1 over history
+    k, v, zk, zv [B, Tmax, G, D] of which lens[b] tokens are valid."""
+    q = np.asarray(q)
+    B = q.shape[0]
+    lens = np.asarray(lens, dtype=np.int64).reshape(B)
+    out = np.zeros(q.shape)
+    for b in range(B):  # sequences have different visible block counts
+        L = int(lens[b])
+        need = visible_blocks(L, cfg.block_m, cfg.n_win) * cfg.block_m
+        sl = slice(b, b + 1)
+        ek = pool(cfg, KEY, np.asarray(k)[sl, :need], np.asarray(zk)[sl, :need], bpos_k, gamma_kv)
+        ev = None if cfg.shared_kv else pool(cfg, VALUE, np.asarray(v)[sl, :need],
+                                             np.asarray(zv)[sl, :need], bpos_v)
+        vv = None if cfg.shared_kv else np.asarray(v)[sl, :L]
+        out[b] = attend(cfg, q[sl, None], np.array([[L - 1]]), ek, ev, np.asarray(k)[sl, :L], vv,
+                        np.array([L]), sink, gamma_q, gamma_kv)[0, 0]
+    return out
+
+
+class Stream:
+    """Token-by-token form of the same definition for one sequence.
+
+    ``append`` adds one raw token; when it completes a block the block is
+    pooled and finalised once and kept.  ``query`` attends one query at the
+    position of the last appended token.  The arithmetic is the C oracle's.
+    """
+
+    def __init__(self, cfg: Config, bpos_k, bpos_v=None, gamma_kv=None):
+        self.cfg = cfg
+        self.bpos_k, self.bpos_v, self.gamma_kv = bpos_k, bpos_v, gamma_kv
+        G, D = cfg.n_kv_heads, cfg.head_dim
+        self.k = np.zeros((0, G, D)); self.zk = np.zeros((0, G, D))
+        self.v = np.zeros((0, G, D)); self.zv = np.zeros((0, G, D))
+        self.ek = np.zeros((0, G, D)); self.ev = np.zeros((0, G, D))
+
+    def extend(self, k, zk, v=None, zv=None):
+        """Append a run of raw tokens [n, G, D] (pools every block it completes)."""
+        m = self.cfg.block_m
+        self.k = np.concatenate([self.k, k]); self.zk = np.concatenate([self.zk, zk])
+        if not self.cfg.shared_kv:
+            self.v = np.concatenate([self.v, v]); self.zv = np.concatenate([self.zv, zv])
+        done = self.k.shape[0] // m
+        have = self.ek.shape[0]
+        if done > have:
+            sl = slice(have * m, done * m)
+            self.ek = np.concatenate([self.ek, pool(self.cfg, KEY, self.k[None, sl], self.zk[None, sl],
+                                                    self.bpos_k, self.gamma_kv, pos0=have * m)[0]])
+            if not self.cfg.shared_kv:
+                self.ev = np.concatenate([self.ev, pool(self.cfg, VALUE, self.v[None, sl],
+                                                        self.zv[None, sl], self.bpos_v)[0]])
+
+    def query(self, q, sink=None, gamma_q=None):
+        """Output [Hq, D] for query q [Hq, D] at the last appended position."""
+        L = self.k.shape[0]
+        v = None if self.cfg.shared_kv else self.v[None]
+        ev = None if self.cfg.shared_kv else self.ev[None]
+        return attend(self.cfg, np.asarray(q)[None, None], np.array([[L - 1]]), self.ek[None], ev,
+                      self.k[None], v, np.array([L]), sink, gamma_q, self.gamma_kv)[0, 0]
+
+
+def cache_entries(T: int, m: int, w: int) -> int:
+    """Entries one LBCA layer stores per kv head for a T-token context:
+    P(T) pooled entries plus the raw tokens from P(T)*m on."""
+    P = visible_blocks(T, m, w)
+    return P + (T - P * m)
+
+
+def kv_cache_bytes(T: int, n_layers: int, n_lbca_layers: int, m: int, w: int,
+                   n_kv_heads: int, head_dim: int, elt_bytes: int = 2) -> int:
+    """Analytic K+V bytes for a model whose LBCA layers store ``cache_entries``
+    per head and whose other layers store every token."""
+    per_entry = 2 * n_kv_heads * head_dim * elt_bytes
+    dense_layers = n_layers - n_lbca_layers
+    return (dense_layers * T + n_lbca_layers * cache_entries(T, m, w)) * per_entry

@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of block-compressed attention on B200.
+
+One step = one decode step of the whole hot path for every sequence of the
+workload: append the new raw token (ring write, running pooling softmax, and
+pooling + finalisation of a block when it completes) and decode its query
+(RoPE / RMSNorm of the query, scores over the visible pooled entries and the
+raw window, softmax with sink, weighted values, split merge).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU, each rank
+decodes its own sequences (weak scaling, no collective on the data path); the
+step time is the max over ranks.  The inputs of the workload are resident in
+HBM before timing; the L2 is flushed (a 256 MiB write) before every timed
+step and outside its CUDA events.  ``e2e`` repeats the steps through the
+public API with the step's inputs copied from pinned host memory and the
+output copied back inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode µs/token"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gqa_decode_32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of the benchmarked GPU during the timed region."""
+    Q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 10 and (self.uuid is None or self.uuid in f[1]):
+                self.rows.append(f)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        rows = self.rows
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[6 + i] and "Not" not in r[6 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------- workload ----
+def bytes_per_decode(w, lens):
+    """Algorithmic HBM bytes of one decode launch: every visible pooled and raw
+    entry read once (K and V, or the shared entry), the queries read and the
+    outputs written once."""
+    esize = 2 if w.dtype == "bf16" else 4
+    series = 1 if w.shared_kv else 2
+    total = 0
+    for L in lens:
+        L = int(L)
+        P = max(0, (L - w.n_win) // w.block_m)
+        total += (P + (L - P * w.block_m)) * w.n_kv_heads * w.head_dim * esize * series
+    total += 2 * len(lens) * w.n_q_heads * w.head_dim * esize
+    return total
+
+
+class DecodeBench:
+    def __init__(self, w, n_steps, rank):
+        import torch
+
+        from block_compressed_long_b200 import lbca as L
+        from block_compressed_long_b200 import synth
+        self.L, self.torch = L, torch
+        self.w = synth.scaled(w, steps=n_steps, seed=w.seed + 7919 * rank)
+        self.inp = synth.make(self.w)
+        w = self.w
+        self.cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win,
+                            w.rope_dims, w.rmsnorm, w.rope_theta, dtype=w.dtype)
+        B = w.batch
+        self.B = B
+        self.max_ctx = int(self.inp.lens.max()) + n_steps
+        d = lambda t: None if t is None else t.cuda()  # noqa: E731
+        self.k, self.v, self.zk, self.zv = (d(t) for t in (self.inp.k, self.inp.v, self.inp.zk, self.inp.zv))
+        self.bpk, self.bpv, self.sink = d(self.inp.bpos_k), d(self.inp.bpos_v), d(self.inp.sink)
+        self.q = d(self.inp.q)
+        self.cache = L.Cache.allocate(self.cfg, B, self.max_ctx)
+        per = self.cache.pool_state.numel() // B
+        ws0 = torch.zeros(16, dtype=torch.uint8, device="cuda")
+        for b in range(B):  # build each sequence's cache with the prefill path (cache only)
+            Lb = int(self.inp.lens[b])
+            c = self.cache
+            sc = L.Cache(self.cfg, 1, c.max_blocks, c.ring_slots, c.pooled_k[b:b + 1],
+                         None if c.pooled_v is None else c.pooled_v[b:b + 1], c.ring_k[b:b + 1],
+                         None if c.ring_v is None else c.ring_v[b:b + 1], c.pool_state[b * per:(b + 1) * per],
+                         c.seq_lens[b:b + 1])
+            s = lambda t: None if t is None else t[b:b + 1, :Lb]  # noqa: E731
+            L.lbca_prefill(self.cfg, None, s(self.k), s(self.v), s(self.zk), s(self.zv), self.bpk, self.bpv,
+                           None, None, None, None, sc, ws0, batch=1, T=Lb)
+        self.ws = torch.zeros(L.lbca_decode_workspace_bytes(self.cfg, B, self.max_ctx), dtype=torch.uint8,
+                              device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        # per-step token inputs, gathered once: [steps, B, G, D]
+        ar = torch.arange(B)
+        pos = torch.as_tensor(self.inp.lens)
+        tok = lambda t: None if t is None else torch.stack(  # noqa: E731
+            [t[ar, pos + i] for i in range(n_steps)]).cuda()
+        self.tk, self.tv, self.tzk, self.tzv = (tok(t) for t in (self.inp.k, self.inp.v, self.inp.zk, self.inp.zv))
+        self.out = torch.empty(B, w.n_q_heads, w.head_dim, dtype=L.torch_dtype(self.cfg), device="cuda")
+        self.i = 0
+
+    def lens_now(self):
+        return self.inp.lens + self.i + 1
+
+    def step(self, ev=None):
+        L, i = self.L, self.i
+        g = lambda t: None if t is None else t[i]  # noqa: E731
+        L.lbca_append(self.cfg, g(self.tk), g(self.tv), g(self.tzk), g(self.tzv), self.bpk, self.bpv, None,
+                      self.cache, self.status)
+        if ev is not None:
+            ev[0].record()
+        L.lbca_decode(self.cfg, self.q[i], self.cache, self.sink, None, self.out, self.ws, self.max_ctx,
+                      self.status)
+        if ev is not None:
+            ev[1].record()
+        self.i += 1
+
+
+def run_ours(args, w, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    n_steps = 2 * (args.warmup + args.steps)
+    bench = DecodeBench(w, n_steps, rank)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        bench.step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    step_ev = [(E(), E()) for _ in range(args.steps)]
+    dec_ev = [(E(), E()) for _ in range(args.steps)]
+    nbytes = 0
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for s in range(args.steps):
+        flush.zero_()
+        nbytes += bytes_per_decode(bench.w, bench.lens_now())
+        step_ev[s][0].record()
+        bench.step(dec_ev[s])
+        step_ev[s][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
+
+    # ---- end to end through the public API: pinned host inputs and output ----
+    w_ = bench.w
+    pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
+    hq = pin(bench.q)
+    htk, htv, htzk, htzv = (pin(t) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv))
+    dq = torch.empty_like(bench.q[0])
+    dtok = [None if t is None else torch.empty_like(t[0]) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)]
+    hout = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
+    L = bench.L
+    h2d = d2h = 0
+
+    def e2e_step():
+        nonlocal h2d, d2h
+        i = bench.i
+        dq.copy_(hq[i], non_blocking=True)
+        for dt, ht in zip(dtok, (htk, htv, htzk, htzv)):
+            if dt is not None:
+                dt.copy_(ht[i], non_blocking=True)
+        L.lbca_append(bench.cfg, dtok[0], dtok[1], dtok[2], dtok[3], bench.bpk, bench.bpv, None, bench.cache,
+                      bench.status)
+        L.lbca_decode(bench.cfg, dq, bench.cache, bench.sink, None, bench.out, bench.ws, bench.max_ctx,
+                      bench.status)
+        hout.copy_(bench.out, non_blocking=True)
+        bench.i += 1
+        h2d = dq.numel() * dq.element_size() + sum(t.numel() * t.element_size() for t in dtok if t is not None)
+        d2h = hout.numel() * hout.element_size()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ev = [(E(), E()) for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.zero_()
+        e2e_ev[s][0].record()
+        e2e_step()
+        e2e_ev[s][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    clocks = sampler.stop()
+    status = int(bench.status.item())
+    if status:
+        raise RuntimeError(f"device status {L.lbca_status_string(status)}")
+
+    t = torch.tensor([step_ms, e2e_ms, dec_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, e2e_ms, dec_ms = t.tolist()
+    tokens = bench.B * world
+    hbm, src = peaks()
+    achieved = nbytes / args.steps / (dec_ms * 1e-3) / 1e9
+    traffic = load_traffic(w_.name)
+    line = {
+        "metric": METRIC, "value": step_ms * 1e3 / tokens, "unit": "µs/token", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
+        "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
+                   "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
+                   "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
+                   "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
+                   "l2": "flushed (256 MiB write) before every timed step, outside its events"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": src, "kernel": "decode_kernel",
+                     "bytes_per_launch": nbytes / args.steps, "launch_us": dec_ms * 1e3,
+                     "traffic": traffic},
+        "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "µs/token", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    return line, bench
+
+
+def load_traffic(workload):
+    """DRAM bytes per decode launch from a committed ncu capture, if the
+    decode source has not changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(p))[workload]
+    except Exception:
+        return None
+    src = os.path.join(ROOT, "block_compressed_long_b200", "csrc", "decode.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes"] if rec.get("decode_cu_sha256_16") == h else None
+
+
+# ----------------------------------------------------- oracle (CPU) timing ----
+def oracle_decode_timing(w, budget_s=12.0, max_steps=None):
+    """The fp64 oracle as it stands, driven step by step on the host cores:
+    each step appends one token per sequence (pooling a block when it
+    completes) and attends its query.  Returns (µs/token, steps, cores, desc)."""
+    from block_compressed_long_b200 import synth
+    from oracle import oracle as orc
+    f64 = synth.f64
+    nb = max_steps or 64
+    ws = synth.scaled(w, steps=nb)
+    inp = synth.make(ws)
+    c = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta)
+    seqs = list(range(min(ws.batch, 4)))  # bounded sample of sequences
+    streams = []
+    for b in seqs:
+        Lb = int(inp.lens[b])
+        st = orc.Stream(c, f64(inp.bpos_k), f64(inp.bpos_v))
+        st.extend(f64(inp.k[b, :Lb]), f64(inp.zk[b, :Lb]), None if w.shared_kv else f64(inp.v[b, :Lb]),
+                  None if w.shared_kv else f64(inp.zv[b, :Lb]))
+        streams.append(st)
+    sink = f64(inp.sink)
+    t0 = time.perf_counter()
+    n = 0
+    while n < nb and (time.perf_counter() - t0) < budget_s:
+        for st, b in zip(streams, seqs):
+            p = int(inp.lens[b]) + n
+            st.extend(f64(inp.k[b, p:p + 1]), f64(inp.zk[b, p:p + 1]),
+                      None if w.shared_kv else f64(inp.v[b, p:p + 1]),
+                      None if w.shared_kv else f64(inp.zv[b, p:p + 1]))
+            st.query(f64(inp.q[n, b]), sink)
+        n += 1
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"{n} decode steps of {len(seqs)} sequence(s) of {w.name} (contexts "
+            f"{[int(inp.lens[b]) for b in seqs]}), fp64 C oracle, cache of pooled entries kept between steps")
+    return dt * 1e6 / (n * len(seqs)), n * len(seqs), cores, desc
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    from block_compressed_long_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if w.kind != "decode":
+        raise SystemExit("bench.py times decode workloads; prefill is timed by its own leg")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        us, n, cores, desc = oracle_decode_timing(w, budget_s=max(5.0, 0.5 * args.steps), max_steps=args.warmup + args.steps)
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": us, "unit": "µs/token", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
+                          "dtype": "f64", "data": "synthetic", "config": {"workload": w.name},
+                          "cpu_baseline": {"value": us, "unit": "µs/token", "cores": cores, "kind": "oracle",
+                                           "sample": desc},
+                          "e2e": {"value": us, "unit": "µs/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    import __graft_entry__
+    __graft_entry__.build()
+    line, _ = run_ours(args, w, rank, world)
+    if rank == 0 and world == 1:
+        us, n, cores, desc = oracle_decode_timing(w)
+        line["cpu_baseline"] = {"value": us, "unit": "µs/token", "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

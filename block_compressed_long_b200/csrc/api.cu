@@ -1,0 +1,300 @@
+// api.cu -- the C ABI: argument validation, device check, launches.
+//
+// Every entry point validates its arguments on the host before any CUDA call
+// (so bad arguments are reported even without a GPU), checks that the current
+// device is sm_100, and enqueues its kernels on the caller's stream.  No entry
+// point allocates device memory or synchronises.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.h"
+#include "lbca.h"
+
+using namespace lbca;
+
+namespace {
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool al16n(const void* p) { return p == nullptr || al16(p); }
+
+int vec_of(int dtype) { return dtype == LBCA_BF16 ? 8 : 4; }
+int esize_of(int dtype) { return dtype == LBCA_BF16 ? 2 : 4; }
+
+lbca_status check_cfg(const lbca_config* c) {
+    if (!c) return LBCA_ERR_ARG;
+    if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) return LBCA_ERR_ARG;
+    if (c->head_dim < 16 || c->head_dim > 512 || c->head_dim % 16) return LBCA_ERR_ARG;
+    if ((c->shared_kv != 0 && c->shared_kv != 1) || (c->rmsnorm != 0 && c->rmsnorm != 1)) return LBCA_ERR_ARG;
+    if (c->block_m < 1 || c->n_win < 0) return LBCA_ERR_ARG;
+    if (c->rope_dims < 0 || c->rope_dims > c->head_dim || (c->rope_dims & 1)) return LBCA_ERR_ARG;
+    if (c->rope_dims > 0 && !(c->rope_theta > 0.0)) return LBCA_ERR_ARG;
+    if (c->rmsnorm && !(c->rms_eps >= 0.f)) return LBCA_ERR_ARG;
+    if (!(c->softmax_scale == c->softmax_scale)) return LBCA_ERR_ARG;  // NaN
+    if (c->dtype != LBCA_F32 && c->dtype != LBCA_BF16) return LBCA_ERR_ARG;
+    if (c->reserved != 0) return LBCA_ERR_ARG;
+    // pooling kernels keep one 16-byte vector of the G*D row per thread (<= 1024 threads)
+    const long long nv = (long long)c->n_kv_heads * c->head_dim / vec_of(c->dtype);
+    if (nv * (c->shared_kv ? 1 : 2) > 1024) return LBCA_ERR_UNSUPPORTED;
+    return LBCA_OK;
+}
+
+float scale_of(const lbca_config* c) {
+    return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt((float)c->head_dim);
+}
+
+int ring_min(const lbca_config* c) {
+    const long long m = c->block_m;
+    long long r = m * ((c->n_win + m - 1 + m - 1) / m);
+    if (r < 1) r = 1;
+    return r > INT32_MAX ? -1 : (int)r;
+}
+
+lbca_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LBCA_ERR_CUDA;
+    static int known[64];  // 0 unknown, 1 sm_100, 2 other
+    if (dev >= 0 && dev < 64 && known[dev]) return known[dev] == 1 ? LBCA_OK : LBCA_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LBCA_ERR_CUDA;
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) known[dev] = ok ? 1 : 2;
+    return ok ? LBCA_OK : LBCA_ERR_UNSUPPORTED;
+}
+
+lbca_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LBCA_OK : LBCA_ERR_CUDA; }
+
+lbca_status check_cache(const lbca_config* c, const lbca_cache* k) {
+    if (!k) return LBCA_ERR_ARG;
+    if (k->batch < 0 || k->max_blocks < 0 || k->reserved != 0) return LBCA_ERR_ARG;
+    const int rmin = ring_min(c);
+    if (rmin < 0 || k->ring_slots < rmin) return LBCA_ERR_CAPACITY;
+    if (!k->pooled_k || !k->ring_k || !k->pool_state || !k->seq_lens) return LBCA_ERR_ARG;
+    if (c->shared_kv) {
+        if (k->pooled_v || k->ring_v) return LBCA_ERR_ARG;
+    } else if (!k->pooled_v || !k->ring_v) {
+        return LBCA_ERR_ARG;
+    }
+    if (!al16(k->pooled_k) || !al16n(k->pooled_v) || !al16(k->ring_k) || !al16n(k->ring_v) ||
+        !al16(k->pool_state))
+        return LBCA_ERR_ALIGN;
+    return LBCA_OK;
+}
+
+// K-side / V-side pointer set: shared form needs exactly the K side.
+lbca_status check_kv(const lbca_config* c, const void* k, const void* v, const void* zk, const void* zv,
+                     const void* bk, const void* bv) {
+    if (!k || !zk || !bk) return LBCA_ERR_ARG;
+    if (c->shared_kv) {
+        if (v || zv || bv) return LBCA_ERR_ARG;
+    } else if (!v || !zv || !bv) {
+        return LBCA_ERR_ARG;
+    }
+    if (!al16(k) || !al16(zk) || !al16(bk) || !al16n(v) || !al16n(zv) || !al16n(bv)) return LBCA_ERR_ALIGN;
+    return LBCA_OK;
+}
+
+#define LBCA_TRY(expr)                    \
+    do {                                  \
+        lbca_status _s = (expr);          \
+        if (_s != LBCA_OK) return _s;     \
+    } while (0)
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t lbca_ring_slots(const lbca_config* cfg) {
+    if (check_cfg(cfg) != LBCA_OK) return -1;
+    return ring_min(cfg);
+}
+
+size_t lbca_pool_state_elems(const lbca_config* cfg, int32_t batch) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0) return 0;
+    return (size_t)batch * (cfg->shared_kv ? 1 : 2) * 3 * cfg->n_kv_heads * cfg->head_dim;
+}
+
+size_t lbca_decode_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return 0;
+    DecodePlan p = plan_decode(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                               cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+    if (!p.ok) return 0;
+    return decode_workspace_bytes(p);
+}
+
+size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t T, int32_t has_cache) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || T < 0) return (size_t)-1;
+    if (has_cache) return 0;
+    const size_t one = (size_t)batch * cfg->n_kv_heads * (T / cfg->block_m) * cfg->head_dim *
+                       esize_of(cfg->dtype);
+    return align256(one) * (cfg->shared_kv ? 1 : 2);
+}
+
+lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                      const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
+                      void* out, int32_t out_blocks, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    if (series != LBCA_KEY && series != LBCA_VALUE) return LBCA_ERR_ARG;
+    if (cfg->shared_kv && series != LBCA_KEY) return LBCA_ERR_ARG;
+    if (!x || !z || !b_pos || !out) return LBCA_ERR_ARG;
+    if (batch < 0 || T < 0 || pos0 < 0 || pos0 % cfg->block_m || out_blocks < 0) return LBCA_ERR_ARG;
+    if ((long long)pos0 / cfg->block_m + T / cfg->block_m > out_blocks) return LBCA_ERR_ARG;
+    if (!al16(x) || !al16(z) || !al16(b_pos) || !al16(out) || !al16n(gamma)) return LBCA_ERR_ALIGN;
+    LBCA_TRY(check_device());
+    PoolArgs a{};
+    a.dtype = cfg->dtype;
+    a.x = x; a.z = z; a.bpos = b_pos; a.gamma = gamma;
+    a.out = out; a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
+    a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
+    a.pos0 = pos0;
+    a.key = series == LBCA_KEY; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
+    a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+    a.state = nullptr; a.S = 1; a.series = 0;
+    return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lbca_status lbca_append(const lbca_config* cfg, const void* k, const void* v, const void* zk,
+                        const void* zv, const void* b_pos_k, const void* b_pos_v, const void* gamma_kv,
+                        const lbca_cache* cache, int32_t* d_status, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v));
+    LBCA_TRY(check_cache(cfg, cache));
+    if (!al16n(gamma_kv)) return LBCA_ERR_ALIGN;
+    LBCA_TRY(check_device());
+    AppendArgs a{};
+    a.dtype = cfg->dtype;
+    a.k = k; a.v = v; a.zk = zk; a.zv = zv; a.bpk = b_pos_k; a.bpv = b_pos_v; a.gamma = gamma_kv;
+    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
+    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
+    a.state = cache->pool_state; a.seq_lens = cache->seq_lens; a.status = d_status;
+    a.B = cache->batch; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
+    a.R = cache->ring_slots; a.max_blocks = cache->max_blocks; a.S = cfg->shared_kv ? 1 : 2;
+    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims; a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+    return cuda_status(launch_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache* cache, const float* sink,
+                        const void* gamma_q, int32_t max_ctx, void* out, void* workspace,
+                        size_t workspace_bytes, int32_t* d_status, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_cache(cfg, cache));
+    if (!q || !out || !workspace) return LBCA_ERR_ARG;
+    if (!al16(q) || !al16(out) || !al16(workspace) || !al16n(gamma_q) || !al16n(sink)) return LBCA_ERR_ALIGN;
+    if (max_ctx <= 0) {
+        const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
+        max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
+    }
+    DecodePlan p = plan_decode(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                               cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+    if (!p.ok) return LBCA_ERR_UNSUPPORTED;
+    if (workspace_bytes < decode_workspace_bytes(p)) return LBCA_ERR_CAPACITY;
+    LBCA_TRY(check_device());
+    char* ws = static_cast<char*>(workspace);
+    DecodeArgs a{};
+    a.dtype = cfg->dtype;
+    a.q = q;
+    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
+    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
+    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    a.part_o = reinterpret_cast<float*>(ws);
+    a.part_ml = reinterpret_cast<float*>(ws + align256(p.part_o_elems * 4));
+    a.counters = reinterpret_cast<uint32_t*>(ws + align256(p.part_o_elems * 4) + align256(p.part_ml_elems * 4));
+    a.status = d_status;
+    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
+    a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
+    a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
+    a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.theta = cfg->rope_theta;
+    return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, const void* v, const void* zk,
+                         const void* zv, const void* b_pos_k, const void* b_pos_v, const float* sink,
+                         const void* gamma_q, const void* gamma_kv, int32_t batch, int32_t T, void* out,
+                         const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
+                         lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v));
+    if (batch < 0 || T < 0) return LBCA_ERR_ARG;
+    if (!out && !cache_out) return LBCA_ERR_ARG;
+    if (out && !q) return LBCA_ERR_ARG;
+    if (!al16n(q) || !al16n(out) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink) ||
+        !al16n(workspace))
+        return LBCA_ERR_ALIGN;
+    const int m = cfg->block_m, NB = T / m;
+    if (cache_out) {
+        LBCA_TRY(check_cache(cfg, cache_out));
+        if (cache_out->batch != batch) return LBCA_ERR_ARG;
+        if (cache_out->max_blocks < NB) return LBCA_ERR_CAPACITY;
+    }
+    const size_t need = lbca_prefill_workspace_bytes(cfg, batch, T, cache_out != nullptr);
+    if (workspace_bytes < need) return LBCA_ERR_CAPACITY;
+    if (need > 0 && !workspace) return LBCA_ERR_ARG;
+    if (out && !prefill_simt_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
+    LBCA_TRY(check_device());
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    // 1. pool every complete block of K and V (and the open block's state)
+    void* pk = cache_out ? cache_out->pooled_k : workspace;
+    void* pv = nullptr;
+    if (!cfg->shared_kv) {
+        const size_t one = (size_t)batch * cfg->n_kv_heads * NB * cfg->head_dim * esize_of(cfg->dtype);
+        pv = cache_out ? cache_out->pooled_v : static_cast<char*>(workspace) + align256(one);
+    }
+    const int stride = cache_out ? cache_out->max_blocks : NB;
+    for (int series = 0; series < (cfg->shared_kv ? 1 : 2); ++series) {
+        PoolArgs a{};
+        a.dtype = cfg->dtype;
+        a.x = series ? v : k; a.z = series ? zv : zk; a.bpos = series ? b_pos_v : b_pos_k;
+        a.gamma = series ? nullptr : gamma_kv;
+        a.out = series ? pv : pk; a.out_blocks = stride; a.blk_off = 0;
+        a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = m; a.pos0 = 0;
+        a.key = series == 0; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
+        a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+        a.state = cache_out ? cache_out->pool_state : nullptr;
+        a.S = cfg->shared_kv ? 1 : 2; a.series = series;
+        LBCA_TRY(cuda_status(launch_pool(a, s)));
+    }
+    // 2. the raw window and the lengths, so decode can continue from T
+    if (cache_out) {
+        RingFillArgs r{};
+        r.dtype = cfg->dtype;
+        r.k = k; r.v = v; r.gamma = gamma_kv;
+        r.ring_k = cache_out->ring_k; r.ring_v = cache_out->ring_v; r.seq_lens = cache_out->seq_lens;
+        r.B = batch; r.T = T; r.G = cfg->n_kv_heads; r.D = cfg->head_dim; r.R = cache_out->ring_slots;
+        r.n = T < r.R ? T : r.R;
+        r.rmsnorm = cfg->rmsnorm; r.rho = cfg->rope_dims; r.theta = cfg->rope_theta; r.eps = cfg->rms_eps;
+        LBCA_TRY(cuda_status(launch_ring_fill(r, s)));
+    }
+    // 3. attention
+    if (out) {
+        PrefillArgs a{};
+        a.dtype = cfg->dtype;
+        a.q = q; a.k = k; a.v = v; a.pooled_k = pk; a.pooled_v = cfg->shared_kv ? pk : pv;
+        a.pool_stride = stride; a.sink = sink; a.gamma_q = gamma_q; a.gamma_kv = gamma_kv; a.out = out;
+        a.B = batch; a.T = T; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
+        a.m = m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
+        a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.theta = cfg->rope_theta;
+        LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
+    }
+    return LBCA_OK;
+}
+
+const char* lbca_status_string(lbca_status status) {
+    switch (status) {
+        case LBCA_OK: return "ok";
+        case LBCA_ERR_ARG: return "invalid argument";
+        case LBCA_ERR_UNSUPPORTED: return "unsupported device or shape";
+        case LBCA_ERR_CAPACITY: return "cache or workspace too small";
+        case LBCA_ERR_CUDA: return "CUDA error";
+        case LBCA_ERR_TIMEOUT: return "bounded device wait timed out";
+        case LBCA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+// kernels.h -- launch interfaces between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lbca.h"
+
+namespace lbca {
+
+// Pool complete blocks (and optionally record the open block's running state).
+struct PoolArgs {
+    int dtype;
+    const void* x;         // [B, T, G, D]
+    const void* z;         // [B, T, G, D]
+    const void* bpos;      // [m, G*D]
+    const void* gamma;     // [D] or null
+    void* out;             // [B, G, out_blocks, D]; block j at blk_off + j
+    int out_blocks, blk_off;
+    int B, T, G, D, m;
+    int64_t pos0;          // absolute position of token 0 of x
+    int key, rmsnorm, rho;
+    double theta;
+    float eps;
+    float* state;          // [B, S, 3, G, D] or null: running state of the partial block
+    int S, series;
+};
+cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
+
+// Write finalised raw keys / raw values of tokens [T - n, T) into the ring and
+// set seq_lens = T.
+struct RingFillArgs {
+    int dtype;
+    const void* k;         // [B, T, G, D]
+    const void* v;         // [B, T, G, D] or null (shared form)
+    const void* gamma;
+    void* ring_k;          // [B, G, R, D]
+    void* ring_v;
+    int32_t* seq_lens;
+    int B, T, G, D, R, n;
+    int rmsnorm, rho;
+    double theta;
+    float eps;
+};
+cudaError_t launch_ring_fill(const RingFillArgs& a, cudaStream_t s);
+
+struct AppendArgs {
+    int dtype;
+    const void* k; const void* v; const void* zk; const void* zv;  // [B, G, D]
+    const void* bpk; const void* bpv;                              // [m, G*D]
+    const void* gamma;
+    void* pooled_k; void* pooled_v;                                // [B, G, max_blocks, D]
+    void* ring_k; void* ring_v;                                    // [B, G, R, D]
+    float* state;                                                  // [B, S, 3, G, D]
+    int32_t* seq_lens;
+    int32_t* status;
+    int B, G, D, m, R, max_blocks, S;
+    int rmsnorm, rho;
+    double theta;
+    float eps;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+    int dtype;
+    const void* q;                                   // [B, Hq, D]
+    const void* pooled_k; const void* pooled_v;      // [B, G, max_blocks, D]
+    const void* ring_k; const void* ring_v;          // [B, G, R, D]
+    const int32_t* seq_lens;
+    const float* sink;
+    const void* gamma_q;
+    void* out;                                       // [B, Hq, D]
+    float* part_o;                                   // [B, Hq, n_split, D]
+    float* part_ml;                                  // [B, Hq, n_split, 2]
+    uint32_t* counters;                              // [B, Hq / heads_per_cta]
+    int32_t* status;
+    int B, Hq, G, D, m, w, rho, rmsnorm, shared, max_blocks, R;
+    int n_split, chunk, heads_per_cta;
+    float eps, scale;
+    double theta;
+};
+// Chooses heads per CTA, chunk and split count for a decode call.
+struct DecodePlan {
+    int heads_per_cta, chunk, n_split;
+    size_t part_o_elems, part_ml_elems, counter_elems;
+    size_t smem_bytes;
+    bool ok;
+};
+DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int shared,
+                       int max_ctx);
+size_t decode_workspace_bytes(const DecodePlan& p);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+struct PrefillArgs {
+    int dtype;
+    const void* q;                                   // [B, T, Hq, D]
+    const void* k; const void* v;                    // raw [B, T, G, D]
+    const void* pooled_k; const void* pooled_v;      // [B, G, pool_stride, D]
+    int pool_stride;
+    const float* sink;
+    const void* gamma_q; const void* gamma_kv;
+    void* out;                                       // [B, T, Hq, D]
+    int B, T, Hq, G, D, m, w, rho, rmsnorm, shared;
+    float eps, scale;
+    double theta;
+};
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+bool prefill_simt_supported(int D);
+
+}  // namespace lbca

@@ -1,0 +1,200 @@
+"""Thin ctypes binding of liblbca.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: tensors become raw device pointers, the current torch
+CUDA stream becomes the ``cudaStream_t``, and a non-OK status raises
+``LbcaError``.  PyTorch is used for device memory and streams only.  Importing
+this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbca.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is not built; run `python -m block_compressed_long_b200.build` "
+                      "(needs nvcc) -- there is no CPU fallback")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+LBCA_OK, LBCA_ERR_ARG, LBCA_ERR_UNSUPPORTED, LBCA_ERR_CAPACITY, LBCA_ERR_CUDA, LBCA_ERR_TIMEOUT, \
+    LBCA_ERR_ALIGN = range(7)
+LBCA_F32, LBCA_BF16 = 0, 1
+LBCA_KEY, LBCA_VALUE = 0, 1
+
+ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspace_bytes",
+                "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
+                "lbca_prefill", "lbca_status_string")
+
+
+class lbca_config(ctypes.Structure):
+    _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("shared_kv", ctypes.c_int32),
+                ("block_m", ctypes.c_int32), ("n_win", ctypes.c_int32),
+                ("rope_dims", ctypes.c_int32), ("rmsnorm", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double), ("rms_eps", ctypes.c_float),
+                ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class lbca_cache(ctypes.Structure):
+    _fields_ = [("pooled_k", ctypes.c_void_p), ("pooled_v", ctypes.c_void_p),
+                ("ring_k", ctypes.c_void_p), ("ring_v", ctypes.c_void_p),
+                ("pool_state", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("ring_slots", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_vp, _i32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+_CP, _KP = ctypes.POINTER(lbca_config), ctypes.POINTER(lbca_cache)
+_lib.lbca_ring_slots.argtypes = [_CP]
+_lib.lbca_ring_slots.restype = _i32
+_lib.lbca_pool_state_elems.argtypes = [_CP, _i32]
+_lib.lbca_pool_state_elems.restype = _sz
+_lib.lbca_decode_workspace_bytes.argtypes = [_CP, _i32, _i32]
+_lib.lbca_decode_workspace_bytes.restype = _sz
+_lib.lbca_prefill_workspace_bytes.argtypes = [_CP, _i32, _i32, _i32]
+_lib.lbca_prefill_workspace_bytes.restype = _sz
+_lib.lbca_pool.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp]
+_lib.lbca_pool.restype = ctypes.c_int
+_lib.lbca_append.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp]
+_lib.lbca_append.restype = ctypes.c_int
+_lib.lbca_decode.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _sz, _vp, _vp]
+_lib.lbca_decode.restype = ctypes.c_int
+_lib.lbca_prefill.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
+                              _KP, _vp, _sz, _vp]
+_lib.lbca_prefill.restype = ctypes.c_int
+_lib.lbca_status_string.argtypes = [ctypes.c_int]
+_lib.lbca_status_string.restype = ctypes.c_char_p
+
+
+class LbcaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {lbca_status_string(status)} (status {status})")
+        self.status = status
+
+
+def lbca_status_string(status: int) -> str:
+    return _lib.lbca_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, st: int):
+    if st != LBCA_OK:
+        raise LbcaError(fn, st)
+
+
+def config(n_q_heads, n_kv_heads, head_dim, shared_kv, block_m, n_win, rope_dims=0, rmsnorm=False,
+           rope_theta=10000.0, rms_eps=1e-6, softmax_scale=0.0, dtype="bf16") -> lbca_config:
+    """Build an ``lbca_config`` (dtype "bf16" or "f32")."""
+    return lbca_config(n_q_heads, n_kv_heads, head_dim, int(shared_kv), block_m, n_win, rope_dims,
+                       int(rmsnorm), float(rope_theta), float(rms_eps), float(softmax_scale),
+                       LBCA_BF16 if dtype == "bf16" else LBCA_F32, 0)
+
+
+def torch_dtype(cfg: lbca_config):
+    return torch.bfloat16 if cfg.dtype == LBCA_BF16 else torch.float32
+
+
+def lbca_ring_slots(cfg: lbca_config) -> int:
+    return int(_lib.lbca_ring_slots(ctypes.byref(cfg)))
+
+
+def lbca_pool_state_elems(cfg: lbca_config, batch: int) -> int:
+    return int(_lib.lbca_pool_state_elems(ctypes.byref(cfg), batch))
+
+
+def lbca_decode_workspace_bytes(cfg: lbca_config, batch: int, max_ctx: int) -> int:
+    return int(_lib.lbca_decode_workspace_bytes(ctypes.byref(cfg), batch, max_ctx))
+
+
+def lbca_prefill_workspace_bytes(cfg: lbca_config, batch: int, T: int, has_cache: bool) -> int:
+    return int(_lib.lbca_prefill_workspace_bytes(ctypes.byref(cfg), batch, T, int(has_cache)))
+
+
+@dataclass
+class Cache:
+    """Device tensors of an ``lbca_cache`` (allocated with torch, zero-filled)."""
+    cfg: lbca_config
+    batch: int
+    max_blocks: int
+    ring_slots: int
+    pooled_k: torch.Tensor
+    pooled_v: torch.Tensor | None
+    ring_k: torch.Tensor
+    ring_v: torch.Tensor | None
+    pool_state: torch.Tensor
+    seq_lens: torch.Tensor
+
+    @staticmethod
+    def allocate(cfg: lbca_config, batch: int, max_ctx: int, device="cuda") -> "Cache":
+        G, D = cfg.n_kv_heads, cfg.head_dim
+        dt = torch_dtype(cfg)
+        nb = max_ctx // cfg.block_m
+        R = lbca_ring_slots(cfg)
+        shared = bool(cfg.shared_kv)
+        z = lambda *s, dtype=dt: torch.zeros(*s, dtype=dtype, device=device)  # noqa: E731
+        return Cache(cfg, batch, nb, R, z(batch, G, nb, D), None if shared else z(batch, G, nb, D),
+                     z(batch, G, R, D), None if shared else z(batch, G, R, D),
+                     z(lbca_pool_state_elems(cfg, batch), dtype=torch.float32),
+                     z(batch, dtype=torch.int32))
+
+    def c(self) -> lbca_cache:
+        return lbca_cache(_ptr(self.pooled_k), _ptr(self.pooled_v), _ptr(self.ring_k), _ptr(self.ring_v),
+                          _ptr(self.pool_state), _ptr(self.seq_lens), self.batch, self.max_blocks,
+                          self.ring_slots, 0)
+
+
+def lbca_pool(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, stream=None):
+    """x, z [B, T, G, D]; out [B, G, out_blocks, D]."""
+    B, T = x.shape[0], x.shape[1]
+    ob = out.shape[2] if out_blocks is None else out_blocks
+    _check("lbca_pool", _lib.lbca_pool(ctypes.byref(cfg), series, _ptr(x), _ptr(z), _ptr(b_pos), _ptr(gamma),
+                                       B, T, pos0, _ptr(out), ob, _stream(stream)))
+
+
+def lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache: Cache, d_status=None, stream=None):
+    """k, v, zk, zv [B, G, D]: one token per sequence."""
+    cc = cache.c()
+    _check("lbca_append", _lib.lbca_append(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv),
+                                           _ptr(b_pos_k), _ptr(b_pos_v), _ptr(gamma_kv), ctypes.byref(cc),
+                                           _ptr(d_status), _stream(stream)))
+
+
+def lbca_decode(cfg, q, cache: Cache, sink, gamma_q, out, workspace, max_ctx=0, d_status=None, stream=None):
+    """q, out [B, Hq, D]; workspace a zero-filled uint8 tensor."""
+    cc = cache.c()
+    _check("lbca_decode", _lib.lbca_decode(ctypes.byref(cfg), _ptr(q), ctypes.byref(cc), _ptr(sink),
+                                           _ptr(gamma_q), max_ctx, _ptr(out), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _ptr(d_status),
+                                           _stream(stream)))
+
+
+def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv, out,
+                 cache_out: Cache | None = None, workspace=None, batch=None, T=None, stream=None):
+    """q, out [B, T, Hq, D]; k, v, zk, zv [B, T, G, D]."""
+    B = k.shape[0] if batch is None else batch
+    TT = k.shape[1] if T is None else T
+    cc = cache_out.c() if cache_out is not None else None
+    wb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lbca_prefill", _lib.lbca_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv),
+                                             _ptr(b_pos_k), _ptr(b_pos_v), _ptr(sink), _ptr(gamma_q),
+                                             _ptr(gamma_kv), B, TT, _ptr(out),
+                                             ctypes.byref(cc) if cc is not None else None,
+                                             _ptr(workspace), wb, _stream(stream)))

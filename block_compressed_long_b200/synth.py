@@ -16,7 +16,9 @@ HCA page and the CSA page's "What is implemented").
 """
 from __future__ import annotations
 
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
 import numpy as np
@@ -77,14 +79,39 @@ def _round(a: np.ndarray, dtype: str) -> torch.Tensor:
     return t.to(torch.bfloat16) if dtype == "bf16" else t
 
 
-def normal(seed: int, tag: str, shape, std: float = 1.0, dtype: str = "bf16") -> torch.Tensor:
-    """N(0, std^2) tensor of ``shape`` rounded to ``dtype``; per-row streams along axis 0."""
+CHUNK = 4096  # tokens per random stream along the sequence axis
+
+
+def normal(seed: int, tag: str, shape, std: float = 1.0, dtype: str = "bf16", row_len=None) -> torch.Tensor:
+    """N(0, std^2) tensor of ``shape`` rounded to ``dtype``.  Streams are keyed
+    by (index along axis 0, chunk of CHUNK entries along axis 1), so any
+    sequence or span can be regenerated alone.  With ``row_len``, row i holds
+    draws only in its first row_len[i] entries of axis 1 and zeros after
+    (ragged sequences)."""
     shape = tuple(int(s) for s in shape)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = torch.zeros(shape, dtype=tdt)
     if len(shape) == 0 or shape[0] == 0:
-        return _round(np.zeros(shape, np.float32), dtype)
-    rows = [(_rng(seed, tag, i).standard_normal(shape[1:], dtype=np.float32) * np.float32(std))
-            for i in range(shape[0])]
-    return _round(np.stack(rows), dtype)
+        return out
+    if len(shape) == 1:
+        out[:] = _round(_rng(seed, tag, 0).standard_normal(shape, dtype=np.float32) * np.float32(std), dtype)
+        return out
+    jobs = []
+    for i in range(shape[0]):
+        n = shape[1] if row_len is None else min(int(row_len[i]), shape[1])
+        for c0 in range(0, n, CHUNK):
+            jobs.append((i, c0, min(n, c0 + CHUNK)))
+
+    def fill(job):
+        i, c0, c1 = job
+        a = _rng(seed, tag, i * 1_000_003 + c0 // CHUNK).standard_normal((c1 - c0,) + shape[2:], dtype=np.float32)
+        if std != 1.0:
+            a *= np.float32(std)
+        out[i, c0:c1] = _round(a, dtype)
+
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, jobs))
+    return out
 
 
 def contexts(w: Workload) -> np.ndarray:
@@ -121,10 +148,11 @@ def make(w: Workload) -> Inputs:
         lens = contexts(w)
         T = int(lens.max()) + w.steps
         q = normal(w.seed, "q", (w.steps, B, Hq, D), dtype=w.dtype)
-    k = normal(w.seed, "k", (B, T, G, D), dtype=w.dtype)
-    v = None if w.shared_kv else normal(w.seed, "v", (B, T, G, D), dtype=w.dtype)
-    zk = normal(w.seed, "zk", (B, T, G, D), dtype=w.dtype)
-    zv = None if w.shared_kv else normal(w.seed, "zv", (B, T, G, D), dtype=w.dtype)
+    rl = None if w.kind == "prefill" else lens + w.steps  # history each sequence reaches
+    k = normal(w.seed, "k", (B, T, G, D), dtype=w.dtype, row_len=rl)
+    v = None if w.shared_kv else normal(w.seed, "v", (B, T, G, D), dtype=w.dtype, row_len=rl)
+    zk = normal(w.seed, "zk", (B, T, G, D), dtype=w.dtype, row_len=rl)
+    zv = None if w.shared_kv else normal(w.seed, "zv", (B, T, G, D), dtype=w.dtype, row_len=rl)
     bpk = normal(w.seed, "bpos_k", (m, G * D), std=w.bpos_std, dtype=w.dtype)
     bpv = None if w.shared_kv else normal(w.seed, "bpos_v", (m, G * D), std=w.bpos_std, dtype=w.dtype)
     if w.sink == "none":

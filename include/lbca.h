@@ -1,0 +1,232 @@
+/*
+ * lbca.h -- C ABI of the B200 (sm_100a) block-compressed attention library.
+ *
+ * Block-compressed attention as in LBCA ("mSeek: learned KV-cache compression
+ * in a 3B model", section "How LBCA works") and HCA ("HCA: Heavily Compressed
+ * Attention", section "What is implemented"):
+ *   - every complete, non-overlapping block of m raw tokens is pooled into one
+ *     entry by a per-channel softmax over the block's positions of content
+ *     logits Z plus a learnable positional bias B_pos (HCA page, Eqs 20-23);
+ *   - a query attends, in one softmax, to every causally visible pooled entry
+ *     plus an exact window of recent raw tokens, plus an optional attention
+ *     sink logit (CSA page, "What is implemented": Eqs 18-19 and Eq 27);
+ *   - key entries take RMSNorm (HCA form) and partial RoPE; pooled entries are
+ *     rotated at their block-start position (CSA page, "Deviations from
+ *     paper"); in the shared K=V form the output's RoPE dims are rotated by
+ *     the negative query position (CSA page, "What is implemented").
+ *
+ * Visibility (the reading under which the mSeek README's cache figures come
+ * out exactly): a query at 0-based position t sees L = t + 1 tokens, the
+ * pooled entries j < P(L) = max(0, floor((L - n_win) / m)), and the raw
+ * tokens s in [P(L) * m, t].  Blocks that are incomplete stay raw.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are caller-owned, row-major, contiguous, and 16-byte
+ *     aligned; the library never allocates device memory.  Pointers named
+ *     "device" must be device (or managed) memory of the current device.
+ *   - I/O tensors have the config's dtype (bf16 or f32); arithmetic is f32.
+ *     Sinks are f32 in natural-log units.  gamma pointers are RMSNorm gains
+ *     [D] in the I/O dtype, or NULL for a gain of one.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return value reports host-side validation and
+ *     launch errors only; it never waits for the GPU.  Conditions found on the
+ *     device are written to the optional device word `d_status` (an
+ *     lbca_status; it is only ever set to a non-zero value, so zero it before
+ *     the calls whose outcome you want to read).
+ *   - Nothing aborts the process: bad arguments return LBCA_ERR_ARG before any
+ *     CUDA call, a device other than sm_100 returns LBCA_ERR_UNSUPPORTED.
+ */
+#ifndef LBCA_H
+#define LBCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LBCA_API __attribute__((visibility("default")))
+#else
+#define LBCA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lbca_stream_t; /* == cudaStream_t */
+
+typedef enum {
+    LBCA_OK = 0,
+    LBCA_ERR_ARG = 1,         /* invalid argument (host-side check)            */
+    LBCA_ERR_UNSUPPORTED = 2, /* device is not sm_100, or shape not supported  */
+    LBCA_ERR_CAPACITY = 3,    /* cache or workspace too small for the request  */
+    LBCA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed          */
+    LBCA_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up            */
+    LBCA_ERR_ALIGN = 6        /* a pointer is not 16-byte aligned              */
+} lbca_status;
+
+typedef enum { LBCA_F32 = 0, LBCA_BF16 = 1 } lbca_dtype;
+
+/* Which pooled series lbca_pool produces: keys are finalised (RMSNorm when
+ * enabled, RoPE at the block start); values are stored as pooled.  In the
+ * shared K=V form the single series is LBCA_KEY. */
+typedef enum { LBCA_KEY = 0, LBCA_VALUE = 1 } lbca_series;
+
+typedef struct {
+    int32_t n_q_heads;     /* Hq >= 1                                                 */
+    int32_t n_kv_heads;    /* G >= 1, Hq % G == 0; query head h uses kv head h/(Hq/G) */
+    int32_t head_dim;      /* D: a multiple of 16 in [16, 512]                        */
+    int32_t shared_kv;     /* 1: one entry serves as key and value (HCA MQA form)     */
+    int32_t block_m;       /* m >= 1 raw tokens per pooled entry                      */
+    int32_t n_win;         /* n_win >= 0 raw window                                   */
+    int32_t rope_dims;     /* rho: RoPE on the last rho dims (even, <= D); 0 = off    */
+    int32_t rmsnorm;       /* 1: RMSNorm on queries and key entries (pooled and raw)  */
+    double  rope_theta;    /* base; pair k of the rotated dims turns by
+                              pos * theta^(-2k/rho); consecutive pairs (2k, 2k+1)    */
+    float   rms_eps;       /* RMSNorm epsilon: x / sqrt(mean(x^2) + eps) * gamma      */
+    float   softmax_scale; /* <= 0 selects 1/sqrt(D)                                  */
+    int32_t dtype;         /* lbca_dtype of every I/O tensor                         */
+    int32_t reserved;      /* must be 0                                               */
+} lbca_config;
+
+/*
+ * Decode-time cache of B sequences (caller-owned device memory; zero-filled
+ * memory with seq_lens = 0 is an empty cache).  Written by lbca_prefill and
+ * lbca_append, read by lbca_decode.
+ *   pooled_k   [B, G, max_blocks, D] finalised pooled key entries (shared form:
+ *              the entries, used as key and value)
+ *   pooled_v   [B, G, max_blocks, D] pooled values; NULL in the shared form
+ *   ring_k     [B, G, ring_slots, D] finalised raw keys; token s in slot s % ring_slots
+ *   ring_v     [B, G, ring_slots, D] raw values; NULL in the shared form
+ *   pool_state [B, S, 3, G, D] f32 running (max, sum, weighted sum) of the
+ *              open block's pooling softmax, S = 2 (K then V) or 1 (shared)
+ *   seq_lens   [B] int32 tokens cached per sequence
+ * ring_slots must be >= lbca_ring_slots(cfg).
+ */
+typedef struct {
+    void*    pooled_k;
+    void*    pooled_v;
+    void*    ring_k;
+    void*    ring_v;
+    float*   pool_state;
+    int32_t* seq_lens;
+    int32_t  batch;
+    int32_t  max_blocks;
+    int32_t  ring_slots;
+    int32_t  reserved;     /* must be 0 */
+} lbca_cache;
+
+/* Minimum ring slots: m * ceil((n_win + m - 1) / m), the most raw tokens a
+ * query can see rounded up to whole blocks.  -1 on an invalid config. */
+LBCA_API int32_t lbca_ring_slots(const lbca_config* cfg);
+
+/* f32 elements of lbca_cache.pool_state for `batch` sequences; 0 on error. */
+LBCA_API size_t lbca_pool_state_elems(const lbca_config* cfg, int32_t batch);
+
+/* Bytes of `workspace` lbca_decode needs for `batch` sequences whose lengths
+ * never exceed max_ctx; 0 on error.  The workspace must be zero-filled before
+ * its first use; lbca_decode leaves it zero-filled again. */
+LBCA_API size_t lbca_decode_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
+
+/* Bytes of `workspace` lbca_prefill needs (0 when a cache receives the
+ * pooled entries); (size_t)-1 on error. */
+LBCA_API size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t T,
+                                    int32_t has_cache);
+
+/*
+ * lbca_pool -- pool the floor(T/m) complete blocks of one series.
+ * (HCA page, "What is implemented": single-series pooling, Eqs 20-23; mSeek
+ * README, "How LBCA works", steps 2-3; entry RoPE at block starts: CSA page,
+ * "Deviations from paper".)
+ *   x, z      device [B, T, G, D] raw values and content logits
+ *   b_pos     device [m, G*D] positional bias, indexed by in-block offset
+ *   gamma     device [D] RMSNorm gain (key series with rmsnorm) or NULL
+ *   pos0      absolute position of x's first token; a multiple of m
+ *   out       device [B, G, out_blocks, D]; block j of this call is written at
+ *             index pos0/m + j, which must be < out_blocks
+ * Per (block j, kv head g, channel c):
+ *   w_i = softmax_i(Z[jm+i, g, c] + B_pos[i, g*D + c]),  out = sum_i w_i X[jm+i, g, c],
+ * then, for LBCA_KEY: RMSNorm (when enabled) and RoPE at position pos0 + j*m.
+ * Errors: LBCA_ERR_ARG (null/bad sizes, pos0 % m != 0, out_blocks too small),
+ * LBCA_ERR_ALIGN, LBCA_ERR_UNSUPPORTED, LBCA_ERR_CUDA.
+ */
+LBCA_API lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                      const void* b_pos, const void* gamma, int32_t batch, int32_t T,
+                      int32_t pos0, void* out, int32_t out_blocks, lbca_stream_t stream);
+
+/*
+ * lbca_append -- add one raw token to every sequence of the cache.
+ * (mSeek README, repository layout: generation through the LBCA cache; "How
+ * LBCA works", step 5: incomplete blocks stay raw.)
+ *   k, v, zk, zv  device [B, G, D] the token's key, value and their content
+ *                 logits (shared form: k = C, zk = Z, v = zv = NULL)
+ *   b_pos_k/_v    device [m, G*D] positional biases (b_pos_v NULL when shared)
+ *   gamma_kv      device [D] key RMSNorm gain or NULL
+ * For sequence b the token's position is p = seq_lens[b]: its finalised key
+ * (RMSNorm, RoPE at p) and raw value go to ring slot p % ring_slots, the
+ * running pooling softmax of block p/m is updated, and when p % m == m - 1 the
+ * block's entry is finalised into pooled_k/v[b, :, p/m].  seq_lens[b] becomes
+ * p + 1.  If block p/m >= max_blocks the entry is dropped and d_status is set
+ * to LBCA_ERR_CAPACITY.
+ */
+LBCA_API lbca_status lbca_append(const lbca_config* cfg, const void* k, const void* v, const void* zk,
+                        const void* zv, const void* b_pos_k, const void* b_pos_v,
+                        const void* gamma_kv, const lbca_cache* cache, int32_t* d_status,
+                        lbca_stream_t stream);
+
+/*
+ * lbca_decode -- attention of one query per sequence at its last position.
+ * (mSeek README, "How LBCA works", step 4; HCA page, "What is implemented":
+ * dense attention over all causally visible compressed entries plus the
+ * sliding window, MQA shared KV, RMSNorm, partial RoPE, sink; CSA page,
+ * "What is implemented": Eqs 18-19, Eq 27, the -i output rotation.)
+ *   q          device [B, Hq, D] queries; sequence b's query sits at position
+ *              t = seq_lens[b] - 1 (call lbca_append for the token first)
+ *   sink       device [Hq] f32 sink logits or NULL
+ *   gamma_q    device [D] query RMSNorm gain or NULL
+ *   max_ctx    upper bound of seq_lens (sizes the split grid); <= 0 derives it
+ *              from the cache capacity
+ *   out        device [B, Hq, D]
+ *   workspace  device, >= lbca_decode_workspace_bytes(cfg, B, max_ctx) bytes,
+ *              zero-filled before first use (left zero-filled)
+ * The visible entries are split into chunks processed by separate CTAs; the
+ * last CTA of each (sequence, head group) merges the partial softmaxes.
+ * A sequence with no tokens yields zeros.  A sequence longer than max_ctx sets
+ * d_status to LBCA_ERR_CAPACITY (its output is then incomplete).
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache* cache,
+                        const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                        void* workspace, size_t workspace_bytes, int32_t* d_status,
+                        lbca_stream_t stream);
+
+/*
+ * lbca_prefill -- causal block-compressed attention over T tokens per sequence.
+ * (mSeek README, "How LBCA works", steps 1-5; HCA page, "What is implemented";
+ * CSA page, "What is implemented" and "Deviations from paper".)
+ *   q            device [B, T, Hq, D]
+ *   k, v, zk, zv device [B, T, G, D] (shared form: k = C, zk = Z, v = zv = NULL)
+ *   b_pos_k/_v   device [m, G*D]
+ *   sink         device [Hq] f32 or NULL; gamma_q, gamma_kv device [D] or NULL
+ *   out          device [B, T, Hq, D], or NULL to only fill `cache_out`
+ *   cache_out    NULL, or a cache that receives the pooled entries, the raw
+ *                window, the open block's pooling state and seq_lens = T, so
+ *                that lbca_append / lbca_decode continue the sequences
+ *   workspace    device, lbca_prefill_workspace_bytes(cfg, B, T, cache_out != NULL)
+ * Errors: LBCA_ERR_ARG, LBCA_ERR_ALIGN, LBCA_ERR_CAPACITY (cache too small),
+ * LBCA_ERR_UNSUPPORTED, LBCA_ERR_CUDA.
+ */
+LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, const void* v,
+                         const void* zk, const void* zv, const void* b_pos_k,
+                         const void* b_pos_v, const float* sink, const void* gamma_q,
+                         const void* gamma_kv, int32_t batch, int32_t T, void* out,
+                         const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
+                         lbca_stream_t stream);
+
+/* Static text for a status code. */
+LBCA_API const char* lbca_status_string(lbca_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LBCA_H */

@@ -197,42 +197,62 @@ def decode(cfg: Config, q, k, v, zk, zv, bpos_k, bpos_v, lens, sink=None,
 class Stream:
     """Token-by-token form of the same definition for one sequence.
 
-    ``append`` adds one raw token; when it completes a block the block is
-    pooled and finalised once and kept.  ``query`` attends one query at the
-    position of the last appended token.  The arithmetic is the C oracle's.
+    ``extend`` adds raw tokens; each block they complete is pooled and
+    finalised once and kept.  ``query`` attends one query at the position of
+    the last appended token.  The arithmetic is the C oracle's; the buffers
+    grow by doubling so that a step does not copy the history.
     """
 
     def __init__(self, cfg: Config, bpos_k, bpos_v=None, gamma_kv=None):
         self.cfg = cfg
         self.bpos_k, self.bpos_v, self.gamma_kv = bpos_k, bpos_v, gamma_kv
-        G, D = cfg.n_kv_heads, cfg.head_dim
-        self.k = np.zeros((0, G, D)); self.zk = np.zeros((0, G, D))
-        self.v = np.zeros((0, G, D)); self.zv = np.zeros((0, G, D))
-        self.ek = np.zeros((0, G, D)); self.ev = np.zeros((0, G, D))
+        self.n = 0
+        self.nb = 0
+        self._buf = {}
+
+    def _grow(self, name, need, row):
+        b = self._buf.get(name)
+        if b is None or b.shape[0] < need:
+            nb = np.zeros((max(need, 2 * (0 if b is None else b.shape[0]), 64),) + row)
+            if b is not None:
+                nb[:b.shape[0]] = b
+            self._buf[name] = nb
+        return self._buf[name]
+
+    def _arr(self, name, n):
+        b = self._buf.get(name)
+        return None if b is None else b[:n]
 
     def extend(self, k, zk, v=None, zv=None):
         """Append a run of raw tokens [n, G, D] (pools every block it completes)."""
         m = self.cfg.block_m
-        self.k = np.concatenate([self.k, k]); self.zk = np.concatenate([self.zk, zk])
-        if not self.cfg.shared_kv:
-            self.v = np.concatenate([self.v, v]); self.zv = np.concatenate([self.zv, zv])
-        done = self.k.shape[0] // m
-        have = self.ek.shape[0]
-        if done > have:
-            sl = slice(have * m, done * m)
-            self.ek = np.concatenate([self.ek, pool(self.cfg, KEY, self.k[None, sl], self.zk[None, sl],
-                                                    self.bpos_k, self.gamma_kv, pos0=have * m)[0]])
+        row = (self.cfg.n_kv_heads, self.cfg.head_dim)
+        new = np.asarray(k).shape[0]
+        names = [("k", k), ("zk", zk)] + ([] if self.cfg.shared_kv else [("v", v), ("zv", zv)])
+        for name, a in names:
+            self._grow(name, self.n + new, row)[self.n:self.n + new] = a
+        self.n += new
+        done = self.n // m
+        if done > self.nb:
+            sl = slice(self.nb * m, done * m)
+            ek = pool(self.cfg, KEY, self._buf["k"][None, sl], self._buf["zk"][None, sl], self.bpos_k,
+                      self.gamma_kv, pos0=self.nb * m)[0]
+            self._grow("ek", done, row)[self.nb:done] = ek
             if not self.cfg.shared_kv:
-                self.ev = np.concatenate([self.ev, pool(self.cfg, VALUE, self.v[None, sl],
-                                                        self.zv[None, sl], self.bpos_v)[0]])
+                ev = pool(self.cfg, VALUE, self._buf["v"][None, sl], self._buf["zv"][None, sl], self.bpos_v)[0]
+                self._grow("ev", done, row)[self.nb:done] = ev
+            self.nb = done
 
     def query(self, q, sink=None, gamma_q=None):
         """Output [Hq, D] for query q [Hq, D] at the last appended position."""
-        L = self.k.shape[0]
-        v = None if self.cfg.shared_kv else self.v[None]
-        ev = None if self.cfg.shared_kv else self.ev[None]
-        return attend(self.cfg, np.asarray(q)[None, None], np.array([[L - 1]]), self.ek[None], ev,
-                      self.k[None], v, np.array([L]), sink, gamma_q, self.gamma_kv)[0, 0]
+        L = self.n
+        shared = self.cfg.shared_kv
+        ek = self._arr("ek", self.nb)
+        ev = None if shared else self._arr("ev", self.nb)
+        return attend(self.cfg, np.asarray(q)[None, None], np.array([[L - 1]]),
+                      None if ek is None else ek[None], None if ev is None else ev[None],
+                      self._arr("k", L)[None], None if shared else self._arr("v", L)[None],
+                      np.array([L]), sink, gamma_q, self.gamma_kv)[0, 0]
 
 
 def cache_entries(T: int, m: int, w: int) -> int:

@@ -1,0 +1,139 @@
+"""Shared helpers for the GPU parity tests: run a workload through the C ABI
+and through the fp64 oracle on the same seeded inputs, and compare.
+
+Tolerances (fixed by the method's target): bf16 I/O -> max-abs <= 1e-2 and
+mean-abs <= 1e-3; f32 I/O -> max-abs <= 1e-5 * max|oracle| (relative 1e-5).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from block_compressed_long_b200 import synth
+from oracle import oracle as orc
+
+f64 = synth.f64
+
+
+def lib():
+    from block_compressed_long_b200 import build
+    build.build()
+    from block_compressed_long_b200 import lbca
+    return lbca
+
+
+def ocfg(w: synth.Workload) -> orc.Config:
+    return orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win,
+                      w.rope_dims, w.rmsnorm, w.rope_theta)
+
+
+def lcfg(L, w: synth.Workload):
+    return L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                    w.rmsnorm, w.rope_theta, dtype=w.dtype)
+
+
+def assert_close(got, want, dtype: str, what: str = ""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    d = np.abs(got - want)
+    if dtype == "bf16":
+        assert d.max() <= 1e-2, f"{what}: max-abs {d.max():.3e}"
+        assert d.mean() <= 1e-3, f"{what}: mean-abs {d.mean():.3e}"
+    else:
+        scale = max(np.abs(want).max(), 1e-30)
+        assert d.max() <= 1e-5 * scale, f"{what}: max-abs {d.max():.3e} vs 1e-5 * {scale:.3e}"
+    return float(d.max()), float(d.mean())
+
+
+def dev(t):
+    return None if t is None else t.cuda()
+
+
+def sub_cache(L, cache, b):
+    """The one-sequence view of sequence b of a batched cache (contiguous slices)."""
+    per = cache.pool_state.numel() // cache.batch
+    sl = slice(b, b + 1)
+    return L.Cache(cache.cfg, 1, cache.max_blocks, cache.ring_slots, cache.pooled_k[sl],
+                   None if cache.pooled_v is None else cache.pooled_v[sl], cache.ring_k[sl],
+                   None if cache.ring_v is None else cache.ring_v[sl],
+                   cache.pool_state[b * per:(b + 1) * per], cache.seq_lens[sl])
+
+
+def gpu_prefill(L, w, inp, cache=None, want_out=True, T=None):
+    """Prefill of the first T tokens (all by default) of every sequence."""
+    cfg = lcfg(L, w)
+    T = inp.k.shape[1] if T is None else T
+    B = inp.k.shape[0]
+    sl = lambda t: None if t is None else t[:, :T].contiguous().cuda()  # noqa: E731
+    q = sl(inp.q) if want_out else None
+    out = torch.empty(B, T, w.n_q_heads, w.head_dim, dtype=L.torch_dtype(cfg), device="cuda") if want_out else None
+    ws = torch.zeros(max(L.lbca_prefill_workspace_bytes(cfg, B, T, cache is not None), 16), dtype=torch.uint8,
+                     device="cuda")
+    L.lbca_prefill(cfg, q, sl(inp.k), sl(inp.v), sl(inp.zk), sl(inp.zv), dev(inp.bpos_k), dev(inp.bpos_v),
+                   dev(inp.sink), None, None, out, cache, ws, batch=B, T=T)
+    return out
+
+
+def oracle_prefill(w, inp, rows=None, T=None):
+    T = inp.k.shape[1] if T is None else T
+    sl = lambda t: None if t is None else f64(t[:, :T])  # noqa: E731
+    return orc.forward(ocfg(w), sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.zk), sl(inp.zv), f64(inp.bpos_k),
+                       f64(inp.bpos_v), f64(inp.sink), rows=rows)
+
+
+class DecodeRun:
+    """Drive a decode workload through the C ABI: prefill every sequence's
+    cached context into the cache, then (append, decode) one token per step."""
+
+    def __init__(self, L, w, inp, steps=None, chunked_prefill=True):
+        self.L, self.w, self.inp = L, w, inp
+        self.cfg = lcfg(L, w)
+        self.B = inp.k.shape[0]
+        self.steps = w.steps if steps is None else steps
+        self.max_ctx = int(inp.lens.max()) + self.steps
+        self.cache = L.Cache.allocate(self.cfg, self.B, self.max_ctx)
+        self.k, self.v, self.zk, self.zv = (dev(t) for t in (inp.k, inp.v, inp.zk, inp.zv))
+        self.bpk, self.bpv, self.sink = dev(inp.bpos_k), dev(inp.bpos_v), dev(inp.sink)
+        self.q = dev(inp.q)
+        for b in range(self.B):
+            Lb = int(inp.lens[b])
+            sc = sub_cache(L, self.cache, b)
+            s = lambda t: None if t is None else t[b:b + 1, :Lb]  # noqa: E731
+            ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
+            L.lbca_prefill(self.cfg, None, s(self.k), s(self.v), s(self.zk), s(self.zv), self.bpk, self.bpv,
+                           None, None, None, None, sc, ws, batch=1, T=Lb)
+        self.ws = torch.zeros(L.lbca_decode_workspace_bytes(self.cfg, self.B, self.max_ctx), dtype=torch.uint8,
+                              device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.pos = torch.as_tensor(inp.lens, device="cuda")
+        self.ar = torch.arange(self.B, device="cuda")
+        self.step_i = 0
+
+    def token(self, t):
+        return None if t is None else t[self.ar, self.pos].contiguous()
+
+    def step(self):
+        L = self.L
+        L.lbca_append(self.cfg, self.token(self.k), self.token(self.v), self.token(self.zk), self.token(self.zv),
+                      self.bpk, self.bpv, None, self.cache, self.status)
+        out = torch.empty(self.B, self.w.n_q_heads, self.w.head_dim, dtype=L.torch_dtype(self.cfg), device="cuda")
+        L.lbca_decode(self.cfg, self.q[self.step_i], self.cache, self.sink, None, out, self.ws, self.max_ctx,
+                      self.status)
+        self.pos += 1
+        self.step_i += 1
+        return out
+
+
+def oracle_decode(w, inp, step, seqs=None):
+    """Oracle output of decode step `step` (0-based) for the sequences `seqs`."""
+    seqs = range(inp.k.shape[0]) if seqs is None else seqs
+    c = ocfg(w)
+    outs = []
+    for b in seqs:
+        Lb = int(inp.lens[b]) + step + 1
+        s = lambda t: None if t is None else f64(t[b:b + 1, :Lb])  # noqa: E731
+        outs.append(orc.decode(c, f64(inp.q[step, b:b + 1]), s(inp.k), s(inp.v), s(inp.zk), s(inp.zv),
+                               f64(inp.bpos_k), f64(inp.bpos_v), [Lb], f64(inp.sink))[0])
+    return np.stack(outs)

@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports every entry point include/lbca.h declares,
+matches the header's struct layouts, and rejects bad arguments on the host
+(before any CUDA call, so these run without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lbca.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_compressed_long_b200 import build
+    build.build()
+    from block_compressed_long_b200 import lbca
+    return lbca
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lbca_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(L._LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.ENTRY_POINTS)
+
+
+def test_struct_layout_matches_header(L, tmp_path):
+    prog = tmp_path / "sz.c"
+    prog.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "lbca.h"\n'
+                    'int main(void){printf("%zu %zu %zu %zu %zu\\n", sizeof(lbca_config), sizeof(lbca_cache),'
+                    ' offsetof(lbca_config, rope_theta), offsetof(lbca_config, dtype),'
+                    ' offsetof(lbca_cache, batch));return 0;}\n')
+    exe = tmp_path / "sz"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)])
+    got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    want = [ctypes.sizeof(L.lbca_config), ctypes.sizeof(L.lbca_cache), L.lbca_config.rope_theta.offset,
+            L.lbca_config.dtype.offset, L.lbca_cache.batch.offset]
+    assert got == want
+
+
+def _cfg(L, **kw):
+    base = dict(n_q_heads=24, n_kv_heads=8, head_dim=128, shared_kv=False, block_m=64, n_win=128,
+                rope_dims=128)
+    base.update(kw)
+    return L.config(**base)
+
+
+def test_ring_slots(L):
+    assert L.lbca_ring_slots(_cfg(L)) == 192                       # m=64, w=128
+    assert L.lbca_ring_slots(_cfg(L, block_m=16)) == 144
+    assert L.lbca_ring_slots(_cfg(L, n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True,
+                                  block_m=128, rope_dims=64)) == 256
+    assert L.lbca_ring_slots(_cfg(L, block_m=1, n_win=0)) == 1
+    assert L.lbca_ring_slots(_cfg(L, block_m=0)) == -1
+
+
+@pytest.mark.parametrize("bad", [dict(n_q_heads=25), dict(head_dim=100), dict(head_dim=1024),
+                                 dict(block_m=0), dict(n_win=-1), dict(rope_dims=3),
+                                 dict(rope_dims=256), dict(rope_theta=0.0)])
+def test_bad_config_rejected(L, bad):
+    cfg = _cfg(L, **bad)
+    A = 0x10000
+    st = L._lib.lbca_pool(ctypes.byref(cfg), 0, A, A, A, None, 1, 64, 0, A, 1, None)
+    assert st == L.LBCA_ERR_ARG
+
+
+def test_pool_argument_checks(L):
+    cfg = _cfg(L)
+    A = 0x10000
+    f = lambda *a: L._lib.lbca_pool(ctypes.byref(cfg), *a)  # noqa: E731
+    assert f(0, None, A, A, None, 1, 64, 0, A, 1, None) == L.LBCA_ERR_ARG        # null x
+    assert f(0, A, A, A, None, 1, 64, 3, A, 8, None) == L.LBCA_ERR_ARG           # pos0 % m
+    assert f(0, A, A, A, None, 1, 640, 0, A, 9, None) == L.LBCA_ERR_ARG          # out_blocks too small
+    assert f(0, A + 8, A, A, None, 1, 64, 0, A, 1, None) == L.LBCA_ERR_ALIGN     # misaligned
+    assert f(7, A, A, A, None, 1, 64, 0, A, 1, None) == L.LBCA_ERR_ARG           # series
+    shared = _cfg(L, n_q_heads=4, n_kv_heads=1, shared_kv=True)
+    assert L._lib.lbca_pool(ctypes.byref(shared), 1, A, A, A, None, 1, 64, 0, A, 1, None) == L.LBCA_ERR_ARG
+    # a valid call with no GPU present must not succeed: there is no CPU fallback
+    assert f(0, A, A, A, None, 1, 64, 0, A, 1, None) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
+
+
+def test_cache_and_decode_checks(L):
+    cfg = _cfg(L)
+    A = 0x10000
+    cache = L.lbca_cache(A, A, A, A, A, A, 1, 600, 192, 0)
+    small = L.lbca_cache(A, A, A, A, A, A, 1, 600, 100, 0)
+    shared_bad = L.lbca_cache(A, None, A, None, A, A, 1, 600, 192, 0)
+    ws = L.lbca_decode_workspace_bytes(cfg, 1, 32769)
+    assert ws > 0
+    dec = lambda c, wsb: L._lib.lbca_decode(ctypes.byref(cfg), A, ctypes.byref(c), None, None, 32769,  # noqa
+                                            A, A, wsb, None, None)
+    assert dec(small, ws) == L.LBCA_ERR_CAPACITY          # ring too small for the window
+    assert dec(shared_bad, ws) == L.LBCA_ERR_ARG          # GQA needs pooled_v / ring_v
+    assert dec(cache, ws - 1) == L.LBCA_ERR_CAPACITY      # workspace too small
+    assert dec(cache, ws) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
+    app = L._lib.lbca_append(ctypes.byref(cfg), A, None, A, A, A, A, None, ctypes.byref(cache), None, None)
+    assert app == L.LBCA_ERR_ARG                          # GQA needs v
+    pre = L._lib.lbca_prefill(ctypes.byref(cfg), A, A, A, A, A, A, A, None, None, None, 1, 64, None, None,
+                              None, 0, None)
+    assert pre == L.LBCA_ERR_ARG                          # neither out nor cache
+    pre = L._lib.lbca_prefill(ctypes.byref(cfg), A, A, A, A, A, A, A, None, None, None, 1, 6400, A, None,
+                              None, 0, None)
+    assert pre == L.LBCA_ERR_CAPACITY                     # pooled entries need a workspace
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.lbca_status_string(s)

@@ -188,12 +188,31 @@ def run_ours(args, w, rank, world):
 
     n_steps = 2 * (args.warmup + args.steps)
     bench = DecodeBench(w, n_steps, rank)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    L = bench.L
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
+    # warm-up: eager launches (first calls set kernel attributes)
     for _ in range(args.warmup):
         flush.zero_()
         bench.step()
+    torch.cuda.synchronize()
+
+    # every step is replayed from CUDA graphs captured up front: the append and
+    # the decode of step i in two graphs, so that events between them time the
+    # decode kernel alone on its stream
+    cap = torch.cuda.Stream()
+    g = lambda t, i: None if t is None else t[i]  # noqa: E731
+    graphs = []
+    for i in range(bench.i, bench.i + args.steps):
+        ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga, stream=cap):
+            L.lbca_append(bench.cfg, g(bench.tk, i), g(bench.tv, i), g(bench.tzk, i), g(bench.tzv, i), bench.bpk,
+                          bench.bpv, None, bench.cache, bench.status)
+        with torch.cuda.graph(gd, stream=cap):
+            L.lbca_decode(bench.cfg, bench.q[i], bench.cache, bench.sink, None, bench.out, bench.ws, bench.max_ctx,
+                          bench.status)
+        graphs.append((ga, gd))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -207,34 +226,37 @@ def run_ours(args, w, rank, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    for s in range(args.steps):
+    for s_, (ga, gd) in enumerate(graphs):
         flush.zero_()
         nbytes += bytes_per_decode(bench.w, bench.lens_now())
-        step_ev[s][0].record()
-        bench.step(dec_ev[s])
-        step_ev[s][1].record()
+        step_ev[s_][0].record()
+        ga.replay()
+        dec_ev[s_][0].record()
+        gd.replay()
+        dec_ev[s_][1].record()
+        step_ev[s_][1].record()
+        bench.i += 1
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     step_ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
+    del graphs
 
     # ---- end to end through the public API: pinned host inputs and output ----
     w_ = bench.w
     pin = lambda t: None if t is None else t.cpu().pin_memory()  # noqa: E731
     hq = pin(bench.q)
-    htk, htv, htzk, htzv = (pin(t) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv))
+    htok = [pin(t) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)]
     dq = torch.empty_like(bench.q[0])
     dtok = [None if t is None else torch.empty_like(t[0]) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)]
     hout = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
-    L = bench.L
-    h2d = d2h = 0
+    h2d = dq.numel() * dq.element_size() + sum(t.numel() * t.element_size() for t in dtok if t is not None)
+    d2h = hout.numel() * hout.element_size()
 
-    def e2e_step():
-        nonlocal h2d, d2h
-        i = bench.i
+    def e2e_body(i):
         dq.copy_(hq[i], non_blocking=True)
-        for dt, ht in zip(dtok, (htk, htv, htzk, htzv)):
+        for dt, ht in zip(dtok, htok):
             if dt is not None:
                 dt.copy_(ht[i], non_blocking=True)
         L.lbca_append(bench.cfg, dtok[0], dtok[1], dtok[2], dtok[3], bench.bpk, bench.bpv, None, bench.cache,
@@ -242,22 +264,29 @@ def run_ours(args, w, rank, world):
         L.lbca_decode(bench.cfg, dq, bench.cache, bench.sink, None, bench.out, bench.ws, bench.max_ctx,
                       bench.status)
         hout.copy_(bench.out, non_blocking=True)
-        bench.i += 1
-        h2d = dq.numel() * dq.element_size() + sum(t.numel() * t.element_size() for t in dtok if t is not None)
-        d2h = hout.numel() * hout.element_size()
 
     for _ in range(args.warmup):
         flush.zero_()
-        e2e_step()
+        e2e_body(bench.i)
+        bench.i += 1
+    torch.cuda.synchronize()
+    egraphs = []
+    for i in range(bench.i, bench.i + args.steps):
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=cap):
+            e2e_body(i)
+        egraphs.append(ge)
     torch.cuda.synchronize()
     e2e_ev = [(E(), E()) for _ in range(args.steps)]
-    for s in range(args.steps):
+    for s_, ge in enumerate(egraphs):
         flush.zero_()
-        e2e_ev[s][0].record()
-        e2e_step()
-        e2e_ev[s][1].record()
+        e2e_ev[s_][0].record()
+        ge.replay()
+        e2e_ev[s_][1].record()
+        bench.i += 1
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    del egraphs
     clocks = sampler.stop()
     status = int(bench.status.item())
     if status:
@@ -279,7 +308,8 @@ def run_ours(args, w, rank, world):
                    "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
                    "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
                    "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
-                   "l2": "flushed (256 MiB write) before every timed step, outside its events"},
+                   "l2": "flushed (512 MiB write) before every timed step, outside its events",
+                   "launch": "each step replayed from CUDA graphs (append, decode)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src, "kernel": "decode_kernel",
                      "bytes_per_launch": nbytes / args.steps, "launch_us": dec_ms * 1e3,

@@ -311,23 +311,50 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
     __syncthreads();
     if (!*flag) return;
     __threadfence();
+    // split weights 2^(m_s - M) per head, staged in shared memory (the group
+    // reduction buffers are free now): all partial statistics load at once
+    float* wsm = red_o;   // [nsp][R] (m, l) pairs, then (weight, l)
+    float* mh = red_ml;   // [R] max, [R, 2R) denominator
+    for (int idx = tid; idx < nsp * R; idx += kThreads) {
+        const int sp = idx / R, h = idx % R;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+            a.part_ml + (((size_t)b * a.Hq + h0 + h) * a.n_split + sp) * 2));
+        wsm[2 * idx] = ml.x;
+        wsm[2 * idx + 1] = ml.y;
+    }
+    __syncthreads();
+    if (warp < R) {
+        const int h = warp;
+        float M = kNegInf;
+        for (int sp = lane; sp < nsp; sp += 32) M = fmaxf(M, wsm[2 * (sp * R + h)]);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float Ls = 0.f;
+        for (int sp = lane; sp < nsp; sp += 32) {
+            const float f = M == kNegInf ? 0.f : ex2(wsm[2 * (sp * R + h)] - M);
+            wsm[2 * (sp * R + h)] = f;
+            Ls = fmaf(f, wsm[2 * (sp * R + h) + 1], Ls);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+        if (lane == 0) {
+            mh[h] = M;
+            mh[R + h] = Ls;
+        }
+    }
+    __syncthreads();
     for (int idx = tid; idx < R * D / 2; idx += kThreads) {
         const int h = idx / (D / 2), d = (idx % (D / 2)) * 2;
-        const size_t pb = ((size_t)b * a.Hq + h0 + h) * a.n_split;
-        float M = kNegInf;
-        for (int s = 0; s < nsp; ++s) M = fmaxf(M, __ldcg(a.part_ml + (pb + s) * 2));
-        float Ls = 0.f, o0 = 0.f, o1 = 0.f;
-        if (M != kNegInf) {
-            for (int s = 0; s < nsp; ++s) {
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + (pb + s) * 2));
-                const float f = ex2(ml.x - M);
-                const float2 ov = __ldcg(reinterpret_cast<const float2*>(a.part_o + (pb + s) * D + d));
-                Ls = fmaf(ml.y, f, Ls);
-                o0 = fmaf(ov.x, f, o0);
-                o1 = fmaf(ov.y, f, o1);
-            }
+        const float* po = a.part_o + ((size_t)b * a.Hq + h0 + h) * a.n_split * D + d;
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll 8
+        for (int sp = 0; sp < nsp; ++sp) {
+            const float f = wsm[2 * (sp * R + h)];
+            const float2 ov = __ldcg(reinterpret_cast<const float2*>(po + (size_t)sp * D));
+            o0 = fmaf(ov.x, f, o0);
+            o1 = fmaf(ov.y, f, o1);
         }
-        finalise(h, d, o0, o1, M, Ls);
+        finalise(h, d, o0, o1, mh[h], mh[R + h]);
     }
     if (tid == 0) *ctr = 0u;
 }
@@ -400,7 +427,8 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int
     p.part_ml_elems = (size_t)B * Hq * p.n_split * 2;
     p.counter_elems = (size_t)B * (Hq / R);
     p.smem_bytes = layout(D, R, chunk, esize, shared).total;
-    p.ok = p.smem_bytes <= 200 * 1024;
+    // the merge stages 2 floats per (split, head) in the group-reduction buffer
+    p.ok = p.smem_bytes <= 200 * 1024 && p.n_split * 2 <= (2048 / D) * D;
     return p;
 }
 

@@ -43,6 +43,11 @@ float scale_of(const lbca_config* c) {
     return c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt((float)c->head_dim);
 }
 
+// theta^(-2/rho): pair k of the rotated dims turns by step^k radians per position
+double rope_step_of(const lbca_config* c) {
+    return c->rope_dims > 0 ? std::pow(c->rope_theta, -2.0 / (double)c->rope_dims) : 1.0;
+}
+
 int ring_min(const lbca_config* c) {
     const long long m = c->block_m;
     long long r = m * ((c->n_win + m - 1 + m - 1) / m);
@@ -84,12 +89,13 @@ lbca_status check_cache(const lbca_config* c, const lbca_cache* k) {
 }
 
 // K-side / V-side pointer set: shared form needs exactly the K side.
+// `need_tokens` is false for a zero-token prefill, whose k, v, zk, zv may be NULL.
 lbca_status check_kv(const lbca_config* c, const void* k, const void* v, const void* zk, const void* zv,
-                     const void* bk, const void* bv) {
-    if (!k || !zk || !bk) return LBCA_ERR_ARG;
+                     const void* bk, const void* bv, bool need_tokens = true) {
+    if ((need_tokens && (!k || !zk)) || !bk) return LBCA_ERR_ARG;
     if (c->shared_kv) {
         if (v || zv || bv) return LBCA_ERR_ARG;
-    } else if (!v || !zv || !bv) {
+    } else if ((need_tokens && (!v || !zv)) || !bv) {
         return LBCA_ERR_ARG;
     }
     if (!al16(k) || !al16(zk) || !al16(bk) || !al16n(v) || !al16n(zv) || !al16n(bv)) return LBCA_ERR_ALIGN;
@@ -152,7 +158,7 @@ lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, con
     a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
     a.pos0 = pos0;
     a.key = series == LBCA_KEY; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
-    a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+    a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
     a.state = nullptr; a.S = 1; a.series = 0;
     return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -173,7 +179,7 @@ lbca_status lbca_append(const lbca_config* cfg, const void* k, const void* v, co
     a.state = cache->pool_state; a.seq_lens = cache->seq_lens; a.status = d_status;
     a.B = cache->batch; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
     a.R = cache->ring_slots; a.max_blocks = cache->max_blocks; a.S = cfg->shared_kv ? 1 : 2;
-    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims; a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims; a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
     return cuda_status(launch_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -208,7 +214,7 @@ lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache*
     a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
     a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
-    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.theta = cfg->rope_theta;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
     return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -218,8 +224,8 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
                          const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
                          lbca_stream_t stream) {
     LBCA_TRY(check_cfg(cfg));
-    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v));
     if (batch < 0 || T < 0) return LBCA_ERR_ARG;
+    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v, T > 0 && batch > 0));
     if (!out && !cache_out) return LBCA_ERR_ARG;
     if (out && !q) return LBCA_ERR_ARG;
     if (!al16n(q) || !al16n(out) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink) ||
@@ -254,7 +260,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.out = series ? pv : pk; a.out_blocks = stride; a.blk_off = 0;
         a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = m; a.pos0 = 0;
         a.key = series == 0; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
-        a.theta = cfg->rope_theta; a.eps = cfg->rms_eps;
+        a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
         a.state = cache_out ? cache_out->pool_state : nullptr;
         a.S = cfg->shared_kv ? 1 : 2; a.series = series;
         LBCA_TRY(cuda_status(launch_pool(a, s)));
@@ -267,7 +273,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         r.ring_k = cache_out->ring_k; r.ring_v = cache_out->ring_v; r.seq_lens = cache_out->seq_lens;
         r.B = batch; r.T = T; r.G = cfg->n_kv_heads; r.D = cfg->head_dim; r.R = cache_out->ring_slots;
         r.n = T < r.R ? T : r.R;
-        r.rmsnorm = cfg->rmsnorm; r.rho = cfg->rope_dims; r.theta = cfg->rope_theta; r.eps = cfg->rms_eps;
+        r.rmsnorm = cfg->rmsnorm; r.rho = cfg->rope_dims; r.rope_step = rope_step_of(cfg); r.eps = cfg->rms_eps;
         LBCA_TRY(cuda_status(launch_ring_fill(r, s)));
     }
     // 3. attention
@@ -278,7 +284,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.pool_stride = stride; a.sink = sink; a.gamma_q = gamma_q; a.gamma_kv = gamma_kv; a.out = out;
         a.B = batch; a.T = T; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
         a.m = m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
-        a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.theta = cfg->rope_theta;
+        a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
         LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
     }
     return LBCA_OK;

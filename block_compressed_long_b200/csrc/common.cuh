@@ -81,14 +81,27 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 }
 
 // ---- RoPE -------------------------------------------------------------------------
-// Pair k (dims D - rho + 2k, +1) turns by pos * theta^(-2k/rho).  The angle is
-// formed and reduced in fp64 (positions reach 1e5+, where an fp32 product loses
-// milliradians) and only the resulting cos/sin are rounded to f32.
-__device__ __forceinline__ float2 rope_cs(double pos, int k, int rho, double theta) {
-    double inv = pow(theta, -2.0 * (double)k / (double)rho);
-    double s, c;
-    sincos(pos * inv, &s, &c);
-    return make_float2((float)c, (float)s);
+// Pair k (dims D - rho + 2k, +1) turns by pos * inv_k radians per position,
+// inv_k = theta^(-2k/rho) = step^k with step = theta^(-2/rho) computed in fp64 on
+// the host.  Positions reach 1e5+, where an fp32 product pos * inv_k would be
+// off by milliradians, so the angle is formed in turns in 64-bit fixed point:
+// F_k = inv_k / (2 pi) * 2^64 and pos * F_k wraps exactly modulo one turn (two's
+// complement makes negative positions come out right too).  The top 24 bits of
+// the fraction (2^-24 turn resolution) then go to sincospif on [0, 2).
+__device__ __forceinline__ float2 rope_cs(int64_t pos, int k, double step) {
+    double inv = 1.0, b = step;
+    for (int e = k; e; e >>= 1) {
+        if (e & 1) inv *= b;
+        b *= b;
+    }
+    const double kTurn = 0.15915494309189535;            // 1 / (2 pi)
+    const double kTwo64 = 18446744073709551616.0;        // 2^64
+    const uint64_t F = (uint64_t)(inv * kTurn * kTwo64);
+    const uint64_t t = (uint64_t)pos * F;
+    const float x = (float)(uint32_t)(t >> 40) * (1.0f / 16777216.0f);
+    float sn, cs;
+    sincospif(2.0f * x, &sn, &cs);
+    return make_float2(cs, sn);
 }
 __device__ __forceinline__ void rotate_pair(float& a, float& b, float2 cs) {
     float x = a, y = b;

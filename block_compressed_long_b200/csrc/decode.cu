@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
     }
 
     // ---- query prep overlaps the copies: RMSNorm, RoPE at t, log2-domain scale ----
-    for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((double)t, k, a.rho, a.theta);
+    for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((int64_t)t, k, a.rope_step);
     for (int idx = tid; idx < R * D / VEC; idx += kThreads) {
         const int h = idx / (D / VEC), c = idx % (D / VEC);
         float v[VEC];
@@ -418,7 +418,7 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int
     const long long groups = (long long)B * (Hq / R);
     int chunk = kMinChunk;
     for (int c = cmax; c >= kMinChunk; c /= 2) {
-        if (groups * ((max_vis + c - 1) / c) >= 2 * 148) { chunk = c; break; }
+        if (groups * ((max_vis + c - 1) / c) >= 148) { chunk = c; break; }  // one wave of SMs
     }
     p.heads_per_cta = R;
     p.chunk = chunk;

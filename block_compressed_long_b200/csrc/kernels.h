@@ -20,7 +20,7 @@ struct PoolArgs {
     int B, T, G, D, m;
     int64_t pos0;          // absolute position of token 0 of x
     int key, rmsnorm, rho;
-    double theta;
+    double rope_step;  // theta^(-2/rho)
     float eps;
     float* state;          // [B, S, 3, G, D] or null: running state of the partial block
     int S, series;
@@ -39,7 +39,7 @@ struct RingFillArgs {
     int32_t* seq_lens;
     int B, T, G, D, R, n;
     int rmsnorm, rho;
-    double theta;
+    double rope_step;  // theta^(-2/rho)
     float eps;
 };
 cudaError_t launch_ring_fill(const RingFillArgs& a, cudaStream_t s);
@@ -56,7 +56,7 @@ struct AppendArgs {
     int32_t* status;
     int B, G, D, m, R, max_blocks, S;
     int rmsnorm, rho;
-    double theta;
+    double rope_step;  // theta^(-2/rho)
     float eps;
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
@@ -77,7 +77,7 @@ struct DecodeArgs {
     int B, Hq, G, D, m, w, rho, rmsnorm, shared, max_blocks, R;
     int n_split, chunk, heads_per_cta;
     float eps, scale;
-    double theta;
+    double rope_step;  // theta^(-2/rho)
 };
 // Chooses heads per CTA, chunk and split count for a decode call.
 struct DecodePlan {
@@ -102,7 +102,7 @@ struct PrefillArgs {
     void* out;                                       // [B, T, Hq, D]
     int B, T, Hq, G, D, m, w, rho, rmsnorm, shared;
     float eps, scale;
-    double theta;
+    double rope_step;  // theta^(-2/rho)
 };
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 bool prefill_simt_supported(int D);

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
     float* part = smem + a.rho;
     if (full && a.key && a.rho)
         for (int k = tid; k < a.rho / 2; k += blockDim.x)
-            cs[k] = rope_cs((double)(a.pos0 + (int64_t)j * a.m), k, a.rho, a.theta);
+            cs[k] = rope_cs(a.pos0 + (int64_t)j * a.m, k, a.rope_step);
     __syncthreads();
 
     const size_t row0 = ((size_t)b * a.T + (size_t)j * a.m) * GD + (size_t)cv * VEC;
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(1024) ring_fill_kernel(const RingFillArgs a) {
     const int cv = active ? tid : 0;
     float2* cs = reinterpret_cast<float2*>(smem);
     float* part = smem + a.rho;
-    for (int k = tid; k < a.rho / 2; k += blockDim.x) cs[k] = rope_cs((double)s, k, a.rho, a.theta);
+    for (int k = tid; k < a.rho / 2; k += blockDim.x) cs[k] = rope_cs((int64_t)s, k, a.rope_step);
     __syncthreads();
     const int g = cv / NVH, d0 = (cv % NVH) * VEC;
     const size_t src = ((size_t)b * a.T + s) * GD + (size_t)cv * VEC;
@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(1024) append_kernel(const AppendArgs a) {
     float2* cs_pool = cs_raw + a.rho / 2;
     float* part = smem + 2 * a.rho;
     for (int k = tid; k < a.rho / 2; k += blockDim.x) {
-        cs_raw[k] = rope_cs((double)pos, k, a.rho, a.theta);
-        if (complete) cs_pool[k] = rope_cs((double)j * a.m, k, a.rho, a.theta);
+        cs_raw[k] = rope_cs((int64_t)pos, k, a.rope_step);
+        if (complete) cs_pool[k] = rope_cs((int64_t)j * a.m, k, a.rope_step);
     }
     __syncthreads();
 

@@ -7,28 +7,38 @@
 // finalised from the pooling kernel.
 //
 // This path serves the f32 I/O dtype (no TF32: every product is an f32 FMA)
-// and the shapes the tensor-core kernel does not cover.  A CTA owns 32 queries
-// of one head; four lanes share a query (D/4 dims each, interleaved so the
-// four read one contiguous 64-byte span of a key row and eight queries of a
-// warp broadcast it).  Key/value tiles of 32 rows are widened to f32 in shared
-// memory; scores are taken eight keys at a time with one rescale.
+// and the shapes the tensor-core kernel does not cover.  TPQ = max(4, D/32)
+// lanes share a query (D/TPQ dims each, interleaved so that they read one
+// contiguous 16*TPQ-byte span of a key row and the queries of a warp broadcast
+// it); a CTA of 128 threads owns 128/TPQ queries of one head.  Key/value tiles
+// (32 rows, 16 for D >= 256) are widened to f32 in shared memory; scores are
+// taken eight keys at a time with one rescale.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace lbca {
 namespace {
 
-constexpr int QT = 32, KT = 32, NT = 128;
+constexpr int NT = 128;
+
+template <int D> struct Shape {
+    static constexpr int TPQ = D / 32 > 4 ? D / 32 : 4;  // lanes per query
+    static constexpr int QT = NT / TPQ;                   // queries per CTA
+    static constexpr int KT = D >= 256 ? 16 : 32;         // key rows per tile
+    static constexpr size_t smem = 2 * (size_t)KT * D * 4;
+};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
-    constexpr int NC = D / 16;  // float4 chunks per thread
-    __shared__ __align__(16) float Ks[KT][D];
-    __shared__ __align__(16) float Vs[KT][D];
+    constexpr int TPQ = Shape<D>::TPQ, QT = Shape<D>::QT, KT = Shape<D>::KT;
+    constexpr int NC = D / (4 * TPQ);  // float4 chunks per thread
+    extern __shared__ __align__(16) float smem[];
+    float (*Ks)[D] = reinterpret_cast<float (*)[D]>(smem);
+    float (*Vs)[D] = reinterpret_cast<float (*)[D]>(smem + KT * D);
 
     const int qt0 = blockIdx.x * QT, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qi = tid >> 2, j4 = tid & 3;
+    const int qi = tid / TPQ, j4 = tid % TPQ;
     const int g = h / (a.Hq / a.G);
     const int t = qt0 + qi;
     const bool qvalid = t < a.T;
@@ -42,7 +52,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
     for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            q[c][i] = to_f<T>(qrow[4 * (j4 + 4 * c) + i]);
+            q[c][i] = to_f<T>(qrow[4 * (j4 + TPQ * c) + i]);
             o[c][i] = 0.f;
         }
     if (a.rmsnorm) {
@@ -51,24 +61,24 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
         for (int c = 0; c < NC; ++c)
 #pragma unroll
             for (int i = 0; i < 4; ++i) ss += q[c][i] * q[c][i];
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+#pragma unroll
+        for (int off = 1; off < TPQ; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
         const T* gm = static_cast<const T*>(a.gamma_q);
 #pragma unroll
         for (int c = 0; c < NC; ++c)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) q[c][i] *= inv * (gm ? to_f<T>(gm[4 * (j4 + 4 * c) + i]) : 1.f);
+            for (int i = 0; i < 4; ++i) q[c][i] *= inv * (gm ? to_f<T>(gm[4 * (j4 + TPQ * c) + i]) : 1.f);
     }
     float2 qcs[NC][2];  // cos/sin at t for this thread's pairs (reused for the output rotation)
 #pragma unroll
     for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr) {
-            const int d = 4 * (j4 + 4 * c) + 2 * pr;
+            const int d = 4 * (j4 + TPQ * c) + 2 * pr;
             qcs[c][pr] = make_float2(1.f, 0.f);
             if (a.rho && d >= D - a.rho) {
-                qcs[c][pr] = rope_cs((double)t, (d - (D - a.rho)) >> 1, a.rho, a.theta);
+                qcs[c][pr] = rope_cs((int64_t)t, (d - (D - a.rho)) >> 1, a.rope_step);
                 rotate_pair(q[c][2 * pr], q[c][2 * pr + 1], qcs[c][pr]);
             }
         }
@@ -124,7 +134,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
                 for (int d = 2 * lane; d < D; d += 64) {
                     if (a.rho && d >= D - a.rho && ok)
                         rotate_pair(Ks[rrow][d], Ks[rrow][d + 1],
-                                    rope_cs((double)e, (d - (D - a.rho)) >> 1, a.rho, a.theta));
+                                    rope_cs((int64_t)e, (d - (D - a.rho)) >> 1, a.rope_step));
                 }
                 __syncwarp();
                 if (a.shared) {
@@ -144,14 +154,14 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
                 float acc = 0.f;
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
-                    const float4 kv = *reinterpret_cast<const float4*>(&Ks[e0 + u][4 * (j4 + 4 * c)]);
+                    const float4 kv = *reinterpret_cast<const float4*>(&Ks[e0 + u][4 * (j4 + TPQ * c)]);
                     acc = fmaf(q[c][0], kv.x, acc);
                     acc = fmaf(q[c][1], kv.y, acc);
                     acc = fmaf(q[c][2], kv.z, acc);
                     acc = fmaf(q[c][3], kv.w, acc);
                 }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+#pragma unroll
+                for (int off = 1; off < TPQ; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
                 const int e = base + e0 + u;
                 const bool vis = qvalid && e < lim && (pooled ? e < Pq : (e >= raw_lo && e <= t));
                 s[u] = vis ? acc : kNegInf;
@@ -172,7 +182,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
                 float4 acc = make_float4(o[c][0] * rr, o[c][1] * rr, o[c][2] * rr, o[c][3] * rr);
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const float4 vv = *reinterpret_cast<const float4*>(&Vs[e0 + u][4 * (j4 + 4 * c)]);
+                    const float4 vv = *reinterpret_cast<const float4*>(&Vs[e0 + u][4 * (j4 + TPQ * c)]);
                     acc.x = fmaf(p[u], vv.x, acc.x);
                     acc.y = fmaf(p[u], vv.y, acc.y);
                     acc.z = fmaf(p[u], vv.z, acc.z);
@@ -196,32 +206,48 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
         if (a.shared && a.rho) {
 #pragma unroll
             for (int pr = 0; pr < 2; ++pr) {
-                const int d = 4 * (j4 + 4 * c) + 2 * pr;
+                const int d = 4 * (j4 + TPQ * c) + 2 * pr;
                 if (d >= D - a.rho)
                     rotate_pair(v[2 * pr], v[2 * pr + 1], make_float2(qcs[c][pr].x, -qcs[c][pr].y));
             }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) orow[4 * (j4 + 4 * c) + i] = from_f<T>(v[i]);
+        for (int i = 0; i < 4; ++i) orow[4 * (j4 + TPQ * c) + i] = from_f<T>(v[i]);
     }
+}
+
+template <typename T, int D>
+cudaError_t launch_d(const PrefillArgs& a, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<T, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<D>::smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid((a.T + Shape<D>::QT - 1) / Shape<D>::QT, a.Hq, a.B);
+    prefill_simt_kernel<T, D><<<grid, NT, Shape<D>::smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t dispatch(const PrefillArgs& a, cudaStream_t s) {
-    dim3 grid((a.T + QT - 1) / QT, a.Hq, a.B);
     switch (a.D) {
-        case 16: prefill_simt_kernel<T, 16><<<grid, NT, 0, s>>>(a); break;
-        case 32: prefill_simt_kernel<T, 32><<<grid, NT, 0, s>>>(a); break;
-        case 64: prefill_simt_kernel<T, 64><<<grid, NT, 0, s>>>(a); break;
-        case 128: prefill_simt_kernel<T, 128><<<grid, NT, 0, s>>>(a); break;
+        case 16: return launch_d<T, 16>(a, s);
+        case 32: return launch_d<T, 32>(a, s);
+        case 64: return launch_d<T, 64>(a, s);
+        case 128: return launch_d<T, 128>(a, s);
+        case 256: return launch_d<T, 256>(a, s);
+        case 512: return launch_d<T, 512>(a, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace
 
-bool prefill_simt_supported(int D) { return D == 16 || D == 32 || D == 64 || D == 128; }
+bool prefill_simt_supported(int D) {
+    return D == 16 || D == 32 || D == 64 || D == 128 || D == 256 || D == 512;
+}
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;

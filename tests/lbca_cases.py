@@ -52,7 +52,9 @@ def assert_close_stored(got, want, dtype: str, what: str = ""):
     an exact value of magnitude |x| is off by up to 2^-9 |x| from rounding
     alone, above 1e-2 once |x| > 5 (RMSNorm'd entries reach that), so each
     element may be off by max(1e-2, 2^-8 |x|): the rounding plus as much again
-    for f32 arithmetic.  Mean-abs stays <= 1e-3; f32 keeps relative 1e-5."""
+    for f32 arithmetic.  Likewise the mean: rounding unit-RMS values to bf16
+    alone costs ~1.07e-3 mean-abs, so the mean bound is 1e-3 plus the mean
+    rounding allowance 2^-9 mean|x|.  f32 keeps relative 1e-5."""
     if dtype != "bf16":
         return assert_close(got, want, dtype, what)
     got = np.asarray(got, dtype=np.float64)
@@ -62,7 +64,8 @@ def assert_close_stored(got, want, dtype: str, what: str = ""):
     bound = np.maximum(1e-2, np.abs(want) * 2.0 ** -8)
     worst = float((d / bound).max())
     assert worst <= 1.0, f"{what}: error {worst:.2f}x the bf16 storage bound"
-    assert d.mean() <= 1e-3, f"{what}: mean-abs {d.mean():.3e}"
+    mean_bound = 1e-3 + 2.0 ** -9 * float(np.abs(want).mean())
+    assert d.mean() <= mean_bound, f"{what}: mean-abs {d.mean():.3e} > {mean_bound:.3e}"
 
 
 def dev(t):

@@ -76,10 +76,11 @@ lbca_status check_cache(const lbca_config* c, const lbca_cache* k) {
     if (k->batch < 0 || k->max_blocks < 0 || k->reserved != 0) return LBCA_ERR_ARG;
     const int rmin = ring_min(c);
     if (rmin < 0 || k->ring_slots < rmin) return LBCA_ERR_CAPACITY;
-    if (!k->pooled_k || !k->ring_k || !k->pool_state || !k->seq_lens) return LBCA_ERR_ARG;
+    const bool pooled = k->max_blocks > 0;  // a cache with no block capacity needs no pooled arrays
+    if ((pooled && !k->pooled_k) || !k->ring_k || !k->pool_state || !k->seq_lens) return LBCA_ERR_ARG;
     if (c->shared_kv) {
         if (k->pooled_v || k->ring_v) return LBCA_ERR_ARG;
-    } else if (!k->pooled_v || !k->ring_v) {
+    } else if ((pooled && !k->pooled_v) || !k->ring_v) {
         return LBCA_ERR_ARG;
     }
     if (!al16(k->pooled_k) || !al16n(k->pooled_v) || !al16(k->ring_k) || !al16n(k->ring_v) ||

@@ -146,7 +146,7 @@ class Cache:
     def allocate(cfg: lbca_config, batch: int, max_ctx: int, device="cuda") -> "Cache":
         G, D = cfg.n_kv_heads, cfg.head_dim
         dt = torch_dtype(cfg)
-        nb = max_ctx // cfg.block_m
+        nb = max(1, max_ctx // cfg.block_m)
         R = lbca_ring_slots(cfg)
         shared = bool(cfg.shared_kv)
         z = lambda *s, dtype=dt: torch.zeros(*s, dtype=dtype, device=device)  # noqa: E731

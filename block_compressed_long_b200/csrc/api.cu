@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "kernels.h"
 #include "lbca.h"
@@ -289,6 +290,77 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
     }
     return LBCA_OK;
+}
+
+// ---- decode without a caller-provided workspace ---------------------------------------
+// For callers that cannot allocate device memory (see lbca_decode_noalloc in the
+// header).  The split partials and merge counters live in this file-scope
+// device array instead of a caller workspace.  Every GPU that loads the library
+// holds it until the process exits, so it is kept to LBCA_NOALLOC_SCRATCH_BYTES.
+static __device__ __align__(256) unsigned char g_decode_scratch[LBCA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64];  // device address of g_decode_scratch, per device ordinal
+
+// In host code `g_decode_scratch` names a host-side shadow, not device memory;
+// the device address is looked up once per device, with that device current.
+lbca_status scratch_for_current_device(void** addr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LBCA_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LBCA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return LBCA_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return LBCA_OK;
+}
+
+}  // namespace
+
+lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbca_cache* cache,
+                                const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                                int32_t* d_status, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_cache(cfg, cache));
+    if (!q || !out) return LBCA_ERR_ARG;
+    if (!al16(q) || !al16(out) || !al16n(gamma_q) || !al16n(sink)) return LBCA_ERR_ALIGN;
+    if (max_ctx <= 0) {
+        const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
+        max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
+    }
+    DecodePlan p = plan_decode(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                               cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+    if (!p.ok) return LBCA_ERR_UNSUPPORTED;
+    if (decode_workspace_bytes(p) > (size_t)LBCA_NOALLOC_SCRATCH_BYTES) return LBCA_ERR_CAPACITY;
+    LBCA_TRY(check_device());
+    void* scratch = nullptr;
+    LBCA_TRY(scratch_for_current_device(&scratch));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(scratch);
+    const size_t ctr_off = align256(p.part_o_elems * 4) + align256(p.part_ml_elems * 4);
+    // the scratch keeps whatever the previous call left: the merge counters must start at zero
+    if (cudaMemsetAsync(ws + ctr_off, 0, p.counter_elems * 4, s) != cudaSuccess) return LBCA_ERR_CUDA;
+    DecodeArgs a{};
+    a.dtype = cfg->dtype;
+    a.q = q;
+    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
+    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
+    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    a.part_o = reinterpret_cast<float*>(ws);
+    a.part_ml = reinterpret_cast<float*>(ws + align256(p.part_o_elems * 4));
+    a.counters = reinterpret_cast<uint32_t*>(ws + ctr_off);
+    a.status = d_status;
+    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
+    a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
+    a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
+    a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
+    return cuda_status(launch_decode(a, s));
 }
 
 const char* lbca_status_string(lbca_status status) {

@@ -27,7 +27,7 @@ LBCA_KEY, LBCA_VALUE = 0, 1
 
 ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspace_bytes",
                 "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
-                "lbca_prefill", "lbca_status_string")
+                "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc")
 
 
 class lbca_config(ctypes.Structure):
@@ -67,6 +67,8 @@ _lib.lbca_decode.restype = ctypes.c_int
 _lib.lbca_prefill.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
                               _KP, _vp, _sz, _vp]
 _lib.lbca_prefill.restype = ctypes.c_int
+_lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _vp]
+_lib.lbca_decode_noalloc.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
 _lib.lbca_status_string.restype = ctypes.c_char_p
 
@@ -198,3 +200,13 @@ def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv
                                              _ptr(gamma_kv), B, TT, _ptr(out),
                                              ctypes.byref(cc) if cc is not None else None,
                                              _ptr(workspace), wb, _stream(stream)))
+
+
+def lbca_decode_noalloc(cfg, q, cache: Cache, sink, gamma_q, out, max_ctx=0, d_status=None, stream=None):
+    """lbca_decode without a workspace, for callers that may not allocate device
+    memory: the library's own static scratch holds the split partials.  Calls
+    that overlap on the GPU race on that scratch."""
+    cc = cache.c()
+    _check("lbca_decode_noalloc", _lib.lbca_decode_noalloc(ctypes.byref(cfg), _ptr(q), ctypes.byref(cc), _ptr(sink),
+                                                           _ptr(gamma_q), max_ctx, _ptr(out), _ptr(d_status),
+                                                           _stream(stream)))

@@ -222,6 +222,32 @@ LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const v
                          const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
                          lbca_stream_t stream);
 
+/*
+ * lbca_decode_noalloc -- lbca_decode for callers that cannot allocate.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that are not allowed to allocate device memory at all -- for example code
+ * running inside a host framework that owns every device allocation, or a
+ * serving loop that must not allocate once it is running -- and so have no
+ * workspace to hand to lbca_decode.  It computes exactly what lbca_decode
+ * computes, with the same arguments minus the workspace; the split partials
+ * and merge counters live in a static device array of the library
+ * (LBCA_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library until
+ * the process exits).
+ *   - A call whose split partials would need more than that returns
+ *     LBCA_ERR_CAPACITY (use lbca_decode with a workspace instead).
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture on that device.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called; each
+ *     call zeroes the merge counters with an asynchronous memset on `stream`.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other host
+ *     threads) race and corrupt each other's results.
+ */
+#define LBCA_NOALLOC_SCRATCH_BYTES (8u << 20)
+LBCA_API lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbca_cache* cache,
+                                         const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                                         int32_t* d_status, lbca_stream_t stream);
+
 /* Static text for a status code. */
 LBCA_API const char* lbca_status_string(lbca_status status);
 

@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa_decode_32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="step", choices=["step", "two-call"],
+                    help="step: lbca_decode_step (one launch); two-call: lbca_append then lbca_decode")
     return ap.parse_args()
 
 
@@ -155,6 +157,8 @@ class DecodeBench:
                            None, None, None, None, sc, ws0, batch=1, T=Lb)
         self.ws = torch.zeros(L.lbca_decode_workspace_bytes(self.cfg, B, self.max_ctx), dtype=torch.uint8,
                               device="cuda")
+        self.step_ws = torch.zeros(max(L.lbca_decode_step_workspace_bytes(self.cfg, B, self.max_ctx), 16),
+                                   dtype=torch.uint8, device="cuda")
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         # per-step token inputs, gathered once: [steps, B, G, D]
         ar = torch.arange(B)
@@ -168,17 +172,26 @@ class DecodeBench:
     def lens_now(self):
         return self.inp.lens + self.i + 1
 
-    def step(self, ev=None):
-        L, i = self.L, self.i
+    def launch(self, i, fused, ev=None, q=None, tok=None, out=None):
+        """Enqueue step i: lbca_decode_step, or lbca_append then lbca_decode."""
+        L = self.L
         g = lambda t: None if t is None else t[i]  # noqa: E731
-        L.lbca_append(self.cfg, g(self.tk), g(self.tv), g(self.tzk), g(self.tzv), self.bpk, self.bpv, None,
-                      self.cache, self.status)
+        k, v, zk, zv = tok if tok is not None else (g(self.tk), g(self.tv), g(self.tzk), g(self.tzv))
+        q = self.q[i] if q is None else q
+        out = self.out if out is None else out
+        if fused:
+            L.lbca_decode_step(self.cfg, k, v, zk, zv, self.bpk, self.bpv, None, q, self.cache, self.sink, None, out,
+                               self.step_ws, self.max_ctx, self.status)
+            return
+        L.lbca_append(self.cfg, k, v, zk, zv, self.bpk, self.bpv, None, self.cache, self.status)
         if ev is not None:
             ev[0].record()
-        L.lbca_decode(self.cfg, self.q[i], self.cache, self.sink, None, self.out, self.ws, self.max_ctx,
-                      self.status)
+        L.lbca_decode(self.cfg, q, self.cache, self.sink, None, out, self.ws, self.max_ctx, self.status)
         if ev is not None:
             ev[1].record()
+
+    def step(self, fused):
+        self.launch(self.i, fused)
         self.i += 1
 
 
@@ -192,27 +205,34 @@ def run_ours(args, w, rank, world):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
+    fused = args.path == "step"
     # warm-up: eager launches (first calls set kernel attributes)
     for _ in range(args.warmup):
         flush.zero_()
-        bench.step()
+        bench.step(fused)
     torch.cuda.synchronize()
 
-    # every step is replayed from CUDA graphs captured up front: the append and
-    # the decode of step i in two graphs, so that events between them time the
-    # decode kernel alone on its stream
+    # every step is replayed from a CUDA graph captured up front; on the
+    # two-call path the append and the decode get separate graphs so that
+    # events between them time the decode kernel alone
     cap = torch.cuda.Stream()
-    g = lambda t, i: None if t is None else t[i]  # noqa: E731
     graphs = []
     for i in range(bench.i, bench.i + args.steps):
-        ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ga, stream=cap):
-            L.lbca_append(bench.cfg, g(bench.tk, i), g(bench.tv, i), g(bench.tzk, i), g(bench.tzv, i), bench.bpk,
-                          bench.bpv, None, bench.cache, bench.status)
-        with torch.cuda.graph(gd, stream=cap):
-            L.lbca_decode(bench.cfg, bench.q[i], bench.cache, bench.sink, None, bench.out, bench.ws, bench.max_ctx,
-                          bench.status)
-        graphs.append((ga, gd))
+        if fused:
+            gs = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs, stream=cap):
+                bench.launch(i, True)
+            graphs.append((gs,))
+        else:
+            ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            g = lambda t: None if t is None else t[i]  # noqa: E731
+            with torch.cuda.graph(ga, stream=cap):
+                L.lbca_append(bench.cfg, g(bench.tk), g(bench.tv), g(bench.tzk), g(bench.tzv), bench.bpk,
+                              bench.bpv, None, bench.cache, bench.status)
+            with torch.cuda.graph(gd, stream=cap):
+                L.lbca_decode(bench.cfg, bench.q[i], bench.cache, bench.sink, None, bench.out, bench.ws,
+                              bench.max_ctx, bench.status)
+            graphs.append((ga, gd))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -226,21 +246,24 @@ def run_ours(args, w, rank, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    for s_, (ga, gd) in enumerate(graphs):
+    for s_, gg in enumerate(graphs):
         flush.zero_()
         nbytes += bytes_per_decode(bench.w, bench.lens_now())
         step_ev[s_][0].record()
-        ga.replay()
-        dec_ev[s_][0].record()
-        gd.replay()
-        dec_ev[s_][1].record()
+        if fused:
+            gg[0].replay()
+        else:
+            gg[0].replay()
+            dec_ev[s_][0].record()
+            gg[1].replay()
+            dec_ev[s_][1].record()
         step_ev[s_][1].record()
         bench.i += 1
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     step_ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
-    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
+    dec_ms = step_ms if fused else sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
     del graphs
 
     # ---- end to end through the public API: pinned host inputs and output ----
@@ -259,10 +282,7 @@ def run_ours(args, w, rank, world):
         for dt, ht in zip(dtok, htok):
             if dt is not None:
                 dt.copy_(ht[i], non_blocking=True)
-        L.lbca_append(bench.cfg, dtok[0], dtok[1], dtok[2], dtok[3], bench.bpk, bench.bpv, None, bench.cache,
-                      bench.status)
-        L.lbca_decode(bench.cfg, dq, bench.cache, bench.sink, None, bench.out, bench.ws, bench.max_ctx,
-                      bench.status)
+        bench.launch(i, fused, q=dq, tok=dtok)
         hout.copy_(bench.out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -309,14 +329,15 @@ def run_ours(args, w, rank, world):
                    "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
                    "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
                    "l2": "flushed (512 MiB write) before every timed step, outside its events",
-                   "launch": "each step replayed from CUDA graphs (append, decode)"},
+                   "launch": ("each step one lbca_decode_step kernel, replayed from a CUDA graph" if fused else
+                              "each step lbca_append + lbca_decode, replayed from CUDA graphs")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "kernel": "decode_kernel",
+                     "peak_source": src, "kernel": "decode_step_kernel" if fused else "decode_kernel",
                      "bytes_per_launch": nbytes / args.steps, "launch_us": dec_ms * 1e3,
                      "traffic": traffic},
         "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "µs/token", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if fused else 2) * args.steps,
         "clocks": clocks,
     }
     return line, bench

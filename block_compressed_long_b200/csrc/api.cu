@@ -220,6 +220,53 @@ lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache*
     return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return 0;
+    StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
+                            cfg->n_win, cfg->shared_kv, max_ctx);
+    if (sp.ok) return align256(sp.arrive_elems * 4);
+    return lbca_decode_workspace_bytes(cfg, batch, max_ctx);  // append + decode fallback
+}
+
+lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk, const void* zv,
+                             const void* b_pos_k, const void* b_pos_v, const void* gamma_kv, const void* q,
+                             const lbca_cache* cache, const float* sink, const void* gamma_q, int32_t max_ctx,
+                             void* out, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                             lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v));
+    LBCA_TRY(check_cache(cfg, cache));
+    if (!q || !out || !workspace) return LBCA_ERR_ARG;
+    if (!al16(q) || !al16(out) || !al16(workspace) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink))
+        return LBCA_ERR_ALIGN;
+    if (max_ctx <= 0) {
+        const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
+        max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
+    }
+    StepPlan sp = plan_step(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                            cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+    if (!sp.ok) {  // shapes the fused kernel does not take: the two-launch path
+        LBCA_TRY(lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache, d_status, stream));
+        return lbca_decode(cfg, q, cache, sink, gamma_q, max_ctx, out, workspace, workspace_bytes, d_status,
+                           stream);
+    }
+    if (workspace_bytes < align256(sp.arrive_elems * 4)) return LBCA_ERR_CAPACITY;
+    LBCA_TRY(check_device());
+    StepArgs a{};
+    a.dtype = cfg->dtype;
+    a.k = k; a.v = v; a.zk = zk; a.zv = zv; a.bpk = b_pos_k; a.bpv = b_pos_v; a.gamma_kv = gamma_kv;
+    a.q = q; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v; a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
+    a.state = cache->pool_state; a.seq_lens = cache->seq_lens;
+    a.arrive = static_cast<uint32_t*>(workspace); a.status = d_status;
+    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
+    a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm; a.shared = cfg->shared_kv;
+    a.max_blocks = cache->max_blocks; a.R = cache->ring_slots; a.S = cfg->shared_kv ? 1 : 2;
+    a.CS = sp.CS; a.SE = sp.SE; a.heads_per_cta = sp.heads_per_cta;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
+    return cuda_status(launch_decode_step(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, const void* v, const void* zk,
                          const void* zv, const void* b_pos_k, const void* b_pos_v, const float* sink,
                          const void* gamma_q, const void* gamma_kv, int32_t batch, int32_t T, void* out,

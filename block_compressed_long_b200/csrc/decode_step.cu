@@ -1,0 +1,567 @@
+// decode_step.cu -- one serving step in one launch: append the new raw token
+// and decode its query, with the split merge done inside a thread-block
+// cluster over distributed shared memory.
+//
+// What is computed is lbca_append followed by lbca_decode (mSeek README, "How
+// LBCA works", steps 2-5; HCA page and CSA page, "What is implemented"): the
+// query at t = L_old sees pooled entries j < P(L_old + 1) and raw tokens
+// [P m, t].  With n_win >= 1 the block the new token may complete is never
+// visible to the same step (it becomes visible n_win tokens later), so the
+// append work (running pooling softmax, block finalisation, ring write) is
+// independent of this step's attention and runs after it, off the critical
+// path.  The newest raw row itself is finalised in shared memory by the CTA
+// that needs it instead of being read back from the ring.
+//
+// B200 mapping: grid (CS, head groups, sequences) with cluster (CS, 1, 1).  The
+// CS CTAs of a cluster split one (sequence, head group)'s visible entries
+// evenly, stream them through a two-stage shared-memory ring filled by bulk
+// async copies (cp.async.bulk, non-multicast), and publish their (max, sum,
+// unnormalised output) partials in shared memory; after a cluster barrier
+// each CTA merges a slice of the head dims by reading its peers' partials over
+// DSMEM.  No global partials, fences or atomics sit between the last entry and
+// the output.  The CTA that arrives last for a sequence advances seq_lens.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace lbca {
+namespace {
+
+constexpr int kThreads = 128;
+
+struct StepLayout {
+    size_t bars, qs, cs, newk, newv, part_o, part_ml, red_o, red_ml, stage, total;
+};
+
+__host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline StepLayout step_layout(int D, int R, int SE, int esize, int shared) {
+    const int NG = 4 * 32 / (D / 16);
+    StepLayout l;
+    l.bars = 0;
+    l.qs = 16;
+    l.cs = l.qs + (size_t)R * D * 4;
+    l.newk = al(l.cs + (size_t)(D / 2) * 8, 16);
+    l.newv = l.newk + (size_t)D * esize;
+    l.part_o = al(l.newv + (size_t)D * esize, 16);
+    l.part_ml = l.part_o + (size_t)R * D * 4;
+    l.red_o = al(l.part_ml + (size_t)R * 2 * 4, 16);
+    l.red_ml = l.red_o + (size_t)NG * R * D * 4;
+    l.stage = al(l.red_ml + (size_t)NG * R * 2 * 4, 128);
+    l.total = l.stage + 2 * (size_t)SE * D * esize * (shared ? 1 : 2);
+    return l;
+}
+
+template <typename T>
+__device__ __forceinline__ void put2(T* p, float a, float b);
+template <> __device__ __forceinline__ void put2<float>(float* p, float a, float b) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+template <> __device__ __forceinline__ void put2<__nv_bfloat16>(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+}
+template <typename T>
+__device__ __forceinline__ float2 get2(const T* p) {
+    return make_float2(to_f<T>(p[0]), to_f<T>(p[1]));
+}
+
+// Block-wide sum over kThreads threads (every thread must call it).
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) s += scratch[i];
+    return s;
+}
+
+template <typename T, int D, int R>
+__global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a) {
+    constexpr int VEC = Vec<T>::N;
+    constexpr int LG = D / 16;
+    constexpr int NCH = 16 / VEC;
+    constexpr int GPW = 32 / LG;
+    constexpr int NG = 4 * GPW;
+    constexpr uint32_t ROW = D * sizeof(T);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(128) unsigned char smem[];
+    const StepLayout lay = step_layout(D, R, a.SE, sizeof(T), a.shared);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars);
+    float* qs = reinterpret_cast<float*>(smem + lay.qs);
+    float2* cs = reinterpret_cast<float2*>(smem + lay.cs);
+    T* newk = reinterpret_cast<T*>(smem + lay.newk);
+    T* newv = reinterpret_cast<T*>(smem + lay.newv);
+    float* part_o = reinterpret_cast<float*>(smem + lay.part_o);
+    float* part_ml = reinterpret_cast<float*>(smem + lay.part_ml);
+    float* red_o = reinterpret_cast<float*>(smem + lay.red_o);
+    float* red_ml = reinterpret_cast<float*>(smem + lay.red_ml);
+    T* kst = reinterpret_cast<T*>(smem + lay.stage);                            // [2][SE][D]
+    T* vst = a.shared ? kst : kst + 2 * (size_t)a.SE * D;                        // [2][SE][D]
+
+    const int CS = a.CS;
+    const int rank = (int)cluster.block_rank();
+    const int hg = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int r = a.Hq / a.G;
+    const int h0 = hg * R;
+    const int g = h0 / r;
+    const int GD = a.G * D;
+
+    // ---- the step: token t = L_old joins, the query sits at t ----
+    const int t = a.seq_lens[b];
+    const int L = t + 1;
+    const int P = visible_blocks(L, a.m, a.w);
+    const int s0 = P * a.m;
+    int n_vis = P + (L - s0);
+    if (P > a.max_blocks || L - s0 > a.R) {
+        if (rank == 0 && hg == 0 && tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
+        n_vis = 0;
+    }
+    const int chunk = (n_vis + CS - 1) / CS;
+    const int e0 = min(n_vis, rank * chunk);
+    const int e1 = min(n_vis, e0 + chunk);
+    const int ne = e1 - e0;
+    const int nst = (ne + a.SE - 1) / a.SE;
+    const int newest = n_vis - 1;  // the raw token t itself: built in shared memory
+
+    auto issue = [&](int st) {  // thread 0 only: bulk copies of stage st into buffer st & 1
+        const int b0 = e0 + st * a.SE, b1 = min(e1, b0 + a.SE);
+        T* kd = kst + (size_t)(st & 1) * a.SE * D;
+        T* vd = vst + (size_t)(st & 1) * a.SE * D;
+        const int c1 = min(b1, newest);  // rows [b0, c1) come from memory
+        const uint32_t rows = c1 > b0 ? (uint32_t)(c1 - b0) : 0u;
+        mbar_arrive_expect_tx(&bars[st & 1], rows * ROW * (a.shared ? 1u : 2u));
+        const size_t pool_head = ((size_t)b * a.G + g) * a.max_blocks;
+        const size_t ring_head = ((size_t)b * a.G + g) * a.R;
+        int e = b0, row = 0;
+        if (e < c1 && e < P) {
+            const int n = min(c1, P) - e;
+            bulk_g2s(kd, static_cast<const T*>(a.pooled_k) + (pool_head + e) * D, n * ROW, &bars[st & 1]);
+            if (!a.shared)
+                bulk_g2s(vd, static_cast<const T*>(a.pooled_v) + (pool_head + e) * D, n * ROW, &bars[st & 1]);
+            e += n;
+            row += n;
+        }
+        while (e < c1) {
+            const int slot = (s0 + (e - P)) % a.R;
+            const int n = min(c1 - e, a.R - slot);
+            bulk_g2s(kd + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + slot) * D, n * ROW,
+                     &bars[st & 1]);
+            if (!a.shared)
+                bulk_g2s(vd + (size_t)row * D, static_cast<const T*>(a.ring_v) + (ring_head + slot) * D, n * ROW,
+                         &bars[st & 1]);
+            e += n;
+            row += n;
+        }
+    };
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if (nst > 0) issue(0);
+        if (nst > 1) issue(1);
+    }
+
+    // ---- query prep and the newest raw row, overlapping the copies ----
+    for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((int64_t)t, k, a.rope_step);
+    for (int idx = tid; idx < R * D / VEC; idx += kThreads) {
+        const int h = idx / (D / VEC), c = idx % (D / VEC);
+        float v[VEC];
+        ld16(static_cast<const T*>(a.q) + ((size_t)b * a.Hq + h0 + h) * D + c * VEC, v);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) qs[h * D + c * VEC + i] = v[i];
+    }
+    // newest row: thread p owns the pair (2p, 2p+1) of kv head g's new key/value
+    const bool pair_owner = tid < D / 2;
+    float2 kx = make_float2(0.f, 0.f);
+    if (pair_owner) kx = get2(static_cast<const T*>(a.k) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+    __syncthreads();  // cs, qs ready
+    {
+        float ss = block_sum(pair_owner ? kx.x * kx.x + kx.y * kx.y : 0.f, red_ml);
+        if (pair_owner) {
+            if (a.rmsnorm) {
+                const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+                const T* gm = static_cast<const T*>(a.gamma_kv);
+                kx.x *= inv * (gm ? to_f<T>(gm[2 * tid]) : 1.f);
+                kx.y *= inv * (gm ? to_f<T>(gm[2 * tid + 1]) : 1.f);
+            }
+            if (a.rho && 2 * tid >= D - a.rho) rotate_pair(kx.x, kx.y, cs[(2 * tid - (D - a.rho)) >> 1]);
+            put2<T>(newk + 2 * tid, kx.x, kx.y);
+            if (!a.shared) {
+                const float2 vx = get2(static_cast<const T*>(a.v) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+                put2<T>(newv + 2 * tid, vx.x, vx.y);
+            }
+        }
+    }
+    if (a.rmsnorm) {
+        for (int h = warp; h < R; h += kThreads / 32) {
+            float ss = 0.f;
+            for (int d = lane; d < D; d += 32) ss += qs[h * D + d] * qs[h * D + d];
+#pragma unroll
+            for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+            const T* gm = static_cast<const T*>(a.gamma_q);
+            for (int d = lane; d < D; d += 32) qs[h * D + d] *= inv * (gm ? to_f<T>(gm[d]) : 1.0f);
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < R * (a.rho / 2); idx += kThreads) {
+        const int h = idx / (a.rho / 2), k = idx % (a.rho / 2);
+        const int d = D - a.rho + 2 * k;
+        rotate_pair(qs[h * D + d], qs[h * D + d + 1], cs[k]);
+    }
+    __syncthreads();
+
+    const int grp = warp * GPW + lane / LG;
+    const int gl = lane % LG;
+    const float qscale = a.scale * kLog2e;
+    float qr[R][16];
+#pragma unroll
+    for (int h = 0; h < R; ++h)
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) qr[h][c * VEC + i] = qs[h * D + (c * LG + gl) * VEC + i] * qscale;
+
+    float mx[R], ls[R], o[R][16];
+#pragma unroll
+    for (int h = 0; h < R; ++h) {
+        mx[h] = kNegInf;
+        ls[h] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[h][i] = 0.f;
+    }
+
+    // ---- stream the CTA's entries through the two-stage ring ----
+    bool ok = true;
+    for (int st = 0; st < nst; ++st) {
+        const int b0 = e0 + st * a.SE;
+        const int n = min(e1, b0 + a.SE) - b0;
+        T* kb = kst + (size_t)(st & 1) * a.SE * D;
+        T* vb = vst + (size_t)(st & 1) * a.SE * D;
+        bool okst = mbar_wait(&bars[st & 1], (uint32_t)((st >> 1) & 1));
+        if (newest >= b0 && newest < b0 + n) {  // the newest row is written, not copied
+            const int row = newest - b0;
+            for (int i = tid; i < D / VEC; i += kThreads) {
+                *reinterpret_cast<uint4*>(kb + (size_t)row * D + i * VEC) = *reinterpret_cast<const uint4*>(newk + i * VEC);
+                if (!a.shared)
+                    *reinterpret_cast<uint4*>(vb + (size_t)row * D + i * VEC) =
+                        *reinterpret_cast<const uint4*>(newv + i * VEC);
+            }
+        }
+        okst = __syncthreads_and(okst);
+        if (!okst) {
+            ok = false;
+            break;
+        }
+        for (int eb = warp * GPW; eb < n; eb += 2 * NG) {
+            const int ea = eb + lane / LG, ebb = ea + NG;
+            const bool va = ea < n, vbb = ebb < n;
+            const T* ka = kb + (size_t)(va ? ea : 0) * D;
+            const T* kbb = kb + (size_t)(vbb ? ebb : 0) * D;
+            float kfa[16], kfb[16];
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                float t0[VEC], t1[VEC];
+                ld16(ka + (c * LG + gl) * VEC, t0);
+                ld16(kbb + (c * LG + gl) * VEC, t1);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { kfa[c * VEC + i] = t0[i]; kfb[c * VEC + i] = t1[i]; }
+            }
+            float sa[R], sb[R];
+#pragma unroll
+            for (int h = 0; h < R; ++h) {
+                float x = 0.f, y = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { x = fmaf(qr[h][i], kfa[i], x); y = fmaf(qr[h][i], kfb[i], y); }
+                sa[h] = x;
+                sb[h] = y;
+            }
+#pragma unroll
+            for (int off = LG / 2; off; off >>= 1)
+#pragma unroll
+                for (int h = 0; h < R; ++h) {
+                    sa[h] += __shfl_xor_sync(0xffffffffu, sa[h], off);
+                    sb[h] += __shfl_xor_sync(0xffffffffu, sb[h], off);
+                }
+            if (!va) continue;
+            const T* vra = vb + (size_t)ea * D;
+            const T* vrb = vb + (size_t)(vbb ? ebb : ea) * D;
+            float vfa[16], vfb[16];
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                float t0[VEC], t1[VEC];
+                ld16(vra + (c * LG + gl) * VEC, t0);
+                ld16(vrb + (c * LG + gl) * VEC, t1);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { vfa[c * VEC + i] = t0[i]; vfb[c * VEC + i] = t1[i]; }
+            }
+#pragma unroll
+            for (int h = 0; h < R; ++h) {
+                const float sbh = vbb ? sb[h] : kNegInf;
+                const float mn = fmaxf(mx[h], fmaxf(sa[h], sbh));
+                const float rr = ex2(mx[h] - mn);
+                const float pa = ex2(sa[h] - mn);
+                const float pb = ex2(sbh - mn);
+                ls[h] = fmaf(ls[h], rr, pa + pb);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[h][i] = fmaf(o[h][i], rr, fmaf(pa, vfa[i], pb * vfb[i]));
+                mx[h] = mn;
+            }
+        }
+        __syncthreads();  // every thread is done with this buffer
+        if (tid == 0 && st + 2 < nst) issue(st + 2);
+    }
+    if (!ok) {
+        if (tid == 0) {
+            set_status(a.status, LBCA_ERR_TIMEOUT);
+            mbar_wait(&bars[0], 0);  // last bounded chance for copies in flight to land
+            mbar_wait(&bars[1], 0);
+        }
+#pragma unroll
+        for (int h = 0; h < R; ++h) {
+            mx[h] = kNegInf;
+            ls[h] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[h][i] = 0.f;
+        }
+    }
+
+    // ---- CTA partial: merge the entry groups ----
+#pragma unroll
+    for (int h = 0; h < R; ++h) {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+#pragma unroll
+            for (int i = 0; i < VEC; ++i)
+                red_o[((size_t)grp * R + h) * D + (c * LG + gl) * VEC + i] = o[h][c * VEC + i];
+        if (gl == 0) {
+            red_ml[(grp * R + h) * 2] = mx[h];
+            red_ml[(grp * R + h) * 2 + 1] = ls[h];
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < R * D; idx += kThreads) {
+        const int h = idx / D, d = idx % D;
+        float M = kNegInf;
+        for (int q = 0; q < NG; ++q) M = fmaxf(M, red_ml[(q * R + h) * 2]);
+        float Ls = 0.f, ov = 0.f;
+        if (M != kNegInf)
+            for (int q = 0; q < NG; ++q) {
+                const float f = ex2(red_ml[(q * R + h) * 2] - M);
+                ov = fmaf(red_o[((size_t)q * R + h) * D + d], f, ov);
+                Ls = fmaf(red_ml[(q * R + h) * 2 + 1], f, Ls);
+            }
+        part_o[h * D + d] = ov;
+        if (d == 0) {
+            part_ml[h * 2] = M;
+            part_ml[h * 2 + 1] = Ls;
+        }
+    }
+
+    // ---- cluster merge: this CTA finalises dims [rank*DS, (rank+1)*DS) of its heads ----
+    cluster.sync();
+    const int DS = D / CS;
+    for (int idx = tid; idx < R * DS / 2; idx += kThreads) {
+        const int h = idx / (DS / 2), d = rank * DS + (idx % (DS / 2)) * 2;
+        float M = kNegInf;
+        for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(part_ml, q)[h * 2]);
+        float Ls = 0.f, o0 = 0.f, o1 = 0.f;
+        if (M != kNegInf)
+            for (int q = 0; q < CS; ++q) {
+                const float* pml = cluster.map_shared_rank(part_ml, q);
+                const float* po = cluster.map_shared_rank(part_o, q);
+                const float f = ex2(pml[h * 2] - M);
+                Ls = fmaf(pml[h * 2 + 1], f, Ls);
+                o0 = fmaf(po[h * D + d], f, o0);
+                o1 = fmaf(po[h * D + d + 1], f, o1);
+            }
+        float den = Ls;
+        if (a.sink) den += (M == kNegInf) ? 1.0f : ex2(a.sink[h0 + h] * kLog2e - M);
+        float v0 = den > 0.f ? o0 / den : 0.f, v1 = den > 0.f ? o1 / den : 0.f;
+        if (a.shared && a.rho && d >= D - a.rho) {
+            const float2 c = cs[(d - (D - a.rho)) >> 1];
+            rotate_pair(v0, v1, make_float2(c.x, -c.y));
+        }
+        put2<T>(static_cast<T*>(a.out) + ((size_t)b * a.Hq + h0 + h) * D + d, v0, v1);
+    }
+    cluster.sync();  // peers stop reading this CTA's partial before it may exit
+
+    // ---- append the new token (one CTA per (sequence, kv head)), off the output path ----
+    if (rank == 0 && h0 % r == 0) {
+        const int i = t % a.m, j = t / a.m;
+        const bool complete = i == a.m - 1;
+        for (int s = 0; s < a.S; ++s) {
+            const bool key = s == 0;
+            float2 x = make_float2(0.f, 0.f), z = x, bp = x;
+            if (pair_owner) {
+                const size_t off = (size_t)b * GD + (size_t)g * D + 2 * tid;
+                x = get2(static_cast<const T*>(key ? a.k : a.v) + off);
+                z = get2(static_cast<const T*>(key ? a.zk : a.zv) + off);
+                bp = get2(static_cast<const T*>(key ? a.bpk : a.bpv) + (size_t)i * GD + (size_t)g * D + 2 * tid);
+            }
+            float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
+            float mxs[2], lss[2], acs[2];
+            const float xv[2] = {x.x, x.y}, av[2] = {(z.x + bp.x) * kLog2e, (z.y + bp.y) * kLog2e};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                if (i == 0 || !pair_owner) {
+                    mxs[e] = av[e]; lss[e] = 1.f; acs[e] = xv[e];
+                } else {
+                    const float m0 = st[e], l0 = st[GD + e], a0 = st[2 * GD + e];
+                    const float mn = fmaxf(m0, av[e]);
+                    const float rr = ex2(m0 - mn), p = ex2(av[e] - mn);
+                    mxs[e] = mn; lss[e] = l0 * rr + p; acs[e] = fmaf(p, xv[e], a0 * rr);
+                }
+            }
+            if (complete) {  // uniform across the CTA
+                float e0v = acs[0] / lss[0], e1v = acs[1] / lss[1];
+                float ss = block_sum(pair_owner && key ? e0v * e0v + e1v * e1v : 0.f, red_ml);
+                if (key && a.rmsnorm) {
+                    const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+                    const T* gm = static_cast<const T*>(a.gamma_kv);
+                    e0v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid]) : 1.f);
+                    e1v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid + 1]) : 1.f);
+                }
+                if (key && a.rho && pair_owner && 2 * tid >= D - a.rho)
+                    rotate_pair(e0v, e1v, rope_cs((int64_t)j * a.m, (2 * tid - (D - a.rho)) >> 1, a.rope_step));
+                if (pair_owner) {
+                    if (j < a.max_blocks)
+                        put2<T>(static_cast<T*>(key ? a.pooled_k : a.pooled_v) +
+                                    (((size_t)b * a.G + g) * a.max_blocks + j) * D + 2 * tid,
+                                e0v, e1v);
+                    else
+                        set_status(a.status, LBCA_ERR_CAPACITY);
+                }
+            } else if (pair_owner) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    st[e] = mxs[e];
+                    st[GD + e] = lss[e];
+                    st[2 * GD + e] = acs[e];
+                }
+            }
+            if (pair_owner) {  // ring slot of token t: the finalised key row, or the raw value
+                T* dst = static_cast<T*>(key ? a.ring_k : a.ring_v) +
+                         (((size_t)b * a.G + g) * a.R + (t % a.R)) * D + 2 * tid;
+                *reinterpret_cast<uint32_t*>(dst) =
+                    *reinterpret_cast<const uint32_t*>((key ? newk : newv) + 2 * tid);
+            }
+        }
+    }
+
+    // ---- the last CTA of this sequence to arrive advances its length ----
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t total = (uint32_t)(CS * (a.Hq / R));
+        if (atomicAdd(&a.arrive[b], 1u) == total - 1) {
+            a.seq_lens[b] = L;
+            a.arrive[b] = 0u;
+        }
+    }
+}
+
+template <typename T, int D, int R>
+cudaError_t launch_step_one(const StepArgs& a, size_t smem, cudaStream_t s) {
+    static bool attr_set = false;
+    auto fn = decode_step_kernel<T, D, R>;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    // 16-CTA clusters are non-portable: fall back to 8 if none fits on this device
+    static int max16 = -1;
+    StepArgs b = a;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (b.CS > 8) {
+        if (max16 < 0) {
+            cfg.gridDim = dim3(16, 1, 1);
+            attr[0].val.clusterDim.x = 16;
+            int n = 0;
+            max16 = cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess ? n : 0;
+            cudaGetLastError();
+        }
+        if (max16 == 0) b.CS = 8;
+    }
+    cfg.gridDim = dim3(b.CS, b.Hq / R, b.B);
+    attr[0].val.clusterDim.x = b.CS;
+    return cudaLaunchKernelEx(&cfg, fn, b);
+}
+template <typename T, int D>
+cudaError_t step_dispatch_r(const StepArgs& a, size_t smem, cudaStream_t s) {
+    switch (a.heads_per_cta) {
+        case 1: return launch_step_one<T, D, 1>(a, smem, s);
+        case 2: return launch_step_one<T, D, 2>(a, smem, s);
+        case 3: return launch_step_one<T, D, 3>(a, smem, s);
+        case 4: return launch_step_one<T, D, 4>(a, smem, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t step_dispatch(const StepArgs& a, size_t smem, cudaStream_t s) {
+    switch (a.D) {
+        case 64: return step_dispatch_r<T, 64>(a, smem, s);
+        case 128: return step_dispatch_r<T, 128>(a, smem, s);
+        case 256: return step_dispatch_r<T, 256>(a, smem, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
+    StepPlan p{};
+    p.ok = false;
+    if ((D != 64 && D != 128 && D != 256) || w < 1) return p;
+    const int r = Hq / G;
+    int R = 1;
+    for (int c : {4, 3, 2, 1})
+        if (r % c == 0) { R = c; break; }
+    const int esize = dtype == LBCA_BF16 ? 2 : 4;
+    const long long groups = (long long)B * (Hq / R);
+    int CS = 1;
+    while (CS < 16 && CS * 2 <= D / 4 && groups * CS < 4 * 148) CS *= 2;
+    p.heads_per_cta = R;
+    p.CS = CS;
+    p.SE = D >= 256 || esize == 4 ? 16 : 32;
+    p.arrive_elems = (size_t)B;
+    p.smem_bytes = step_layout(D, R, p.SE, esize, shared).total;
+    p.ok = p.smem_bytes <= 200 * 1024;
+    (void)m; (void)max_ctx;
+    return p;
+}
+
+cudaError_t launch_decode_step(const StepArgs& a, cudaStream_t s) {
+    if (a.B == 0) return cudaSuccess;
+    const size_t smem = step_layout(a.D, a.heads_per_cta, a.SE, a.dtype == LBCA_BF16 ? 2 : 4, a.shared).total;
+    if (a.dtype == LBCA_BF16) return step_dispatch<__nv_bfloat16>(a, smem, s);
+    return step_dispatch<float>(a, smem, s);
+}
+
+}  // namespace lbca

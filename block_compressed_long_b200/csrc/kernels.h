@@ -91,6 +91,30 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int
 size_t decode_workspace_bytes(const DecodePlan& p);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
+// One serving step (append + decode) in one cluster launch.
+struct StepArgs {
+    int dtype;
+    const void* k; const void* v; const void* zk; const void* zv;  // [B, G, D] the new token
+    const void* bpk; const void* bpv; const void* gamma_kv;
+    const void* q; const float* sink; const void* gamma_q;         // q [B, Hq, D]
+    void* out;                                                     // [B, Hq, D]
+    void* pooled_k; void* pooled_v; void* ring_k; void* ring_v;
+    float* state; int32_t* seq_lens;
+    uint32_t* arrive;                                              // [B] arrival counters (zeroed)
+    int32_t* status;
+    int B, Hq, G, D, m, w, rho, rmsnorm, shared, max_blocks, R, S;
+    int CS, SE, heads_per_cta;
+    float eps, scale;
+    double rope_step;  // theta^(-2/rho)
+};
+struct StepPlan {
+    int heads_per_cta, CS, SE;
+    size_t arrive_elems, smem_bytes;
+    bool ok;
+};
+StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+cudaError_t launch_decode_step(const StepArgs& a, cudaStream_t s);
+
 struct PrefillArgs {
     int dtype;
     const void* q;                                   // [B, T, Hq, D]

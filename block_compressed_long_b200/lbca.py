@@ -27,7 +27,8 @@ LBCA_KEY, LBCA_VALUE = 0, 1
 
 ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspace_bytes",
                 "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
-                "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc")
+                "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc",
+                "lbca_decode_step_workspace_bytes", "lbca_decode_step")
 
 
 class lbca_config(ctypes.Structure):
@@ -67,6 +68,11 @@ _lib.lbca_decode.restype = ctypes.c_int
 _lib.lbca_prefill.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
                               _KP, _vp, _sz, _vp]
 _lib.lbca_prefill.restype = ctypes.c_int
+_lib.lbca_decode_step_workspace_bytes.argtypes = [_CP, _i32, _i32]
+_lib.lbca_decode_step_workspace_bytes.restype = _sz
+_lib.lbca_decode_step.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _sz,
+                                  _vp, _vp]
+_lib.lbca_decode_step.restype = ctypes.c_int
 _lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _vp]
 _lib.lbca_decode_noalloc.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
@@ -186,6 +192,20 @@ def lbca_decode(cfg, q, cache: Cache, sink, gamma_q, out, workspace, max_ctx=0, 
                                            _ptr(gamma_q), max_ctx, _ptr(out), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), _ptr(d_status),
                                            _stream(stream)))
+
+
+def lbca_decode_step_workspace_bytes(cfg: lbca_config, batch: int, max_ctx: int) -> int:
+    return int(_lib.lbca_decode_step_workspace_bytes(ctypes.byref(cfg), batch, max_ctx))
+
+
+def lbca_decode_step(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, q, cache: Cache, sink, gamma_q, out,
+                     workspace, max_ctx=0, d_status=None, stream=None):
+    """Append the token (k, v, zk, zv [B, G, D]) and decode q [B, Hq, D] in one step."""
+    cc = cache.c()
+    _check("lbca_decode_step", _lib.lbca_decode_step(
+        ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv), _ptr(b_pos_k), _ptr(b_pos_v), _ptr(gamma_kv),
+        _ptr(q), ctypes.byref(cc), _ptr(sink), _ptr(gamma_q), max_ctx, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(d_status), _stream(stream)))
 
 
 def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv, out,

@@ -200,6 +200,27 @@ LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lb
                         lbca_stream_t stream);
 
 /*
+ * lbca_decode_step -- one serving step: lbca_append of the token (k, v, zk, zv)
+ * followed by lbca_decode of q, in one launch where the shapes allow.
+ * (mSeek README, repository layout: generation through the LBCA cache; "How
+ * LBCA works", steps 2-5.)  Arguments as in lbca_append and lbca_decode;
+ * `workspace` (zero-filled before first use, left zero-filled) must hold
+ * lbca_decode_step_workspace_bytes(cfg, B, max_ctx) bytes.  With n_win >= 1,
+ * D in {64, 128, 256} and up to 4 query heads per kv head per CTA group, the
+ * step runs as one cluster kernel (the appended token's block cannot be
+ * visible to the same query, so appending and attending are independent);
+ * other shapes run lbca_append then lbca_decode.  Results equal those of the
+ * two calls.
+ */
+LBCA_API size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
+LBCA_API lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk,
+                                      const void* zv, const void* b_pos_k, const void* b_pos_v,
+                                      const void* gamma_kv, const void* q, const lbca_cache* cache,
+                                      const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                                      void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                      lbca_stream_t stream);
+
+/*
  * lbca_prefill -- causal block-compressed attention over T tokens per sequence.
  * (mSeek README, "How LBCA works", steps 1-5; HCA page, "What is implemented";
  * CSA page, "What is implemented" and "Deviations from paper".)

@@ -147,6 +147,21 @@ class DecodeRun:
         return out
 
 
+def fused_step(run: DecodeRun):
+    """The same step as DecodeRun.step through lbca_decode_step (one launch)."""
+    L = run.L
+    if not hasattr(run, "step_ws"):
+        run.step_ws = torch.zeros(max(L.lbca_decode_step_workspace_bytes(run.cfg, run.B, run.max_ctx), 16),
+                                  dtype=torch.uint8, device="cuda")
+    out = torch.empty(run.B, run.w.n_q_heads, run.w.head_dim, dtype=L.torch_dtype(run.cfg), device="cuda")
+    L.lbca_decode_step(run.cfg, run.token(run.k), run.token(run.v), run.token(run.zk), run.token(run.zv), run.bpk,
+                       run.bpv, None, run.q[run.step_i], run.cache, run.sink, None, out, run.step_ws, run.max_ctx,
+                       run.status)
+    run.pos += 1
+    run.step_i += 1
+    return out
+
+
 def oracle_decode(w, inp, step, seqs=None):
     """Oracle output of decode step `step` (0-based) for the sequences `seqs`."""
     seqs = range(inp.k.shape[0]) if seqs is None else seqs

@@ -23,7 +23,7 @@ def L():
     ("gqa_decode_32k", dict(ctx=(5, 5), n_win=3, block_m=4), 40),
     ("ragged_gqa_decode_append", dict(ctx=(0, 2500), batch=7), 66),
     ("hca_mqa_decode_128k", dict(ctx=(700, 900), batch=2, n_q_heads=4, head_dim=128, rope_dims=32), 130),
-    ("tiny_f32_prefill", dict(kind="decode", ctx=(300, 300), n_kv_heads=1, n_q_heads=4, steps=20), 20),
+    ("tiny_f32_prefill", dict(kind="decode", ctx=(300, 300), n_kv_heads=1, n_q_heads=4), 20),
 ])
 def test_step_matches_oracle(L, name, kw, steps):
     w = synth.scaled(W[name], steps=steps, **kw)

@@ -457,8 +457,9 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
             if (pair_owner) {  // ring slot of token t: the finalised key row, or the raw value
                 T* dst = static_cast<T*>(key ? a.ring_k : a.ring_v) +
                          (((size_t)b * a.G + g) * a.R + (t % a.R)) * D + 2 * tid;
-                *reinterpret_cast<uint32_t*>(dst) =
-                    *reinterpret_cast<const uint32_t*>((key ? newk : newv) + 2 * tid);
+                const T* src = (key ? newk : newv) + 2 * tid;
+                dst[0] = src[0];
+                dst[1] = src[1];
             }
         }
     }

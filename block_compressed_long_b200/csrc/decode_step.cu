@@ -35,24 +35,26 @@ namespace {
 constexpr int kThreads = 128;
 
 struct StepLayout {
-    size_t bars, qs, cs, newk, newv, part_o, part_ml, red_o, red_ml, stage, total;
+    size_t bars, misc, qs, cs, newk, newv, wred_o, wred_ml, recv_o, recv_ml, stage, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline StepLayout step_layout(int D, int R, int SE, int esize, int shared) {
-    const int NG = 4 * 32 / (D / 16);
+constexpr int kWarps = kThreads / 32;
+
+__host__ __device__ inline StepLayout step_layout(int D, int R, int SE, int esize, int shared, int CS) {
     StepLayout l;
     l.bars = 0;
-    l.qs = 16;
+    l.misc = 16;                                   // broadcast of t + block_sum scratch
+    l.qs = 64;
     l.cs = l.qs + (size_t)R * D * 4;
     l.newk = al(l.cs + (size_t)(D / 2) * 8, 16);
     l.newv = l.newk + (size_t)D * esize;
-    l.part_o = al(l.newv + (size_t)D * esize, 16);
-    l.part_ml = l.part_o + (size_t)R * D * 4;
-    l.red_o = al(l.part_ml + (size_t)R * 2 * 4, 16);
-    l.red_ml = l.red_o + (size_t)NG * R * D * 4;
-    l.stage = al(l.red_ml + (size_t)NG * R * 2 * 4, 128);
+    l.wred_o = al(l.newv + (size_t)D * esize, 16);
+    l.wred_ml = l.wred_o + (size_t)kWarps * R * D * 4;
+    l.recv_o = al(l.wred_ml + (size_t)kWarps * R * 2 * 4, 16);
+    l.recv_ml = l.recv_o + (size_t)R * D * 4;      // CS slices of D / CS dims
+    l.stage = al(l.recv_ml + (size_t)CS * R * 2 * 4, 128);
     l.total = l.stage + 2 * (size_t)SE * D * esize * (shared ? 1 : 2);
     return l;
 }
@@ -79,35 +81,45 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
     __syncthreads();
     float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < kThreads / 32; ++i) s += scratch[i];
+    for (int i = 0; i < kWarps; ++i) s += scratch[i];
+    __syncthreads();
     return s;
+}
+
+// Online-softmax merge weights of two partials with maxima ma, mb.
+__device__ __forceinline__ void merge_weights(float ma, float mb, float& M, float& fa, float& fb) {
+    M = fmaxf(ma, mb);
+    fa = ma == kNegInf ? 0.f : ex2(ma - M);
+    fb = mb == kNegInf ? 0.f : ex2(mb - M);
 }
 
 template <typename T, int D, int R>
 __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a) {
     constexpr int VEC = Vec<T>::N;
-    constexpr int LG = D / 16;
-    constexpr int NCH = 16 / VEC;
-    constexpr int GPW = 32 / LG;
-    constexpr int NG = 4 * GPW;
+    constexpr int LG = D / 16;       // lanes per entry
+    constexpr int NCH = 16 / VEC;    // 16-byte chunks per lane
+    constexpr int GPW = 32 / LG;     // entry groups per warp
+    constexpr int NG = kWarps * GPW; // entry groups per CTA
     constexpr uint32_t ROW = D * sizeof(T);
 
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(128) unsigned char smem[];
-    const StepLayout lay = step_layout(D, R, a.SE, sizeof(T), a.shared);
+    const int CS = a.CS;
+    const StepLayout lay = step_layout(D, R, a.SE, sizeof(T), a.shared, CS);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars);
+    int* tsh = reinterpret_cast<int*>(smem + lay.misc);
+    float* scratch = reinterpret_cast<float*>(smem + lay.misc + 16);
     float* qs = reinterpret_cast<float*>(smem + lay.qs);
     float2* cs = reinterpret_cast<float2*>(smem + lay.cs);
     T* newk = reinterpret_cast<T*>(smem + lay.newk);
     T* newv = reinterpret_cast<T*>(smem + lay.newv);
-    float* part_o = reinterpret_cast<float*>(smem + lay.part_o);
-    float* part_ml = reinterpret_cast<float*>(smem + lay.part_ml);
-    float* red_o = reinterpret_cast<float*>(smem + lay.red_o);
-    float* red_ml = reinterpret_cast<float*>(smem + lay.red_ml);
-    T* kst = reinterpret_cast<T*>(smem + lay.stage);                            // [2][SE][D]
-    T* vst = a.shared ? kst : kst + 2 * (size_t)a.SE * D;                        // [2][SE][D]
+    float* wred_o = reinterpret_cast<float*>(smem + lay.wred_o);
+    float* wred_ml = reinterpret_cast<float*>(smem + lay.wred_ml);
+    float* recv_o = reinterpret_cast<float*>(smem + lay.recv_o);
+    float* recv_ml = reinterpret_cast<float*>(smem + lay.recv_ml);
+    T* kst = reinterpret_cast<T*>(smem + lay.stage);        // [2][SE][D]
+    T* vst = a.shared ? kst : kst + 2 * (size_t)a.SE * D;    // [2][SE][D]
 
-    const int CS = a.CS;
     const int rank = (int)cluster.block_rank();
     const int hg = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -115,9 +127,17 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     const int h0 = hg * R;
     const int g = h0 / r;
     const int GD = a.G * D;
+    const int DS = D / CS;  // dims this CTA finalises
 
     // ---- the step: token t = L_old joins, the query sits at t ----
-    const int t = a.seq_lens[b];
+    if (tid == 0) {
+        *tsh = a.seq_lens[b];  // read once, broadcast
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int t = *tsh;
     const int L = t + 1;
     const int P = visible_blocks(L, a.m, a.w);
     const int s0 = P * a.m;
@@ -165,14 +185,37 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     };
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
         if (nst > 0) issue(0);
         if (nst > 1) issue(1);
+        // Every CTA of the sequence has read its length once it has arrived
+        // here, so the last to arrive may advance it (latency hidden behind
+        // the copies).
+        const uint32_t total = (uint32_t)(CS * (a.Hq / R));
+        if (atomicAdd(&a.arrive[b], 1u) == total - 1) {
+            a.seq_lens[b] = L;
+            a.arrive[b] = 0u;
+        }
+    }
+
+    // ---- the appending CTA (one per sequence and kv head) prefetches its inputs ----
+    const bool app = rank == 0 && h0 % r == 0;
+    const bool pair_owner = tid < D / 2;
+    const int ai = t % a.m, aj = t / a.m;
+    float2 ax[2], az[2], abp[2], am[2], al_[2], aa[2];
+    if (app && pair_owner) {
+        for (int s = 0; s < a.S; ++s) {
+            const bool key = s == 0;
+            const size_t off = (size_t)b * GD + (size_t)g * D + 2 * tid;
+            ax[s] = get2(static_cast<const T*>(key ? a.k : a.v) + off);
+            az[s] = get2(static_cast<const T*>(key ? a.zk : a.zv) + off);
+            abp[s] = get2(static_cast<const T*>(key ? a.bpk : a.bpv) + (size_t)ai * GD + (size_t)g * D + 2 * tid);
+            if (ai > 0) {
+                const float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
+                am[s] = *reinterpret_cast<const float2*>(st);
+                al_[s] = *reinterpret_cast<const float2*>(st + GD);
+                aa[s] = *reinterpret_cast<const float2*>(st + 2 * GD);
+            }
+        }
     }
 
     // ---- query prep and the newest raw row, overlapping the copies ----
@@ -184,13 +227,14 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
 #pragma unroll
         for (int i = 0; i < VEC; ++i) qs[h * D + c * VEC + i] = v[i];
     }
-    // newest row: thread p owns the pair (2p, 2p+1) of kv head g's new key/value
-    const bool pair_owner = tid < D / 2;
-    float2 kx = make_float2(0.f, 0.f);
-    if (pair_owner) kx = get2(static_cast<const T*>(a.k) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+    float2 kx = make_float2(0.f, 0.f), vx = kx;
+    if (pair_owner) {
+        kx = get2(static_cast<const T*>(a.k) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+        if (!a.shared) vx = get2(static_cast<const T*>(a.v) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+    }
     __syncthreads();  // cs, qs ready
     {
-        float ss = block_sum(pair_owner ? kx.x * kx.x + kx.y * kx.y : 0.f, red_ml);
+        const float ss = a.rmsnorm ? block_sum(pair_owner ? kx.x * kx.x + kx.y * kx.y : 0.f, scratch) : 0.f;
         if (pair_owner) {
             if (a.rmsnorm) {
                 const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
@@ -200,14 +244,11 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
             }
             if (a.rho && 2 * tid >= D - a.rho) rotate_pair(kx.x, kx.y, cs[(2 * tid - (D - a.rho)) >> 1]);
             put2<T>(newk + 2 * tid, kx.x, kx.y);
-            if (!a.shared) {
-                const float2 vx = get2(static_cast<const T*>(a.v) + (size_t)b * GD + (size_t)g * D + 2 * tid);
-                put2<T>(newv + 2 * tid, vx.x, vx.y);
-            }
+            if (!a.shared) put2<T>(newv + 2 * tid, vx.x, vx.y);
         }
     }
     if (a.rmsnorm) {
-        for (int h = warp; h < R; h += kThreads / 32) {
+        for (int h = warp; h < R; h += kWarps) {
             float ss = 0.f;
             for (int d = lane; d < D; d += 32) ss += qs[h * D + d] * qs[h * D + d];
 #pragma unroll
@@ -225,7 +266,6 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     }
     __syncthreads();
 
-    const int grp = warp * GPW + lane / LG;
     const int gl = lane % LG;
     const float qscale = a.scale * kLog2e;
     float qr[R][16];
@@ -340,54 +380,73 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         }
     }
 
-    // ---- CTA partial: merge the entry groups ----
+    // ---- merge the entry groups of each warp with shuffles, then the warps ----
 #pragma unroll
-    for (int h = 0; h < R; ++h) {
+    for (int off = LG; off < 32; off <<= 1)
 #pragma unroll
-        for (int c = 0; c < NCH; ++c)
+        for (int h = 0; h < R; ++h) {
+            const float mo = __shfl_xor_sync(0xffffffffu, mx[h], off);
+            const float lo = __shfl_xor_sync(0xffffffffu, ls[h], off);
+            float M, fa, fb;
+            merge_weights(mx[h], mo, M, fa, fb);
+            ls[h] = ls[h] * fa + lo * fb;
 #pragma unroll
-            for (int i = 0; i < VEC; ++i)
-                red_o[((size_t)grp * R + h) * D + (c * LG + gl) * VEC + i] = o[h][c * VEC + i];
-        if (gl == 0) {
-            red_ml[(grp * R + h) * 2] = mx[h];
-            red_ml[(grp * R + h) * 2 + 1] = ls[h];
+            for (int i = 0; i < 16; ++i) o[h][i] = o[h][i] * fa + __shfl_xor_sync(0xffffffffu, o[h][i], off) * fb;
+            mx[h] = M;
+        }
+    if (lane < LG) {
+#pragma unroll
+        for (int h = 0; h < R; ++h) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int i = 0; i < VEC; ++i)
+                    wred_o[((size_t)warp * R + h) * D + (c * LG + gl) * VEC + i] = o[h][c * VEC + i];
+            if (lane == 0) {
+                wred_ml[(warp * R + h) * 2] = mx[h];
+                wred_ml[(warp * R + h) * 2 + 1] = ls[h];
+            }
         }
     }
     __syncthreads();
+    // CTA partial, pushed slice by slice into the owning CTA's receive buffer
     for (int idx = tid; idx < R * D; idx += kThreads) {
         const int h = idx / D, d = idx % D;
         float M = kNegInf;
-        for (int q = 0; q < NG; ++q) M = fmaxf(M, red_ml[(q * R + h) * 2]);
+#pragma unroll
+        for (int q = 0; q < kWarps; ++q) M = fmaxf(M, wred_ml[(q * R + h) * 2]);
         float Ls = 0.f, ov = 0.f;
-        if (M != kNegInf)
-            for (int q = 0; q < NG; ++q) {
-                const float f = ex2(red_ml[(q * R + h) * 2] - M);
-                ov = fmaf(red_o[((size_t)q * R + h) * D + d], f, ov);
-                Ls = fmaf(red_ml[(q * R + h) * 2 + 1], f, Ls);
+        if (M != kNegInf) {
+#pragma unroll
+            for (int q = 0; q < kWarps; ++q) {
+                const float f = ex2(wred_ml[(q * R + h) * 2] - M);
+                ov = fmaf(wred_o[((size_t)q * R + h) * D + d], f, ov);
+                Ls = fmaf(wred_ml[(q * R + h) * 2 + 1], f, Ls);
             }
-        part_o[h * D + d] = ov;
-        if (d == 0) {
-            part_ml[h * 2] = M;
-            part_ml[h * 2 + 1] = Ls;
+        }
+        const int owner = d / DS;
+        float* ro = cluster.map_shared_rank(recv_o, owner);
+        ro[(rank * R + h) * DS + (d - owner * DS)] = ov;
+        if (d % DS == 0) {
+            float* rm = cluster.map_shared_rank(recv_ml, owner);
+            rm[(rank * R + h) * 2] = M;
+            rm[(rank * R + h) * 2 + 1] = Ls;
         }
     }
+    cluster.sync();  // every slice has landed; nothing remote is read after this
 
-    // ---- cluster merge: this CTA finalises dims [rank*DS, (rank+1)*DS) of its heads ----
-    cluster.sync();
-    const int DS = D / CS;
+    // ---- this CTA finalises dims [rank*DS, (rank+1)*DS) of its heads ----
     for (int idx = tid; idx < R * DS / 2; idx += kThreads) {
-        const int h = idx / (DS / 2), d = rank * DS + (idx % (DS / 2)) * 2;
+        const int h = idx / (DS / 2), dl = (idx % (DS / 2)) * 2, d = rank * DS + dl;
         float M = kNegInf;
-        for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(part_ml, q)[h * 2]);
+        for (int q = 0; q < CS; ++q) M = fmaxf(M, recv_ml[(q * R + h) * 2]);
         float Ls = 0.f, o0 = 0.f, o1 = 0.f;
         if (M != kNegInf)
             for (int q = 0; q < CS; ++q) {
-                const float* pml = cluster.map_shared_rank(part_ml, q);
-                const float* po = cluster.map_shared_rank(part_o, q);
-                const float f = ex2(pml[h * 2] - M);
-                Ls = fmaf(pml[h * 2 + 1], f, Ls);
-                o0 = fmaf(po[h * D + d], f, o0);
-                o1 = fmaf(po[h * D + d + 1], f, o1);
+                const float f = ex2(recv_ml[(q * R + h) * 2] - M);
+                Ls = fmaf(recv_ml[(q * R + h) * 2 + 1], f, Ls);
+                o0 = fmaf(recv_o[(q * R + h) * DS + dl], f, o0);
+                o1 = fmaf(recv_o[(q * R + h) * DS + dl + 1], f, o1);
             }
         float den = Ls;
         if (a.sink) den += (M == kNegInf) ? 1.0f : ex2(a.sink[h0 + h] * kLog2e - M);
@@ -398,38 +457,33 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         }
         put2<T>(static_cast<T*>(a.out) + ((size_t)b * a.Hq + h0 + h) * D + d, v0, v1);
     }
-    cluster.sync();  // peers stop reading this CTA's partial before it may exit
 
     // ---- append the new token (one CTA per (sequence, kv head)), off the output path ----
-    if (rank == 0 && h0 % r == 0) {
-        const int i = t % a.m, j = t / a.m;
-        const bool complete = i == a.m - 1;
+    if (app) {
+        const bool complete = ai == a.m - 1;
         for (int s = 0; s < a.S; ++s) {
             const bool key = s == 0;
-            float2 x = make_float2(0.f, 0.f), z = x, bp = x;
+            float mxs[2] = {0.f, 0.f}, lss[2] = {1.f, 1.f}, acs[2] = {0.f, 0.f};
             if (pair_owner) {
-                const size_t off = (size_t)b * GD + (size_t)g * D + 2 * tid;
-                x = get2(static_cast<const T*>(key ? a.k : a.v) + off);
-                z = get2(static_cast<const T*>(key ? a.zk : a.zv) + off);
-                bp = get2(static_cast<const T*>(key ? a.bpk : a.bpv) + (size_t)i * GD + (size_t)g * D + 2 * tid);
-            }
-            float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
-            float mxs[2], lss[2], acs[2];
-            const float xv[2] = {x.x, x.y}, av[2] = {(z.x + bp.x) * kLog2e, (z.y + bp.y) * kLog2e};
+                const float xv[2] = {ax[s].x, ax[s].y};
+                const float av[2] = {(az[s].x + abp[s].x) * kLog2e, (az[s].y + abp[s].y) * kLog2e};
+                const float m0[2] = {am[s].x, am[s].y}, l0[2] = {al_[s].x, al_[s].y}, a0[2] = {aa[s].x, aa[s].y};
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                if (i == 0 || !pair_owner) {
-                    mxs[e] = av[e]; lss[e] = 1.f; acs[e] = xv[e];
-                } else {
-                    const float m0 = st[e], l0 = st[GD + e], a0 = st[2 * GD + e];
-                    const float mn = fmaxf(m0, av[e]);
-                    const float rr = ex2(m0 - mn), p = ex2(av[e] - mn);
-                    mxs[e] = mn; lss[e] = l0 * rr + p; acs[e] = fmaf(p, xv[e], a0 * rr);
+                for (int e = 0; e < 2; ++e) {
+                    if (ai == 0) {
+                        mxs[e] = av[e]; lss[e] = 1.f; acs[e] = xv[e];
+                    } else {
+                        const float mn = fmaxf(m0[e], av[e]);
+                        const float rr = ex2(m0[e] - mn), p = ex2(av[e] - mn);
+                        mxs[e] = mn; lss[e] = l0[e] * rr + p; acs[e] = fmaf(p, xv[e], a0[e] * rr);
+                    }
                 }
             }
+            float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
             if (complete) {  // uniform across the CTA
                 float e0v = acs[0] / lss[0], e1v = acs[1] / lss[1];
-                float ss = block_sum(pair_owner && key ? e0v * e0v + e1v * e1v : 0.f, red_ml);
+                const float ss = (key && a.rmsnorm)
+                                     ? block_sum(pair_owner ? e0v * e0v + e1v * e1v : 0.f, scratch) : 0.f;
                 if (key && a.rmsnorm) {
                     const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
                     const T* gm = static_cast<const T*>(a.gamma_kv);
@@ -437,22 +491,19 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
                     e1v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid + 1]) : 1.f);
                 }
                 if (key && a.rho && pair_owner && 2 * tid >= D - a.rho)
-                    rotate_pair(e0v, e1v, rope_cs((int64_t)j * a.m, (2 * tid - (D - a.rho)) >> 1, a.rope_step));
+                    rotate_pair(e0v, e1v, rope_cs((int64_t)aj * a.m, (2 * tid - (D - a.rho)) >> 1, a.rope_step));
                 if (pair_owner) {
-                    if (j < a.max_blocks)
+                    if (aj < a.max_blocks)
                         put2<T>(static_cast<T*>(key ? a.pooled_k : a.pooled_v) +
-                                    (((size_t)b * a.G + g) * a.max_blocks + j) * D + 2 * tid,
+                                    (((size_t)b * a.G + g) * a.max_blocks + aj) * D + 2 * tid,
                                 e0v, e1v);
                     else
                         set_status(a.status, LBCA_ERR_CAPACITY);
                 }
             } else if (pair_owner) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    st[e] = mxs[e];
-                    st[GD + e] = lss[e];
-                    st[2 * GD + e] = acs[e];
-                }
+                *reinterpret_cast<float2*>(st) = make_float2(mxs[0], mxs[1]);
+                *reinterpret_cast<float2*>(st + GD) = make_float2(lss[0], lss[1]);
+                *reinterpret_cast<float2*>(st + 2 * GD) = make_float2(acs[0], acs[1]);
             }
             if (pair_owner) {  // ring slot of token t: the finalised key row, or the raw value
                 T* dst = static_cast<T*>(key ? a.ring_k : a.ring_v) +
@@ -461,17 +512,6 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
                 dst[0] = src[0];
                 dst[1] = src[1];
             }
-        }
-    }
-
-    // ---- the last CTA of this sequence to arrive advances its length ----
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const uint32_t total = (uint32_t)(CS * (a.Hq / R));
-        if (atomicAdd(&a.arrive[b], 1u) == total - 1) {
-            a.seq_lens[b] = L;
-            a.arrive[b] = 0u;
         }
     }
 }
@@ -552,7 +592,7 @@ StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int sha
     p.CS = CS;
     p.SE = D >= 256 || esize == 4 ? 16 : 32;
     p.arrive_elems = (size_t)B;
-    p.smem_bytes = step_layout(D, R, p.SE, esize, shared).total;
+    p.smem_bytes = step_layout(D, R, p.SE, esize, shared, CS).total;
     p.ok = p.smem_bytes <= 200 * 1024;
     (void)m; (void)max_ctx;
     return p;
@@ -560,7 +600,7 @@ StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int sha
 
 cudaError_t launch_decode_step(const StepArgs& a, cudaStream_t s) {
     if (a.B == 0) return cudaSuccess;
-    const size_t smem = step_layout(a.D, a.heads_per_cta, a.SE, a.dtype == LBCA_BF16 ? 2 : 4, a.shared).total;
+    const size_t smem = step_layout(a.D, a.heads_per_cta, a.SE, a.dtype == LBCA_BF16 ? 2 : 4, a.shared, a.CS).total;
     if (a.dtype == LBCA_BF16) return step_dispatch<__nv_bfloat16>(a, smem, s);
     return step_dispatch<float>(a, smem, s);
 }

@@ -12,10 +12,12 @@ raw window, softmax with sink, weighted values, split merge).
 Prints one JSON line (rank 0).  Multi-GPU: one process per GPU, each rank
 decodes its own sequences (weak scaling, no collective on the data path); the
 step time is the max over ranks.  The inputs of the workload are resident in
-HBM before timing; the L2 is flushed (a 256 MiB write) before every timed
-step and outside its CUDA events.  ``e2e`` repeats the steps through the
-public API with the step's inputs copied from pinned host memory and the
-output copied back inside the timed region.
+HBM before timing.  Steps rotate over enough independent cache replicas
+(more than 3x the L2 in total) that every step reads cold data, as the caches
+of a model's layers and sequences are at every decode step; the K timed steps
+are replayed back to back from one CUDA graph.  ``e2e`` repeats the steps
+through the public API with each step's inputs copied from pinned host memory
+and its output copied back inside the timed region.
 """
 from __future__ import annotations
 
@@ -46,8 +48,6 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa_decode_32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="step", choices=["step", "two-call"],
-                    help="step: lbca_decode_step (one launch); two-call: lbca_append then lbca_decode")
     return ap.parse_args()
 
 
@@ -124,115 +124,104 @@ def bytes_per_decode(w, lens):
 
 
 class DecodeBench:
-    def __init__(self, w, n_steps, rank):
+    """Decode workload state on one GPU: NR replicas of the workload's cache,
+    each advanced by its own steps.  Steps rotate over the replicas so that
+    the data of each step has been evicted from L2 by the other replicas'
+    traffic (the replicas together hold more than 3x the L2 size), the way the
+    caches of a model's many layers and sequences are cold at every step."""
+
+    def __init__(self, w, rank, min_steps):
         import torch
 
         from block_compressed_long_b200 import lbca as L
         from block_compressed_long_b200 import synth
         self.L, self.torch = L, torch
-        self.w = synth.scaled(w, steps=n_steps, seed=w.seed + 7919 * rank)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        base = synth.scaled(w, steps=1)
+        lens0 = synth.contexts(base)
+        step_bytes = bytes_per_decode(base, lens0 + 1)
+        self.NR = max(1, -(-3 * l2 // step_bytes))
+        self.local_steps = -(-min_steps // self.NR) + 1
+        self.w = synth.scaled(w, steps=self.local_steps, seed=w.seed + 7919 * rank)
         self.inp = synth.make(self.w)
         w = self.w
         self.cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win,
                             w.rope_dims, w.rmsnorm, w.rope_theta, dtype=w.dtype)
         B = w.batch
         self.B = B
-        self.max_ctx = int(self.inp.lens.max()) + n_steps
+        self.max_ctx = int(self.inp.lens.max()) + self.local_steps
         d = lambda t: None if t is None else t.cuda()  # noqa: E731
-        self.k, self.v, self.zk, self.zv = (d(t) for t in (self.inp.k, self.inp.v, self.inp.zk, self.inp.zv))
+        k, v, zk, zv = (d(t) for t in (self.inp.k, self.inp.v, self.inp.zk, self.inp.zv))
         self.bpk, self.bpv, self.sink = d(self.inp.bpos_k), d(self.inp.bpos_v), d(self.inp.sink)
         self.q = d(self.inp.q)
-        self.cache = L.Cache.allocate(self.cfg, B, self.max_ctx)
-        per = self.cache.pool_state.numel() // B
+        c0 = L.Cache.allocate(self.cfg, B, self.max_ctx)
+        per = c0.pool_state.numel() // B
         ws0 = torch.zeros(16, dtype=torch.uint8, device="cuda")
         for b in range(B):  # build each sequence's cache with the prefill path (cache only)
             Lb = int(self.inp.lens[b])
-            c = self.cache
-            sc = L.Cache(self.cfg, 1, c.max_blocks, c.ring_slots, c.pooled_k[b:b + 1],
-                         None if c.pooled_v is None else c.pooled_v[b:b + 1], c.ring_k[b:b + 1],
-                         None if c.ring_v is None else c.ring_v[b:b + 1], c.pool_state[b * per:(b + 1) * per],
-                         c.seq_lens[b:b + 1])
+            sc = L.Cache(self.cfg, 1, c0.max_blocks, c0.ring_slots, c0.pooled_k[b:b + 1],
+                         None if c0.pooled_v is None else c0.pooled_v[b:b + 1], c0.ring_k[b:b + 1],
+                         None if c0.ring_v is None else c0.ring_v[b:b + 1], c0.pool_state[b * per:(b + 1) * per],
+                         c0.seq_lens[b:b + 1])
             s = lambda t: None if t is None else t[b:b + 1, :Lb]  # noqa: E731
-            L.lbca_prefill(self.cfg, None, s(self.k), s(self.v), s(self.zk), s(self.zv), self.bpk, self.bpv,
+            L.lbca_prefill(self.cfg, None, s(k), s(v), s(zk), s(zv), self.bpk, self.bpv,
                            None, None, None, None, sc, ws0, batch=1, T=Lb)
-        self.ws = torch.zeros(L.lbca_decode_workspace_bytes(self.cfg, B, self.max_ctx), dtype=torch.uint8,
-                              device="cuda")
-        self.step_ws = torch.zeros(max(L.lbca_decode_step_workspace_bytes(self.cfg, B, self.max_ctx), 16),
-                                   dtype=torch.uint8, device="cuda")
+        cl = lambda t: None if t is None else t.clone()  # noqa: E731
+        self.caches = [c0] + [L.Cache(self.cfg, B, c0.max_blocks, c0.ring_slots, cl(c0.pooled_k), cl(c0.pooled_v),
+                                      cl(c0.ring_k), cl(c0.ring_v), cl(c0.pool_state), cl(c0.seq_lens))
+                              for _ in range(self.NR - 1)]
+        del k, v, zk, zv
+        wsb = max(L.lbca_decode_step_workspace_bytes(self.cfg, B, self.max_ctx), 16)
+        self.step_ws = [torch.zeros(wsb, dtype=torch.uint8, device="cuda") for _ in range(self.NR)]
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
-        # per-step token inputs, gathered once: [steps, B, G, D]
+        # per-step token inputs, gathered once: [local_steps, B, G, D]
         ar = torch.arange(B)
         pos = torch.as_tensor(self.inp.lens)
         tok = lambda t: None if t is None else torch.stack(  # noqa: E731
-            [t[ar, pos + i] for i in range(n_steps)]).cuda()
+            [t[ar, pos + i] for i in range(self.local_steps)]).cuda()
         self.tk, self.tv, self.tzk, self.tzv = (tok(t) for t in (self.inp.k, self.inp.v, self.inp.zk, self.inp.zv))
-        self.out = torch.empty(B, w.n_q_heads, w.head_dim, dtype=L.torch_dtype(self.cfg), device="cuda")
-        self.i = 0
+        self.outs = [torch.empty(B, w.n_q_heads, w.head_dim, dtype=L.torch_dtype(self.cfg), device="cuda")
+                     for _ in range(self.NR)]
+        self.i = 0  # global step counter; step i uses replica i % NR, local step i // NR
 
-    def lens_now(self):
-        return self.inp.lens + self.i + 1
+    def lens_at(self, i):
+        return self.inp.lens + i // self.NR + 1
 
-    def launch(self, i, fused, ev=None, q=None, tok=None, out=None):
-        """Enqueue step i: lbca_decode_step, or lbca_append then lbca_decode."""
+    def launch(self, i, q=None, tok=None):
+        """Enqueue global step i (lbca_decode_step on replica i % NR)."""
         L = self.L
-        g = lambda t: None if t is None else t[i]  # noqa: E731
+        rep, j = i % self.NR, i // self.NR
+        g = lambda t: None if t is None else t[j]  # noqa: E731
         k, v, zk, zv = tok if tok is not None else (g(self.tk), g(self.tv), g(self.tzk), g(self.tzv))
-        q = self.q[i] if q is None else q
-        out = self.out if out is None else out
-        if fused:
-            L.lbca_decode_step(self.cfg, k, v, zk, zv, self.bpk, self.bpv, None, q, self.cache, self.sink, None, out,
-                               self.step_ws, self.max_ctx, self.status)
-            return
-        L.lbca_append(self.cfg, k, v, zk, zv, self.bpk, self.bpv, None, self.cache, self.status)
-        if ev is not None:
-            ev[0].record()
-        L.lbca_decode(self.cfg, q, self.cache, self.sink, None, out, self.ws, self.max_ctx, self.status)
-        if ev is not None:
-            ev[1].record()
-
-    def step(self, fused):
-        self.launch(self.i, fused)
-        self.i += 1
+        q = self.q[j] if q is None else q
+        L.lbca_decode_step(self.cfg, k, v, zk, zv, self.bpk, self.bpv, None, q, self.caches[rep], self.sink, None,
+                           self.outs[rep], self.step_ws[rep], self.max_ctx, self.status)
 
 
 def run_ours(args, w, rank, world):
     import torch
     import torch.distributed as dist
 
-    n_steps = 2 * (args.warmup + args.steps)
-    bench = DecodeBench(w, n_steps, rank)
+    K, W = args.steps, args.warmup
+    bench = DecodeBench(w, rank, 2 * (W + K))
     L = bench.L
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-
-    fused = args.path == "step"
-    # warm-up: eager launches (first calls set kernel attributes)
-    for _ in range(args.warmup):
-        flush.zero_()
-        bench.step(fused)
-    torch.cuda.synchronize()
-
-    # every step is replayed from a CUDA graph captured up front; on the
-    # two-call path the append and the decode get separate graphs so that
-    # events between them time the decode kernel alone
     cap = torch.cuda.Stream()
-    graphs = []
-    for i in range(bench.i, bench.i + args.steps):
-        if fused:
-            gs = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gs, stream=cap):
-                bench.launch(i, True)
-            graphs.append((gs,))
-        else:
-            ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            g = lambda t: None if t is None else t[i]  # noqa: E731
-            with torch.cuda.graph(ga, stream=cap):
-                L.lbca_append(bench.cfg, g(bench.tk), g(bench.tv), g(bench.tzk), g(bench.tzv), bench.bpk,
-                              bench.bpv, None, bench.cache, bench.status)
-            with torch.cuda.graph(gd, stream=cap):
-                L.lbca_decode(bench.cfg, bench.q[i], bench.cache, bench.sink, None, bench.out, bench.ws,
-                              bench.max_ctx, bench.status)
-            graphs.append((ga, gd))
+
+    def graph_of(first, n, body):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap):
+            for i in range(first, first + n):
+                body(i)
+        return gr
+
+    # warm-up (eager, sets kernel attributes), then K steps captured in one graph
+    for _ in range(W):
+        bench.launch(bench.i)
+        bench.i += 1
+    torch.cuda.synchronize()
+    nbytes = sum(bytes_per_decode(bench.w, bench.lens_at(i)) for i in range(bench.i, bench.i + K))
+    g_main = graph_of(bench.i, K, bench.launch)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -240,111 +229,89 @@ def run_ours(args, w, rank, world):
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
-    step_ev = [(E(), E()) for _ in range(args.steps)]
-    dec_ev = [(E(), E()) for _ in range(args.steps)]
-    nbytes = 0
+    e0, e1 = E(), E()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    for s_, gg in enumerate(graphs):
-        flush.zero_()
-        nbytes += bytes_per_decode(bench.w, bench.lens_now())
-        step_ev[s_][0].record()
-        if fused:
-            gg[0].replay()
-        else:
-            gg[0].replay()
-            dec_ev[s_][0].record()
-            gg[1].replay()
-            dec_ev[s_][1].record()
-        step_ev[s_][1].record()
-        bench.i += 1
+    e0.record()
+    g_main.replay()
+    e1.record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
-    dec_ms = step_ms if fused else sum(a.elapsed_time(b) for a, b in dec_ev) / args.steps
-    del graphs
+    step_ms = e0.elapsed_time(e1) / K
+    bench.i += K
+    del g_main
 
     # ---- end to end through the public API: pinned host inputs and output ----
     # each step's inputs (q and the new token's k, v, z_k, z_v) sit packed in
     # one pinned host buffer and cross with one copy; the output comes back
     # with one copy
-    w_ = bench.w
     parts = [bench.q] + [t for t in (bench.tk, bench.tv, bench.tzk, bench.tzv) if t is not None]
     sizes = [t[0].numel() * t[0].element_size() for t in parts]
     offs = np.cumsum([0] + sizes)
-    nstep = bench.q.shape[0]
-    hstage = torch.empty(nstep, int(offs[-1]), dtype=torch.uint8).pin_memory()
+    nloc = bench.q.shape[0]
+    hstage = torch.empty(nloc, int(offs[-1]), dtype=torch.uint8).pin_memory()
     for pi, t in enumerate(parts):
-        hstage[:, offs[pi]:offs[pi + 1]] = t.cpu().contiguous().view(nstep, -1).view(torch.uint8)
+        hstage[:, offs[pi]:offs[pi + 1]] = t.cpu().contiguous().view(nloc, -1).view(torch.uint8)
     dstage = torch.empty(int(offs[-1]), dtype=torch.uint8, device="cuda")
     views = [dstage[offs[pi]:offs[pi + 1]].view(parts[pi].dtype).view(parts[pi][0].shape) for pi in range(len(parts))]
     dq = views[0]
     it = iter(views[1:])
     dtok = [None if t is None else next(it) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)]
-    hout = torch.empty(bench.out.shape, dtype=bench.out.dtype).pin_memory()
+    hout = torch.empty(bench.outs[0].shape, dtype=bench.outs[0].dtype).pin_memory()
     h2d = int(offs[-1])
     d2h = hout.numel() * hout.element_size()
 
     def e2e_body(i):
-        dstage.copy_(hstage[i], non_blocking=True)
-        bench.launch(i, fused, q=dq, tok=dtok)
-        hout.copy_(bench.out, non_blocking=True)
+        dstage.copy_(hstage[i // bench.NR], non_blocking=True)
+        bench.launch(i, q=dq, tok=dtok)
+        hout.copy_(bench.outs[i % bench.NR], non_blocking=True)
 
-    for _ in range(args.warmup):
-        flush.zero_()
+    for _ in range(W):
         e2e_body(bench.i)
         bench.i += 1
     torch.cuda.synchronize()
-    egraphs = []
-    for i in range(bench.i, bench.i + args.steps):
-        ge = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ge, stream=cap):
-            e2e_body(i)
-        egraphs.append(ge)
+    g_e2e = graph_of(bench.i, K, e2e_body)
     torch.cuda.synchronize()
-    e2e_ev = [(E(), E()) for _ in range(args.steps)]
-    for s_, ge in enumerate(egraphs):
-        flush.zero_()
-        e2e_ev[s_][0].record()
-        ge.replay()
-        e2e_ev[s_][1].record()
-        bench.i += 1
+    e0.record()
+    g_e2e.replay()
+    e1.record()
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
-    del egraphs
+    e2e_ms = e0.elapsed_time(e1) / K
+    bench.i += K
+    del g_e2e
     clocks = sampler.stop()
     status = int(bench.status.item())
     if status:
         raise RuntimeError(f"device status {L.lbca_status_string(status)}")
 
-    t = torch.tensor([step_ms, e2e_ms, dec_ms], dtype=torch.float64, device="cuda")
+    t = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms, dec_ms = t.tolist()
+    step_ms, e2e_ms = t.tolist()
     tokens = bench.B * world
     hbm, src = peaks()
-    achieved = nbytes / args.steps / (dec_ms * 1e-3) / 1e9
-    traffic = load_traffic(w_.name)
+    achieved = nbytes / K / (step_ms * 1e-3) / 1e9
+    w_ = bench.w
     line = {
         "metric": METRIC, "value": step_ms * 1e3 / tokens, "unit": "µs/token", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False,
+        "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
         "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
                    "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
                    "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
                    "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
-                   "l2": "flushed (512 MiB write) before every timed step, outside its events",
-                   "launch": ("each step one lbca_decode_step kernel, replayed from a CUDA graph" if fused else
-                              "each step lbca_append + lbca_decode, replayed from CUDA graphs")},
+                   "l2": (f"inputs larger than L2: steps rotate over {bench.NR} cache replicas "
+                          f"(>= 3x L2 of data in total), each step's data cold"),
+                   "launch": "K steps of one lbca_decode_step kernel each, back to back from one CUDA graph"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "kernel": "decode_step_kernel" if fused else "decode_kernel",
-                     "bytes_per_launch": nbytes / args.steps, "launch_us": dec_ms * 1e3,
-                     "traffic": traffic},
+                     "peak_source": src, "kernel": "decode_step_kernel",
+                     "bytes_per_launch": nbytes / K, "launch_us": step_ms * 1e3,
+                     "traffic": load_traffic(w_.name)},
         "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "µs/token", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": (1 if fused else 2) * args.steps,
+        "gpu_launches": K,
         "clocks": clocks,
     }
     return line, bench

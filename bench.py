@@ -325,9 +325,9 @@ def load_traffic(workload):
         rec = json.load(open(p))[workload]
     except Exception:
         return None
-    src = os.path.join(ROOT, "block_compressed_long_b200", "csrc", "decode.cu")
+    src = os.path.join(ROOT, "block_compressed_long_b200", "csrc", rec["source"])
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes"] if rec.get("decode_cu_sha256_16") == h else None
+    return rec["bytes"] if rec.get("source_sha256_16") == h else None
 
 
 # ----------------------------------------------------- oracle (CPU) timing ----

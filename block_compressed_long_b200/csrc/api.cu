@@ -136,10 +136,15 @@ size_t lbca_decode_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_
 
 size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t T, int32_t has_cache) {
     if (check_cfg(cfg) != LBCA_OK || batch < 0 || T < 0) return (size_t)-1;
-    if (has_cache) return 0;
-    const size_t one = (size_t)batch * cfg->n_kv_heads * (T / cfg->block_m) * cfg->head_dim *
-                       esize_of(cfg->dtype);
-    return align256(one) * (cfg->shared_kv ? 1 : 2);
+    size_t bytes = 0;
+    if (!has_cache) {
+        const size_t one = (size_t)batch * cfg->n_kv_heads * (T / cfg->block_m) * cfg->head_dim *
+                           esize_of(cfg->dtype);
+        bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
+    }
+    if (prefill_tc_supported(cfg->dtype, cfg->head_dim, cfg->rmsnorm, cfg->shared_kv))
+        bytes += align256(prefill_tc_scratch_bytes(batch, T, cfg->n_kv_heads, cfg->rope_dims));
+    return bytes;
 }
 
 lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
@@ -271,7 +276,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
                          const void* zv, const void* b_pos_k, const void* b_pos_v, const float* sink,
                          const void* gamma_q, const void* gamma_kv, int32_t batch, int32_t T, void* out,
                          const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
-                         lbca_stream_t stream) {
+                         int32_t* d_status, lbca_stream_t stream) {
     LBCA_TRY(check_cfg(cfg));
     if (batch < 0 || T < 0) return LBCA_ERR_ARG;
     LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v, T > 0 && batch > 0));
@@ -289,7 +294,8 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
     const size_t need = lbca_prefill_workspace_bytes(cfg, batch, T, cache_out != nullptr);
     if (workspace_bytes < need) return LBCA_ERR_CAPACITY;
     if (need > 0 && !workspace) return LBCA_ERR_ARG;
-    if (out && !prefill_simt_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
+    const bool use_tc = out && prefill_tc_supported(cfg->dtype, cfg->head_dim, cfg->rmsnorm, cfg->shared_kv);
+    if (out && !use_tc && !prefill_simt_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
     LBCA_TRY(check_device());
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
@@ -334,7 +340,17 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.B = batch; a.T = T; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
         a.m = m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
         a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
-        LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
+        if (use_tc) {
+            size_t pooled_bytes = 0;
+            if (!cache_out) {
+                const size_t one = (size_t)batch * cfg->n_kv_heads * NB * cfg->head_dim * esize_of(cfg->dtype);
+                pooled_bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
+            }
+            void* scratch = static_cast<char*>(workspace) + pooled_bytes;
+            LBCA_TRY(cuda_status(launch_prefill_tc(a, scratch, d_status, s)));
+        } else {
+            LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
+        }
     }
     return LBCA_OK;
 }

@@ -129,6 +129,11 @@ struct PrefillArgs {
     double rope_step;  // theta^(-2/rho)
 };
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+// Tensor-core prefill (bf16, D = 128, GQA form without RMSNorm); `scratch` holds
+// prefill_tc_scratch_bytes (finalised raw keys and the RoPE table).
+bool prefill_tc_supported(int dtype, int D, int rmsnorm, int shared);
+size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, void* scratch, int32_t* status, cudaStream_t s);
 bool prefill_simt_supported(int D);
 
 }  // namespace lbca

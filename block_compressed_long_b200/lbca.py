@@ -66,7 +66,7 @@ _lib.lbca_append.restype = ctypes.c_int
 _lib.lbca_decode.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _sz, _vp, _vp]
 _lib.lbca_decode.restype = ctypes.c_int
 _lib.lbca_prefill.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
-                              _KP, _vp, _sz, _vp]
+                              _KP, _vp, _sz, _vp, _vp]
 _lib.lbca_prefill.restype = ctypes.c_int
 _lib.lbca_decode_step_workspace_bytes.argtypes = [_CP, _i32, _i32]
 _lib.lbca_decode_step_workspace_bytes.restype = _sz
@@ -209,7 +209,7 @@ def lbca_decode_step(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, q, cache: Ca
 
 
 def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv, out,
-                 cache_out: Cache | None = None, workspace=None, batch=None, T=None, stream=None):
+                 cache_out: Cache | None = None, workspace=None, batch=None, T=None, d_status=None, stream=None):
     """q, out [B, T, Hq, D]; k, v, zk, zv [B, T, G, D]."""
     B = k.shape[0] if batch is None else batch
     TT = k.shape[1] if T is None else T
@@ -219,7 +219,7 @@ def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv
                                              _ptr(b_pos_k), _ptr(b_pos_v), _ptr(sink), _ptr(gamma_q),
                                              _ptr(gamma_kv), B, TT, _ptr(out),
                                              ctypes.byref(cc) if cc is not None else None,
-                                             _ptr(workspace), wb, _stream(stream)))
+                                             _ptr(workspace), wb, _ptr(d_status), _stream(stream)))
 
 
 def lbca_decode_noalloc(cfg, q, cache: Cache, sink, gamma_q, out, max_ctx=0, d_status=None, stream=None):

@@ -233,6 +233,11 @@ LBCA_API lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, con
  *                window, the open block's pooling state and seq_lens = T, so
  *                that lbca_append / lbca_decode continue the sequences
  *   workspace    device, lbca_prefill_workspace_bytes(cfg, B, T, cache_out != NULL)
+ *   d_status     nullable device word for device-side conditions (a bounded
+ *                wait of the tensor-core kernel giving up: LBCA_ERR_TIMEOUT)
+ * bf16 I/O with D = 128, no RMSNorm and separate K/V runs QK^T and PV on the
+ * tensor cores (tcgen05, TMEM accumulators, TMA-fed tiles); every other
+ * shape runs the f32 CUDA-core kernel (no TF32).
  * Errors: LBCA_ERR_ARG, LBCA_ERR_ALIGN, LBCA_ERR_CAPACITY (cache too small),
  * LBCA_ERR_UNSUPPORTED, LBCA_ERR_CUDA.
  */
@@ -241,7 +246,7 @@ LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const v
                          const void* b_pos_v, const float* sink, const void* gamma_q,
                          const void* gamma_kv, int32_t batch, int32_t T, void* out,
                          const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
-                         lbca_stream_t stream);
+                         int32_t* d_status, lbca_stream_t stream);
 
 /*
  * lbca_decode_noalloc -- lbca_decode for callers that cannot allocate.

@@ -107,10 +107,10 @@ def test_cache_and_decode_checks(L):
     app = L._lib.lbca_append(ctypes.byref(cfg), A, None, A, A, A, A, None, ctypes.byref(cache), None, None)
     assert app == L.LBCA_ERR_ARG                          # GQA needs v
     pre = L._lib.lbca_prefill(ctypes.byref(cfg), A, A, A, A, A, A, A, None, None, None, 1, 64, None, None,
-                              None, 0, None)
+                              None, 0, None, None)
     assert pre == L.LBCA_ERR_ARG                          # neither out nor cache
     pre = L._lib.lbca_prefill(ctypes.byref(cfg), A, A, A, A, A, A, A, None, None, None, 1, 6400, A, None,
-                              None, 0, None)
+                              None, 0, None, None)
     assert pre == L.LBCA_ERR_CAPACITY                     # pooled entries need a workspace
 
 

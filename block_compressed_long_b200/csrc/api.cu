@@ -143,7 +143,7 @@ size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32
         bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
     }
     if (prefill_tc_supported(cfg->dtype, cfg->head_dim, cfg->rmsnorm, cfg->shared_kv))
-        bytes += align256(prefill_tc_scratch_bytes(batch, T, cfg->n_kv_heads, cfg->rope_dims));
+        bytes += align256(prefill_tc_scratch_bytes(batch, T, cfg->n_kv_heads, cfg->rope_dims, cfg->block_m));
     return bytes;
 }
 
@@ -307,6 +307,12 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         pv = cache_out ? cache_out->pooled_v : static_cast<char*>(workspace) + align256(one);
     }
     const int stride = cache_out ? cache_out->max_blocks : NB;
+    size_t pooled_bytes = 0;
+    if (!cache_out) {
+        const size_t one = (size_t)batch * cfg->n_kv_heads * NB * cfg->head_dim * esize_of(cfg->dtype);
+        pooled_bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
+    }
+    char* tc_scratch = static_cast<char*>(workspace) + pooled_bytes;
     for (int series = 0; series < (cfg->shared_kv ? 1 : 2); ++series) {
         PoolArgs a{};
         a.dtype = cfg->dtype;
@@ -318,6 +324,11 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
         a.state = cache_out ? cache_out->pool_state : nullptr;
         a.S = cfg->shared_kv ? 1 : 2; a.series = series;
+        if (use_tc && series == 0) {
+            // the tensor-core QK^T reads a dense fp16 copy of the pooled keys, [B, G, NB, D]
+            a.out_f16 = tc_scratch + prefill_tc_pooled_f16_offset(batch, T, cfg->n_kv_heads, cfg->rope_dims);
+            a.out_f16_blocks = NB;
+        }
         LBCA_TRY(cuda_status(launch_pool(a, s)));
     }
     // 2. the raw window and the lengths, so decode can continue from T
@@ -341,13 +352,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.m = m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
         a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
         if (use_tc) {
-            size_t pooled_bytes = 0;
-            if (!cache_out) {
-                const size_t one = (size_t)batch * cfg->n_kv_heads * NB * cfg->head_dim * esize_of(cfg->dtype);
-                pooled_bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
-            }
-            void* scratch = static_cast<char*>(workspace) + pooled_bytes;
-            LBCA_TRY(cuda_status(launch_prefill_tc(a, scratch, d_status, s)));
+            LBCA_TRY(cuda_status(launch_prefill_tc(a, tc_scratch, d_status, s)));
         } else {
             LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
         }

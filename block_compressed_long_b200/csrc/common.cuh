@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -56,6 +57,19 @@ __device__ __forceinline__ void ld16_cs(const __nv_bfloat16* p, float (&o)[8]) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+// 8 floats -> 8 fp16 (16 bytes)
+__device__ __forceinline__ void st16_f16(__half* p, const float (&o)[8]) {
+    uint4 v;
+    v.x = pack_f16x2(o[0], o[1]);
+    v.y = pack_f16x2(o[2], o[3]);
+    v.z = pack_f16x2(o[4], o[5]);
+    v.w = pack_f16x2(o[6], o[7]);
+    *reinterpret_cast<uint4*>(p) = v;
 }
 __device__ __forceinline__ void st16(float* p, const float (&o)[4]) {
     *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);

@@ -24,6 +24,8 @@ struct PoolArgs {
     float eps;
     float* state;          // [B, S, 3, G, D] or null: running state of the partial block
     int S, series;
+    void* out_f16;         // optional fp16 copy [B, G, out_f16_blocks, D] (bf16 input only)
+    int out_f16_blocks;
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 
@@ -132,7 +134,9 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // Tensor-core prefill (bf16, D = 128, GQA form without RMSNorm); `scratch` holds
 // prefill_tc_scratch_bytes (finalised raw keys and the RoPE table).
 bool prefill_tc_supported(int dtype, int D, int rmsnorm, int shared);
-size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho);
+size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m);
+// where, inside that scratch, the pool pass leaves the fp16 copy of the pooled keys
+size_t prefill_tc_pooled_f16_offset(int B, int T, int G, int rho);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, void* scratch, int32_t* status, cudaStream_t s);
 bool prefill_simt_supported(int D);
 

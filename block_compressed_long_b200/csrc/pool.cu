@@ -173,12 +173,17 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
             finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma),
                                  a.rho, cs);
         if (active) {
-            T* o = static_cast<T*>(a.out) +
-                   (((size_t)b * a.G + g) * a.out_blocks + a.blk_off + j) * a.D + d0;
+            const size_t oi = (((size_t)b * a.G + g) * a.out_blocks + a.blk_off + j) * a.D + d0;
             float tmp[VEC];
 #pragma unroll
             for (int i = 0; i < VEC; ++i) tmp[i] = e[i];
-            st16(o, tmp);
+            st16(static_cast<T*>(a.out) + oi, tmp);
+            if constexpr (VEC == 8) {
+                if (a.out_f16) {  // the f32 value, rounded once to fp16
+                    const size_t oi16 = (((size_t)b * a.G + g) * a.out_f16_blocks + a.blk_off + j) * a.D + d0;
+                    st16_f16(static_cast<__half*>(a.out_f16) + oi16, tmp);
+                }
+            }
         }
     } else if (a.state && active) {
         float* st = a.state + (((size_t)b * a.S + a.series) * 3) * GD + (size_t)cv * VEC;

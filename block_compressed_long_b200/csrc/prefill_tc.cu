@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idS = idesc_bf16_f32(BM, BN, false);
+            const uint32_t idS = idesc_f16_f32(BM, BN);
             const uint32_t idP = idesc_bf16_f32(BM, HD, true);
             const uint32_t sq = smem_addr(smem + OFF_Q), sp = smem_addr(smem + OFF_P);
             auto issue_s = [&](int i) {
@@ -194,8 +194,8 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         const int half = a.rho / 2;
 
         bool ok = __all_sync(0xffffffffu, wait_or_fail(&bars[B_QFULL], 0, fail, a.status));
-        if (ok && valid && a.rho) {  // rotate this query row in place (RoPE at t)
-            const float2* tab = a.tab + (size_t)t * half;
+        if (ok) {  // this query row, in place: bf16 -> f32, RoPE at t, -> fp16 (QK^T runs in fp16)
+            const float2* tab = a.tab + (size_t)(valid ? t : 0) * half;
             for (int q = 0; q < HD / 8; ++q) {
                 uint4* p = reinterpret_cast<uint4*>(smem + OFF_Q + sw128_off(r, 8 * q, REGION));
                 uint4 u = *p;
@@ -203,11 +203,9 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int d = 8 * q + 2 * e;
-                    if (d >= HD - a.rho) {
-                        float x = __uint_as_float(wv[e] << 16), y = __uint_as_float(wv[e] & 0xffff0000u);
-                        rotate_pair(x, y, tab[(d - (HD - a.rho)) >> 1]);
-                        wv[e] = pack_bf16x2(x, y);
-                    }
+                    float x = __uint_as_float(wv[e] << 16), y = __uint_as_float(wv[e] & 0xffff0000u);
+                    if (valid && d >= HD - a.rho) rotate_pair(x, y, tab[(d - (HD - a.rho)) >> 1]);
+                    wv[e] = pack_f16x2(x, y);
                 }
                 *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
@@ -338,8 +336,9 @@ __global__ void rope_table_kernel(float2* tab, int T, int half, double step) {
         tab[i] = rope_cs(i / half, (int)(i % half), step);
 }
 
-// Finalised raw keys: RoPE at s applied once, bf16 out, same [B, T, G, D] layout.
-__global__ void finalise_keys_kernel(const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ out,
+// Finalised raw keys: RoPE at s applied once, fp16 out (the QK^T operand type),
+// same [B, T, G, D] layout.
+__global__ void finalise_keys_kernel(const __nv_bfloat16* __restrict__ k, __half* __restrict__ out,
                                      const float2* __restrict__ tab, int64_t n_vec, int G, int T, int rho) {
     const int half = rho / 2;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec; i += (int64_t)gridDim.x * blockDim.x) {
@@ -353,7 +352,7 @@ __global__ void finalise_keys_kernel(const __nv_bfloat16* __restrict__ k, __nv_b
             const int d = d0 + e;
             if (d >= HD - rho) rotate_pair(v[e], v[e + 1], tab[(size_t)s * half + ((d - (HD - rho)) >> 1)]);
         }
-        st16(out + i * 8, v);
+        st16_f16(out + i * 8, v);
     }
 }
 
@@ -371,12 +370,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 4-D bf16 map with a box of (64, b1, b2, 1) and 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides_bytes[3],
-              uint32_t box1, uint32_t box2) {
+              uint32_t box1, uint32_t box2, bool f16 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t box[4] = {64, box1, box2, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides_bytes, box, estr,
+    CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                    const_cast<void*>(base), dims, strides_bytes, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -388,22 +388,31 @@ bool prefill_tc_supported(int dtype, int D, int rmsnorm, int shared) {
     return dtype == LBCA_BF16 && D == HD && !rmsnorm && !shared;
 }
 
-size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho) {
+size_t prefill_tc_pooled_f16_offset(int B, int T, int G, int rho) {
     const size_t keys = (size_t)B * T * G * HD * 2;
-    const size_t tab = (size_t)T * (rho / 2) * sizeof(float2);
+    const size_t tab = (size_t)T * std::max(rho / 2, 1) * sizeof(float2);
     return (keys + 255) / 256 * 256 + (tab + 255) / 256 * 256;
+}
+
+// fp16 finalised raw keys, the cos/sin table, and an fp16 copy of the pooled keys
+size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m) {
+    const size_t pooled = (size_t)B * G * (T / m) * HD * 2;
+    return prefill_tc_pooled_f16_offset(B, T, G, rho) + (pooled + 255) / 256 * 256;
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* status, cudaStream_t s) {
     if (p.B == 0 || p.T == 0) return cudaSuccess;
     const int G = p.G, T = p.T, B = p.B, Hq = p.Hq;
-    __nv_bfloat16* keys = static_cast<__nv_bfloat16*>(scratch);
+    __half* keys = static_cast<__half*>(scratch);
     const size_t keys_bytes = ((size_t)B * T * G * HD * 2 + 255) / 256 * 256;
     float2* tab = reinterpret_cast<float2*>(static_cast<char*>(scratch) + keys_bytes);
+    const void* pooled_k16 = static_cast<char*>(scratch) + prefill_tc_pooled_f16_offset(B, T, G, p.rho);
     const int half = p.rho / 2;
     if (half > 0) {
         const int64_t n = (int64_t)T * half;
         rope_table_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 148 * 16), 256, 0, s>>>(tab, T, half, p.rope_step);
+    }
+    {
         const int64_t nv = (int64_t)B * T * G * (HD / 8);
         finalise_keys_kernel<<<(int)std::min<int64_t>((nv + 255) / 256, 148 * 32), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(p.k), keys, tab, nv, G, T, p.rho);
@@ -421,14 +430,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     {   // pooled [B, G, stride, D], valid rows NB
         const uint64_t dims[4] = {HD, (uint64_t)std::max(NB, 1), (uint64_t)G, (uint64_t)B};
         const uint64_t str[3] = {HD * e, ps * HD * e, (uint64_t)G * ps * HD * e};
-        if (!make_map(&a.tpk, p.pooled_k, dims, str, BN, 1)) return cudaErrorInvalidValue;
         if (!make_map(&a.tpv, p.pooled_v, dims, str, BN, 1)) return cudaErrorInvalidValue;
+        // fp16 pooled keys in the scratch, [B, G, NB, D]
+        const uint64_t nb = (uint64_t)std::max(NB, 1);
+        const uint64_t str16[3] = {HD * e, nb * HD * e, (uint64_t)G * nb * HD * e};
+        if (!make_map(&a.tpk, pooled_k16, dims, str16, BN, 1, true)) return cudaErrorInvalidValue;
     }
     {   // raw [B, T, G, D]
         const uint64_t dims[4] = {HD, (uint64_t)G, (uint64_t)T, (uint64_t)B};
         const uint64_t str[3] = {HD * e, (uint64_t)G * HD * e, (uint64_t)T * G * HD * e};
-        if (!make_map(&a.trk, half > 0 ? static_cast<const void*>(keys) : p.k, dims, str, 1, BN))
-            return cudaErrorInvalidValue;
+        if (!make_map(&a.trk, keys, dims, str, 1, BN, true)) return cudaErrorInvalidValue;
         if (!make_map(&a.trv, p.v, dims, str, 1, BN)) return cudaErrorInvalidValue;
     }
     a.tab = tab;

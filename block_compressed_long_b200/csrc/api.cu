@@ -291,10 +291,14 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         if (cache_out->batch != batch) return LBCA_ERR_ARG;
         if (cache_out->max_blocks < NB) return LBCA_ERR_CAPACITY;
     }
-    const size_t need = lbca_prefill_workspace_bytes(cfg, batch, T, cache_out != nullptr);
+    const bool use_tc = out && prefill_tc_supported(cfg->dtype, cfg->head_dim, cfg->rmsnorm, cfg->shared_kv);
+    size_t need = 0;  // what this call uses: pooled entries without a cache, tensor-core scratch with an output
+    if (!cache_out)
+        need += align256((size_t)batch * cfg->n_kv_heads * NB * cfg->head_dim * esize_of(cfg->dtype)) *
+                (cfg->shared_kv ? 1 : 2);
+    if (use_tc) need += align256(prefill_tc_scratch_bytes(batch, T, cfg->n_kv_heads, cfg->rope_dims, cfg->block_m));
     if (workspace_bytes < need) return LBCA_ERR_CAPACITY;
     if (need > 0 && !workspace) return LBCA_ERR_ARG;
-    const bool use_tc = out && prefill_tc_supported(cfg->dtype, cfg->head_dim, cfg->rmsnorm, cfg->shared_kv);
     if (out && !use_tc && !prefill_simt_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
     LBCA_TRY(check_device());
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -13,15 +13,16 @@
 //              two-stage ring, 128-byte swizzled, no multicast.
 //   warp 1     TMEM owner and MMA issuer: S = Q K^T (tcgen05.mma M=128 N=128,
 //              K-major operands) into one of two TMEM S buffers, and
-//              O += P V (P from shared memory, V as an MN-major operand) into
+//              O += P V (fp16 P from shared memory, fp16 V as an MN-major operand) into
 //              the TMEM O accumulator; completion is signalled by
 //              tcgen05.commit on mbarriers.  S(i+1) is issued before PV(i) so
 //              the tensor core works on the next tile while the softmax runs.
+//   warps 2-3  convert each V tile in place from bf16 to fp16 once it lands.
 //   warps 4-7  softmax: thread r owns query row r and TMEM lane r.  It rotates
 //              its Q row in shared memory once, then per tile loads its S row,
 //              applies the causal-block / window mask, keeps an online max
 //              (rescaling O in TMEM only when the max grows by more than 2^8),
-//              writes P in bf16 into the swizzled P tile, and finally
+//              writes P in fp16 into the swizzled P tile, and finally
 //              normalises its O row (plus the sink) and stores it.
 // Raw keys arrive already rotated (a pre-pass writes the finalised keys once,
 // instead of every query tile rotating them again); Q is rotated in shared
@@ -46,8 +47,8 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers, + alignmen
 constexpr uint32_t TMEM_COLS = 512;                    // S0, S1, O (128 columns each)
 constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;
 
-enum { B_QFULL, B_QROT, B_KFULL0, B_KFULL1, B_VFULL0, B_VFULL1, B_KVEMPTY0, B_KVEMPTY1, B_SFULL0, B_SFULL1,
-       B_SFREE0, B_SFREE1, B_PFULL, B_ODONE, B_COUNT };
+enum { B_QFULL, B_QROT, B_KFULL0, B_KFULL1, B_VFULL0, B_VFULL1, B_VCONV0, B_VCONV1, B_KVEMPTY0, B_KVEMPTY1,
+       B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL, B_ODONE, B_COUNT };
 
 struct TcArgs {
     CUtensorMap tq;   // q [B, T, Hq, D]          dims (D, Hq, T, B)
@@ -92,7 +93,8 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             const bool softmax_arrivals = i == B_QROT || i == B_SFREE0 || i == B_SFREE1 || i == B_PFULL;
-            mbar_init(&bars[i], softmax_arrivals ? 128u : 1u);
+            const bool convert_arrivals = i == B_VCONV0 || i == B_VCONV1;
+            mbar_init(&bars[i], softmax_arrivals ? 128u : convert_arrivals ? 64u : 1u);
         }
         *fail = 0;
         fence_barrier_init();
@@ -142,8 +144,8 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idS = idesc_f16_f32(BM, BN);
-            const uint32_t idP = idesc_bf16_f32(BM, HD, true);
+            const uint32_t idS = idesc_f16_f32(BM, BN, false);
+            const uint32_t idP = idesc_f16_f32(BM, HD, true);
             const uint32_t sq = smem_addr(smem + OFF_Q), sp = smem_addr(smem + OFF_P);
             auto issue_s = [&](int i) {
                 const int s = i & 1;
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                     issue_s(n);
                 }
                 ok = wait_or_fail(&bars[B_PFULL], i & 1, fail, a.status) &&
-                     wait_or_fail(&bars[B_VFULL0 + (i & 1)], (i >> 1) & 1, fail, a.status);
+                     wait_or_fail(&bars[B_VCONV0 + (i & 1)], (i >> 1) & 1, fail, a.status);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sv = smem_addr(smem + OFF_V + (i & 1) * TILE);
@@ -182,6 +184,27 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 tc_commit(&bars[B_ODONE]);
                 tc_commit(&bars[B_KVEMPTY0 + (i & 1)]);
             }
+        }
+    } else if (warp == 2 || warp == 3) {
+        // ----------------------------------------- V tiles: bf16 -> fp16 in place
+        // (P V runs in fp16: P in [0, 256] keeps 11 mantissa bits; bf16 values
+        // widen exactly to fp16 in its normal range; element-wise, so the
+        // swizzled layout is untouched)
+        const int ct = threadIdx.x - 64;
+        for (int i = 0; i < ntile; ++i) {
+            const int s = i & 1;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&bars[B_VFULL0 + s], (i >> 1) & 1, fail, a.status))) break;
+            uint4* vt = reinterpret_cast<uint4*>(smem + OFF_V + s * TILE);
+            for (int q = ct; q < (int)(TILE / 16); q += 64) {
+                uint4 u = vt[q];
+                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    wv[e] = pack_f16x2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
+                vt[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&bars[B_VCONV0 + s]);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------- softmax
@@ -279,10 +302,10 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
 #pragma unroll
             for (int q = 0; q < BN / 8; ++q) {
                 uint4 u;
-                u.x = pack_bf16x2(s[8 * q + 0], s[8 * q + 1]);
-                u.y = pack_bf16x2(s[8 * q + 2], s[8 * q + 3]);
-                u.z = pack_bf16x2(s[8 * q + 4], s[8 * q + 5]);
-                u.w = pack_bf16x2(s[8 * q + 6], s[8 * q + 7]);
+                u.x = pack_f16x2(s[8 * q + 0], s[8 * q + 1]);
+                u.y = pack_f16x2(s[8 * q + 2], s[8 * q + 3]);
+                u.z = pack_f16x2(s[8 * q + 4], s[8 * q + 5]);
+                u.w = pack_f16x2(s[8 * q + 6], s[8 * q + 7]);
                 *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(r, 8 * q, REGION)) = u;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

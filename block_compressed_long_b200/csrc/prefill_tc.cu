@@ -39,28 +39,50 @@
 namespace lbca {
 namespace {
 
-constexpr int BM = 128, BN = 128, HD = 128;
-constexpr uint32_t REGION = 128 * 64 * 2;  // [128 rows][64 cols] bf16, one 128-byte swizzle span per row
-constexpr uint32_t TILE = 2 * REGION;      // a [128][128] bf16 tile
-constexpr uint32_t OFF_Q = 0, OFF_K = TILE, OFF_V = 3 * TILE, OFF_P = 5 * TILE, OFF_BAR = 6 * TILE;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t TMEM_COLS = 512;                    // S0, S1, O (128 columns each)
+constexpr int BM = 128;     // query rows per softmax warpgroup (one M=128 MMA)
+constexpr int NQ = 2;       // query tiles per CTA
+constexpr int BN = 64;      // entries per K/V tile
+constexpr int HD = 128;     // head dim
+constexpr int NSTAGE = 3;   // K/V ring depth
+constexpr uint32_t QREG = BM * 64 * 2;   // [128 rows][64 cols] 16-bit: one 128-byte swizzle span per row
+constexpr uint32_t QTILE = 2 * QREG;     // [128][128]
+constexpr uint32_t KREG = BN * 64 * 2;   // [64 rows][64 cols]
+constexpr uint32_t KTILE = 2 * KREG;     // [64][128]
+constexpr uint32_t PTILE = BM * BN * 2;  // [128 rows][64 entries] fp16
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + NQ * QTILE;
+constexpr uint32_t OFF_V = OFF_K + NSTAGE * KTILE;
+constexpr uint32_t OFF_P = OFF_V + NSTAGE * KTILE;
+constexpr uint32_t OFF_BAR = OFF_P + NQ * PTILE;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + barriers, + alignment slack
+constexpr uint32_t TMEM_COLS = 512;  // S[q][2] (64 columns each) at 0..255, O[q] (128 columns) at 256..511
+constexpr int kThreads = 384;        // warps 0 producer, 1 MMA, 2-3 V converters, 4-7 / 8-11 softmax
 constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;
 
-enum { B_QFULL, B_QROT, B_KFULL0, B_KFULL1, B_VFULL0, B_VFULL1, B_VCONV0, B_VCONV1, B_KVEMPTY0, B_KVEMPTY1,
-       B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL, B_ODONE, B_COUNT };
+// barrier slots
+constexpr int B_QFULL = 0;
+constexpr int B_QROT = 1;                      // [NQ]
+constexpr int B_KFULL = B_QROT + NQ;           // [NSTAGE]
+constexpr int B_VFULL = B_KFULL + NSTAGE;      // [NSTAGE]
+constexpr int B_VCONV = B_VFULL + NSTAGE;      // [NSTAGE]
+constexpr int B_KVEMPTY = B_VCONV + NSTAGE;    // [NSTAGE]
+constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ][2]
+constexpr int B_SFREE = B_SFULL + 2 * NQ;      // [NQ][2]
+constexpr int B_PFULL = B_SFREE + 2 * NQ;      // [NQ]
+constexpr int B_ODONE = B_PFULL + NQ;          // [NQ]
+constexpr int B_COUNT = B_ODONE + NQ;
 
 struct TcArgs {
-    CUtensorMap tq;   // q [B, T, Hq, D]          dims (D, Hq, T, B)
-    CUtensorMap tpk;  // pooled keys [B, G, *, D]  dims (D, NB, G, B)
-    CUtensorMap tpv;  // pooled values
-    CUtensorMap trk;  // finalised raw keys [B, T, G, D] dims (D, G, T, B)
-    CUtensorMap trv;  // raw values
+    CUtensorMap tq;   // q [B, T, Hq, D] bf16          dims (D, Hq, T, B)
+    CUtensorMap tpk;  // pooled keys fp16 [B, G, NB, D] dims (D, NB, G, B)
+    CUtensorMap tpv;  // pooled values bf16 [B, G, *, D]
+    CUtensorMap trk;  // finalised raw keys fp16 [B, T, G, D] dims (D, G, T, B)
+    CUtensorMap trv;  // raw values bf16
     const float2* tab;  // [T][rho/2] cos/sin
     const float* sink;
     void* out;          // [B, T, Hq, D] bf16
     int32_t* status;
-    int T, Hq, G, m, w, rho, n_qtiles;
+    int T, Hq, G, m, w, rho, n_ctiles;
     float scale;
 };
 
@@ -71,8 +93,11 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, int
     set_status(status, LBCA_ERR_TIMEOUT);
     return false;
 }
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* fail, int32_t* status) {
+    return __all_sync(0xffffffffu, wait_or_fail(bar, parity, fail, status));
+}
 
-__global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -80,10 +105,10 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     int* fail = reinterpret_cast<int*>(tmem_sh + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, qt = a.n_qtiles - 1 - (int)blockIdx.y, b = blockIdx.z;  // heavy tiles first
+    const int h = blockIdx.x, ct = a.n_ctiles - 1 - (int)blockIdx.y, b = blockIdx.z;  // heavy tiles first
     const int g = h / (a.Hq / a.G);
-    const int t0 = qt * BM;
-    const int t_last = min(t0 + BM, a.T) - 1;
+    const int t0 = ct * NQ * BM;
+    const int t_last = min(t0 + NQ * BM, a.T) - 1;
     const int Pmax = visible_blocks(t_last + 1, a.m, a.w);
     const int s_lo = visible_blocks(t0 + 1, a.m, a.w) * a.m;
     const int npt = (Pmax + BN - 1) / BN;
@@ -92,9 +117,12 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            const bool softmax_arrivals = i == B_QROT || i == B_SFREE0 || i == B_SFREE1 || i == B_PFULL;
-            const bool convert_arrivals = i == B_VCONV0 || i == B_VCONV1;
-            mbar_init(&bars[i], softmax_arrivals ? 128u : convert_arrivals ? 64u : 1u);
+            uint32_t cnt = 1;
+            if ((i >= B_QROT && i < B_QROT + NQ) || (i >= B_SFREE && i < B_SFREE + 2 * NQ) ||
+                (i >= B_PFULL && i < B_PFULL + NQ))
+                cnt = 128;
+            if (i >= B_VCONV && i < B_VCONV + NSTAGE) cnt = 64;
+            mbar_init(&bars[i], cnt);
         }
         *fail = 0;
         fence_barrier_init();
@@ -103,41 +131,43 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_sh;
-    const uint32_t tO = tbase + 256;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&bars[B_QFULL], TILE);
-            tma_load_4d(smem + OFF_Q, &a.tq, 0, h, t0, b, &bars[B_QFULL]);
-            tma_load_4d(smem + OFF_Q + REGION, &a.tq, 64, h, t0, b, &bars[B_QFULL]);
+            mbar_arrive_expect_tx(&bars[B_QFULL], NQ * QTILE);
+            for (int q = 0; q < NQ; ++q)
+                for (int rg = 0; rg < 2; ++rg)
+                    tma_load_4d(smem + OFF_Q + q * QTILE + rg * QREG, &a.tq, 64 * rg, h, t0 + q * BM, b,
+                                &bars[B_QFULL]);
             int issued = 0;
             for (int i = 0; i < ntile; ++i) {
-                const int s = i & 1;
-                if (i >= 2 && !wait_or_fail(&bars[B_KVEMPTY0 + s], ((i >> 1) - 1) & 1, fail, a.status)) break;
-                uint8_t* kd = smem + OFF_K + s * TILE;
-                uint8_t* vd = smem + OFF_V + s * TILE;
-                mbar_arrive_expect_tx(&bars[B_KFULL0 + s], TILE);
-                mbar_arrive_expect_tx(&bars[B_VFULL0 + s], TILE);
+                const int s = i % NSTAGE;
+                if (i >= NSTAGE && !wait_or_fail(&bars[B_KVEMPTY + s], ((i / NSTAGE) - 1) & 1, fail, a.status))
+                    break;
+                uint8_t* kd = smem + OFF_K + s * KTILE;
+                uint8_t* vd = smem + OFF_V + s * KTILE;
+                mbar_arrive_expect_tx(&bars[B_KFULL + s], KTILE);
+                mbar_arrive_expect_tx(&bars[B_VFULL + s], KTILE);
                 if (i < npt) {
                     const int j0 = i * BN;
-                    tma_load_4d(kd, &a.tpk, 0, j0, g, b, &bars[B_KFULL0 + s]);
-                    tma_load_4d(kd + REGION, &a.tpk, 64, j0, g, b, &bars[B_KFULL0 + s]);
-                    tma_load_4d(vd, &a.tpv, 0, j0, g, b, &bars[B_VFULL0 + s]);
-                    tma_load_4d(vd + REGION, &a.tpv, 64, j0, g, b, &bars[B_VFULL0 + s]);
+                    for (int rg = 0; rg < 2; ++rg) {
+                        tma_load_4d(kd + rg * KREG, &a.tpk, 64 * rg, j0, g, b, &bars[B_KFULL + s]);
+                        tma_load_4d(vd + rg * KREG, &a.tpv, 64 * rg, j0, g, b, &bars[B_VFULL + s]);
+                    }
                 } else {
                     const int s0 = s_lo + (i - npt) * BN;
-                    tma_load_4d(kd, &a.trk, 0, g, s0, b, &bars[B_KFULL0 + s]);
-                    tma_load_4d(kd + REGION, &a.trk, 64, g, s0, b, &bars[B_KFULL0 + s]);
-                    tma_load_4d(vd, &a.trv, 0, g, s0, b, &bars[B_VFULL0 + s]);
-                    tma_load_4d(vd + REGION, &a.trv, 64, g, s0, b, &bars[B_VFULL0 + s]);
+                    for (int rg = 0; rg < 2; ++rg) {
+                        tma_load_4d(kd + rg * KREG, &a.trk, 64 * rg, g, s0, b, &bars[B_KFULL + s]);
+                        tma_load_4d(vd + rg * KREG, &a.trv, 64 * rg, g, s0, b, &bars[B_VFULL + s]);
+                    }
                 }
                 issued = i + 1;
             }
             // drain: never leave copies in flight into shared memory (bounded)
-            for (int i = max(0, issued - 2); i < issued; ++i) {
-                mbar_wait(&bars[B_KFULL0 + (i & 1)], (i >> 1) & 1, kWaitNs);
-                mbar_wait(&bars[B_VFULL0 + (i & 1)], (i >> 1) & 1, kWaitNs);
+            for (int i = max(0, issued - NSTAGE); i < issued; ++i) {
+                mbar_wait(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, kWaitNs);
+                mbar_wait(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, kWaitNs);
             }
             mbar_wait(&bars[B_QFULL], 0, kWaitNs);
         }
@@ -146,43 +176,47 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
-            const uint32_t sq = smem_addr(smem + OFF_Q), sp = smem_addr(smem + OFF_P);
-            auto issue_s = [&](int i) {
-                const int s = i & 1;
-                const uint32_t sk = smem_addr(smem + OFF_K + s * TILE);
-                tc_fence_after();
+            bool ok = true;
+            for (int q = 0; ok && q < NQ; ++q) ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
+            for (int i = 0; ok && i <= ntile; ++i) {
+                if (i < ntile) {  // S_q(i) = Q_q K_i^T for both query tiles
+                    const int s = i % NSTAGE;
+                    ok = wait_or_fail(&bars[B_KFULL + s], (i / NSTAGE) & 1, fail, a.status);
+                    const uint32_t sk = smem_addr(smem + OFF_K + s * KTILE);
+                    for (int q = 0; ok && q < NQ; ++q) {
+                        if (i >= 2) ok = wait_or_fail(&bars[B_SFREE + 2 * q + (i & 1)], ((i >> 1) - 1) & 1, fail,
+                                                      a.status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
+                        const uint32_t dS = tbase + (uint32_t)(2 * q + (i & 1)) * BN;
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * REGION + (kk & 3) * 32;
-                    tc_mma_bf16(tbase + 128 * s, smem_desc_sw128(sq + off, 16, 1024),
-                                smem_desc_sw128(sk + off, 16, 1024), idS, kk > 0);
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            tc_mma_bf16(dS, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
+                                        smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+                        }
+                        tc_commit(&bars[B_SFULL + 2 * q + (i & 1)]);
+                    }
                 }
-                tc_commit(&bars[B_SFULL0 + s]);
-            };
-            bool ok = wait_or_fail(&bars[B_QROT], 0, fail, a.status);
-            if (ok && ntile > 0) ok = wait_or_fail(&bars[B_KFULL0], 0, fail, a.status);
-            if (ok && ntile > 0) issue_s(0);
-            for (int i = 0; ok && i < ntile; ++i) {
-                const int n = i + 1;
-                if (n < ntile) {
-                    ok = wait_or_fail(&bars[B_KFULL0 + (n & 1)], (n >> 1) & 1, fail, a.status);
-                    if (ok && n >= 2) ok = wait_or_fail(&bars[B_SFREE0 + (n & 1)], ((n >> 1) - 1) & 1, fail, a.status);
-                    if (!ok) break;
-                    issue_s(n);
-                }
-                ok = wait_or_fail(&bars[B_PFULL], i & 1, fail, a.status) &&
-                     wait_or_fail(&bars[B_VCONV0 + (i & 1)], (i >> 1) & 1, fail, a.status);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t sv = smem_addr(smem + OFF_V + (i & 1) * TILE);
+                if (ok && i >= 1) {  // O_q += P_q(j) V_j for the previous tile j
+                    const int j = i - 1, sj = j % NSTAGE;
+                    ok = wait_or_fail(&bars[B_VCONV + sj], (j / NSTAGE) & 1, fail, a.status);
+                    const uint32_t sv = smem_addr(smem + OFF_V + sj * KTILE);
+                    for (int q = 0; ok && q < NQ; ++q) {
+                        ok = wait_or_fail(&bars[B_PFULL + q], j & 1, fail, a.status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sp = smem_addr(smem + OFF_P + q * PTILE);
+                        const uint32_t dO = tbase + 256 + (uint32_t)q * HD;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint32_t poff = (kk >> 2) * REGION + (kk & 3) * 32;
-                    tc_mma_bf16(tO, smem_desc_sw128(sp + poff, 16, 1024),
-                                smem_desc_sw128(sv + kk * 2048, REGION, 1024), idP, (i > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BN / 16; ++kk) {
+                            tc_mma_bf16(dO, smem_desc_sw128(sp + kk * 32, 16, 1024),
+                                        smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&bars[B_ODONE + q]);
+                    }
+                    if (ok) tc_commit(&bars[B_KVEMPTY + sj]);
                 }
-                tc_commit(&bars[B_ODONE]);
-                tc_commit(&bars[B_KVEMPTY0 + (i & 1)]);
             }
         }
     } else if (warp == 2 || warp == 3) {
@@ -190,42 +224,48 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
         // (P V runs in fp16: P in [0, 256] keeps 11 mantissa bits; bf16 values
         // widen exactly to fp16 in its normal range; element-wise, so the
         // swizzled layout is untouched)
-        const int ct = threadIdx.x - 64;
+        const int cthr = threadIdx.x - 64;
         for (int i = 0; i < ntile; ++i) {
-            const int s = i & 1;
-            if (!__all_sync(0xffffffffu, wait_or_fail(&bars[B_VFULL0 + s], (i >> 1) & 1, fail, a.status))) break;
-            uint4* vt = reinterpret_cast<uint4*>(smem + OFF_V + s * TILE);
-            for (int q = ct; q < (int)(TILE / 16); q += 64) {
-                uint4 u = vt[q];
+            const int s = i % NSTAGE;
+            if (!warp_wait(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status)) break;
+            uint4* vt = reinterpret_cast<uint4*>(smem + OFF_V + s * KTILE);
+#pragma unroll 4
+            for (int qv = cthr; qv < (int)(KTILE / 16); qv += 64) {
+                uint4 u = vt[qv];
                 uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     wv[e] = pack_f16x2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
-                vt[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                vt[qv] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&bars[B_VCONV0 + s]);
+            mbar_arrive(&bars[B_VCONV + s]);
         }
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------------------- softmax
-        const int r = threadIdx.x - 128;
-        const int t = t0 + r;
+        const int q = (warp - 4) >> 2;           // query tile of this warpgroup
+        const int r = threadIdx.x - 128 - 128 * q;
+        const int t = t0 + q * BM + r;
         const bool valid = t < a.T;
         const int Pq = visible_blocks(t + 1, a.m, a.w);
         const int lo = Pq * a.m;
-        const uint32_t lane_f = (uint32_t)(32 * (warp - 4)) << 16;
+        const uint32_t lane_f = (uint32_t)(32 * (warp & 3)) << 16;
         const int half = a.rho / 2;
+        const uint32_t tS0 = tbase + (uint32_t)(2 * q) * BN;
+        const uint32_t tO = tbase + 256 + (uint32_t)q * HD;
+        uint8_t* sQ = smem + OFF_Q + q * QTILE;
+        uint8_t* sP = smem + OFF_P + q * PTILE;
 
-        bool ok = __all_sync(0xffffffffu, wait_or_fail(&bars[B_QFULL], 0, fail, a.status));
+        bool ok = warp_wait(&bars[B_QFULL], 0, fail, a.status);
         if (ok) {  // this query row, in place: bf16 -> f32, RoPE at t, -> fp16 (QK^T runs in fp16)
             const float2* tab = a.tab + (size_t)(valid ? t : 0) * half;
-            for (int q = 0; q < HD / 8; ++q) {
-                uint4* p = reinterpret_cast<uint4*>(smem + OFF_Q + sw128_off(r, 8 * q, REGION));
+            for (int c8 = 0; c8 < HD / 8; ++c8) {
+                uint4* p = reinterpret_cast<uint4*>(sQ + sw128_off(r, 8 * c8, QREG));
                 uint4 u = *p;
                 uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int d = 8 * q + 2 * e;
+                    const int d = 8 * c8 + 2 * e;
                     float x = __uint_as_float(wv[e] << 16), y = __uint_as_float(wv[e] & 0xffff0000u);
                     if (valid && d >= HD - a.rho) rotate_pair(x, y, tab[(d - (HD - a.rho)) >> 1]);
                     wv[e] = pack_f16x2(x, y);
@@ -234,53 +274,62 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&bars[B_QROT]);
+        mbar_arrive(&bars[B_QROT + q]);
 
-        const float sc = a.scale * kLog2e;
-        float m_ref = kNegInf, l = 0.f;
+        const float sc = a.scale * kLog2e;  // scores enter the exponent as s * sc (log2 units)
+        float m_ref = kNegInf, l = 0.f;     // running max (unscaled score units) and sum
         for (int i = 0; ok && i < ntile; ++i) {
             const bool pooled = i < npt;
             const int base = pooled ? i * BN : s_lo + (i - npt) * BN;
-            ok = __all_sync(0xffffffffu, wait_or_fail(&bars[B_SFULL0 + (i & 1)], (i >> 1) & 1, fail, a.status));
+            ok = warp_wait(&bars[B_SFULL + 2 * q + (i & 1)], (i >> 1) & 1, fail, a.status);
             if (!ok) break;
             tc_fence_after();
             float s[BN];
+            {
+                float v0[32], v1[32];
+                tmem_ld32(tS0 + (uint32_t)(i & 1) * BN + lane_f, v0);
+                tmem_ld32(tS0 + (uint32_t)(i & 1) * BN + lane_f + 32, v1);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                float v[32];
-                tmem_ld32(tbase + 128 * (i & 1) + lane_f + 32 * c, v);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) s[32 * c + k] = v[k];
+                for (int k = 0; k < 32; ++k) { s[k] = v0[k]; s[32 + k] = v1[k]; }
             }
-            tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&bars[B_SFREE0 + (i & 1)]);
+            mbar_arrive(&bars[B_SFREE + 2 * q + (i & 1)]);
 
+            // visible columns of this row in this tile: [c_lo, c_hi)
+            int c_lo, c_hi;
+            if (pooled) { c_lo = 0; c_hi = min(BN, Pq - base); }
+            else { c_lo = max(0, lo - base); c_hi = min(BN, t - base + 1); }
+            if (!valid) c_hi = 0;
+            c_hi = max(c_hi, c_lo);  // an empty range masks every column
+            if (c_lo > 0 || c_hi < BN) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if ((unsigned)(c - c_lo) >= (unsigned)(c_hi - c_lo)) s[c] = kNegInf;
+            }
             float mx = kNegInf;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const int e = base + c;
-                const bool vis = valid && (pooled ? e < Pq : (e >= lo && e <= t));
-                s[c] = vis ? s[c] * sc : kNegInf;
-                mx = fmaxf(mx, s[c]);
-            }
-            const float m_new = fmaxf(m_ref, mx);
+            for (int c = 0; c < BN; c += 2) mx = fmaxf(mx, fmaxf(s[c], s[c + 1]));
+            // lazy rescale: only when the row max grows by more than 2^8 in probability
             float alpha = 1.f;
             bool rescale = false;
-            if (m_new > m_ref + 8.f) {  // also covers the first visible score (m_ref = -inf)
-                alpha = m_ref == kNegInf ? 0.f : ex2(m_ref - m_new);
+            if (mx * sc > m_ref * sc + 8.f || (m_ref == kNegInf && mx != kNegInf)) {
+                alpha = m_ref == kNegInf ? 0.f : ex2((m_ref - mx) * sc);
                 rescale = m_ref != kNegInf;
-                m_ref = m_new;
+                m_ref = mx;
             }
-            float psum = 0.f;
+            const float mneg = m_ref == kNegInf ? 0.f : -m_ref * sc;
+            float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                s[c] = m_ref == kNegInf ? 0.f : ex2(s[c] - m_ref);
-                psum += s[c];
+            for (int c = 0; c < BN; c += 2) {
+                s[c] = ex2(fmaf(s[c], sc, mneg));
+                s[c + 1] = ex2(fmaf(s[c + 1], sc, mneg));
+                ps0 += s[c];
+                ps1 += s[c + 1];
             }
-            l = l * alpha + psum;
+            l = l * alpha + (ps0 + ps1);
             if (i >= 1) {
-                ok = __all_sync(0xffffffffu, wait_or_fail(&bars[B_ODONE], (i - 1) & 1, fail, a.status));
+                ok = warp_wait(&bars[B_ODONE + q], (i - 1) & 1, fail, a.status);
                 if (!ok) break;
                 tc_fence_after();
                 // TMEM loads/stores are warp-collective: the warp rescales together,
@@ -300,24 +349,23 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
                 }
             }
 #pragma unroll
-            for (int q = 0; q < BN / 8; ++q) {
+            for (int c8 = 0; c8 < BN / 8; ++c8) {
                 uint4 u;
-                u.x = pack_f16x2(s[8 * q + 0], s[8 * q + 1]);
-                u.y = pack_f16x2(s[8 * q + 2], s[8 * q + 3]);
-                u.z = pack_f16x2(s[8 * q + 4], s[8 * q + 5]);
-                u.w = pack_f16x2(s[8 * q + 6], s[8 * q + 7]);
-                *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(r, 8 * q, REGION)) = u;
+                u.x = pack_f16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
+                u.y = pack_f16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
+                u.z = pack_f16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
+                u.w = pack_f16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
+                *reinterpret_cast<uint4*>(sP + sw128_off(r, 8 * c8, PTILE)) = u;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
-            mbar_arrive(&bars[B_PFULL]);
+            mbar_arrive(&bars[B_PFULL + q]);
         }
         // ---- epilogue: normalise the O row and store it ----
-        if (ok && ntile > 0)
-            ok = __all_sync(0xffffffffu, wait_or_fail(&bars[B_ODONE], (ntile - 1) & 1, fail, a.status));
+        if (ok && ntile > 0) ok = warp_wait(&bars[B_ODONE + q], (ntile - 1) & 1, fail, a.status);
         tc_fence_after();
         float den = l;
-        if (a.sink) den += m_ref == kNegInf ? 1.f : ex2(a.sink[h] * kLog2e - m_ref);
+        if (a.sink) den += m_ref == kNegInf ? 1.f : ex2(a.sink[h] * kLog2e - m_ref * sc);
         const float inv = den > 0.f ? 1.f / den : 0.f;
         const bool have_o = ok && ntile > 0;  // warp-uniform
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + (valid ? t : 0)) * a.Hq + h) * HD;
@@ -333,13 +381,13 @@ __global__ void __launch_bounds__(256, 1) prefill_tc_kernel(const __grid_constan
             }
             if (valid) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int c8 = 0; c8 < 4; ++c8) {
                     uint4 u;
-                    u.x = pack_bf16x2(v[8 * q + 0] * inv, v[8 * q + 1] * inv);
-                    u.y = pack_bf16x2(v[8 * q + 2] * inv, v[8 * q + 3] * inv);
-                    u.z = pack_bf16x2(v[8 * q + 4] * inv, v[8 * q + 5] * inv);
-                    u.w = pack_bf16x2(v[8 * q + 6] * inv, v[8 * q + 7] * inv);
-                    *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = u;
+                    u.x = pack_bf16x2(v[8 * c8 + 0] * inv, v[8 * c8 + 1] * inv);
+                    u.y = pack_bf16x2(v[8 * c8 + 2] * inv, v[8 * c8 + 3] * inv);
+                    u.z = pack_bf16x2(v[8 * c8 + 4] * inv, v[8 * c8 + 5] * inv);
+                    u.w = pack_bf16x2(v[8 * c8 + 6] * inv, v[8 * c8 + 7] * inv);
+                    *reinterpret_cast<uint4*>(orow + 32 * c + 8 * c8) = u;
                 }
             }
         }
@@ -446,7 +494,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     {   // q [B, T, Hq, D]
         const uint64_t dims[4] = {HD, (uint64_t)Hq, (uint64_t)T, (uint64_t)B};
         const uint64_t str[3] = {HD * e, (uint64_t)Hq * HD * e, (uint64_t)T * Hq * HD * e};
-        if (!make_map(&a.tq, p.q, dims, str, 1, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&a.tq, p.q, dims, str, 1, BM)) return cudaErrorInvalidValue;  // box 64 x 1 x 128
     }
     const int NB = T / p.m;
     const uint64_t ps = (uint64_t)std::max(p.pool_stride, 1);
@@ -470,7 +518,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     a.out = p.out;
     a.status = status;
     a.T = T; a.Hq = Hq; a.G = G; a.m = p.m; a.w = p.w; a.rho = p.rho;
-    a.n_qtiles = (T + BM - 1) / BM;
+    a.n_ctiles = (T + NQ * BM - 1) / (NQ * BM);
     a.scale = p.scale;
     static bool attr_set = false;
     if (!attr_set) {
@@ -479,8 +527,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
         if (err != cudaSuccess) return err;
         attr_set = true;
     }
-    dim3 grid(Hq, a.n_qtiles, B);
-    prefill_tc_kernel<<<grid, 256, SMEM_BYTES, s>>>(a);
+    dim3 grid(Hq, a.n_ctiles, B);
+    prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError();
 }
 

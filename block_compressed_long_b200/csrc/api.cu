@@ -328,9 +328,12 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
         a.state = cache_out ? cache_out->pool_state : nullptr;
         a.S = cfg->shared_kv ? 1 : 2; a.series = series;
-        if (use_tc && series == 0) {
-            // the tensor-core QK^T reads a dense fp16 copy of the pooled keys, [B, G, NB, D]
-            a.out_f16 = tc_scratch + prefill_tc_pooled_f16_offset(batch, T, cfg->n_kv_heads, cfg->rope_dims);
+        if (use_tc) {
+            // the tensor-core MMAs read dense fp16 copies of the pooled keys and values, [B, G, NB, D]
+            a.out_f16 = tc_scratch + (series == 0
+                                          ? prefill_tc_pooled_f16_offset(batch, T, cfg->n_kv_heads, cfg->rope_dims)
+                                          : prefill_tc_pooled_v_f16_offset(batch, T, cfg->n_kv_heads,
+                                                                           cfg->rope_dims, m));
             a.out_f16_blocks = NB;
         }
         LBCA_TRY(cuda_status(launch_pool(a, s)));

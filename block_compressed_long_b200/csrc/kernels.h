@@ -137,6 +137,7 @@ bool prefill_tc_supported(int dtype, int D, int rmsnorm, int shared);
 size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m);
 // where, inside that scratch, the pool pass leaves the fp16 copy of the pooled keys
 size_t prefill_tc_pooled_f16_offset(int B, int T, int G, int rho);
+size_t prefill_tc_pooled_v_f16_offset(int B, int T, int G, int rho, int m);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, void* scratch, int32_t* status, cudaStream_t s);
 bool prefill_simt_supported(int D);
 

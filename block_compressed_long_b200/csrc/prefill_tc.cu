@@ -17,16 +17,15 @@
 //              the TMEM O accumulator; completion is signalled by
 //              tcgen05.commit on mbarriers.  S(i+1) is issued before PV(i) so
 //              the tensor core works on the next tile while the softmax runs.
-//   warps 2-3  convert each V tile in place from bf16 to fp16 once it lands.
 //   warps 4-7  softmax: thread r owns query row r and TMEM lane r.  It rotates
 //              its Q row in shared memory once, then per tile loads its S row,
 //              applies the causal-block / window mask, keeps an online max
 //              (rescaling O in TMEM only when the max grows by more than 2^8),
 //              writes P in fp16 into the swizzled P tile, and finally
 //              normalises its O row (plus the sink) and stores it.
-// Raw keys arrive already rotated (a pre-pass writes the finalised keys once,
-// instead of every query tile rotating them again); Q is rotated in shared
-// memory from a per-position cos/sin table.  Rows past a tensor's valid extent
+// Raw keys arrive already rotated and, like the values, in fp16 (a pre-pass
+// writes them once instead of every query tile converting them again); Q is
+// rotated in shared memory from a per-position cos/sin table.  Rows past a tensor's valid extent
 // are zero-filled by TMA, so masked products never meet garbage.
 #include <cudaTypedefs.h>
 
@@ -64,8 +63,7 @@ constexpr int B_QFULL = 0;
 constexpr int B_QROT = 1;                      // [NQ]
 constexpr int B_KFULL = B_QROT + NQ;           // [NSTAGE]
 constexpr int B_VFULL = B_KFULL + NSTAGE;      // [NSTAGE]
-constexpr int B_VCONV = B_VFULL + NSTAGE;      // [NSTAGE]
-constexpr int B_KVEMPTY = B_VCONV + NSTAGE;    // [NSTAGE]
+constexpr int B_KVEMPTY = B_VFULL + NSTAGE;    // [NSTAGE]
 constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ][2]
 constexpr int B_SFREE = B_SFULL + 2 * NQ;      // [NQ][2]
 constexpr int B_PFULL = B_SFREE + 2 * NQ;      // [NQ]
@@ -121,7 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if ((i >= B_QROT && i < B_QROT + NQ) || (i >= B_SFREE && i < B_SFREE + 2 * NQ) ||
                 (i >= B_PFULL && i < B_PFULL + NQ))
                 cnt = 128;
-            if (i >= B_VCONV && i < B_VCONV + NSTAGE) cnt = 64;
             mbar_init(&bars[i], cnt);
         }
         *fail = 0;
@@ -200,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 }
                 if (ok && i >= 1) {  // O_q += P_q(j) V_j for the previous tile j
                     const int j = i - 1, sj = j % NSTAGE;
-                    ok = wait_or_fail(&bars[B_VCONV + sj], (j / NSTAGE) & 1, fail, a.status);
+                    ok = wait_or_fail(&bars[B_VFULL + sj], (j / NSTAGE) & 1, fail, a.status);
                     const uint32_t sv = smem_addr(smem + OFF_V + sj * KTILE);
                     for (int q = 0; ok && q < NQ; ++q) {
                         ok = wait_or_fail(&bars[B_PFULL + q], j & 1, fail, a.status);
@@ -220,28 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
         }
     } else if (warp == 2 || warp == 3) {
-        // ----------------------------------------- V tiles: bf16 -> fp16 in place
-        // (P V runs in fp16: P in [0, 256] keeps 11 mantissa bits; bf16 values
-        // widen exactly to fp16 in its normal range; element-wise, so the
-        // swizzled layout is untouched)
-        const int cthr = threadIdx.x - 64;
-        for (int i = 0; i < ntile; ++i) {
-            const int s = i % NSTAGE;
-            if (!warp_wait(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status)) break;
-            uint4* vt = reinterpret_cast<uint4*>(smem + OFF_V + s * KTILE);
-#pragma unroll 4
-            for (int qv = cthr; qv < (int)(KTILE / 16); qv += 64) {
-                uint4 u = vt[qv];
-                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    wv[e] = pack_f16x2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
-                vt[qv] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&bars[B_VCONV + s]);
-        }
-    } else {
+        // idle: the tiles arrive in their MMA operand types
+    } else if (warp >= 4) {
         // ------------------------------------------------------------- softmax
         const int q = (warp - 4) >> 2;           // query tile of this warpgroup
         const int r = threadIdx.x - 128 - 128 * q;
@@ -256,18 +233,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         uint8_t* sQ = smem + OFF_Q + q * QTILE;
         uint8_t* sP = smem + OFF_P + q * PTILE;
 
+        // this query row's cos/sin, fetched in one batch while Q lands
+        float2 cs_row[HD / 2];
+        {
+            const int base = HD / 2 - half;  // pairs below `base` are not rotated
+            const float2* tab = a.tab + (size_t)(valid ? t : 0) * half;
+#pragma unroll
+            for (int k = 0; k < HD / 2; ++k)
+                cs_row[k] = (valid && k >= base) ? __ldg(tab + (k - base)) : make_float2(1.f, 0.f);
+        }
         bool ok = warp_wait(&bars[B_QFULL], 0, fail, a.status);
         if (ok) {  // this query row, in place: bf16 -> f32, RoPE at t, -> fp16 (QK^T runs in fp16)
-            const float2* tab = a.tab + (size_t)(valid ? t : 0) * half;
+#pragma unroll
             for (int c8 = 0; c8 < HD / 8; ++c8) {
                 uint4* p = reinterpret_cast<uint4*>(sQ + sw128_off(r, 8 * c8, QREG));
                 uint4 u = *p;
                 uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int d = 8 * c8 + 2 * e;
                     float x = __uint_as_float(wv[e] << 16), y = __uint_as_float(wv[e] & 0xffff0000u);
-                    if (valid && d >= HD - a.rho) rotate_pair(x, y, tab[(d - (HD - a.rho)) >> 1]);
+                    rotate_pair(x, y, cs_row[4 * c8 + e]);
                     wv[e] = pack_f16x2(x, y);
                 }
                 *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -407,23 +392,26 @@ __global__ void rope_table_kernel(float2* tab, int T, int half, double step) {
         tab[i] = rope_cs(i / half, (int)(i % half), step);
 }
 
-// Finalised raw keys: RoPE at s applied once, fp16 out (the QK^T operand type),
-// same [B, T, G, D] layout.
-__global__ void finalise_keys_kernel(const __nv_bfloat16* __restrict__ k, __half* __restrict__ out,
-                                     const float2* __restrict__ tab, int64_t n_vec, int G, int T, int rho) {
+// Finalised raw keys (RoPE at s applied once) and raw values, both widened to
+// fp16, the operand type of the tensor-core MMAs; same [B, T, G, D] layout.
+__global__ void finalise_kv_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                                   __half* __restrict__ ko, __half* __restrict__ vo, const float2* __restrict__ tab,
+                                   int64_t n_vec, int G, int T, int rho) {
     const int half = rho / 2;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec; i += (int64_t)gridDim.x * blockDim.x) {
         const int d0 = (int)(i % (HD / 8)) * 8;
         const int64_t row = i / (HD / 8);            // (b, s, g)
         const int s = (int)((row / G) % T);
-        float v[8];
-        ld16(k + i * 8, v);
+        float x[8], y[8];
+        ld16(k + i * 8, x);
+        ld16(v + i * 8, y);
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
             const int d = d0 + e;
-            if (d >= HD - rho) rotate_pair(v[e], v[e + 1], tab[(size_t)s * half + ((d - (HD - rho)) >> 1)]);
+            if (d >= HD - rho) rotate_pair(x[e], x[e + 1], tab[(size_t)s * half + ((d - (HD - rho)) >> 1)]);
         }
-        st16_f16(out + i * 8, v);
+        st16_f16(ko + i * 8, x);
+        st16_f16(vo + i * 8, y);
     }
 }
 
@@ -459,25 +447,29 @@ bool prefill_tc_supported(int dtype, int D, int rmsnorm, int shared) {
     return dtype == LBCA_BF16 && D == HD && !rmsnorm && !shared;
 }
 
+// scratch: [fp16 raw keys][fp16 raw values][cos/sin table][fp16 pooled keys][fp16 pooled values]
+static size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 size_t prefill_tc_pooled_f16_offset(int B, int T, int G, int rho) {
-    const size_t keys = (size_t)B * T * G * HD * 2;
-    const size_t tab = (size_t)T * std::max(rho / 2, 1) * sizeof(float2);
-    return (keys + 255) / 256 * 256 + (tab + 255) / 256 * 256;
+    const size_t raw = a256((size_t)B * T * G * HD * 2);
+    const size_t tab = a256((size_t)T * std::max(rho / 2, 1) * sizeof(float2));
+    return 2 * raw + tab;
 }
-
-// fp16 finalised raw keys, the cos/sin table, and an fp16 copy of the pooled keys
+size_t prefill_tc_pooled_v_f16_offset(int B, int T, int G, int rho, int m) {
+    return prefill_tc_pooled_f16_offset(B, T, G, rho) + a256((size_t)B * G * (T / m) * HD * 2);
+}
 size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m) {
-    const size_t pooled = (size_t)B * G * (T / m) * HD * 2;
-    return prefill_tc_pooled_f16_offset(B, T, G, rho) + (pooled + 255) / 256 * 256;
+    return prefill_tc_pooled_v_f16_offset(B, T, G, rho, m) + a256((size_t)B * G * (T / m) * HD * 2);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* status, cudaStream_t s) {
     if (p.B == 0 || p.T == 0) return cudaSuccess;
     const int G = p.G, T = p.T, B = p.B, Hq = p.Hq;
+    const size_t raw_bytes = a256((size_t)B * T * G * HD * 2);
     __half* keys = static_cast<__half*>(scratch);
-    const size_t keys_bytes = ((size_t)B * T * G * HD * 2 + 255) / 256 * 256;
-    float2* tab = reinterpret_cast<float2*>(static_cast<char*>(scratch) + keys_bytes);
+    __half* vals = reinterpret_cast<__half*>(static_cast<char*>(scratch) + raw_bytes);
+    float2* tab = reinterpret_cast<float2*>(static_cast<char*>(scratch) + 2 * raw_bytes);
     const void* pooled_k16 = static_cast<char*>(scratch) + prefill_tc_pooled_f16_offset(B, T, G, p.rho);
+    const void* pooled_v16 = static_cast<char*>(scratch) + prefill_tc_pooled_v_f16_offset(B, T, G, p.rho, p.m);
     const int half = p.rho / 2;
     if (half > 0) {
         const int64_t n = (int64_t)T * half;
@@ -485,8 +477,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     }
     {
         const int64_t nv = (int64_t)B * T * G * (HD / 8);
-        finalise_keys_kernel<<<(int)std::min<int64_t>((nv + 255) / 256, 148 * 32), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(p.k), keys, tab, nv, G, T, p.rho);
+        finalise_kv_kernel<<<(int)std::min<int64_t>((nv + 255) / 256, 148 * 32), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v), keys, vals, tab, nv, G, T,
+            p.rho);
     }
     TcArgs a;
     memset(&a, 0, sizeof(a));
@@ -501,17 +494,18 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     {   // pooled [B, G, stride, D], valid rows NB
         const uint64_t dims[4] = {HD, (uint64_t)std::max(NB, 1), (uint64_t)G, (uint64_t)B};
         const uint64_t str[3] = {HD * e, ps * HD * e, (uint64_t)G * ps * HD * e};
-        if (!make_map(&a.tpv, p.pooled_v, dims, str, BN, 1)) return cudaErrorInvalidValue;
-        // fp16 pooled keys in the scratch, [B, G, NB, D]
+        // fp16 pooled keys and values in the scratch, [B, G, NB, D]
         const uint64_t nb = (uint64_t)std::max(NB, 1);
         const uint64_t str16[3] = {HD * e, nb * HD * e, (uint64_t)G * nb * HD * e};
         if (!make_map(&a.tpk, pooled_k16, dims, str16, BN, 1, true)) return cudaErrorInvalidValue;
+        if (!make_map(&a.tpv, pooled_v16, dims, str16, BN, 1, true)) return cudaErrorInvalidValue;
+        (void)str;
     }
     {   // raw [B, T, G, D]
         const uint64_t dims[4] = {HD, (uint64_t)G, (uint64_t)T, (uint64_t)B};
         const uint64_t str[3] = {HD * e, (uint64_t)G * HD * e, (uint64_t)T * G * HD * e};
         if (!make_map(&a.trk, keys, dims, str, 1, BN, true)) return cudaErrorInvalidValue;
-        if (!make_map(&a.trv, p.v, dims, str, 1, BN)) return cudaErrorInvalidValue;
+        if (!make_map(&a.trv, vals, dims, str, 1, BN, true)) return cudaErrorInvalidValue;
     }
     a.tab = tab;
     a.sink = p.sink;

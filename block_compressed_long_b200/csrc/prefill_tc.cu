@@ -7,21 +7,23 @@
 // "Deviations from paper").  This kernel serves the GQA form with bf16 I/O,
 // head_dim 128 and no RMSNorm; other shapes use the CUDA-core kernel.
 //
-// B200 mapping (one CTA = 128 queries of one head, 256 threads):
-//   warp 0     TMA producer: the Q tile once, then K and V tiles of 128
-//              entries (pooled tiles first, then the raw band) into a
-//              two-stage ring, 128-byte swizzled, no multicast.
+// B200 mapping (one CTA = 2 x 128 queries of one head, 384 threads):
+//   warp 0     TMA producer: the two Q tiles once, then fp16 K and V tiles
+//              of 128 entries (pooled tiles first, then the raw band) into
+//              a two-stage ring, 128-byte swizzled, no multicast.
 //   warp 1     TMEM owner and MMA issuer: S = Q K^T (tcgen05.mma M=128 N=128,
-//              K-major operands) into one of two TMEM S buffers, and
-//              O += P V (fp16 P from shared memory, fp16 V as an MN-major operand) into
-//              the TMEM O accumulator; completion is signalled by
-//              tcgen05.commit on mbarriers.  S(i+1) is issued before PV(i) so
-//              the tensor core works on the next tile while the softmax runs.
-//   warps 4-7  softmax: thread r owns query row r and TMEM lane r.  It rotates
+//              fp16 K-major operands from shared memory) into the query tile's
+//              TMEM S columns, and O += P V with P read from TMEM (the
+//              softmax overwrites S with P) and fp16 V as an MN-major operand;
+//              completion is signalled by tcgen05.commit on mbarriers.  Two
+//              query tiles per CTA interleave (PV0, S0', PV1, S1') so the
+//              tensor core works on one tile while the other's softmax runs.
+//   warps 4-7, 8-11  softmax of query tiles 0 and 1: thread r owns query row r
+//              and TMEM lane r.  It rotates
 //              its Q row in shared memory once, then per tile loads its S row,
 //              applies the causal-block / window mask, keeps an online max
 //              (rescaling O in TMEM only when the max grows by more than 2^8),
-//              writes P in fp16 into the swizzled P tile, and finally
+//              writes P in fp16 into TMEM over its S row, and finally
 //              normalises its O row (plus the sink) and stores it.
 // Raw keys arrive already rotated and, like the values, in fp16 (a pre-pass
 // writes them once instead of every query tile converting them again); Q is
@@ -40,22 +42,20 @@ namespace {
 
 constexpr int BM = 128;     // query rows per softmax warpgroup (one M=128 MMA)
 constexpr int NQ = 2;       // query tiles per CTA
-constexpr int BN = 64;      // entries per K/V tile
+constexpr int BN = 128;     // entries per K/V tile
 constexpr int HD = 128;     // head dim
-constexpr int NSTAGE = 3;   // K/V ring depth
+constexpr int NSTAGE = 2;   // K/V ring depth
 constexpr uint32_t QREG = BM * 64 * 2;   // [128 rows][64 cols] 16-bit: one 128-byte swizzle span per row
 constexpr uint32_t QTILE = 2 * QREG;     // [128][128]
-constexpr uint32_t KREG = BN * 64 * 2;   // [64 rows][64 cols]
-constexpr uint32_t KTILE = 2 * KREG;     // [64][128]
-constexpr uint32_t PTILE = BM * BN * 2;  // [128 rows][64 entries] fp16
+constexpr uint32_t KREG = BN * 64 * 2;   // [128 rows][64 cols]
+constexpr uint32_t KTILE = 2 * KREG;     // [128][128]
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + NQ * QTILE;
 constexpr uint32_t OFF_V = OFF_K + NSTAGE * KTILE;
-constexpr uint32_t OFF_P = OFF_V + NSTAGE * KTILE;
-constexpr uint32_t OFF_BAR = OFF_P + NQ * PTILE;
+constexpr uint32_t OFF_BAR = OFF_V + NSTAGE * KTILE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t TMEM_COLS = 512;  // S[q][2] (64 columns each) at 0..255, O[q] (128 columns) at 256..511
-constexpr int kThreads = 384;        // warps 0 producer, 1 MMA, 2-3 V converters, 4-7 / 8-11 softmax
+constexpr uint32_t TMEM_COLS = 512;  // per query tile q: S/P at 256q (128 columns), O at 256q + 128
+constexpr int kThreads = 384;        // warps 0 producer, 1 MMA, 2-3 idle, 4-7 / 8-11 softmax
 constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;
 
 // barrier slots
@@ -64,18 +64,17 @@ constexpr int B_QROT = 1;                      // [NQ]
 constexpr int B_KFULL = B_QROT + NQ;           // [NSTAGE]
 constexpr int B_VFULL = B_KFULL + NSTAGE;      // [NSTAGE]
 constexpr int B_KVEMPTY = B_VFULL + NSTAGE;    // [NSTAGE]
-constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ][2]
-constexpr int B_SFREE = B_SFULL + 2 * NQ;      // [NQ][2]
-constexpr int B_PFULL = B_SFREE + 2 * NQ;      // [NQ]
+constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ]
+constexpr int B_PFULL = B_SFULL + NQ;          // [NQ]
 constexpr int B_ODONE = B_PFULL + NQ;          // [NQ]
 constexpr int B_COUNT = B_ODONE + NQ;
 
 struct TcArgs {
     CUtensorMap tq;   // q [B, T, Hq, D] bf16          dims (D, Hq, T, B)
     CUtensorMap tpk;  // pooled keys fp16 [B, G, NB, D] dims (D, NB, G, B)
-    CUtensorMap tpv;  // pooled values bf16 [B, G, *, D]
+    CUtensorMap tpv;  // pooled values fp16
     CUtensorMap trk;  // finalised raw keys fp16 [B, T, G, D] dims (D, G, T, B)
-    CUtensorMap trv;  // raw values bf16
+    CUtensorMap trv;  // raw values fp16
     const float2* tab;  // [T][rho/2] cos/sin
     const float* sink;
     void* out;          // [B, T, Hq, D] bf16
@@ -115,11 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            uint32_t cnt = 1;
-            if ((i >= B_QROT && i < B_QROT + NQ) || (i >= B_SFREE && i < B_SFREE + 2 * NQ) ||
-                (i >= B_PFULL && i < B_PFULL + NQ))
-                cnt = 128;
-            mbar_init(&bars[i], cnt);
+            const bool softmax_arrivals = (i >= B_QROT && i < B_QROT + NQ) || (i >= B_PFULL && i < B_PFULL + NQ);
+            mbar_init(&bars[i], softmax_arrivals ? 128u : 1u);
         }
         *fail = 0;
         fence_barrier_init();
@@ -148,16 +144,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 mbar_arrive_expect_tx(&bars[B_VFULL + s], KTILE);
                 if (i < npt) {
                     const int j0 = i * BN;
-                    for (int rg = 0; rg < 2; ++rg) {
-                        tma_load_4d(kd + rg * KREG, &a.tpk, 64 * rg, j0, g, b, &bars[B_KFULL + s]);
-                        tma_load_4d(vd + rg * KREG, &a.tpv, 64 * rg, j0, g, b, &bars[B_VFULL + s]);
-                    }
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.tpk, 64 * rg, j0, g, b, &bars[B_KFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.tpv, 64 * rg, j0, g, b, &bars[B_VFULL + s]);
                 } else {
                     const int s0 = s_lo + (i - npt) * BN;
-                    for (int rg = 0; rg < 2; ++rg) {
-                        tma_load_4d(kd + rg * KREG, &a.trk, 64 * rg, g, s0, b, &bars[B_KFULL + s]);
-                        tma_load_4d(vd + rg * KREG, &a.trv, 64 * rg, g, s0, b, &bars[B_VFULL + s]);
-                    }
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.trk, 64 * rg, g, s0, b, &bars[B_KFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.trv, 64 * rg, g, s0, b, &bars[B_VFULL + s]);
                 }
                 issued = i + 1;
             }
@@ -170,54 +162,55 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
+        // order: S0(0) S1(0) | PV0(i) S0(i+1) PV1(i) S1(i+1) | ...  P_q(i) lives in
+        // S_q's TMEM columns, so S_q(i+1) waits until PV_q(i) has read it.
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
+            auto issue_s = [&](int q, int i) {
+                const int s = i % NSTAGE;
+                const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
+                const uint32_t sk = smem_addr(smem + OFF_K + s * KTILE);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    tc_mma_bf16(tbase + 256 * q, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
+                                smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+                tc_commit(&bars[B_SFULL + q]);
+            };
+            auto issue_pv = [&](int q, int i) {
+                const int s = i % NSTAGE;
+                const uint32_t sv = smem_addr(smem + OFF_V + s * KTILE);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)  // A = P_q(i): 8 fp16x2 columns per 16 entries
+                    tc_mma_ts(tbase + 256 * q + 128, tbase + 256 * q + kk * 8,
+                              smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&bars[B_ODONE + q]);
+            };
             bool ok = true;
             for (int q = 0; ok && q < NQ; ++q) ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
-            for (int i = 0; ok && i <= ntile; ++i) {
-                if (i < ntile) {  // S_q(i) = Q_q K_i^T for both query tiles
-                    const int s = i % NSTAGE;
-                    ok = wait_or_fail(&bars[B_KFULL + s], (i / NSTAGE) & 1, fail, a.status);
-                    const uint32_t sk = smem_addr(smem + OFF_K + s * KTILE);
-                    for (int q = 0; ok && q < NQ; ++q) {
-                        if (i >= 2) ok = wait_or_fail(&bars[B_SFREE + 2 * q + (i & 1)], ((i >> 1) - 1) & 1, fail,
-                                                      a.status);
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
-                        const uint32_t dS = tbase + (uint32_t)(2 * q + (i & 1)) * BN;
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            tc_mma_bf16(dS, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
-                                        smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
-                        }
-                        tc_commit(&bars[B_SFULL + 2 * q + (i & 1)]);
+            if (ok && ntile > 0) {
+                ok = wait_or_fail(&bars[B_KFULL], 0, fail, a.status);
+                if (ok) { issue_s(0, 0); issue_s(1, 0); }
+            }
+            for (int i = 0; ok && i < ntile; ++i) {
+                const int s = i % NSTAGE, n = i + 1, sn = n % NSTAGE;
+                ok = wait_or_fail(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status);
+                const bool more = n < ntile;
+                if (ok && more) ok = wait_or_fail(&bars[B_KFULL + sn], (n / NSTAGE) & 1, fail, a.status);
+                for (int q = 0; ok && q < NQ; ++q) {
+                    ok = wait_or_fail(&bars[B_PFULL + q], i & 1, fail, a.status);
+                    if (!ok) break;
+                    issue_pv(q, i);
+                    if (q == NQ - 1) tc_commit(&bars[B_KVEMPTY + s]);
+                    if (more) {
+                        ok = wait_or_fail(&bars[B_ODONE + q], i & 1, fail, a.status);
+                        if (ok) issue_s(q, n);
                     }
-                }
-                if (ok && i >= 1) {  // O_q += P_q(j) V_j for the previous tile j
-                    const int j = i - 1, sj = j % NSTAGE;
-                    ok = wait_or_fail(&bars[B_VFULL + sj], (j / NSTAGE) & 1, fail, a.status);
-                    const uint32_t sv = smem_addr(smem + OFF_V + sj * KTILE);
-                    for (int q = 0; ok && q < NQ; ++q) {
-                        ok = wait_or_fail(&bars[B_PFULL + q], j & 1, fail, a.status);
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint32_t sp = smem_addr(smem + OFF_P + q * PTILE);
-                        const uint32_t dO = tbase + 256 + (uint32_t)q * HD;
-#pragma unroll
-                        for (int kk = 0; kk < BN / 16; ++kk) {
-                            tc_mma_bf16(dO, smem_desc_sw128(sp + kk * 32, 16, 1024),
-                                        smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (j > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        tc_commit(&bars[B_ODONE + q]);
-                    }
-                    if (ok) tc_commit(&bars[B_KVEMPTY + sj]);
                 }
             }
         }
-    } else if (warp == 2 || warp == 3) {
-        // idle: the tiles arrive in their MMA operand types
     } else if (warp >= 4) {
         // ------------------------------------------------------------- softmax
         const int q = (warp - 4) >> 2;           // query tile of this warpgroup
@@ -228,10 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int lo = Pq * a.m;
         const uint32_t lane_f = (uint32_t)(32 * (warp & 3)) << 16;
         const int half = a.rho / 2;
-        const uint32_t tS0 = tbase + (uint32_t)(2 * q) * BN;
-        const uint32_t tO = tbase + 256 + (uint32_t)q * HD;
+        const uint32_t tS = tbase + 256 * q + lane_f;
+        const uint32_t tO = tS + 128;
         uint8_t* sQ = smem + OFF_Q + q * QTILE;
-        uint8_t* sP = smem + OFF_P + q * PTILE;
 
         // this query row's cos/sin, fetched in one batch while Q lands
         float2 cs_row[HD / 2];
@@ -266,20 +258,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         for (int i = 0; ok && i < ntile; ++i) {
             const bool pooled = i < npt;
             const int base = pooled ? i * BN : s_lo + (i - npt) * BN;
-            ok = warp_wait(&bars[B_SFULL + 2 * q + (i & 1)], (i >> 1) & 1, fail, a.status);
+            ok = warp_wait(&bars[B_SFULL + q], i & 1, fail, a.status);
             if (!ok) break;
             tc_fence_after();
             float s[BN];
-            {
-                float v0[32], v1[32];
-                tmem_ld32(tS0 + (uint32_t)(i & 1) * BN + lane_f, v0);
-                tmem_ld32(tS0 + (uint32_t)(i & 1) * BN + lane_f + 32, v1);
-                tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 32; ++k) { s[k] = v0[k]; s[32 + k] = v1[k]; }
+            for (int c = 0; c < BN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tS + 32 * c, v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) s[32 * c + k] = v[k];
             }
-            tc_fence_before();
-            mbar_arrive(&bars[B_SFREE + 2 * q + (i & 1)]);
+            tmem_wait_ld();
 
             // visible columns of this row in this tile: [c_lo, c_hi)
             int c_lo, c_hi;
@@ -292,57 +282,54 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 for (int c = 0; c < BN; ++c)
                     if ((unsigned)(c - c_lo) >= (unsigned)(c_hi - c_lo)) s[c] = kNegInf;
             }
-            float mx = kNegInf;
+            float mx0 = kNegInf, mx1 = kNegInf;
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) mx = fmaxf(mx, fmaxf(s[c], s[c + 1]));
+            for (int c = 0; c < BN; c += 2) { mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); }
+            const float mx = fmaxf(mx0, mx1);
             // lazy rescale: only when the row max grows by more than 2^8 in probability
             float alpha = 1.f;
             bool rescale = false;
-            if (mx * sc > m_ref * sc + 8.f || (m_ref == kNegInf && mx != kNegInf)) {
+            if (mx * sc > m_ref * sc + 8.f) {  // also the first visible score (m_ref = -inf)
                 alpha = m_ref == kNegInf ? 0.f : ex2((m_ref - mx) * sc);
                 rescale = m_ref != kNegInf;
                 m_ref = mx;
             }
             const float mneg = m_ref == kNegInf ? 0.f : -m_ref * sc;
             float ps0 = 0.f, ps1 = 0.f;
+            uint32_t pk[BN / 2];
 #pragma unroll
             for (int c = 0; c < BN; c += 2) {
-                s[c] = ex2(fmaf(s[c], sc, mneg));
-                s[c + 1] = ex2(fmaf(s[c + 1], sc, mneg));
-                ps0 += s[c];
-                ps1 += s[c + 1];
+                const float p0 = ex2(fmaf(s[c], sc, mneg));
+                const float p1 = ex2(fmaf(s[c + 1], sc, mneg));
+                ps0 += p0;
+                ps1 += p1;
+                pk[c / 2] = pack_f16x2(p0, p1);
             }
             l = l * alpha + (ps0 + ps1);
-            if (i >= 1) {
-                ok = warp_wait(&bars[B_ODONE + q], (i - 1) & 1, fail, a.status);
-                if (!ok) break;
-                tc_fence_after();
-                // TMEM loads/stores are warp-collective: the warp rescales together,
-                // rows whose max did not move scale by one
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float f = rescale ? alpha : 1.f;
+            // PV_q(i-1) finished before S_q(i) was issued: O is quiet, rescale it if needed
+            if (__any_sync(0xffffffffu, rescale)) {
+                const float f = rescale ? alpha : 1.f;
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(tO + lane_f + 32 * c, v);
-                        tmem_wait_ld();
+                for (int c = 0; c < HD / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tO + 32 * c, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] *= f;
-                        tmem_st32(tO + lane_f + 32 * c, v);
-                    }
-                    tmem_wait_st();
+                    for (int k = 0; k < 32; ++k) v[k] *= f;
+                    tmem_st32(tO + 32 * c, v);
                 }
             }
+            // P_q(i) (fp16 pairs) into the first 64 columns of S_q's TMEM
+            {
+                float v[32];
 #pragma unroll
-            for (int c8 = 0; c8 < BN / 8; ++c8) {
-                uint4 u;
-                u.x = pack_f16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
-                u.y = pack_f16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
-                u.z = pack_f16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
-                u.w = pack_f16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
-                *reinterpret_cast<uint4*>(sP + sw128_off(r, 8 * c8, PTILE)) = u;
+                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(pk[k]);
+                tmem_st32(tS, v);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(pk[32 + k]);
+                tmem_st32(tS + 32, v);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + q]);
         }
@@ -358,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         for (int c = 0; c < HD / 32; ++c) {
             float v[32];
             if (have_o) {  // every lane loads (warp-collective); rows past T do not store
-                tmem_ld32(tO + lane_f + 32 * c, v);
+                tmem_ld32(tO + 32 * c, v);
                 tmem_wait_ld();
             } else {
 #pragma unroll

@@ -24,7 +24,8 @@
 //              applies the causal-block / window mask, keeps an online max
 //              (rescaling O in TMEM only when the max grows by more than 2^8),
 //              writes P in fp16 into TMEM over its S row, and finally
-//              normalises its O row (plus the sink) and stores it.
+//              normalises its O row (plus the sink) into shared memory, from
+//              where one thread TMA-stores the tile.
 // Raw keys arrive already rotated and, like the values, in fp16 (a pre-pass
 // writes them once instead of every query tile converting them again); Q is
 // rotated in shared memory from a per-position cos/sin table.  Rows past a tensor's valid extent
@@ -75,7 +76,8 @@ struct TcArgs {
     CUtensorMap tpv;  // pooled values fp16
     CUtensorMap trk;  // finalised raw keys fp16 [B, T, G, D] dims (D, G, T, B)
     CUtensorMap trv;  // raw values fp16
-    const float2* tab;  // [T][rho/2] cos/sin
+    CUtensorMap to;   // out [B, T, Hq, D] bf16       dims (D, Hq, T, B)
+    const float2* tab;  // [rho/2][T] cos/sin
     const float* sink;
     void* out;          // [B, T, Hq, D] bf16
     int32_t* status;
@@ -198,14 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 const int s = i % NSTAGE, n = i + 1, sn = n % NSTAGE;
                 ok = wait_or_fail(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status);
                 const bool more = n < ntile;
-                if (ok && more) ok = wait_or_fail(&bars[B_KFULL + sn], (n / NSTAGE) & 1, fail, a.status);
                 for (int q = 0; ok && q < NQ; ++q) {
                     ok = wait_or_fail(&bars[B_PFULL + q], i & 1, fail, a.status);
                     if (!ok) break;
                     issue_pv(q, i);
                     if (q == NQ - 1) tc_commit(&bars[B_KVEMPTY + s]);
-                    if (more) {
-                        ok = wait_or_fail(&bars[B_ODONE + q], i & 1, fail, a.status);
+                    if (more) {  // S_q(i+1) needs the next K tile and P_q(i) consumed
+                        if (q == 0) ok = wait_or_fail(&bars[B_KFULL + sn], (n / NSTAGE) & 1, fail, a.status);
+                        if (ok) ok = wait_or_fail(&bars[B_ODONE + q], i & 1, fail, a.status);
                         if (ok) issue_s(q, n);
                     }
                 }
@@ -229,10 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         float2 cs_row[HD / 2];
         {
             const int base = HD / 2 - half;  // pairs below `base` are not rotated
-            const float2* tab = a.tab + (size_t)(valid ? t : 0) * half;
+            const float2* tab = a.tab + (valid ? t : 0);  // pair-major: a warp's 32 rows are contiguous
 #pragma unroll
             for (int k = 0; k < HD / 2; ++k)
-                cs_row[k] = (valid && k >= base) ? __ldg(tab + (k - base)) : make_float2(1.f, 0.f);
+                cs_row[k] = (valid && k >= base) ? __ldg(tab + (size_t)(k - base) * a.T) : make_float2(1.f, 0.f);
         }
         bool ok = warp_wait(&bars[B_QFULL], 0, fail, a.status);
         if (ok) {  // this query row, in place: bf16 -> f32, RoPE at t, -> fp16 (QK^T runs in fp16)
@@ -333,35 +335,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + q]);
         }
-        // ---- epilogue: normalise the O row and store it ----
+        // ---- epilogue: normalise the O row into this query tile's shared memory
+        // (free: the last S MMA that read Q is complete), then TMA-store the tile
         if (ok && ntile > 0) ok = warp_wait(&bars[B_ODONE + q], (ntile - 1) & 1, fail, a.status);
         tc_fence_after();
         float den = l;
         if (a.sink) den += m_ref == kNegInf ? 1.f : ex2(a.sink[h] * kLog2e - m_ref * sc);
         const float inv = den > 0.f ? 1.f / den : 0.f;
         const bool have_o = ok && ntile > 0;  // warp-uniform
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + (valid ? t : 0)) * a.Hq + h) * HD;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
             float v[32];
-            if (have_o) {  // every lane loads (warp-collective); rows past T do not store
+            if (have_o) {  // every lane loads (warp-collective)
                 tmem_ld32(tO + 32 * c, v);
                 tmem_wait_ld();
             } else {
 #pragma unroll
                 for (int k = 0; k < 32; ++k) v[k] = 0.f;
             }
-            if (valid) {
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    uint4 u;
-                    u.x = pack_bf16x2(v[8 * c8 + 0] * inv, v[8 * c8 + 1] * inv);
-                    u.y = pack_bf16x2(v[8 * c8 + 2] * inv, v[8 * c8 + 3] * inv);
-                    u.z = pack_bf16x2(v[8 * c8 + 4] * inv, v[8 * c8 + 5] * inv);
-                    u.w = pack_bf16x2(v[8 * c8 + 6] * inv, v[8 * c8 + 7] * inv);
-                    *reinterpret_cast<uint4*>(orow + 32 * c + 8 * c8) = u;
-                }
+            for (int c8 = 0; c8 < 4; ++c8) {
+                uint4 u;
+                u.x = pack_bf16x2(v[8 * c8 + 0] * inv, v[8 * c8 + 1] * inv);
+                u.y = pack_bf16x2(v[8 * c8 + 2] * inv, v[8 * c8 + 3] * inv);
+                u.z = pack_bf16x2(v[8 * c8 + 4] * inv, v[8 * c8 + 5] * inv);
+                u.w = pack_bf16x2(v[8 * c8 + 6] * inv, v[8 * c8 + 7] * inv);
+                *reinterpret_cast<uint4*>(sQ + sw128_off(r, 32 * c + 8 * c8, QREG)) = u;
             }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_barrier(1 + q, 128);
+        if (r == 0) {
+            tma_store_4d(&a.to, sQ, 0, h, t0 + q * BM, b);
+            tma_store_4d(&a.to, sQ + QREG, 64, h, t0 + q * BM, b);
+            tma_store_commit_and_wait_read();
         }
     }
     tc_fence_before();
@@ -372,11 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
 }
 
-// cos/sin of every (position, pair) the queries and raw keys need.
+// cos/sin of every (pair, position) the queries and raw keys need, pair-major
+// ([half][T]) so that consecutive positions of one pair are contiguous.
 __global__ void rope_table_kernel(float2* tab, int T, int half, double step) {
     const int64_t n = (int64_t)T * half;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        tab[i] = rope_cs(i / half, (int)(i % half), step);
+        tab[i] = rope_cs(i % T, (int)(i / T), step);
 }
 
 // Finalised raw keys (RoPE at s applied once) and raw values, both widened to
@@ -395,7 +403,7 @@ __global__ void finalise_kv_kernel(const __nv_bfloat16* __restrict__ k, const __
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
             const int d = d0 + e;
-            if (d >= HD - rho) rotate_pair(x[e], x[e + 1], tab[(size_t)s * half + ((d - (HD - rho)) >> 1)]);
+            if (d >= HD - rho) rotate_pair(x[e], x[e + 1], tab[(size_t)((d - (HD - rho)) >> 1) * T + s]);
         }
         st16_f16(ko + i * 8, x);
         st16_f16(vo + i * 8, y);
@@ -475,6 +483,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
         const uint64_t dims[4] = {HD, (uint64_t)Hq, (uint64_t)T, (uint64_t)B};
         const uint64_t str[3] = {HD * e, (uint64_t)Hq * HD * e, (uint64_t)T * Hq * HD * e};
         if (!make_map(&a.tq, p.q, dims, str, 1, BM)) return cudaErrorInvalidValue;  // box 64 x 1 x 128
+        if (!make_map(&a.to, p.out, dims, str, 1, BM)) return cudaErrorInvalidValue;
     }
     const int NB = T / p.m;
     const uint64_t ps = (uint64_t)std::max(p.pool_stride, 1);

@@ -298,14 +298,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
             const float mneg = m_ref == kNegInf ? 0.f : -m_ref * sc;
             float ps0 = 0.f, ps1 = 0.f;
-            uint32_t pk[BN / 2];
+            // P as fp16 pairs, written over S in two halves of 32 columns (64 entries)
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                const float p0 = ex2(fmaf(s[c], sc, mneg));
-                const float p1 = ex2(fmaf(s[c + 1], sc, mneg));
-                ps0 += p0;
-                ps1 += p1;
-                pk[c / 2] = pack_f16x2(p0, p1);
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int c = 64 * hh + 2 * k;
+                    const float p0 = ex2(fmaf(s[c], sc, mneg));
+                    const float p1 = ex2(fmaf(s[c + 1], sc, mneg));
+                    ps0 += p0;
+                    ps1 += p1;
+                    v[k] = __uint_as_float(pack_f16x2(p0, p1));
+                }
+                tmem_st32(tS + 32 * hh, v);  // columns [32 hh, 32 hh + 32) of S_q: already read
             }
             l = l * alpha + (ps0 + ps1);
             // PV_q(i-1) finished before S_q(i) was issued: O is quiet, rescale it if needed
@@ -320,16 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     for (int k = 0; k < 32; ++k) v[k] *= f;
                     tmem_st32(tO + 32 * c, v);
                 }
-            }
-            // P_q(i) (fp16 pairs) into the first 64 columns of S_q's TMEM
-            {
-                float v[32];
-#pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(pk[k]);
-                tmem_st32(tS, v);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(pk[32 + k]);
-                tmem_st32(tS + 32, v);
             }
             tmem_wait_st();
             tc_fence_before();

@@ -317,6 +317,102 @@ def run_ours(args, w, rank, world):
     return line, bench
 
 
+def peak_tflops():
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 burst; fp16 has the same dense rate)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_flops(w):
+    """Algorithmic FLOPs: 4 D Hq per visible (query, entry) pair."""
+    T, m, n = w.seq_len, w.block_m, w.n_win
+    pairs = 0
+    for L in range(1, T + 1):
+        P = max(0, (L - n) // m)
+        pairs += P + (L - P * m)
+    return 4.0 * w.head_dim * w.n_q_heads * pairs * w.batch
+
+
+def extra_prefill(reps=10):
+    """lbca_prefill of the 16K-token GQA layer (pool pass, RoPE table, finalised
+    keys, tensor-core attention), inputs resident (> L2), CUDA events."""
+    import torch
+
+    from block_compressed_long_b200 import lbca as L
+    from block_compressed_long_b200 import synth
+    w = synth.WORKLOADS["gqa_prefill_16k"]
+    inp = synth.make(w)
+    cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta, dtype=w.dtype)
+    d = lambda t: None if t is None else t.cuda()  # noqa: E731
+    q, k, v, zk, zv, bpk, bpv = (d(t) for t in (inp.q, inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v))
+    out = torch.empty_like(q)
+    ws = torch.zeros(L.lbca_prefill_workspace_bytes(cfg, w.batch, w.seq_len, False), dtype=torch.uint8,
+                     device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, out, None, ws, d_status=st)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, out, None, ws, d_status=st)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.item()):
+        raise RuntimeError(f"prefill device status {L.lbca_status_string(int(st.item()))}")
+    ms = e0.elapsed_time(e1) / reps
+    fl = prefill_flops(w)
+    tf = fl / (ms * 1e-3) / 1e12
+    pk, src = peak_tflops()
+    return {"workload": w.name, "metric": "prefill TFLOP/s", "value": tf, "unit": "TFLOP/s", "ms_per_call": ms,
+            "dtype": "bf16 I/O, fp16 tensor-core operands, f32 accumulate",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+                         "peak_source": src, "kernel": "prefill_tc_kernel (whole lbca_prefill call timed)",
+                         "flops_per_call": fl}}
+
+
+def extra_pool(reps=10):
+    """lbca_pool of both series of the 32K-token GQA prefix (HBM-bound)."""
+    import torch
+
+    from block_compressed_long_b200 import lbca as L
+    from block_compressed_long_b200 import synth
+    w = synth.scaled(synth.WORKLOADS["gqa_decode_32k"], kind="prefill", seq_len=32768)
+    inp = synth.make(w)
+    cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   dtype=w.dtype)
+    d = lambda t: t.cuda()  # noqa: E731
+    k, v, zk, zv, bpk, bpv = (d(t) for t in (inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v))
+    nb = w.seq_len // w.block_m
+    ok_ = torch.empty(1, w.n_kv_heads, nb, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    ov_ = torch.empty_like(ok_)
+
+    def run():
+        L.lbca_pool(cfg, L.LBCA_KEY, k, zk, bpk, None, ok_)
+        L.lbca_pool(cfg, L.LBCA_VALUE, v, zv, bpv, None, ov_)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = 2 * (2 * k.numel() * 2 + ok_.numel() * 2)  # K and V series: read X and Z, write entries
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    hbm, src = peaks()
+    return {"workload": "gqa_decode_32k prefix (32768 tokens, K and V series)", "metric": "pool GB/s", "value": gbs,
+            "unit": "GB/s", "ms_per_call": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_source": src, "kernel": "pool_kernel", "bytes_per_call": nbytes}}
+
+
 def load_traffic(workload):
     """DRAM bytes per decode launch from a committed ncu capture, if the
     decode source has not changed since it was taken."""
@@ -402,6 +498,8 @@ def main():
     import __graft_entry__
     __graft_entry__.build()
     line, _ = run_ours(args, w, rank, world)
+    if world == 1 and args.workload == "gqa_decode_32k":
+        line["also"] = [extra_prefill(), extra_pool()]
     if rank == 0 and world == 1:
         us, n, cores, desc = oracle_decode_timing(w)
         line["cpu_baseline"] = {"value": us, "unit": "µs/token", "cores": cores, "kind": "oracle", "sample": desc}

@@ -15,10 +15,9 @@
 //              fp16 K-major operands from shared memory) into the query tile's
 //              TMEM S columns, and O += P V with P read from TMEM (the
 //              softmax overwrites S with P) and fp16 V as an MN-major operand;
-//              completion is signalled by tcgen05.commit on mbarriers.  It
-//              polls all pending work and issues whatever is ready, so the
-//              two query tiles of a CTA interleave on the tensor core while
-//              the other tile's softmax runs.
+//              completion is signalled by tcgen05.commit on mbarriers.  Two
+//              query tiles per CTA interleave (PV0, S0', PV1, S1') so the
+//              tensor core works on one tile while the other's softmax runs.
 //   warps 4-7, 8-11  softmax of query tiles 0 and 1: thread r owns query row r
 //              and TMEM lane r.  It rotates
 //              its Q row in shared memory once, then per tile loads its S row,
@@ -165,12 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        // P_q(i) lives in S_q's TMEM columns, so S_q(i+1) waits until PV_q(i)
-        // has read it; the two query tiles otherwise proceed independently.
+        // order: S0(0) S1(0) | PV0(i) S0(i+1) PV1(i) S1(i+1) | ...  P_q(i) lives in
+        // S_q's TMEM columns, so S_q(i+1) waits until PV_q(i) has read it.
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
-            auto issue_s = [&](int q, int i) {  // S_q(i) = Q_q K_i^T
+            auto issue_s = [&](int q, int i) {
                 const int s = i % NSTAGE;
                 const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
                 const uint32_t sk = smem_addr(smem + OFF_K + s * KTILE);
@@ -193,54 +192,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             };
             bool ok = true;
             for (int q = 0; ok && q < NQ; ++q) ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
-            // event loop: issue whichever S or PV is ready, so that one query
-            // tile's wait never holds up the other's work
-            int next_s[NQ], next_pv[NQ];
-            for (int q = 0; q < NQ; ++q) { next_s[q] = 0; next_pv[q] = 0; }
-            int pv_pairs = 0;  // tiles whose PV has been issued for every query tile
-            uint64_t t_start = globaltimer_ns();
-            while (ok) {
-                bool done = true, progressed = false;
-                for (int q = 0; q < NQ; ++q) {
-                    // S_q(i): K_i loaded, and PV_q(i-1) has read P_q(i-1) from the S columns
-                    const int i = next_s[q];
-                    if (i < ntile) {
-                        done = false;
-                        if (next_pv[q] == i && mbar_test(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1) &&
-                            (i == 0 || mbar_test(&bars[B_ODONE + q], (i - 1) & 1))) {
-                            issue_s(q, i);
-                            next_s[q] = i + 1;
-                            progressed = true;
-                        }
-                    }
-                    // PV_q(j): P_q(j) written and V_j loaded
-                    const int j = next_pv[q];
-                    if (j < ntile) {
-                        done = false;
-                        if (j < next_s[q] && mbar_test(&bars[B_PFULL + q], j & 1) &&
-                            mbar_test(&bars[B_VFULL + j % NSTAGE], (j / NSTAGE) & 1)) {
-                            issue_pv(q, j);
-                            next_pv[q] = j + 1;
-                            progressed = true;
-                        }
+            if (ok && ntile > 0) {
+                ok = wait_or_fail(&bars[B_KFULL], 0, fail, a.status);
+                if (ok) { issue_s(0, 0); issue_s(1, 0); }
+            }
+            for (int i = 0; ok && i < ntile; ++i) {
+                const int s = i % NSTAGE, n = i + 1, sn = n % NSTAGE;
+                ok = wait_or_fail(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status);
+                const bool more = n < ntile;
+                for (int q = 0; ok && q < NQ; ++q) {
+                    ok = wait_or_fail(&bars[B_PFULL + q], i & 1, fail, a.status);
+                    if (!ok) break;
+                    issue_pv(q, i);
+                    if (q == NQ - 1) tc_commit(&bars[B_KVEMPTY + s]);
+                    if (more) {  // S_q(i+1) needs the next K tile and P_q(i) consumed
+                        if (q == 0) ok = wait_or_fail(&bars[B_KFULL + sn], (n / NSTAGE) & 1, fail, a.status);
+                        if (ok) ok = wait_or_fail(&bars[B_ODONE + q], i & 1, fail, a.status);
+                        if (ok) issue_s(q, n);
                     }
                 }
-                // a stage is free once every query tile's PV of its tile has been issued (and completes)
-                int both = ntile;
-                for (int q = 0; q < NQ; ++q) both = min(both, next_pv[q]);
-                while (pv_pairs < both) {
-                    tc_commit(&bars[B_KVEMPTY + pv_pairs % NSTAGE]);
-                    ++pv_pairs;
-                }
-                if (done) break;
-                if (progressed) {
-                    t_start = globaltimer_ns();
-                } else if (globaltimer_ns() - t_start > kWaitNs) {  // no progress for the wait bound
-                    *reinterpret_cast<volatile int*>(fail) = 1;
-                    set_status(a.status, LBCA_ERR_TIMEOUT);
-                    ok = false;
-                }
-                if (*reinterpret_cast<volatile int*>(fail)) ok = false;
             }
         }
     } else if (warp >= 4) {

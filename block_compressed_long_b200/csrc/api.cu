@@ -112,6 +112,15 @@ lbca_status check_kv(const lbca_config* c, const void* k, const void* v, const v
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// The decode launch: the tensor-core kernel for the shared-entry form where it
+// applies (it needs no workspace), else the CUDA-core split-KV kernel.
+lbca_status run_decode(const lbca_config* cfg, DecodeArgs& a, int32_t max_ctx, cudaStream_t s) {
+    a.tc_cs = plan_decode_mqa_tc(cfg->dtype, a.B, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
+                                 cfg->n_win, cfg->shared_kv, max_ctx);
+    if (a.tc_cs > 0) return cuda_status(launch_decode_mqa_tc(a, s));
+    return cuda_status(launch_decode(a, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -222,7 +231,7 @@ lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache*
     a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
-    return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+    return run_decode(cfg, a, max_ctx, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
@@ -231,6 +240,13 @@ size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, i
                             cfg->n_win, cfg->shared_kv, max_ctx);
     if (sp.ok) return align256(sp.arrive_elems * 4);
     return lbca_decode_workspace_bytes(cfg, batch, max_ctx);  // append + decode fallback
+}
+
+int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return -1;
+    const StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
+                                  cfg->n_win, cfg->shared_kv, max_ctx);
+    return sp.ok ? 1 : 2;
 }
 
 lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk, const void* zv,
@@ -435,7 +451,7 @@ lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbc
     a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
-    return cuda_status(launch_decode(a, s));
+    return run_decode(cfg, a, max_ctx, s);
 }
 
 const char* lbca_status_string(lbca_status status) {

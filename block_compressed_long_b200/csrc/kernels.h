@@ -78,6 +78,7 @@ struct DecodeArgs {
     int32_t* status;
     int B, Hq, G, D, m, w, rho, rmsnorm, shared, max_blocks, R;
     int n_split, chunk, heads_per_cta;
+    int tc_cs;         // tensor-core shared-entry path: CTAs per cluster (0 = CUDA-core path)
     float eps, scale;
     double rope_step;  // theta^(-2/rho)
 };
@@ -92,6 +93,10 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int
                        int max_ctx);
 size_t decode_workspace_bytes(const DecodePlan& p);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+// Tensor-core decode of the shared-entry form (bf16, 64 query heads per kv head,
+// D in {256, 512}): the cluster size for this call, or 0 when it does not apply.
+int plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+cudaError_t launch_decode_mqa_tc(const DecodeArgs& a, cudaStream_t s);
 
 // One serving step (append + decode) in one cluster launch.
 struct StepArgs {

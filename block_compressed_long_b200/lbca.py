@@ -28,7 +28,7 @@ LBCA_KEY, LBCA_VALUE = 0, 1
 ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspace_bytes",
                 "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
                 "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc",
-                "lbca_decode_step_workspace_bytes", "lbca_decode_step")
+                "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches")
 
 
 class lbca_config(ctypes.Structure):
@@ -73,6 +73,8 @@ _lib.lbca_decode_step_workspace_bytes.restype = _sz
 _lib.lbca_decode_step.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _sz,
                                   _vp, _vp]
 _lib.lbca_decode_step.restype = ctypes.c_int
+_lib.lbca_decode_step_launches.argtypes = [_CP, _i32, _i32]
+_lib.lbca_decode_step_launches.restype = _i32
 _lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _vp]
 _lib.lbca_decode_noalloc.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
@@ -196,6 +198,10 @@ def lbca_decode(cfg, q, cache: Cache, sink, gamma_q, out, workspace, max_ctx=0, 
 
 def lbca_decode_step_workspace_bytes(cfg: lbca_config, batch: int, max_ctx: int) -> int:
     return int(_lib.lbca_decode_step_workspace_bytes(ctypes.byref(cfg), batch, max_ctx))
+
+
+def lbca_decode_step_launches(cfg: lbca_config, batch: int, max_ctx: int) -> int:
+    return int(_lib.lbca_decode_step_launches(ctypes.byref(cfg), batch, max_ctx))
 
 
 def lbca_decode_step(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, q, cache: Cache, sink, gamma_q, out,

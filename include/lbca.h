@@ -213,6 +213,10 @@ LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lb
  * two calls.
  */
 LBCA_API size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
+/* Kernel launches one lbca_decode_step call makes for these shapes: 1 when the
+ * step runs as one fused kernel, 2 when it runs lbca_append then lbca_decode,
+ * -1 for an invalid configuration.  Host-only; needs no GPU. */
+LBCA_API int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
 LBCA_API lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk,
                                       const void* zv, const void* b_pos_k, const void* b_pos_v,
                                       const void* gamma_kv, const void* q, const lbca_cache* cache,

@@ -114,6 +114,16 @@ def test_cache_and_decode_checks(L):
     assert pre == L.LBCA_ERR_CAPACITY                     # pooled entries need a workspace
 
 
+def test_decode_step_launches(L):
+    """One fused kernel for the GQA step shapes, append + decode for the
+    shared-entry D = 512 form (and for no window); -1 for a bad config."""
+    assert L.lbca_decode_step_launches(_cfg(L), 1, 32769) == 1
+    assert L.lbca_decode_step_launches(_cfg(L, n_win=0), 1, 32769) == 2
+    hca = _cfg(L, n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128, rope_dims=64)
+    assert L.lbca_decode_step_launches(hca, 8, 131073) == 2
+    assert L.lbca_decode_step_launches(_cfg(L, block_m=0), 1, 100) == -1
+
+
 def test_status_strings(L):
     for s in range(7):
         assert L.lbca_status_string(s)

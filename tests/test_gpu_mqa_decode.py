@@ -1,0 +1,112 @@
+"""Decode of the shared-entry (MQA, HCA) form on the tensor-core path.
+
+bf16 shapes with 64 query heads per kv head and head_dim 256 or 512 take the
+tcgen05 kernel (entry tiles as the M operand, one cluster per sequence and kv
+head, merge in distributed shared memory).  Every case here runs through the
+C ABI on seeded inputs and is compared element by element with the fp64
+oracle: ragged batches that put 0, 1, 15, 16, 17, 127, 128 ... entries into
+a CTA's chunk, the variants of the form (no sink, no RMSNorm, no RoPE, RoPE
+dims that split a 16-byte chunk, D = 256, two kv heads, no window), a
+sequence whose visible list fills every CTA of a 16-CTA cluster with exactly
+128 entries, an empty sequence, and the one-launch step entry point.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_compressed_long_b200 import synth
+from lbca_cases import (DecodeRun, assert_close, assert_close_few_entries, entry_magnitudes, f64, fused_step, lib,
+                        oracle_decode, visible_entries)
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS["hca_mqa_decode_128k"]
+
+
+@pytest.fixture(scope="module")
+def L():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return lib()
+
+
+def _inputs(w, lens, steps):
+    """Inputs whose every row is drawn, then the per-sequence cached lengths."""
+    top = int(max(lens))
+    w = synth.scaled(w, ctx=(top, top), batch=len(lens), steps=steps)
+    inp = synth.make(w)
+    inp.lens = np.asarray(lens, dtype=np.int64)
+    return w, inp
+
+
+def _check_steps(L, w, lens, steps, what):
+    """Every step against the oracle: the plain bf16 bound for every sequence
+    that sees 32 or more entries, the entry-rounding bound for the others."""
+    w, inp = _inputs(w, lens, steps)
+    run = DecodeRun(L, w, inp, steps=steps)
+    for s in range(steps):
+        got = f64(run.step())
+        torch.cuda.synchronize()
+        want = oracle_decode(w, inp, s)
+        few = np.array([visible_entries(w, int(n) + s + 1) < 32 for n in inp.lens])
+        if (~few).any():
+            assert_close(got[~few], want[~few], "bf16", f"{what} step {s}")
+        if few.any():
+            emax = entry_magnitudes(w, inp, s, np.flatnonzero(few))
+            assert_close_few_entries(got[few], want[few], emax, f"{what} step {s}, < 32 entries")
+    assert int(run.status.item()) == 0
+
+
+def test_ragged_chunk_sizes(L):
+    """Visible lists of 1 ... ~2000 entries in one batch: chunks of 0 to 128
+    rows, pooled and raw rows in the same chunk, ring wrap-around."""
+    lens = [0, 1, 4, 15, 16, 17, 127, 128, 255, 256, 300, 1000, 2900, 131072 // 64]
+    _check_steps(L, W, lens, 2, "hca ragged")
+
+
+@pytest.mark.parametrize("kw", [
+    dict(sink="none"),
+    dict(rmsnorm=False),
+    dict(rope_dims=0),
+    dict(rope_dims=6),
+    dict(head_dim=256),
+    dict(n_kv_heads=2, n_q_heads=128),
+    dict(n_win=0, block_m=64),
+    dict(sink="zero", rope_dims=512),
+], ids=["no-sink", "no-rmsnorm", "no-rope", "rope6", "d256", "two-kv-heads", "no-window", "full-rope"])
+def test_form_variants(L, kw):
+    _check_steps(L, synth.scaled(W, **kw), [50, 700, 2100], 2, f"hca {kw}")
+
+
+def test_full_tiles_in_a_16_cta_cluster(L):
+    """m = 16, n_win = 16 and 32303 tokens give 2017 pooled + 31 raw = 2048
+    visible entries: 16 CTAs with 128 entries each (the largest chunk)."""
+    w = synth.scaled(W, block_m=16, n_win=16)
+    _check_steps(L, w, [32300], 3, "hca 2048 entries")
+
+
+def test_empty_sequence_gives_zeros(L):
+    """No visible entry: zeros, with or without the sink in the denominator."""
+    w, inp = _inputs(W, [0, 0], 1)
+    run = DecodeRun(L, w, inp, steps=1)
+    run.cache.seq_lens.zero_()
+    for sink in (None, run.sink):
+        out = torch.full((2, w.n_q_heads, w.head_dim), 3.0, dtype=torch.bfloat16, device="cuda")
+        L.lbca_decode(run.cfg, run.q[0], run.cache, sink, None, out, run.ws, 1, run.status)
+        torch.cuda.synchronize()
+        assert torch.all(out == 0)
+    assert int(run.status.item()) == 0
+
+
+def test_step_entry_point_equals_append_then_decode(L):
+    """lbca_decode_step on this form runs append then the tensor-core decode:
+    bit-identical to the two calls."""
+    w, inp = _inputs(W, [300, 1500, 40], 3)
+    a = DecodeRun(L, w, inp, steps=3)
+    b = DecodeRun(L, w, inp, steps=3)
+    for s in range(3):
+        x = a.step()
+        y = fused_step(b)
+        torch.cuda.synchronize()
+        assert torch.equal(x, y), f"step {s}"
+        assert_close(f64(y), oracle_decode(w, inp, s), "bf16", f"step {s}")
+    assert int(a.status.item()) == 0 and int(b.status.item()) == 0

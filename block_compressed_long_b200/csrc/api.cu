@@ -115,9 +115,13 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // The decode launch: the tensor-core kernel for the shared-entry form where it
 // applies (it needs no workspace), else the CUDA-core split-KV kernel.
 lbca_status run_decode(const lbca_config* cfg, DecodeArgs& a, int32_t max_ctx, cudaStream_t s) {
-    a.tc_cs = plan_decode_mqa_tc(cfg->dtype, a.B, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
-                                 cfg->n_win, cfg->shared_kv, max_ctx);
-    if (a.tc_cs > 0) return cuda_status(launch_decode_mqa_tc(a, s));
+    const MqaTcPlan tc = plan_decode_mqa_tc(cfg->dtype, a.B, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                                            cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+    a.tc_cs = tc.cs;
+    if (tc.cs > 0) {
+        a.chunk = tc.rows;
+        return cuda_status(launch_decode_mqa_tc(a, s));
+    }
     return cuda_status(launch_decode(a, s));
 }
 

@@ -25,55 +25,73 @@
 // fp16, whose 11-bit significand keeps the weights 8x closer than bf16 would.
 // An element beyond the fp16 range sets d_status to LBCA_ERR_UNSUPPORTED.
 //
-// B200 mapping: grid (CS, G, B) with cluster (CS, 1, 1).  The CS CTAs of a
-// cluster split one (sequence, kv head)'s visible list into CS chunks of at
-// most 128 entries.  A CTA copies its chunk (pooled rows, then ring rows) into
-// 128-byte-swizzled shared memory with 16-byte cp.async, prepares the NH
-// queries meanwhile (RMSNorm, RoPE at t, fp16, swizzled), issues the S^T MMAs
-// (one thread), takes the per-head max and sum over its entries with
-// transposing warp butterflies, writes P^T (fp16) and issues the O^T MMAs.
-// The partials are merged inside the cluster through distributed shared
-// memory: after one cluster barrier every CTA reads all CTAs' (max, sum) per
-// head, scales its O^T by 2^(m - M) / denominator (the sink joins the
-// denominator), and pushes slice d / (D / CS) of it to the CTA that owns those
-// dims; after a second barrier each CTA sums its slice, turns the rotated dims
-// back by -t and writes the output.  No workspace, no second launch.
-#include <cooperative_groups.h>
-
+// B200 mapping: grid (CS, G, B), cluster (CS, 1, 1), 16 warps per CTA.  The CS
+// CTAs of a cluster share one (sequence, kv head):
+//   1. Each CTA copies its chunk of the visible list (<= C rows: pooled rows,
+//      then ring rows) into 128-byte-swizzled shared memory with 16-byte
+//      cp.async and widens it to fp16 in place.  Meanwhile up to 8 CTAs each
+//      prepare a share of the queries (RMSNorm, RoPE at t, fp16) and
+//      bulk-copy it into every other CTA's query tile (shared memory to
+//      shared memory across the cluster, one destination per copy).
+//   2. One thread issues S^T; warps take each head's max over the chunk with
+//      a transposing butterfly, and every CTA pushes its maxima to all CTAs.
+//      After one cluster barrier every CTA holds the same per-head reference
+//      max M (the sink included), so the CTAs' partial outputs share one
+//      scale and simply add.
+//   3. P = 2^(s - M) (fp16) -> P^T tile; per-head sums; O^T on tcgen05.
+//   4. Each CTA rounds its O^T to fp16, lays it out by owner (dims
+//      [r SW, (r+1) SW) belong to CTA r) and bulk-copies one slice, plus its
+//      sums, to each owner.  An owner waits for its CS slices on an mbarrier,
+//      adds them, divides by the summed sums plus the sink term, turns the
+//      rotated dims back by -t and writes bf16.
+// A sequence whose whole visible list fits one chunk skips the exchange: its
+// first CTA takes every entry and writes the output straight from TMEM.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace lbca {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int NH = 64;          // query heads per kv head (N of both MMAs)
-constexpr int TE = 128;         // entry rows per CTA tile (M of S^T)
+constexpr int NGRP = NH / 8;    // 8-head groups of the query tile
+constexpr int kMaxCS = 16;
 constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;
 
-template <int D>
+// Output dims owned by each CTA of a CS-CTA cluster (even, so RoPE pairs never split).
+__host__ __device__ inline int owned_dims(int D, int CS) { return ((D + CS - 1) / CS + 1) & ~1; }
+
+// Shared-memory plan for head dim D, C entry rows per CTA (a multiple of 16, <= 128)
+// and CS CTAs per cluster.
 struct MqaLayout {
-    static constexpr uint32_t EREG = TE * 128;               // one 64-dim column region of E
-    static constexpr uint32_t QREG = NH * 128;               // one 64-dim column region of Q
-    static constexpr uint32_t OFF_E = 0;
-    static constexpr uint32_t OFF_Q = OFF_E + (D / 64) * EREG;
-    static constexpr uint32_t OFF_P = OFF_Q + (D / 64) * QREG;
-    static constexpr uint32_t OFF_CS = OFF_P + TE * NH * 2;  // [D/2] float2 cos/sin at t
-    static constexpr uint32_t OFF_RED = OFF_CS + (D / 2) * 8;  // [2][4][NH] warp partials
-    static constexpr uint32_t OFF_MH = OFF_RED + 2 * 4 * NH * 4;  // [NH] CTA max
-    static constexpr uint32_t OFF_ML = OFF_MH + NH * 4;            // [2][NH] published (max, sum)
-    static constexpr uint32_t OFF_F = OFF_ML + 2 * NH * 4;         // [NH] merge factor
-    static constexpr uint32_t OFF_BAR = OFF_F + NH * 4;            // 2 mbarriers, TMEM base, flag
-    static constexpr uint32_t TOTAL = OFF_BAR + 64;
-    static constexpr uint32_t SMEM = TOTAL + 1024;                 // slack for 1024-byte alignment
-    // the merge's receive buffer [CS][NH/4][D/CS][4] f32 = NH * D * 4 bytes aliases E and Q
-    static_assert((uint32_t)NH * D * 4 <= OFF_P, "receive buffer must fit in the E and Q regions");
-    static constexpr uint32_t TMEM_COLS = (NH + (D / 128) * NH) <= 256 ? 256 : 512;
+    uint32_t EREG, GS, SLICE;
+    uint32_t OFF_E, OFF_Q, OFF_P, OFF_MALL, OFF_LRECV, OFF_CS, OFF_RED, OFF_MH, OFF_LLOC, OFF_DEN, OFF_BAR;
+    uint32_t TOTAL, SMEM;
+    __host__ __device__ MqaLayout(int D, int C, int CS) {
+        EREG = (uint32_t)C * 128u;                          // one 64-dim column region of E
+        GS = (uint32_t)(D / 64) * 1024u;                    // one 8-head group of Q (all regions)
+        SLICE = (uint32_t)(NH / 4) * owned_dims(D, CS) * 8u;  // fp16 [NH/4][SW][4] per owner
+        const uint32_t e_bytes = (uint32_t)(D / 64) * EREG;
+        const uint32_t xfer = (uint32_t)CS * SLICE;          // O^T staging (aliases E) / receive (aliases Q)
+        const uint32_t q_bytes = (uint32_t)NH * D * 2u;
+        OFF_E = 0;
+        OFF_Q = ((e_bytes > xfer ? e_bytes : xfer) + 1023u) & ~1023u;
+        OFF_P = (OFF_Q + (q_bytes > xfer ? q_bytes : xfer) + 1023u) & ~1023u;
+        OFF_MALL = OFF_P + (uint32_t)C * 128u;              // [kMaxCS][NH] f32 pushed maxima
+        OFF_LRECV = OFF_MALL + kMaxCS * NH * 4u;            // [kMaxCS][NH] f32 pushed sums
+        OFF_CS = OFF_LRECV + kMaxCS * NH * 4u;              // [D/2] float2 cos/sin at t
+        OFF_RED = OFF_CS + (uint32_t)(D / 2) * 8u;          // [4][NH] warp partials
+        OFF_MH = OFF_RED + 4u * NH * 4u;                    // [NH] reference max
+        OFF_LLOC = OFF_MH + NH * 4u;                        // [NH] this CTA's sums
+        OFF_DEN = OFF_LLOC + NH * 4u;                       // [NH] denominators
+        OFF_BAR = OFF_DEN + NH * 4u;                        // 4 mbarriers + TMEM base
+        TOTAL = OFF_BAR + 64u;
+        SMEM = TOTAL + 1024u;                               // slack for 1024-byte alignment
+    }
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -88,13 +106,12 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Butterfly over the 32 lanes of a warp that leaves lane l holding the
-// reduction over all lanes of v[l]: each step trades half of the remaining
-// values with the partner lane, 31 shuffles in all.
+// Butterfly over the 32 lanes of a warp for 16 values per lane: lane l ends up
+// holding the reduction over all 32 lanes of v[l % 16] (16 shuffles).
 template <bool kMax>
-__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
+__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lane) {
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
+    for (int o = 8; o >= 1; o >>= 1) {
         const bool up = (lane & o) != 0;
 #pragma unroll
         for (int i = 0; i < o; ++i) {
@@ -104,7 +121,8 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
             v[i] = kMax ? fmaxf(keep, got) : keep + got;
         }
     }
-    return v[0];
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], 16);
+    return kMax ? fmaxf(v[0], got) : v[0] + got;
 }
 
 // kind::f16 instruction descriptor with both operands MN-major (fp16 in, f32 out).
@@ -121,28 +139,36 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& ovf) {
     return pack_f16x2(lo, hi);
 }
 
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    return __half22float2(h);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const DecodeArgs a) {
-    using Lay = MqaLayout<D>;
+    constexpr int CPR = D / 8;    // 16-byte chunks per entry row
     constexpr int CPL = D / 256;  // 16-byte query chunks per lane per head
     static_assert(D % 256 == 0 && D <= 512, "D must be 256 or 512");
+    const int C = a.chunk;        // entry rows per CTA (multiple of 16, <= 128)
+    const int CS = a.tc_cs;
+    const MqaLayout lay(D, C, CS);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
-    uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(smem + Lay::OFF_BAR + 16);
-    float2* cs = reinterpret_cast<float2*>(smem + Lay::OFF_CS);
-    float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
-    float* mh = reinterpret_cast<float*>(smem + Lay::OFF_MH);
-    float* ml = reinterpret_cast<float*>(smem + Lay::OFF_ML);
-    float* fh = reinterpret_cast<float*>(smem + Lay::OFF_F);
-    float* recv = reinterpret_cast<float*>(smem + Lay::OFF_E);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.OFF_BAR);  // S done, O done, Q in, slices in
+    uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(smem + lay.OFF_BAR + 32);
+    float2* cs = reinterpret_cast<float2*>(smem + lay.OFF_CS);
+    float* red = reinterpret_cast<float*>(smem + lay.OFF_RED);
+    float* mh = reinterpret_cast<float*>(smem + lay.OFF_MH);
+    float* lloc = reinterpret_cast<float*>(smem + lay.OFF_LLOC);
+    float* den = reinterpret_cast<float*>(smem + lay.OFF_DEN);
+    const float* mall = reinterpret_cast<const float*>(smem + lay.OFF_MALL);
+    const float* lrecv = reinterpret_cast<const float*>(smem + lay.OFF_LRECV);
 
-    cg::cluster_group cluster = cg::this_cluster();
-    const int CS = a.tc_cs;
     const int rank = (int)blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int SW = D / CS;  // output dims owned by each CTA of the cluster
+    const int quad = warp & 3, hq = warp >> 2;  // TMEM lane quarter, head group of 16
+    const int SW = owned_dims(D, CS);
 
     // ---- visible set of this sequence (block-aligned partition) and this CTA's chunk ----
     const int L = a.seq_lens[b];
@@ -150,87 +176,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     const int P = visible_blocks(L, a.m, a.w);
     const int s0 = P * a.m;
     int n_vis = L > 0 ? P + (L - s0) : 0;
-    if (P > a.max_blocks || L - s0 > a.R || n_vis > TE * CS) {  // cache or split grid cannot hold it
+    if (P > a.max_blocks || L - s0 > a.R || n_vis > C * CS) {  // cache or split grid cannot hold it
         if (rank == 0 && g == 0 && tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
         n_vis = 0;
     }
-    const int chunk = (n_vis + CS - 1) / CS;
-    const int e0 = rank * chunk;
-    const int n = max(0, min(n_vis, e0 + chunk) - e0);
+    const bool single = n_vis <= C;  // one CTA takes the whole list: no exchange (uniform per cluster)
+    const int chunk = single ? n_vis : (n_vis + CS - 1) / CS;
+    const int e0 = single ? 0 : rank * chunk;
+    const int n = single ? (rank == 0 ? n_vis : 0) : max(0, min(n_vis, e0 + chunk) - e0);
     const int n16 = (n + 15) & ~15;
 
+    // query groups this CTA prepares for the whole cluster
+    const int preppers = CS >= 8 ? 8 : (CS >= 4 ? 4 : (CS >= 2 ? 2 : 1));
+    const int gpc = NGRP / preppers;
+    const bool prepper = rank < preppers;
+    const uint32_t my_q_bytes = prepper ? (uint32_t)gpc * lay.GS : 0u;
+
+    const uint32_t sE = smem_addr(smem + lay.OFF_E), sQ = smem_addr(smem + lay.OFF_Q);
+    const uint32_t sP = smem_addr(smem + lay.OFF_P);
+    const uint32_t bar_q = smem_addr(&bars[2]), bar_r = smem_addr(&bars[3]);
+
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_barrier_init();
+        mbar_arrive_expect_tx(&bars[2], (uint32_t)NH * D * 2u - my_q_bytes);
+        mbar_arrive_expect_tx(&bars[3], single ? 0u : (uint32_t)CS * (lay.SLICE + NH * 4u));
     }
     __syncwarp();
-    if (warp == 0) tmem_alloc(tmem_sh, Lay::TMEM_COLS);
+    if (warp == 0) tmem_alloc(tmem_sh, 512);
+    cluster_arrive_relaxed();  // this CTA's barriers exist (waited for before the first push)
 
     // ---- stage the chunk's entry rows (bf16), 128-byte swizzled; rows [n, n16) zero ----
-    const uint32_t sE = smem_addr(smem + Lay::OFF_E);
-    {
-        const size_t pool_head = ((size_t)b * a.G + g) * a.max_blocks;
-        const size_t ring_head = ((size_t)b * a.G + g) * a.R;
-        const __nv_bfloat16* pk = static_cast<const __nv_bfloat16*>(a.pooled_k);
-        const __nv_bfloat16* rk = static_cast<const __nv_bfloat16*>(a.ring_k);
-        constexpr int CPR = D / 8;  // 16-byte chunks per row
-        for (int c = tid; c < n16 * CPR; c += kThreads) {
-            const int row = c / CPR, ch = c % CPR;
-            const uint32_t dst = sE + (uint32_t)(ch >> 3) * Lay::EREG + (uint32_t)(row >> 3) * 1024u +
-                                 (uint32_t)(row & 7) * 128u + ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
-            const void* src = a.q;  // any valid address for the zero-filled rows
-            uint32_t bytes = 0;
-            if (row < n) {
-                const int idx = e0 + row;
-                src = idx < P ? pk + (pool_head + idx) * D + ch * 8
-                              : rk + (ring_head + (s0 + (idx - P)) % a.R) * D + ch * 8;
-                bytes = 16;
-            }
-            cp_async16(dst, src, bytes);
+    const size_t pool_head = ((size_t)b * a.G + g) * a.max_blocks;
+    const size_t ring_head = ((size_t)b * a.G + g) * a.R;
+    const __nv_bfloat16* pk = static_cast<const __nv_bfloat16*>(a.pooled_k);
+    const __nv_bfloat16* rk = static_cast<const __nv_bfloat16*>(a.ring_k);
+    for (int row = warp; row < n16; row += kWarps) {
+        const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.q);  // any valid address (zero fill)
+        uint32_t bytes = 0;
+        if (row < n) {
+            const int idx = e0 + row;
+            src = idx < P ? pk + (pool_head + idx) * D : rk + (ring_head + (s0 + (idx - P)) % a.R) * D;
+            bytes = 16;
+        }
+        const uint32_t rbase = sE + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+#pragma unroll
+        for (int j = 0; j < CPR / 32; ++j) {
+            const int ch = j * 32 + lane;
+            cp_async16(rbase + (uint32_t)(ch >> 3) * lay.EREG + ((uint32_t)((ch & 7) ^ (row & 7)) << 4),
+                       bytes ? src + ch * 8 : src, bytes);
         }
     }
 
-    // ---- cos/sin at t, then the NH queries: RMSNorm, RoPE, fp16, swizzled (K-major) ----
+    // ---- cos/sin at t; this CTA's query groups: RMSNorm, RoPE, fp16, group-major swizzled ----
     for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((int64_t)t, k, a.rope_step);
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_sh;
     bool ovf = false;
-    {
+    if (prepper) {
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.Hq + (size_t)g * NH) * D;
         const __nv_bfloat16* gm = static_cast<const __nv_bfloat16*>(a.gamma_q);
-        float gam[CPL][8];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            if (gm && a.rmsnorm) {
-                ld16(gm + (c * 32 + lane) * 8, gam[c]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) gam[c][i] = 1.f;
-            }
-        }
-        constexpr int HPW = NH / (kThreads / 32);  // heads per warp
-        uint4 raw[HPW][CPL];
-#pragma unroll
-        for (int hi = 0; hi < HPW; ++hi)
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                raw[hi][c] = __ldg(reinterpret_cast<const uint4*>(qg + (size_t)(warp * HPW + hi) * D) + c * 32 + lane);
         const int rope0 = D - a.rho;
-#pragma unroll
-        for (int hi = 0; hi < HPW; ++hi) {
-            const int h = warp * HPW + hi;
+        for (int hi = warp; hi < gpc * 8; hi += kWarps) {
+            const int h = rank * gpc * 8 + hi;
             float x[CPL][8];
             float ss = 0.f;
 #pragma unroll
             for (int c = 0; c < CPL; ++c) {
-                const uint32_t wv[4] = {raw[hi][c].x, raw[hi][c].y, raw[hi][c].z, raw[hi][c].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[c][2 * e] = __uint_as_float(wv[e] << 16);
-                    x[c][2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
-                }
+                ld16(qg + (size_t)h * D + (c * 32 + lane) * 8, x[c]);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ss = fmaf(x[c][i], x[c][i], ss);
             }
@@ -239,13 +253,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
                 for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
                 const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
 #pragma unroll
-                for (int c = 0; c < CPL; ++c)
+                for (int c = 0; c < CPL; ++c) {
+                    float gam[8];
+                    if (gm) {
+                        ld16(gm + (c * 32 + lane) * 8, gam);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) x[c][i] *= inv * gam[c][i];
+                        for (int i = 0; i < 8; ++i) gam[i] = 1.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[c][i] *= inv * gam[i];
+                }
             }
 #pragma unroll
             for (int c = 0; c < CPL; ++c) {
-                const int d0 = (c * 32 + lane) * 8;
+                const int ch = c * 32 + lane, d0 = ch * 8;
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     if (a.rho > 0 && d0 + 2 * e >= rope0)
@@ -257,18 +279,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
                 o.y = pack_f16x2(x[c][2], x[c][3]);
                 o.z = pack_f16x2(x[c][4], x[c][5]);
                 o.w = pack_f16x2(x[c][6], x[c][7]);
-                *reinterpret_cast<uint4*>(smem + Lay::OFF_Q + sw128_off(h, d0, Lay::QREG)) = o;
+                const int hr = h & 7;
+                *reinterpret_cast<uint4*>(smem + lay.OFF_Q + (uint32_t)(h >> 3) * lay.GS + (uint32_t)(ch >> 3) * 1024u +
+                                          (uint32_t)hr * 128u + ((uint32_t)((ch & 7) ^ hr) << 4)) = o;
             }
         }
+        fence_async_smem();
     }
-    // this thread's own copies have landed: widen them to fp16 in place
+    __syncthreads();
+    cluster_wait_acquire();  // every CTA's barriers exist
+    const bool q_sender = prepper && tid < CS && tid != rank;
+    if (q_sender) {  // this CTA's query groups to CTA `tid`
+        for (int G = rank * gpc; G < rank * gpc + gpc; ++G) {
+            const uint32_t off = sQ + (uint32_t)G * lay.GS;
+            bulk_to_peer(peer_addr(off, tid), off, lay.GS, peer_addr(bar_q, tid));
+        }
+        bulk_commit();
+    }
+
+    // ---- this thread's entry copies have landed: widen them to fp16 in place ----
     cp_async_wait_all();
-    {
-        constexpr int CPR = D / 8;
-        for (int c = tid; c < n16 * CPR; c += kThreads) {
-            const int row = c / CPR, ch = c % CPR;
-            uint4* p = reinterpret_cast<uint4*>(smem + Lay::OFF_E + (uint32_t)(ch >> 3) * Lay::EREG +
-                                                (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+    for (int row = warp; row < n16; row += kWarps) {
+        uint8_t* rbase = smem + lay.OFF_E + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+#pragma unroll
+        for (int j = 0; j < CPR / 32; ++j) {
+            const int ch = j * 32 + lane;
+            uint4* p = reinterpret_cast<uint4*>(rbase + (uint32_t)(ch >> 3) * lay.EREG +
                                                 ((uint32_t)((ch & 7) ^ (row & 7)) << 4));
             uint4 u = *p;
             u.x = bf16x2_to_f16x2(u.x, ovf);
@@ -281,215 +317,259 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     fence_async_smem();
     if (__syncthreads_or(ovf) && tid == 0) set_status(a.status, LBCA_ERR_UNSUPPORTED);
 
-    // ---- S^T = E . Q^T  (TMEM columns [0, NH), lane = entry row) ----
-    const uint32_t sQ = smem_addr(smem + Lay::OFF_Q);
-    const uint32_t sP = smem_addr(smem + Lay::OFF_P);
-    if (tid == 0 && n > 0) {
+    // ---- the other CTAs' query groups, then S^T = E . Q^T (TMEM columns [0, NH)) ----
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait(&bars[2], 0, kWaitNs);
+    ok = __syncthreads_and(ok);
+    if (tid == 0 && ok && n > 0) {
         tc_fence_after();
-        constexpr uint32_t idS = idesc_f16_f32(TE, NH, false);
+        constexpr uint32_t idS = idesc_f16_f32(128, NH, false);
 #pragma unroll 4
         for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma_bf16(tbase, smem_desc_sw128(sE + (kk >> 2) * Lay::EREG + (kk & 3) * 32, 16, 1024),
-                        smem_desc_sw128(sQ + (kk >> 2) * Lay::QREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+            tc_mma_bf16(tbase, smem_desc_sw128(sE + (kk >> 2) * lay.EREG + (kk & 3) * 32, 16, 1024),
+                        smem_desc_sw128(sQ + (kk >> 2) * 1024 + (kk & 3) * 32, 16, lay.GS), idS, kk > 0);
         tc_commit(&bars[0]);
     }
-
-    // ---- per-head max and sum over this chunk; P^T (fp16) into shared memory ----
-    // warp w reads TMEM lanes 32 (w & 3).. (entry rows) and heads 32 (w >> 2)..
-    const int quad = warp & 3, hh = warp >> 2;
-    const uint32_t lane_f = (uint32_t)(32 * quad) << 16;
-    const int e = 32 * quad + lane;
-    const bool valid = e < n;
-    bool ok = true;
-    if (n > 0) ok = mbar_wait(&bars[0], 0, kWaitNs);
+    if (ok && n > 0 && tid == 0) ok = mbar_wait(&bars[0], 0, kWaitNs);
     ok = __syncthreads_and(ok);
     if (!ok && tid == 0) set_status(a.status, LBCA_ERR_TIMEOUT);
     const bool live = ok && n > 0;
+
+    // ---- per-head max over this chunk; warp (quad, hq) holds entry rows 32 quad.. x heads 16 hq.. ----
+    const uint32_t lane_f = (uint32_t)(32 * quad) << 16;
+    const int e = 32 * quad + lane;
+    const bool valid = e < n;
     const float sc = a.scale * kLog2e;
-    float v[32];
+    float s[16];
     if (live) {
         tc_fence_after();
-        tmem_ld32(tbase + lane_f + 32 * hh, v);
+        tmem_ld16(tbase + lane_f + 16 * hq, s);
         tmem_wait_ld();
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = (live && valid) ? v[i] * sc : kNegInf;
-    float s[32];
+    for (int i = 0; i < 16; ++i) s[i] = (live && valid) ? s[i] * sc : kNegInf;
+    {
+        float v[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) s[i] = v[i];
-    red[quad * NH + 32 * hh + lane] = warp_transpose_reduce<true>(v, lane);
+        for (int i = 0; i < 16; ++i) v[i] = s[i];
+        const float r = warp_transpose_reduce16<true>(v, lane);
+        if (lane < 16) red[quad * NH + 16 * hq + lane] = r;
+    }
     __syncthreads();
+    const float sink_l2 = (a.sink && tid < NH) ? a.sink[g * NH + tid] * kLog2e : kNegInf;
     if (tid < NH) {
-        float M = red[tid];
-#pragma unroll
-        for (int q = 1; q < 4; ++q) M = fmaxf(M, red[q * NH + tid]);
-        mh[tid] = M;
+        const float m = fmaxf(fmaxf(red[tid], red[NH + tid]), fmaxf(red[2 * NH + tid], red[3 * NH + tid]));
+        if (single) {
+            mh[tid] = fmaxf(m, sink_l2);
+        } else {
+            const uint32_t dst = smem_addr(smem + lay.OFF_MALL) + (uint32_t)(rank * NH + tid) * 4u;
+            for (int r = 0; r < CS; ++r) st_peer_f32(peer_addr(dst, r), m);
+        }
+    }
+    if (q_sender) bulk_wait_read_all();  // the query tile is overwritten by the slices below
+    if (!single) {
+        cluster_arrive_release();
+        cluster_wait_acquire();  // every CTA's maxima have landed everywhere; every S^T is done
+        if (tid < NH) {
+            float m = sink_l2;
+            for (int r = 0; r < CS; ++r) m = fmaxf(m, mall[r * NH + tid]);
+            mh[tid] = m;
+        }
     }
     __syncthreads();
+
+    // ---- P = 2^(s - M) (fp16) into the P^T tile; per-head sums ----
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float M = mh[32 * hh + i];
-        s[i] = (s[i] == kNegInf) ? 0.f : ex2(s[i] - M);
-    }
+    for (int i = 0; i < 16; ++i) s[i] = s[i] == kNegInf ? 0.f : ex2(s[i] - mh[16 * hq + i]);
+    if (e < C) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint4 o;
-        o.x = pack_f16x2(s[8 * c + 0], s[8 * c + 1]);
-        o.y = pack_f16x2(s[8 * c + 2], s[8 * c + 3]);
-        o.z = pack_f16x2(s[8 * c + 4], s[8 * c + 5]);
-        o.w = pack_f16x2(s[8 * c + 6], s[8 * c + 7]);
-        *reinterpret_cast<uint4*>(smem + Lay::OFF_P + sw128_off(e, 32 * hh + 8 * c, 0)) = o;
+        for (int c = 0; c < 2; ++c) {
+            uint4 o;
+            o.x = pack_f16x2(s[8 * c + 0], s[8 * c + 1]);
+            o.y = pack_f16x2(s[8 * c + 2], s[8 * c + 3]);
+            o.z = pack_f16x2(s[8 * c + 4], s[8 * c + 5]);
+            o.w = pack_f16x2(s[8 * c + 6], s[8 * c + 7]);
+            *reinterpret_cast<uint4*>(smem + lay.OFF_P + sw128_off(e, 16 * hq + 8 * c, 0)) = o;
+        }
     }
     fence_async_smem();
-    red[4 * NH + quad * NH + 32 * hh + lane] = warp_transpose_reduce<false>(s, lane);
-    __syncthreads();
-    if (tid < NH) {
-        float l = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) l += red[4 * NH + q * NH + tid];
-        ml[tid] = mh[tid];
-        ml[NH + tid] = l;
+    {
+        const float r = warp_transpose_reduce16<false>(s, lane);
+        if (lane < 16) red[quad * NH + 16 * hq + lane] = r;
     }
+    __syncthreads();
+    if (tid < NH) lloc[tid] = red[tid] + red[NH + tid] + red[2 * NH + tid] + red[3 * NH + tid];
 
-    // ---- O^T = E^T . P^T  (TMEM columns [NH + NH mt, ...), lane = dim within tile mt) ----
+    // ---- O^T = E^T . P^T (TMEM columns [NH + NH mt, ...), lane = dim within tile mt) ----
     if (tid == 0 && live) {
         tc_fence_after();
         constexpr uint32_t idO = idesc_f16_f32_mn_mn(128, NH);
         for (int mt = 0; mt < D / 128; ++mt)
             for (int kk = 0; kk < n16 / 16; ++kk)
-                tc_mma_bf16(tbase + NH + NH * mt, smem_desc_sw128(sE + 2 * mt * Lay::EREG + kk * 2048, Lay::EREG, 1024),
-                            smem_desc_sw128(sP + kk * 2048, Lay::EREG, 1024), idO, kk > 0);
+                tc_mma_bf16(tbase + NH + NH * mt, smem_desc_sw128(sE + 2 * mt * lay.EREG + kk * 2048, lay.EREG, 1024),
+                            smem_desc_sw128(sP + kk * 2048, 8192, 1024), idO, kk > 0);
         tc_commit(&bars[1]);
     }
     bool ok2 = true;
-    if (live) ok2 = mbar_wait(&bars[1], 0, kWaitNs);
+    if (live && tid == 0) ok2 = mbar_wait(&bars[1], 0, kWaitNs);
     ok2 = __syncthreads_and(ok2);
     if (!ok2 && tid == 0) set_status(a.status, LBCA_ERR_TIMEOUT);
     const bool have_o = live && ok2;
     tc_fence_after();
-    fence_async_smem();  // E and Q are rewritten by the generic-proxy merge below
 
-    // ---- merge across the cluster ----
-    cluster.sync();  // every CTA's (max, sum) published; every CTA's MMAs have read E
-    if (tid < NH) {
-        const int hg = g * NH + tid;
-        float Ms[16], Ls[16];
-        float M = kNegInf;
-        for (int r = 0; r < CS; ++r) {
-            const float* rm = cluster.map_shared_rank(ml, r);
-            Ms[r] = rm[tid];
-            Ls[r] = rm[NH + tid];
-            M = fmaxf(M, Ms[r]);
-        }
-        const float sk = a.sink ? a.sink[hg] * kLog2e : kNegInf;
-        M = fmaxf(M, sk);
-        float den = 0.f;
-        if (M != kNegInf) {
-            for (int r = 0; r < CS; ++r) den = fmaf(Ls[r], Ms[r] == kNegInf ? 0.f : ex2(Ms[r] - M), den);
-            if (a.sink) den += ex2(sk - M);
-        }
-        const float mine = ml[tid];
-        fh[tid] = (den > 0.f && mine != kNegInf) ? ex2(mine - M) / den : 0.f;
-    }
-    __syncthreads();
-    // push this CTA's scaled O^T slices: dim d goes to rank d / SW
-#pragma unroll 1
-    for (int mt = 0; mt < D / 128; ++mt) {
-        if (have_o) {
-            tmem_ld32(tbase + lane_f + NH + NH * mt + 32 * hh, v);
-            tmem_wait_ld();
-        }
-        const int d = 128 * mt + 32 * quad + lane;
-        const int owner = d / SW, dd = d % SW;
-        float* dst = cluster.map_shared_rank(recv, owner);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int h4 = 8 * hh + j;  // heads 4 h4 .. 4 h4 + 3
-            float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (have_o) {
-                o.x = v[4 * j + 0] * fh[4 * h4 + 0];
-                o.y = v[4 * j + 1] * fh[4 * h4 + 1];
-                o.z = v[4 * j + 2] * fh[4 * h4 + 2];
-                o.w = v[4 * j + 3] * fh[4 * h4 + 3];
-            }
-            *reinterpret_cast<float4*>(dst + (((size_t)rank * (NH / 4) + h4) * SW + dd) * 4) = o;
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, Lay::TMEM_COLS);
-    cluster.sync();  // every slice has landed; nothing remote is touched after this
-
-    // ---- sum the slices, turn the rotated dims back by -t, write bf16 ----
     const int rope0 = D - a.rho;
     __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out) + ((size_t)b * a.Hq + (size_t)g * NH) * D;
-    for (int u = tid; u < SW * (NH / 4); u += kThreads) {  // SW * 16 is a multiple of 256: no divergence
-        const int dd = u % SW, h4 = u / SW;
-        const int d = rank * SW + dd;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int r = 0; r < CS; ++r) {
-            const float4 x = *reinterpret_cast<const float4*>(recv + (((size_t)r * (NH / 4) + h4) * SW + dd) * 4);
-            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-        }
-        float4 p;  // the pair partner: pairs (d, d + 1) sit in lanes (2i, 2i + 1)
-        p.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
-        p.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
-        p.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
-        p.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
-        if (a.shared && a.rho > 0 && d >= rope0) {
-            const float2 c = cs[(d - rope0) >> 1];
-            if ((d & 1) == 0) {  // x' = x c + y s
-                acc.x = acc.x * c.x + p.x * c.y; acc.y = acc.y * c.x + p.y * c.y;
-                acc.z = acc.z * c.x + p.z * c.y; acc.w = acc.w * c.x + p.w * c.y;
-            } else {             // y' = y c - x s
-                acc.x = acc.x * c.x - p.x * c.y; acc.y = acc.y * c.x - p.y * c.y;
-                acc.z = acc.z * c.x - p.z * c.y; acc.w = acc.w * c.x - p.w * c.y;
+    if (single) {
+        // ---- the whole list was this CTA's: normalise and write straight from TMEM ----
+        if (rank == 0) {
+            if (tid < NH) {
+                const float M = mh[tid];
+                float dn = lloc[tid];
+                if (a.sink && M != kNegInf) dn += ex2(sink_l2 - M);
+                den[tid] = dn;
+            }
+            __syncthreads();
+#pragma unroll 1
+            for (int mt = 0; mt < D / 128; ++mt) {
+                float o[16];
+                if (have_o) {
+                    tmem_ld16(tbase + lane_f + NH + NH * mt + 16 * hq, o);
+                    tmem_wait_ld();
+                }
+                const int d = 128 * mt + 32 * quad + lane;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float dn = den[16 * hq + i];
+                    float x = (have_o && dn > 0.f) ? o[i] / dn : 0.f;
+                    const float y = __shfl_xor_sync(0xffffffffu, x, 1);  // pair partner (d ^ 1)
+                    if (a.rho > 0 && d >= rope0) {
+                        const float2 c = cs[(d - rope0) >> 1];
+                        x = (d & 1) == 0 ? x * c.x + y * c.y : x * c.x - y * c.y;
+                    }
+                    outp[(size_t)(16 * hq + i) * D + d] = __float2bfloat16_rn(x);
+                }
             }
         }
-        outp[(size_t)(4 * h4 + 0) * D + d] = __float2bfloat16_rn(acc.x);
-        outp[(size_t)(4 * h4 + 1) * D + d] = __float2bfloat16_rn(acc.y);
-        outp[(size_t)(4 * h4 + 2) * D + d] = __float2bfloat16_rn(acc.z);
-        outp[(size_t)(4 * h4 + 3) * D + d] = __float2bfloat16_rn(acc.w);
+    } else {
+        // ---- fp16 O^T slices to their owners, with this CTA's sums ----
+        uint8_t* stage = smem + lay.OFF_E;  // [owner][NH/4][SW][4] fp16
+#pragma unroll 1
+        for (int mt = 0; mt < D / 128; ++mt) {
+            float o[16];
+            if (have_o) {
+                tmem_ld16(tbase + lane_f + NH + NH * mt + 16 * hq, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = 0.f;
+            }
+            const int d = 128 * mt + 32 * quad + lane;
+            const int owner = d / SW, dd = d - owner * SW;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int h4 = 4 * hq + j;
+                uint2 w2;
+                w2.x = pack_f16x2(o[4 * j + 0], o[4 * j + 1]);
+                w2.y = pack_f16x2(o[4 * j + 2], o[4 * j + 3]);
+                *reinterpret_cast<uint2*>(stage + (size_t)owner * lay.SLICE + ((size_t)h4 * SW + dd) * 8) = w2;
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid < CS) {
+            const uint32_t rb = peer_addr(bar_r, tid);
+            bulk_to_peer(peer_addr(sQ + (uint32_t)rank * lay.SLICE, tid), smem_addr(stage) + tid * lay.SLICE,
+                         lay.SLICE, rb);
+            const uint32_t lo = smem_addr(smem + lay.OFF_LRECV) + (uint32_t)rank * NH * 4u;
+            bulk_to_peer(peer_addr(lo, tid), smem_addr(lloc), NH * 4u, rb);
+            bulk_commit();
+        }
+        // ---- owner: add the CS slices, normalise, rotate back, write ----
+        const bool ok3 = __syncthreads_and(mbar_wait(&bars[3], 0, kWaitNs));
+        if (!ok3 && tid == 0) set_status(a.status, LBCA_ERR_TIMEOUT);
+        if (tid < NH) {
+            const float M = mh[tid];
+            float dn = 0.f;
+            for (int r = 0; r < CS; ++r) dn += lrecv[r * NH + tid];
+            if (a.sink && M != kNegInf) dn += ex2(sink_l2 - M);
+            den[tid] = dn;
+        }
+        __syncthreads();
+        const uint8_t* recv = smem + lay.OFF_Q;  // [src][NH/4][SW][4] fp16
+        for (int u = tid; u < SW * (NH / 4); u += kThreads) {  // whole warps: SW * 16 is a multiple of 32
+            const int h4 = u / SW, dd = u - h4 * SW;
+            const int d = rank * SW + dd;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ok3 && d < D) {
+                for (int r = 0; r < CS; ++r) {
+                    const uint2 w2 = *reinterpret_cast<const uint2*>(recv + (size_t)r * lay.SLICE +
+                                                                     ((size_t)h4 * SW + dd) * 8);
+                    const float2 p0 = unpack_f16x2(w2.x), p1 = unpack_f16x2(w2.y);
+                    acc[0] += p0.x; acc[1] += p0.y; acc[2] += p1.x; acc[3] += p1.y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float dn = den[4 * h4 + j];
+                float x = dn > 0.f ? acc[j] / dn : 0.f;
+                const float y = __shfl_xor_sync(0xffffffffu, x, 1);  // pair partner (d ^ 1)
+                if (a.rho > 0 && d >= rope0 && d < D) {
+                    const float2 c = cs[(d - rope0) >> 1];
+                    x = (d & 1) == 0 ? x * c.x + y * c.y : x * c.x - y * c.y;
+                }
+                if (d < D) outp[(size_t)(4 * h4 + j) * D + d] = __float2bfloat16_rn(x);
+            }
+        }
+        if (tid < CS) bulk_wait_read_all();  // the staging is read out before this CTA exits
     }
+    if (q_sender) bulk_wait_read_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
-// Largest cluster size (16, else 8) this kernel can be scheduled with, cached.
+// How many CS-CTA clusters of this kernel fit on the device at once with `smem`
+// bytes of shared memory per CTA (0: none).  Cached per cluster size.
 template <int D>
-int max_cluster() {
-    static int best = -1;
-    if (best >= 0) return best;
+int max_active_clusters(int cs, uint32_t smem) {
     auto fn = decode_mqa_tc_kernel<D>;
-    best = 0;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, MqaLayout<D>::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-        cudaGetLastError();
-        return best;
-    }
-    for (int cs : {16, 8, 4, 2, 1}) {
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = cs;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(cs, 1, 1);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = MqaLayout<D>::SMEM;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int nclu = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclu, fn, &cfg) == cudaSuccess && nclu > 0) {
-            best = cs;
-            break;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
         }
-        cudaGetLastError();
+        attr = true;
     }
-    return best;
+    static uint32_t key[kMaxCS + 1];
+    static int val[kMaxCS + 1];
+    if (key[cs] == smem) return val[cs];
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(cs, 1, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int nclu = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclu, fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        nclu = 0;
+    }
+    key[cs] = smem;
+    val[cs] = nclu;
+    return nclu;
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
     auto fn = decode_mqa_tc_kernel<D>;
+    const MqaLayout lay(D, a.chunk, a.tc_cs);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -498,7 +578,7 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(a.tc_cs, a.G, a.B);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = MqaLayout<D>::SMEM;
+    cfg.dynamicSmemBytes = lay.SMEM;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -507,17 +587,31 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-int plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
-    if (dtype != LBCA_BF16 || !shared || G < 1 || Hq != NH * G || (D != 256 && D != 512)) return 0;
-    if (B < 1 || max_ctx < 1) return 0;
+MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
+    MqaTcPlan p{0, 0};
+    if (dtype != LBCA_BF16 || !shared || G < 1 || Hq != NH * G || (D != 256 && D != 512)) return p;
+    if (B < 1 || max_ctx < 1) return p;
     const long long P = max_ctx - w > 0 ? (long long)(max_ctx - w) / m : 0;
     const long long max_vis = std::min<long long>(max_ctx, P + w + m - 1);
-    const int cap = D == 512 ? max_cluster<512>() : max_cluster<256>();
-    int cs = 1;
-    while ((long long)cs * TE < max_vis) cs *= 2;
-    if (cs > cap) return 0;
-    while (cs < cap && (long long)B * G * cs < 148) cs *= 2;  // spread short batches over the SMs
-    return cs;
+    const int cs_min = (int)std::max<long long>(1, (max_vis + 127) / 128);
+    if (cs_min > kMaxCS) return p;
+    // fewest waves of clusters first, then the widest cluster (the most SMs streaming)
+    const long long groups = (long long)B * G;
+    long long best_waves = 0;
+    for (int cs = kMaxCS; cs >= cs_min; --cs) {
+        const int rows = std::max<int>(16, (int)(((max_vis + cs - 1) / cs + 15) / 16 * 16));
+        const MqaLayout lay(D, rows, cs);
+        if (lay.SMEM > 227u * 1024u) continue;
+        const int act = D == 512 ? max_active_clusters<512>(cs, lay.SMEM) : max_active_clusters<256>(cs, lay.SMEM);
+        if (act < 1) continue;
+        const long long waves = (groups + act - 1) / act;
+        if (p.cs == 0 || waves < best_waves) {
+            p.cs = cs;
+            p.rows = rows;
+            best_waves = waves;
+        }
+    }
+    return p;
 }
 
 cudaError_t launch_decode_mqa_tc(const DecodeArgs& a, cudaStream_t s) {

@@ -94,8 +94,12 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int G, int D, int m, int w, int
 size_t decode_workspace_bytes(const DecodePlan& p);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 // Tensor-core decode of the shared-entry form (bf16, 64 query heads per kv head,
-// D in {256, 512}): the cluster size for this call, or 0 when it does not apply.
-int plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+// D in {256, 512}): CTAs per cluster (0 when the kernel does not apply) and
+// entry rows per CTA.  Launch with DecodeArgs.tc_cs = cs and .chunk = rows.
+struct MqaTcPlan {
+    int cs, rows;
+};
+MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
 cudaError_t launch_decode_mqa_tc(const DecodeArgs& a, cudaStream_t s);
 
 // One serving step (append + decode) in one cluster launch.

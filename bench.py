@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gqa_decode_32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--leg", default="decode", choices=["decode", "prefill", "pool"],
+                    help="decode: the decode-step benchmark (default, with the prefill and pool legs appended); "
+                         "prefill / pool: that leg alone (one JSON line)")
     return ap.parse_args()
 
 
@@ -134,7 +137,7 @@ class DecodeBench:
         import torch
 
         from block_compressed_long_b200 import lbca as L
-        from block_compressed_long_b200 import synth
+        from block_compressed_long_b200 import ranks, synth
         self.L, self.torch = L, torch
         l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
         base = synth.scaled(w, steps=1)
@@ -142,7 +145,7 @@ class DecodeBench:
         step_bytes = bytes_per_decode(base, lens0 + 1)
         self.NR = max(1, -(-3 * l2 // step_bytes))
         self.local_steps = -(-min_steps // self.NR) + 1
-        self.w = synth.scaled(w, steps=self.local_steps, seed=w.seed + 7919 * rank)
+        self.w = synth.scaled(ranks.rank_workload(w, rank), steps=self.local_steps)
         self.inp = synth.make(self.w)
         w = self.w
         self.cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win,
@@ -215,6 +218,8 @@ class DecodeBench:
 def run_ours(args, w, rank, world):
     import torch
     import torch.distributed as dist
+
+    from block_compressed_long_b200 import ranks
 
     K, W = args.steps, args.warmup
     bench = DecodeBench(w, rank, 2 * (W + K))
@@ -313,16 +318,13 @@ def run_ours(args, w, rank, world):
     if status:
         raise RuntimeError(f"device status {L.lbca_status_string(status)}")
 
-    t = torch.tensor([step_ms, e2e_ms, kernel_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms, kernel_ms = t.tolist()
-    tokens = bench.B * world
+    step_ms, e2e_ms, kernel_ms = ranks.max_over_ranks([step_ms, e2e_ms, kernel_ms], device="cuda")
     hbm, src = peaks()
     achieved = nbytes / K / (kernel_ms * 1e-3) / 1e9
     w_ = bench.w
     line = {
-        "metric": METRIC, "value": step_ms * 1e3 / tokens, "unit": "µs/token", "n_gpus": world,
+        "metric": METRIC, "value": ranks.job_us_per_token(step_ms, bench.B, world), "unit": "µs/token",
+        "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
         "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
@@ -339,7 +341,8 @@ def run_ours(args, w, rank, world):
                                 "the decode launch of the step (timed alone over the same replicas)"),
                      "bytes_per_launch": nbytes / K, "launch_us": kernel_ms * 1e3,
                      "traffic": load_traffic(w_.name)},
-        "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "µs/token", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": ranks.job_us_per_token(e2e_ms, bench.B, world), "unit": "µs/token",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": K * bench.launches,
         "clocks": clocks,
@@ -365,7 +368,7 @@ def prefill_flops(w):
     return 4.0 * w.head_dim * w.n_q_heads * pairs * w.batch
 
 
-def extra_prefill(reps=10):
+def extra_prefill(reps=10, warm=3):
     """lbca_prefill of the 16K-token GQA layer (pool pass, RoPE table, finalised
     keys, tensor-core attention), inputs resident (> L2), CUDA events."""
     import torch
@@ -382,7 +385,7 @@ def extra_prefill(reps=10):
     ws = torch.zeros(L.lbca_prefill_workspace_bytes(cfg, w.batch, w.seq_len, False), dtype=torch.uint8,
                      device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for _ in range(3):
+    for _ in range(warm):
         L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, out, None, ws, d_status=st)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -404,7 +407,7 @@ def extra_prefill(reps=10):
                          "flops_per_call": fl}}
 
 
-def extra_pool(reps=10):
+def extra_pool(reps=10, warm=3):
     """lbca_pool of both series of the 32K-token GQA prefix (HBM-bound)."""
     import torch
 
@@ -424,7 +427,7 @@ def extra_pool(reps=10):
         L.lbca_pool(cfg, L.LBCA_KEY, k, zk, bpk, None, ok_)
         L.lbca_pool(cfg, L.LBCA_VALUE, v, zv, bpv, None, ov_)
 
-    for _ in range(3):
+    for _ in range(warm):
         run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -497,9 +500,8 @@ def oracle_decode_timing(w, budget_s=12.0, max_steps=None):
 
 def main():
     args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    from block_compressed_long_b200 import synth
+    from block_compressed_long_b200 import ranks, synth
+    rank, world, local_rank = ranks.from_env()
     w = synth.WORKLOADS[args.workload]
     if w.kind != "decode":
         raise SystemExit("bench.py times decode workloads; prefill is timed by its own leg")
@@ -521,12 +523,17 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     else:
         torch.cuda.set_device(0)
     import __graft_entry__
     __graft_entry__.build()
+    if args.leg != "decode":  # one leg alone, on this GPU
+        if rank == 0:
+            leg = extra_prefill if args.leg == "prefill" else extra_pool
+            print(json.dumps(leg(reps=args.steps, warm=args.warmup)), flush=True)
+        return
     line, _ = run_ours(args, w, rank, world)
     if world == 1 and args.workload == "gqa_decode_32k":
         line["also"] = [extra_prefill(), extra_pool()]

@@ -12,8 +12,9 @@
 // thread owns one 16-byte vector of channels (8 bf16 / 4 f32) of the G*D row,
 // so every token row is read with fully coalesced 128-bit streaming loads.
 // The per-channel softmax runs online in registers, four tokens per step with
-// the next four already in flight, one rescale per step and base-2
-// exponentials on the SFU.  RMSNorm needs a per-head reduction, done
+// the loads of a step issued together, one rescale per step and base-2
+// exponentials on the SFU.  Registers are kept low enough that a whole launch
+// of the common shapes is resident at once (memory parallelism from warps).  RMSNorm needs a per-head reduction, done
 // deterministically through shared memory.
 #include <algorithm>
 
@@ -69,7 +70,7 @@ __device__ __forceinline__ void finalise_key(float (&e)[VEC], int d0, int D, boo
 
 // CTA = (block j, sequence b, slice of whole kv heads); <= 256 threads.
 template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     constexpr int VEC = Vec<T>::N;
     constexpr int U = 4;  // tokens per online-softmax step
     extern __shared__ __align__(16) float smem[];
@@ -98,24 +99,19 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
     for (int e = 0; e < VEC; ++e) { mx[e] = kNegInf; l[e] = 0.f; acc[e] = 0.f; }
 
     if (active) {
-        uint4 cx[U], cz[U], cb[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (u < n_tok) {
-                cx[u] = __ldcs(xp + (size_t)u * rstride);
-                cz[u] = __ldcs(zp + (size_t)u * rstride);
-                cb[u] = __ldg(bp + (size_t)u * rstride);
-            }
+        // U tokens per step: their X, Z and B_pos vectors are loaded together
+        // (12 x 16 bytes in flight per thread), then one rescale and U
+        // accumulations.  Memory parallelism comes from many resident warps
+        // (few registers per thread) rather than from a register prefetch.
         for (int i0 = 0; i0 < n_tok; i0 += U) {
-            uint4 nx[U], nz[U], nb[U];
+            uint4 cx[U], cz[U], cb[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (i0 + U + u < n_tok) {
-                    nx[u] = __ldcs(xp + (size_t)(i0 + U + u) * rstride);
-                    nz[u] = __ldcs(zp + (size_t)(i0 + U + u) * rstride);
-                    nb[u] = __ldg(bp + (size_t)(i0 + U + u) * rstride);
+                if (i0 + u < n_tok) {
+                    cx[u] = __ldcs(xp + (size_t)(i0 + u) * rstride);
+                    cz[u] = __ldcs(zp + (size_t)(i0 + u) * rstride);
+                    cb[u] = __ldg(bp + (size_t)(i0 + u) * rstride);
                 }
-            float av[U][VEC];
             float cmax[VEC];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) cmax[e] = mx[e];
@@ -126,10 +122,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
                     unpack<T>(cz[u], zf);
                     unpack<T>(cb[u], bf);
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) {
-                        av[u][e] = (zf[e] + bf[e]) * kLog2e;
-                        cmax[e] = fmaxf(cmax[e], av[u][e]);
-                    }
+                    for (int e = 0; e < VEC; ++e) cmax[e] = fmaxf(cmax[e], (zf[e] + bf[e]) * kLog2e);
                 }
             }
 #pragma unroll
@@ -142,18 +135,18 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (i0 + u < n_tok) {
-                    float xf[VEC];
+                    float xf[VEC], zf[VEC], bf[VEC];
                     unpack<T>(cx[u], xf);
+                    unpack<T>(cz[u], zf);
+                    unpack<T>(cb[u], bf);
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) {
-                        const float p = ex2(av[u][e] - mx[e]);
+                        const float p = ex2((zf[e] + bf[e]) * kLog2e - mx[e]);
                         l[e] += p;
                         acc[e] = fmaf(p, xf[e], acc[e]);
                     }
                 }
             }
-#pragma unroll
-            for (int u = 0; u < U; ++u) { cx[u] = nx[u]; cz[u] = nz[u]; cb[u] = nb[u]; }
         }
     }
 

@@ -96,6 +96,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* f
     return __all_sync(0xffffffffu, wait_or_fail(bar, parity, fail, status));
 }
 
+// The K/V tiles of a CTA run over the pooled entries [0, npt BN) and then the
+// raw band [s_lo, t_last]; query tile q needs only a prefix of the pooled
+// tiles and a sub-range of the raw tiles.  Tiles no row of q can see are not
+// multiplied for q at all.
+struct Need {
+    int np;      // pooled tiles [0, np)
+    int r0, r1;  // raw tiles [npt + r0, npt + r1)
+    __device__ bool operator()(int i, int npt) const {
+        return i < npt ? i < np : (i - npt >= r0 && i - npt < r1);
+    }
+};
+__device__ __forceinline__ Need need_of(const TcArgs& a, int q, int t0, int s_lo, int nrt) {
+    Need n{0, 0, 0};
+    const int tf = t0 + q * BM;
+    if (tf >= a.T) return n;
+    const int tl = min(tf + BM, a.T) - 1;
+    n.np = (visible_blocks(tl + 1, a.m, a.w) + BN - 1) / BN;
+    const int lo = visible_blocks(tf + 1, a.m, a.w) * a.m;  // >= s_lo
+    n.r0 = (lo - s_lo) / BN;
+    n.r1 = min(nrt, tl >= s_lo ? (tl - s_lo) / BN + 1 : 0);
+    n.r1 = max(n.r1, n.r0);
+    return n;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -164,8 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        // order: S0(0) S1(0) | PV0(i) S0(i+1) PV1(i) S1(i+1) | ...  P_q(i) lives in
-        // S_q's TMEM columns, so S_q(i+1) waits until PV_q(i) has read it.
+        // order per K/V tile i: S_q(i) for the query tiles that need it (unless
+        // issued ahead), then PV_q(i) and at once S_q(i+1).  P_q(i) lives in
+        // S_q's TMEM columns, so S_q(i+1) waits until PV_q(i) has read it; a
+        // query tile skips the tiles none of its rows can see.
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
@@ -180,37 +206,53 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                                 smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
                 tc_commit(&bars[B_SFULL + q]);
             };
-            auto issue_pv = [&](int q, int i) {
+            auto issue_pv = [&](int q, int i, bool acc) {
                 const int s = i % NSTAGE;
                 const uint32_t sv = smem_addr(smem + OFF_V + s * KTILE);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)  // A = P_q(i): 8 fp16x2 columns per 16 entries
                     tc_mma_ts(tbase + 256 * q + 128, tbase + 256 * q + kk * 8,
-                              smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (i > 0 || kk > 0) ? 1u : 0u);
+                              smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (acc || kk > 0) ? 1u : 0u);
                 tc_commit(&bars[B_ODONE + q]);
             };
+            Need nd[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) nd[q] = need_of(a, q, t0, s_lo, nrt);
+            int npv[NQ] = {0, 0};    // P V products issued per query tile (its ODONE phases)
+            int s_at[NQ] = {-1, -1}; // tile of the latest S issued per query tile
             bool ok = true;
             for (int q = 0; ok && q < NQ; ++q) ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
-            if (ok && ntile > 0) {
-                ok = wait_or_fail(&bars[B_KFULL], 0, fail, a.status);
-                if (ok) { issue_s(0, 0); issue_s(1, 0); }
-            }
             for (int i = 0; ok && i < ntile; ++i) {
-                const int s = i % NSTAGE, n = i + 1, sn = n % NSTAGE;
-                ok = wait_or_fail(&bars[B_VFULL + s], (i / NSTAGE) & 1, fail, a.status);
-                const bool more = n < ntile;
-                for (int q = 0; ok && q < NQ; ++q) {
-                    ok = wait_or_fail(&bars[B_PFULL + q], i & 1, fail, a.status);
+                const int s = i % NSTAGE;
+                const uint32_t ph = (i / NSTAGE) & 1;
+                bool any = false;
+                for (int q = 0; ok && q < NQ; ++q) {  // S_q(i), unless issued ahead
+                    if (!nd[q](i, npt)) continue;
+                    any = true;
+                    if (s_at[q] == i) continue;
+                    ok = wait_or_fail(&bars[B_KFULL + s], ph, fail, a.status);
+                    if (ok && npv[q] > 0) ok = wait_or_fail(&bars[B_ODONE + q], (npv[q] - 1) & 1, fail, a.status);
+                    if (ok) { issue_s(q, i); s_at[q] = i; }
+                }
+                if (!ok) break;
+                // the stage's data must have landed before it is released
+                ok = wait_or_fail(&bars[B_VFULL + s], ph, fail, a.status);
+                if (ok && !any) ok = wait_or_fail(&bars[B_KFULL + s], ph, fail, a.status);
+                for (int q = 0; ok && any && q < NQ; ++q) {
+                    if (!nd[q](i, npt)) continue;
+                    ok = wait_or_fail(&bars[B_PFULL + q], npv[q] & 1, fail, a.status);
                     if (!ok) break;
-                    issue_pv(q, i);
-                    if (q == NQ - 1) tc_commit(&bars[B_KVEMPTY + s]);
-                    if (more) {  // S_q(i+1) needs the next K tile and P_q(i) consumed
-                        if (q == 0) ok = wait_or_fail(&bars[B_KFULL + sn], (n / NSTAGE) & 1, fail, a.status);
-                        if (ok) ok = wait_or_fail(&bars[B_ODONE + q], i & 1, fail, a.status);
-                        if (ok) issue_s(q, n);
+                    issue_pv(q, i, npv[q] > 0);
+                    ++npv[q];
+                    const int n = i + 1;
+                    if (n < ntile && nd[q](n, npt)) {  // S_q(i+1) as soon as P_q(i) is consumed
+                        ok = wait_or_fail(&bars[B_KFULL + n % NSTAGE], (n / NSTAGE) & 1, fail, a.status);
+                        if (ok) ok = wait_or_fail(&bars[B_ODONE + q], (npv[q] - 1) & 1, fail, a.status);
+                        if (ok) { issue_s(q, n); s_at[q] = n; }
                     }
                 }
+                if (ok) tc_commit(&bars[B_KVEMPTY + s]);
             }
         }
     } else if (warp >= 4) {
@@ -257,10 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
         const float sc = a.scale * kLog2e;  // scores enter the exponent as s * sc (log2 units)
         float m_ref = kNegInf, l = 0.f;     // running max (unscaled score units) and sum
+        const Need nd = need_of(a, q, t0, s_lo, nrt);
+        int k = 0;                          // tiles of this query tile so far
         for (int i = 0; ok && i < ntile; ++i) {
+            if (!nd(i, npt)) continue;      // uniform over the warpgroup
             const bool pooled = i < npt;
             const int base = pooled ? i * BN : s_lo + (i - npt) * BN;
-            ok = warp_wait(&bars[B_SFULL + q], i & 1, fail, a.status);
+            ok = warp_wait(&bars[B_SFULL + q], k & 1, fail, a.status);
+            ++k;
             if (!ok) break;
             tc_fence_after();
             float s[BN];
@@ -333,12 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         // ---- epilogue: normalise the O row into this query tile's shared memory
         // (free: the last S MMA that read Q is complete), then TMA-store the tile
-        if (ok && ntile > 0) ok = warp_wait(&bars[B_ODONE + q], (ntile - 1) & 1, fail, a.status);
+        if (ok && k > 0) ok = warp_wait(&bars[B_ODONE + q], (k - 1) & 1, fail, a.status);
         tc_fence_after();
         float den = l;
         if (a.sink) den += m_ref == kNegInf ? 1.f : ex2(a.sink[h] * kLog2e - m_ref * sc);
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        const bool have_o = ok && ntile > 0;  // warp-uniform
+        const bool have_o = ok && k > 0;  // warp-uniform
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
             float v[32];

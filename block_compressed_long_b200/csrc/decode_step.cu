@@ -67,6 +67,34 @@ template <> __device__ __forceinline__ void put2<float>(float* p, float a, float
 template <> __device__ __forceinline__ void put2<__nv_bfloat16>(__nv_bfloat16* p, float a, float b) {
     *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
 }
+// Two consecutive I/O elements, loaded as raw bits (so that the load can be
+// issued early and converted where it is used).
+template <typename T> struct Pair;
+template <> struct Pair<float> {
+    using Raw = float2;
+    static __device__ __forceinline__ Raw load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+    static __device__ __forceinline__ float2 cvt(Raw r) { return r; }
+};
+template <> struct Pair<__nv_bfloat16> {
+    using Raw = uint32_t;
+    static __device__ __forceinline__ Raw load(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+    static __device__ __forceinline__ float2 cvt(Raw w) {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+};
+template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float (&o)[Vec<T>::N]);
+template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, float (&o)[4]) {
+    o[0] = __uint_as_float(u.x); o[1] = __uint_as_float(u.y); o[2] = __uint_as_float(u.z); o[3] = __uint_as_float(u.w);
+}
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float (&o)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o[2 * i] = __uint_as_float(w[i] << 16);
+        o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
 template <typename T>
 __device__ __forceinline__ float2 get2(const T* p) {
     return make_float2(to_f<T>(p[0]), to_f<T>(p[1]));
@@ -128,6 +156,37 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     const int g = h0 / r;
     const int GD = a.G * D;
     const int DS = D / CS;  // dims this CTA finalises
+
+    // ---- loads that do not depend on the length go out first ----
+    const bool app = rank == 0 && h0 % r == 0;  // the CTA that appends for (sequence, kv head)
+    const bool pair_owner = tid < D / 2;
+    constexpr int QV = (R * D / VEC + kThreads - 1) / kThreads;
+    uint4 qv[QV];
+#pragma unroll
+    for (int j = 0; j < QV; ++j) {
+        const int idx = tid + j * kThreads;
+        if (idx < R * D / VEC)
+            qv[j] = *reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((size_t)b * a.Hq + h0 + idx / (D / VEC)) * D +
+                                                    (idx % (D / VEC)) * VEC);
+    }
+    const size_t tok = (size_t)b * GD + (size_t)g * D + 2 * tid;  // this thread's pair of the new token
+    typename Pair<T>::Raw kraw{}, vraw{}, zraw[2]{};
+    float2 am[2], al_[2], aa[2];  // running pooling state of the open block
+    if (pair_owner) {
+        kraw = Pair<T>::load(static_cast<const T*>(a.k) + tok);
+        if (!a.shared) vraw = Pair<T>::load(static_cast<const T*>(a.v) + tok);
+        if (app) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {  // series: key (or shared entry), value
+                if (s >= a.S) break;
+                zraw[s] = Pair<T>::load(static_cast<const T*>(s == 0 ? a.zk : a.zv) + tok);
+                const float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
+                am[s] = *reinterpret_cast<const float2*>(st);
+                al_[s] = *reinterpret_cast<const float2*>(st + GD);
+                aa[s] = *reinterpret_cast<const float2*>(st + 2 * GD);
+            }
+        }
+    }
 
     // ---- the step: token t = L_old joins, the query sits at t ----
     if (tid == 0) {
@@ -197,40 +256,32 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         }
     }
 
-    // ---- the appending CTA (one per sequence and kv head) prefetches its inputs ----
-    const bool app = rank == 0 && h0 % r == 0;
-    const bool pair_owner = tid < D / 2;
+    // ---- the appending CTA: B_pos row of the new token's offset in its block ----
     const int ai = t % a.m, aj = t / a.m;
-    float2 ax[2], az[2], abp[2], am[2], al_[2], aa[2];
-    if (app && pair_owner) {
-        for (int s = 0; s < a.S; ++s) {
-            const bool key = s == 0;
-            const size_t off = (size_t)b * GD + (size_t)g * D + 2 * tid;
-            ax[s] = get2(static_cast<const T*>(key ? a.k : a.v) + off);
-            az[s] = get2(static_cast<const T*>(key ? a.zk : a.zv) + off);
-            abp[s] = get2(static_cast<const T*>(key ? a.bpk : a.bpv) + (size_t)ai * GD + (size_t)g * D + 2 * tid);
-            if (ai > 0) {
-                const float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
-                am[s] = *reinterpret_cast<const float2*>(st);
-                al_[s] = *reinterpret_cast<const float2*>(st + GD);
-                aa[s] = *reinterpret_cast<const float2*>(st + 2 * GD);
-            }
-        }
-    }
+    float2 abp[2];
+    if (app && pair_owner)
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+            if (s < a.S) abp[s] = get2(static_cast<const T*>(s == 0 ? a.bpk : a.bpv) + (size_t)ai * GD + (size_t)g * D + 2 * tid);
 
     // ---- query prep and the newest raw row, overlapping the copies ----
     for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((int64_t)t, k, a.rope_step);
-    for (int idx = tid; idx < R * D / VEC; idx += kThreads) {
-        const int h = idx / (D / VEC), c = idx % (D / VEC);
-        float v[VEC];
-        ld16(static_cast<const T*>(a.q) + ((size_t)b * a.Hq + h0 + h) * D + c * VEC, v);
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) qs[h * D + c * VEC + i] = v[i];
+    for (int j = 0; j < QV; ++j) {
+        const int idx = tid + j * kThreads;
+        if (idx < R * D / VEC) {
+            float v[VEC];
+            unpack16<T>(qv[j], v);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) qs[(idx / (D / VEC)) * D + (idx % (D / VEC)) * VEC + i] = v[i];
+        }
     }
+    float2 kraw_f = make_float2(0.f, 0.f);  // the new raw key before RMSNorm / RoPE (pooled raw)
     float2 kx = make_float2(0.f, 0.f), vx = kx;
     if (pair_owner) {
-        kx = get2(static_cast<const T*>(a.k) + (size_t)b * GD + (size_t)g * D + 2 * tid);
-        if (!a.shared) vx = get2(static_cast<const T*>(a.v) + (size_t)b * GD + (size_t)g * D + 2 * tid);
+        kx = Pair<T>::cvt(kraw);
+        kraw_f = kx;
+        if (!a.shared) vx = Pair<T>::cvt(vraw);
     }
     __syncthreads();  // cs, qs ready
     {
@@ -265,6 +316,69 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         rotate_pair(qs[h * D + d], qs[h * D + d + 1], cs[k]);
     }
     __syncthreads();
+
+    // ---- append the new token (one CTA per (sequence, kv head)) while the copies
+    // land: running pooling softmax, block finalisation, ring write.  Nothing
+    // it writes is visible to this step (the ring slot of t holds token t - R,
+    // the block it may complete becomes visible n_win tokens later).
+    if (app) {
+        const bool complete = ai == a.m - 1;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            if (s >= a.S) break;
+            const bool key = s == 0;
+            float mxs[2] = {0.f, 0.f}, lss[2] = {1.f, 1.f}, acs[2] = {0.f, 0.f};
+            if (pair_owner) {
+                const float2 xs = key ? kraw_f : vx, zs = Pair<T>::cvt(zraw[s]);
+                const float xv[2] = {xs.x, xs.y};
+                const float av[2] = {(zs.x + abp[s].x) * kLog2e, (zs.y + abp[s].y) * kLog2e};
+                const float m0[2] = {am[s].x, am[s].y}, l0[2] = {al_[s].x, al_[s].y}, a0[2] = {aa[s].x, aa[s].y};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (ai == 0) {
+                        mxs[e] = av[e]; lss[e] = 1.f; acs[e] = xv[e];
+                    } else {
+                        const float mn = fmaxf(m0[e], av[e]);
+                        const float rr = ex2(m0[e] - mn), p = ex2(av[e] - mn);
+                        mxs[e] = mn; lss[e] = l0[e] * rr + p; acs[e] = fmaf(p, xv[e], a0[e] * rr);
+                    }
+                }
+            }
+            float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
+            if (complete) {  // uniform across the CTA
+                float e0v = acs[0] / lss[0], e1v = acs[1] / lss[1];
+                const float ss = (key && a.rmsnorm)
+                                     ? block_sum(pair_owner ? e0v * e0v + e1v * e1v : 0.f, scratch) : 0.f;
+                if (key && a.rmsnorm) {
+                    const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+                    const T* gm = static_cast<const T*>(a.gamma_kv);
+                    e0v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid]) : 1.f);
+                    e1v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid + 1]) : 1.f);
+                }
+                if (key && a.rho && pair_owner && 2 * tid >= D - a.rho)
+                    rotate_pair(e0v, e1v, rope_cs((int64_t)aj * a.m, (2 * tid - (D - a.rho)) >> 1, a.rope_step));
+                if (pair_owner) {
+                    if (aj < a.max_blocks)
+                        put2<T>(static_cast<T*>(key ? a.pooled_k : a.pooled_v) +
+                                    (((size_t)b * a.G + g) * a.max_blocks + aj) * D + 2 * tid,
+                                e0v, e1v);
+                    else
+                        set_status(a.status, LBCA_ERR_CAPACITY);
+                }
+            } else if (pair_owner) {
+                *reinterpret_cast<float2*>(st) = make_float2(mxs[0], mxs[1]);
+                *reinterpret_cast<float2*>(st + GD) = make_float2(lss[0], lss[1]);
+                *reinterpret_cast<float2*>(st + 2 * GD) = make_float2(acs[0], acs[1]);
+            }
+            if (pair_owner) {  // ring slot of token t: the finalised key row, or the raw value
+                T* dst = static_cast<T*>(key ? a.ring_k : a.ring_v) +
+                         (((size_t)b * a.G + g) * a.R + (t % a.R)) * D + 2 * tid;
+                const T* src = (key ? newk : newv) + 2 * tid;
+                dst[0] = src[0];
+                dst[1] = src[1];
+            }
+        }
+    }
 
     const int gl = lane % LG;
     const float qscale = a.scale * kLog2e;
@@ -435,19 +549,34 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     }
     cluster.sync();  // every slice has landed; nothing remote is read after this
 
-    // ---- this CTA finalises dims [rank*DS, (rank+1)*DS) of its heads ----
-    for (int idx = tid; idx < R * DS / 2; idx += kThreads) {
-        const int h = idx / (DS / 2), dl = (idx % (DS / 2)) * 2, d = rank * DS + dl;
+    // ---- this CTA finalises dims [rank*DS, (rank+1)*DS) of its heads: GS threads
+    // per output pair, each over every GS-th rank, joined by shuffles ----
+    constexpr int GS = 4;
+    const int items = R * (DS / 2) * GS;
+    for (int base = 0; base < items; base += kThreads) {  // every thread runs every round
+        const int idx = base + tid;
+        const bool act = idx < items;
+        const int pr = act ? idx / GS : 0, sub = idx % GS;
+        const int h = pr / (DS / 2), dl = (pr % (DS / 2)) * 2, d = rank * DS + dl;
         float M = kNegInf;
-        for (int q = 0; q < CS; ++q) M = fmaxf(M, recv_ml[(q * R + h) * 2]);
+        for (int q = sub; q < CS; q += GS) M = fmaxf(M, recv_ml[(q * R + h) * 2]);
+#pragma unroll
+        for (int off = 1; off < GS; off <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float Ls = 0.f, o0 = 0.f, o1 = 0.f;
         if (M != kNegInf)
-            for (int q = 0; q < CS; ++q) {
+            for (int q = sub; q < CS; q += GS) {
                 const float f = ex2(recv_ml[(q * R + h) * 2] - M);
                 Ls = fmaf(recv_ml[(q * R + h) * 2 + 1], f, Ls);
                 o0 = fmaf(recv_o[(q * R + h) * DS + dl], f, o0);
                 o1 = fmaf(recv_o[(q * R + h) * DS + dl + 1], f, o1);
             }
+#pragma unroll
+        for (int off = 1; off < GS; off <<= 1) {
+            Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+            o0 += __shfl_xor_sync(0xffffffffu, o0, off);
+            o1 += __shfl_xor_sync(0xffffffffu, o1, off);
+        }
+        if (!act || sub != 0) continue;
         float den = Ls;
         if (a.sink) den += (M == kNegInf) ? 1.0f : ex2(a.sink[h0 + h] * kLog2e - M);
         float v0 = den > 0.f ? o0 / den : 0.f, v1 = den > 0.f ? o1 / den : 0.f;
@@ -456,63 +585,6 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
             rotate_pair(v0, v1, make_float2(c.x, -c.y));
         }
         put2<T>(static_cast<T*>(a.out) + ((size_t)b * a.Hq + h0 + h) * D + d, v0, v1);
-    }
-
-    // ---- append the new token (one CTA per (sequence, kv head)), off the output path ----
-    if (app) {
-        const bool complete = ai == a.m - 1;
-        for (int s = 0; s < a.S; ++s) {
-            const bool key = s == 0;
-            float mxs[2] = {0.f, 0.f}, lss[2] = {1.f, 1.f}, acs[2] = {0.f, 0.f};
-            if (pair_owner) {
-                const float xv[2] = {ax[s].x, ax[s].y};
-                const float av[2] = {(az[s].x + abp[s].x) * kLog2e, (az[s].y + abp[s].y) * kLog2e};
-                const float m0[2] = {am[s].x, am[s].y}, l0[2] = {al_[s].x, al_[s].y}, a0[2] = {aa[s].x, aa[s].y};
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    if (ai == 0) {
-                        mxs[e] = av[e]; lss[e] = 1.f; acs[e] = xv[e];
-                    } else {
-                        const float mn = fmaxf(m0[e], av[e]);
-                        const float rr = ex2(m0[e] - mn), p = ex2(av[e] - mn);
-                        mxs[e] = mn; lss[e] = l0[e] * rr + p; acs[e] = fmaf(p, xv[e], a0[e] * rr);
-                    }
-                }
-            }
-            float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
-            if (complete) {  // uniform across the CTA
-                float e0v = acs[0] / lss[0], e1v = acs[1] / lss[1];
-                const float ss = (key && a.rmsnorm)
-                                     ? block_sum(pair_owner ? e0v * e0v + e1v * e1v : 0.f, scratch) : 0.f;
-                if (key && a.rmsnorm) {
-                    const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
-                    const T* gm = static_cast<const T*>(a.gamma_kv);
-                    e0v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid]) : 1.f);
-                    e1v *= inv * (gm && pair_owner ? to_f<T>(gm[2 * tid + 1]) : 1.f);
-                }
-                if (key && a.rho && pair_owner && 2 * tid >= D - a.rho)
-                    rotate_pair(e0v, e1v, rope_cs((int64_t)aj * a.m, (2 * tid - (D - a.rho)) >> 1, a.rope_step));
-                if (pair_owner) {
-                    if (aj < a.max_blocks)
-                        put2<T>(static_cast<T*>(key ? a.pooled_k : a.pooled_v) +
-                                    (((size_t)b * a.G + g) * a.max_blocks + aj) * D + 2 * tid,
-                                e0v, e1v);
-                    else
-                        set_status(a.status, LBCA_ERR_CAPACITY);
-                }
-            } else if (pair_owner) {
-                *reinterpret_cast<float2*>(st) = make_float2(mxs[0], mxs[1]);
-                *reinterpret_cast<float2*>(st + GD) = make_float2(lss[0], lss[1]);
-                *reinterpret_cast<float2*>(st + 2 * GD) = make_float2(acs[0], acs[1]);
-            }
-            if (pair_owner) {  // ring slot of token t: the finalised key row, or the raw value
-                T* dst = static_cast<T*>(key ? a.ring_k : a.ring_v) +
-                         (((size_t)b * a.G + g) * a.R + (t % a.R)) * D + 2 * tid;
-                const T* src = (key ? newk : newv) + 2 * tid;
-                dst[0] = src[0];
-                dst[1] = src[1];
-            }
-        }
     }
 }
 

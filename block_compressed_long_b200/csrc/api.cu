@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "common.cuh"
 #include "kernels.h"
 #include "lbca.h"
 
@@ -242,7 +243,7 @@ size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, i
     if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return 0;
     StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
                             cfg->n_win, cfg->shared_kv, max_ctx);
-    if (sp.ok) return align256(sp.arrive_elems * 4);
+    if (sp.ok) return step_workspace_bytes(sp);
     return lbca_decode_workspace_bytes(cfg, batch, max_ctx);  // append + decode fallback
 }
 
@@ -251,6 +252,13 @@ int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch, int32_t
     const StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
                                   cfg->n_win, cfg->shared_kv, max_ctx);
     return sp.ok ? 1 : 2;
+}
+
+int32_t lbca_decode_step_form(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return -1;
+    const StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
+                                  cfg->n_win, cfg->shared_kv, max_ctx);
+    return !sp.ok ? LBCA_STEP_TWO_CALLS : sp.flat ? LBCA_STEP_PERSISTENT : LBCA_STEP_CLUSTER;
 }
 
 lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk, const void* zv,
@@ -275,7 +283,7 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
         return lbca_decode(cfg, q, cache, sink, gamma_q, max_ctx, out, workspace, workspace_bytes, d_status,
                            stream);
     }
-    if (workspace_bytes < align256(sp.arrive_elems * 4)) return LBCA_ERR_CAPACITY;
+    if (workspace_bytes < step_workspace_bytes(sp)) return LBCA_ERR_CAPACITY;
     LBCA_TRY(check_device());
     StepArgs a{};
     a.dtype = cfg->dtype;
@@ -289,6 +297,17 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
     a.max_blocks = cache->max_blocks; a.R = cache->ring_slots; a.S = cfg->shared_kv ? 1 : 2;
     a.CS = sp.CS; a.SE = sp.SE; a.heads_per_cta = sp.heads_per_cta;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
+    if (sp.flat) {
+        for (int kk = 0; kk < cfg->rope_dims / 2 && kk < 128; ++kk) a.rope_f[kk] = rope_turns(kk, a.rope_step);  // workspace: [arrival counter][segment counters][partial max, sum][partial outputs]
+        char* ws = static_cast<char*>(workspace);
+        const size_t o1 = align256(4), o2 = o1 + align256(sp.seg_elems * 4), o3 = o2 + align256(sp.part_ml_elems * 4);
+        a.seg_count = reinterpret_cast<uint32_t*>(ws + o1);
+        a.part_ml = reinterpret_cast<float*>(ws + o2);
+        a.part_o = reinterpret_cast<float*>(ws + o3);
+        a.C = sp.C;
+        a.maxc = sp.maxc;
+        LBCA_TRY(cuda_status(flat_grid(&a.grid, a.dtype, a.D, a.heads_per_cta, sp.smem_bytes)));
+    }
     return cuda_status(launch_decode_step(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

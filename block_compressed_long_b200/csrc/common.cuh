@@ -102,7 +102,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // F_k = inv_k / (2 pi) * 2^64 and pos * F_k wraps exactly modulo one turn (two's
 // complement makes negative positions come out right too).  The top 24 bits of
 // the fraction (2^-24 turn resolution) then go to sincospif on [0, 2).
-__device__ __forceinline__ float2 rope_cs(int64_t pos, int k, double step) {
+// F_k of pair k (fixed-point turns per position): step^k / (2 pi) * 2^64, with
+// step^k by repeated squaring in fp64.  Host and device compute it alike.
+__host__ __device__ __forceinline__ uint64_t rope_turns(int k, double step) {
     double inv = 1.0, b = step;
     for (int e = k; e; e >>= 1) {
         if (e & 1) inv *= b;
@@ -110,17 +112,27 @@ __device__ __forceinline__ float2 rope_cs(int64_t pos, int k, double step) {
     }
     const double kTurn = 0.15915494309189535;            // 1 / (2 pi)
     const double kTwo64 = 18446744073709551616.0;        // 2^64
-    const uint64_t F = (uint64_t)(inv * kTurn * kTwo64);
+    return (uint64_t)(inv * kTurn * kTwo64);
+}
+// cos / sin of position pos on the pair whose turns per position are F.
+__device__ __forceinline__ float2 rope_cs_turns(int64_t pos, uint64_t F) {
     const uint64_t t = (uint64_t)pos * F;
     const float x = (float)(uint32_t)(t >> 40) * (1.0f / 16777216.0f);
     float sn, cs;
     sincospif(2.0f * x, &sn, &cs);
     return make_float2(cs, sn);
 }
+__device__ __forceinline__ float2 rope_cs(int64_t pos, int k, double step) {
+    return rope_cs_turns(pos, rope_turns(k, step));
+}
+// (x, y) turned by the angle whose cosine and sine are cs.  Spelt out as one
+// rounded product and one fused multiply-add per component so that every
+// kernel rounds a rotation identically (the compiler may not contract it
+// differently from one kernel to the next).
 __device__ __forceinline__ void rotate_pair(float& a, float& b, float2 cs) {
-    float x = a, y = b;
-    a = x * cs.x - y * cs.y;
-    b = x * cs.y + y * cs.x;
+    const float x = a, y = b;
+    a = __fmaf_rn(x, cs.x, -__fmul_rn(y, cs.y));
+    b = __fmaf_rn(x, cs.y, __fmul_rn(y, cs.x));
 }
 
 // ---- status -------------------------------------------------------------------------

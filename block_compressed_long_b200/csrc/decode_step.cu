@@ -25,6 +25,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "decode_common.cuh"
 #include "kernels.h"
 
 namespace cg = cooperative_groups;
@@ -59,47 +60,6 @@ __host__ __device__ inline StepLayout step_layout(int D, int R, int SE, int esiz
     return l;
 }
 
-template <typename T>
-__device__ __forceinline__ void put2(T* p, float a, float b);
-template <> __device__ __forceinline__ void put2<float>(float* p, float a, float b) {
-    *reinterpret_cast<float2*>(p) = make_float2(a, b);
-}
-template <> __device__ __forceinline__ void put2<__nv_bfloat16>(__nv_bfloat16* p, float a, float b) {
-    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
-}
-// Two consecutive I/O elements, loaded as raw bits (so that the load can be
-// issued early and converted where it is used).
-template <typename T> struct Pair;
-template <> struct Pair<float> {
-    using Raw = float2;
-    static __device__ __forceinline__ Raw load(const float* p) { return *reinterpret_cast<const float2*>(p); }
-    static __device__ __forceinline__ float2 cvt(Raw r) { return r; }
-};
-template <> struct Pair<__nv_bfloat16> {
-    using Raw = uint32_t;
-    static __device__ __forceinline__ Raw load(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
-    static __device__ __forceinline__ float2 cvt(Raw w) {
-        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    }
-};
-template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float (&o)[Vec<T>::N]);
-template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, float (&o)[4]) {
-    o[0] = __uint_as_float(u.x); o[1] = __uint_as_float(u.y); o[2] = __uint_as_float(u.z); o[3] = __uint_as_float(u.w);
-}
-template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float (&o)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o[2 * i] = __uint_as_float(w[i] << 16);
-        o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
-template <typename T>
-__device__ __forceinline__ float2 get2(const T* p) {
-    return make_float2(to_f<T>(p[0]), to_f<T>(p[1]));
-}
-
 // Block-wide sum over kThreads threads (every thread must call it).
 __device__ __forceinline__ float block_sum(float v, float* scratch) {
 #pragma unroll
@@ -112,13 +72,6 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
     for (int i = 0; i < kWarps; ++i) s += scratch[i];
     __syncthreads();
     return s;
-}
-
-// Online-softmax merge weights of two partials with maxima ma, mb.
-__device__ __forceinline__ void merge_weights(float ma, float mb, float& M, float& fa, float& fb) {
-    M = fmaxf(ma, mb);
-    fa = ma == kNegInf ? 0.f : ex2(ma - M);
-    fb = mb == kNegInf ? 0.f : ex2(mb - M);
 }
 
 template <typename T, int D, int R>
@@ -658,9 +611,30 @@ StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int sha
         if (r % c == 0) { R = c; break; }
     const int esize = dtype == LBCA_BF16 ? 2 : 4;
     const long long groups = (long long)B * (Hq / R);
+    p.heads_per_cta = R;
+    // Many (sequence, head group) segments: the persistent evenly-split kernel
+    // (one launch, no clusters), whose CTAs each take an equal share of all the
+    // step's entries however unequal the contexts.
+    const int S = shared ? 1 : 2;
+    const int C = std::min(128, std::max(16, 32768 / (D * esize * S)));
+    if (groups >= 96 && B <= 4096) {
+        const long long mc = std::max(1, max_ctx);
+        const long long P = mc > w ? (mc - w) / m : 0;
+        const long long max_vis = std::min<long long>(mc, P + w + m - 1);
+        p.flat = true;
+        p.C = C;
+        p.maxc = (int)((max_vis + C - 1) / C + 2);
+        p.seg_elems = (size_t)groups;
+        p.part_ml_elems = (size_t)groups * p.maxc * R * 2;
+        p.part_o_elems = (size_t)groups * p.maxc * R * D;
+        p.arrive_elems = 1;
+        p.smem_bytes = flat_smem_bytes(dtype, B, D, R, C, shared);
+        p.ok = p.smem_bytes <= 200 * 1024;
+        if (p.ok) return p;
+        p.flat = false;
+    }
     int CS = 1;
     while (CS < 16 && CS * 2 <= D / 4 && groups * CS < 4 * 148) CS *= 2;
-    p.heads_per_cta = R;
     p.CS = CS;
     p.SE = D >= 256 || esize == 4 ? 16 : 32;
     p.arrive_elems = (size_t)B;
@@ -670,8 +644,15 @@ StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int sha
     return p;
 }
 
+static size_t a256(size_t x) { return (x + 255) / 256 * 256; }
+size_t step_workspace_bytes(const StepPlan& p) {
+    if (!p.flat) return a256(p.arrive_elems * 4);
+    return a256(p.arrive_elems * 4) + a256(p.seg_elems * 4) + a256(p.part_ml_elems * 4) + a256(p.part_o_elems * 4);
+}
+
 cudaError_t launch_decode_step(const StepArgs& a, cudaStream_t s) {
     if (a.B == 0) return cudaSuccess;
+    if (a.C > 0) return launch_decode_flat(a, s);
     const size_t smem = step_layout(a.D, a.heads_per_cta, a.SE, a.dtype == LBCA_BF16 ? 2 : 4, a.shared, a.CS).total;
     if (a.dtype == LBCA_BF16) return step_dispatch<__nv_bfloat16>(a, smem, s);
     return step_dispatch<float>(a, smem, s);

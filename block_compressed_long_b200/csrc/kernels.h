@@ -117,14 +117,29 @@ struct StepArgs {
     int CS, SE, heads_per_cta;
     float eps, scale;
     double rope_step;  // theta^(-2/rho)
+    // persistent evenly-split form (decode_flat.cu): arrive is one grid-wide counter
+    float* part_o;                                                 // [segments][maxc][R][D]
+    float* part_ml;                                                // [segments][maxc][R][2]
+    uint32_t* seg_count;                                           // [segments], zeroed
+    int C, grid, maxc;
+    uint64_t rope_f[128];  // persistent form: fixed-point turns per position of each RoPE pair (rope_turns)
 };
 struct StepPlan {
     int heads_per_cta, CS, SE;
     size_t arrive_elems, smem_bytes;
     bool ok;
+    // persistent evenly-split form: chosen for large batches
+    bool flat;
+    int C, maxc;
+    size_t seg_elems, part_o_elems, part_ml_elems;
 };
 StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+size_t step_workspace_bytes(const StepPlan& p);
 cudaError_t launch_decode_step(const StepArgs& a, cudaStream_t s);
+size_t flat_smem_bytes(int dtype, int B, int D, int R, int C, int shared);
+cudaError_t launch_decode_flat(const StepArgs& a, cudaStream_t s);
+// CTAs of the persistent grid on the current device (every SM filled).
+cudaError_t flat_grid(int* grid, int dtype, int D, int R, size_t smem);
 
 struct PrefillArgs {
     int dtype;

@@ -28,7 +28,8 @@ LBCA_KEY, LBCA_VALUE = 0, 1
 ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspace_bytes",
                 "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
                 "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc",
-                "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches")
+                "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches",
+                "lbca_decode_step_form")
 
 
 class lbca_config(ctypes.Structure):
@@ -75,6 +76,8 @@ _lib.lbca_decode_step.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _
 _lib.lbca_decode_step.restype = ctypes.c_int
 _lib.lbca_decode_step_launches.argtypes = [_CP, _i32, _i32]
 _lib.lbca_decode_step_launches.restype = _i32
+_lib.lbca_decode_step_form.argtypes = [_CP, _i32, _i32]
+_lib.lbca_decode_step_form.restype = _i32
 _lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _vp]
 _lib.lbca_decode_noalloc.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
@@ -202,6 +205,13 @@ def lbca_decode_step_workspace_bytes(cfg: lbca_config, batch: int, max_ctx: int)
 
 def lbca_decode_step_launches(cfg: lbca_config, batch: int, max_ctx: int) -> int:
     return int(_lib.lbca_decode_step_launches(ctypes.byref(cfg), batch, max_ctx))
+
+
+LBCA_STEP_TWO_CALLS, LBCA_STEP_CLUSTER, LBCA_STEP_PERSISTENT = range(3)
+
+
+def lbca_decode_step_form(cfg: lbca_config, batch: int, max_ctx: int) -> int:
+    return int(_lib.lbca_decode_step_form(ctypes.byref(cfg), batch, max_ctx))
 
 
 def lbca_decode_step(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, q, cache: Cache, sink, gamma_q, out,

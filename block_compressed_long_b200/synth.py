@@ -136,16 +136,17 @@ class Inputs:
     lens: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))  # decode: context per sequence
 
 
-def make(w: Workload) -> Inputs:
+def make(w: Workload, lens: np.ndarray | None = None) -> Inputs:
     """Draw a workload's inputs.  Order of draws: Q, K (or C), V, Z_K (or Z),
-    Z_V, B_pos_K, B_pos_V, sink; each from its own keyed stream."""
+    Z_V, B_pos_K, B_pos_V, sink; each from its own keyed stream.  A decode
+    workload's cached contexts come from `contexts(w)` unless given."""
     B, Hq, G, D, m = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_m
     if w.kind == "prefill":
         T = w.seq_len
         q = normal(w.seed, "q", (B, T, Hq, D), dtype=w.dtype)
         lens = np.full(B, T, dtype=np.int64)
     else:
-        lens = contexts(w)
+        lens = contexts(w) if lens is None else np.asarray(lens, dtype=np.int64)
         T = int(lens.max()) + w.steps
         q = normal(w.seed, "q", (w.steps, B, Hq, D), dtype=w.dtype)
     rl = None if w.kind == "prefill" else lens + w.steps  # history each sequence reaches

@@ -207,16 +207,28 @@ LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lb
  * `workspace` (zero-filled before first use, left zero-filled) must hold
  * lbca_decode_step_workspace_bytes(cfg, B, max_ctx) bytes.  With n_win >= 1,
  * D in {64, 128, 256} and up to 4 query heads per kv head per CTA group, the
- * step runs as one cluster kernel (the appended token's block cannot be
- * visible to the same query, so appending and attending are independent);
- * other shapes run lbca_append then lbca_decode.  Results equal those of the
- * two calls.
+ * step runs as one kernel (the appended token's block cannot be visible to
+ * the same query, so appending and attending are independent): for a few
+ * (sequence, head group) pairs a cluster kernel that splits each pair's
+ * entries over the CTAs of a cluster, for many pairs (96 or more) a
+ * persistent kernel whose CTAs each take an equal share of all the step's
+ * entries, whatever the mix of context lengths.  Other shapes run lbca_append
+ * then lbca_decode.  Results equal those of the two calls.  A sequence longer
+ * than max_ctx sets d_status to LBCA_ERR_CAPACITY.
  */
 LBCA_API size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
 /* Kernel launches one lbca_decode_step call makes for these shapes: 1 when the
  * step runs as one fused kernel, 2 when it runs lbca_append then lbca_decode,
  * -1 for an invalid configuration.  Host-only; needs no GPU. */
 LBCA_API int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
+/* Which form lbca_decode_step takes for these shapes (host-only; needs no GPU). */
+typedef enum {
+    LBCA_STEP_TWO_CALLS = 0,   /* lbca_append, then lbca_decode */
+    LBCA_STEP_CLUSTER = 1,     /* one cluster kernel */
+    LBCA_STEP_PERSISTENT = 2   /* one persistent, evenly split kernel */
+} lbca_step_form;
+/* Returns an lbca_step_form, or -1 for an invalid configuration. */
+LBCA_API int32_t lbca_decode_step_form(const lbca_config* cfg, int32_t batch, int32_t max_ctx);
 LBCA_API lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk,
                                       const void* zv, const void* b_pos_k, const void* b_pos_v,
                                       const void* gamma_kv, const void* q, const lbca_cache* cache,

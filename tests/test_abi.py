@@ -124,6 +124,20 @@ def test_decode_step_launches(L):
     assert L.lbca_decode_step_launches(_cfg(L, block_m=0), 1, 100) == -1
 
 
+def test_decode_step_form(L):
+    """A few (sequence, head group) pairs take the cluster kernel, many (the
+    32-sequence ragged batch: 256 pairs) the persistent evenly split one; the
+    persistent form's workspace grows with the longest context it may meet."""
+    cfg = _cfg(L)
+    assert L.lbca_decode_step_form(cfg, 1, 32769) == L.LBCA_STEP_CLUSTER
+    assert L.lbca_decode_step_form(cfg, 32, 65600) == L.LBCA_STEP_PERSISTENT
+    assert L.lbca_decode_step_form(_cfg(L, n_win=0), 32, 65600) == L.LBCA_STEP_TWO_CALLS
+    assert L.lbca_decode_step_form(_cfg(L, block_m=0), 32, 100) == -1
+    small = L.lbca_decode_step_workspace_bytes(cfg, 32, 4096)
+    big = L.lbca_decode_step_workspace_bytes(cfg, 32, 65600)
+    assert 0 < small < big
+
+
 def test_status_strings(L):
     for s in range(7):
         assert L.lbca_status_string(s)

@@ -174,10 +174,13 @@ class DecodeBench:
                                       cl(c0.ring_k), cl(c0.ring_v), cl(c0.pool_state), cl(c0.seq_lens))
                               for _ in range(self.NR - 1)]
         del k, v, zk, zv
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()  # the raw token history is no longer needed: hand its memory back
         wsb = max(L.lbca_decode_step_workspace_bytes(self.cfg, B, self.max_ctx), 16)
         self.step_ws = [torch.zeros(wsb, dtype=torch.uint8, device="cuda") for _ in range(self.NR)]
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.launches = L.lbca_decode_step_launches(self.cfg, B, self.max_ctx)
+        self.form = L.lbca_decode_step_form(self.cfg, B, self.max_ctx)
         self.dec_ws = []
         if self.launches == 2:
             dwb = max(L.lbca_decode_workspace_bytes(self.cfg, B, self.max_ctx), 16)
@@ -337,8 +340,9 @@ def run_ours(args, w, rank, world):
                               f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src,
-                     "kernel": ("decode_step_kernel" if bench.launches == 1 else
-                                "the decode launch of the step (timed alone over the same replicas)"),
+                     "kernel": ({L.LBCA_STEP_CLUSTER: "decode_step_kernel (cluster form)",
+                                 L.LBCA_STEP_PERSISTENT: "decode_flat_kernel (persistent evenly split form)"}
+                                .get(bench.form, "the decode launch of the step (timed alone over the same replicas)")),
                      "bytes_per_launch": nbytes / K, "launch_us": kernel_ms * 1e3,
                      "traffic": load_traffic(w_.name)},
         "e2e": {"value": ranks.job_us_per_token(e2e_ms, bench.B, world), "unit": "µs/token",

@@ -27,6 +27,8 @@ POOL_CASES = [
     ("gqa_prefill_16k", dict(seq_len=16 * 9 + 3)),
     ("hca_mqa_decode_128k", dict(seq_len=128 * 4 + 100, batch=3)),
     ("ragged_gqa_decode_append", dict(seq_len=64 * 3, batch=2)),
+    # more blocks than the GPU holds CTAs at once, and a ragged tail
+    ("gqa_prefill_16k", dict(seq_len=16 * 1100 + 5, batch=1)),
 ]
 
 

@@ -9,23 +9,25 @@
 //
 // B200 mapping (one CTA = 2 x 128 queries of one head, 384 threads):
 //   warp 0     TMA producer: the two Q tiles once, then fp16 K and V tiles
-//              of 128 entries (pooled tiles first, then the raw band) into
-//              a two-stage ring, 128-byte swizzled, no multicast.
-//   warp 1     TMEM owner and MMA issuer: S = Q K^T (tcgen05.mma M=128 N=128,
-//              fp16 K-major operands from shared memory) into the query tile's
-//              TMEM S columns, and O += P V with P read from TMEM (the
-//              softmax overwrites S with P) and fp16 V as an MN-major operand;
-//              completion is signalled by tcgen05.commit on mbarriers.  Two
-//              query tiles per CTA interleave (PV0, S0', PV1, S1') so the
-//              tensor core works on one tile while the other's softmax runs.
+//              of 64 entries (pooled tiles first, then the raw band) into a
+//              four-stage ring, 128-byte swizzled, no multicast.
+//   warps 1-2  MMA issuers, one per query tile q: S_q = Q_q K^T (tcgen05.mma
+//              M=128 N=64, fp16 K-major operands from shared memory) into
+//              q's TMEM S columns, and O_q += P V with P read from TMEM (one
+//              of two P buffers) and fp16 V as an MN-major operand; completion
+//              is signalled by tcgen05.commit on mbarriers.  S, P and O have
+//              TMEM columns of their own, so S_q of the next tile is issued
+//              as soon as the softmax has read the current one -- the tensor
+//              core computes it while the exponentials of the current tile
+//              run -- and P V of a tile runs behind.
 //   warps 4-7, 8-11  softmax of query tiles 0 and 1: thread r owns query row r
-//              and TMEM lane r.  It rotates
-//              its Q row in shared memory once, then per tile loads its S row,
-//              applies the causal-block / window mask, keeps an online max
-//              (rescaling O in TMEM only when the max grows by more than 2^8),
-//              writes P in fp16 into TMEM over its S row, and finally
-//              normalises its O row (plus the sink) into shared memory, from
-//              where one thread TMA-stores the tile.
+//              and TMEM lane r.  It rotates its Q row in shared memory once,
+//              then per tile loads its S row, releases S, applies the
+//              causal-block / window mask, keeps an online max (rescaling O
+//              in TMEM only when the max grows by more than 2^8), writes P in
+//              fp16 into the free P buffer, and finally normalises its O row
+//              (plus the sink) into shared memory, from where one thread
+//              TMA-stores the tile.
 // Raw keys arrive already rotated and, like the values, in fp16 (a pre-pass
 // writes them once instead of every query tile converting them again); Q is
 // rotated in shared memory from a per-position cos/sin table.  Rows past a tensor's valid extent
@@ -43,32 +45,36 @@ namespace {
 
 constexpr int BM = 128;     // query rows per softmax warpgroup (one M=128 MMA)
 constexpr int NQ = 2;       // query tiles per CTA
-constexpr int BN = 128;     // entries per K/V tile
+constexpr int BN = 64;      // entries per K/V tile
 constexpr int HD = 128;     // head dim
-constexpr int NSTAGE = 2;   // K/V ring depth
+constexpr int NSTAGE = 4;   // K/V ring depth
 constexpr uint32_t QREG = BM * 64 * 2;   // [128 rows][64 cols] 16-bit: one 128-byte swizzle span per row
 constexpr uint32_t QTILE = 2 * QREG;     // [128][128]
-constexpr uint32_t KREG = BN * 64 * 2;   // [128 rows][64 cols]
-constexpr uint32_t KTILE = 2 * KREG;     // [128][128]
+constexpr uint32_t KREG = BN * 64 * 2;   // [64 rows][64 cols]
+constexpr uint32_t KTILE = 2 * KREG;     // [64][128]
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + NQ * QTILE;
 constexpr uint32_t OFF_V = OFF_K + NSTAGE * KTILE;
 constexpr uint32_t OFF_BAR = OFF_V + NSTAGE * KTILE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t TMEM_COLS = 512;  // per query tile q: S/P at 256q (128 columns), O at 256q + 128
-constexpr int kThreads = 384;        // warps 0 producer, 1 MMA, 2-3 idle, 4-7 / 8-11 softmax
+// TMEM columns of query tile q, from 256 q: S [0, 64) f32, P buffers [64, 96) and
+// [96, 128) (fp16 pairs: 64 entries in 32 columns), O [128, 256) f32.
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_S = 0, T_P = 64, T_O = 128;
+constexpr int kThreads = 384;        // warps 0 producer, 1-2 MMA issuers, 3 idle, 4-7 / 8-11 softmax
 constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;
 
 // barrier slots
 constexpr int B_QFULL = 0;
-constexpr int B_QROT = 1;                      // [NQ]
+constexpr int B_QROT = 1;                      // [NQ] softmax warpgroup q has rotated its Q rows
 constexpr int B_KFULL = B_QROT + NQ;           // [NSTAGE]
 constexpr int B_VFULL = B_KFULL + NSTAGE;      // [NSTAGE]
-constexpr int B_KVEMPTY = B_VFULL + NSTAGE;    // [NSTAGE]
-constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ]
-constexpr int B_PFULL = B_SFULL + NQ;          // [NQ]
-constexpr int B_ODONE = B_PFULL + NQ;          // [NQ]
-constexpr int B_COUNT = B_ODONE + NQ;
+constexpr int B_KVEMPTY = B_VFULL + NSTAGE;    // [NSTAGE] both issuers are done with the stage
+constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ] S_q computed
+constexpr int B_SFREE = B_SFULL + NQ;          // [NQ] S_q read by the softmax
+constexpr int B_PFULL = B_SFREE + NQ;          // [NQ] P_q written
+constexpr int B_PVDONE = B_PFULL + NQ;         // [NQ][2] P V from P buffer b of query tile q done
+constexpr int B_COUNT = B_PVDONE + 2 * NQ;
 
 struct TcArgs {
     CUtensorMap tq;   // q [B, T, Hq, D] bf16          dims (D, Hq, T, B)
@@ -94,6 +100,20 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, int
 }
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* fail, int32_t* status) {
     return __all_sync(0xffffffffu, wait_or_fail(bar, parity, fail, status));
+}
+
+// 2^x on the FMA pipe, after Cody and Waite's range reduction: x = n + f with
+// n = rint(x) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial (a weighted
+// least-squares fit of 2^f on that interval, relative error below 7.5e-5, under
+// half an fp16 ulp, the precision P is kept in); 2^n added to the exponent
+// field.  Inputs below -125 (masked scores are -inf) give 2^-125, which is 0 in
+// fp16; inputs are at most 8 here (the lazy rescale bounds them).
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
+    const float f = x - (t - 12582912.0f);
+    const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // The K/V tiles of a CTA run over the pooled entries [0, npt BN) and then the
@@ -140,8 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            const bool softmax_arrivals = (i >= B_QROT && i < B_QROT + NQ) || (i >= B_PFULL && i < B_PFULL + NQ);
-            mbar_init(&bars[i], softmax_arrivals ? 128u : 1u);
+            const bool softmax_arrivals = (i >= B_QROT && i < B_QROT + NQ) || (i >= B_SFREE && i < B_SFREE + NQ) ||
+                                          (i >= B_PFULL && i < B_PFULL + NQ);
+            const bool both_issuers = i >= B_KVEMPTY && i < B_KVEMPTY + NSTAGE;
+            mbar_init(&bars[i], softmax_arrivals ? 128u : both_issuers ? (uint32_t)NQ : 1u);
         }
         *fail = 0;
         fence_barrier_init();
@@ -186,74 +208,65 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
             mbar_wait(&bars[B_QFULL], 0, kWaitNs);
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
-        // order per K/V tile i: S_q(i) for the query tiles that need it (unless
-        // issued ahead), then PV_q(i) and at once S_q(i+1).  P_q(i) lives in
-        // S_q's TMEM columns, so S_q(i+1) waits until PV_q(i) has read it; a
-        // query tile skips the tiles none of its rows can see.
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------- MMA issuers, one per query tile
+        // For each tile i this query tile needs: S(i) once K(i) has landed and
+        // the softmax has read S of the previous tile, then P V of the previous
+        // tile (so the tensor core computes S(i) while the softmax of the
+        // previous tile runs).  A stage is released (KVEMPTY, two issuers) after
+        // its P V; a tile no row of q can see is released once its data has
+        // landed.  A pending P V is issued early when the next wait would need
+        // the stage it holds.
+        const int q = warp - 1;
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
-            auto issue_s = [&](int q, int i) {
-                const int s = i % NSTAGE;
-                const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
-                const uint32_t sk = smem_addr(smem + OFF_K + s * KTILE);
+            const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
+            const uint32_t tq = tbase + 256 * q;
+            const Need nd = need_of(a, q, t0, s_lo, nrt);
+            bool ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
+            int k = 0;      // needed tiles whose S has been issued
+            int prev = -1;  // tile whose P V is still to be issued (the (k-1)-th needed one)
+            auto issue_pv = [&](int i, int kk) {  // P V of tile i, the kk-th needed tile of q
+                ok = wait_or_fail(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
+                if (ok) ok = wait_or_fail(&bars[B_PFULL + q], kk & 1, fail, a.status);
+                if (!ok) return;
+                const uint32_t sv = smem_addr(smem + OFF_V + (i % NSTAGE) * KTILE);
+                tc_fence_after();
+#pragma unroll
+                for (int e = 0; e < BN / 16; ++e)  // A = P (16 entries = 8 fp16-pair columns)
+                    tc_mma_ts(tq + T_O, tq + T_P + 32 * (kk & 1) + 8 * e, smem_desc_sw128(sv + e * 2048, KREG, 1024),
+                              idP, (kk > 0 || e > 0) ? 1u : 0u);
+                tc_commit(&bars[B_PVDONE + 2 * q + (kk & 1)]);
+                tc_commit(&bars[B_KVEMPTY + i % NSTAGE]);
+            };
+            for (int i = 0; ok && i < ntile; ++i) {
+                if (prev >= 0 && prev <= i - NSTAGE) {  // tile i reuses prev's stage
+                    issue_pv(prev, k - 1);
+                    prev = -1;
+                    if (!ok) break;
+                }
+                if (!nd(i, npt)) {
+                    ok = wait_or_fail(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status) &&
+                         wait_or_fail(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
+                    if (ok) tc_commit(&bars[B_KVEMPTY + i % NSTAGE]);
+                    continue;
+                }
+                ok = wait_or_fail(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
+                if (ok && k > 0) ok = wait_or_fail(&bars[B_SFREE + q], (k - 1) & 1, fail, a.status);
+                if (!ok) break;
+                const uint32_t sk = smem_addr(smem + OFF_K + (i % NSTAGE) * KTILE);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    tc_mma_bf16(tbase + 256 * q, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
+                    tc_mma_bf16(tq + T_S, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
                                 smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
                 tc_commit(&bars[B_SFULL + q]);
-            };
-            auto issue_pv = [&](int q, int i, bool acc) {
-                const int s = i % NSTAGE;
-                const uint32_t sv = smem_addr(smem + OFF_V + s * KTILE);
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)  // A = P_q(i): 8 fp16x2 columns per 16 entries
-                    tc_mma_ts(tbase + 256 * q + 128, tbase + 256 * q + kk * 8,
-                              smem_desc_sw128(sv + kk * 2048, KREG, 1024), idP, (acc || kk > 0) ? 1u : 0u);
-                tc_commit(&bars[B_ODONE + q]);
-            };
-            Need nd[NQ];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) nd[q] = need_of(a, q, t0, s_lo, nrt);
-            int npv[NQ] = {0, 0};    // P V products issued per query tile (its ODONE phases)
-            int s_at[NQ] = {-1, -1}; // tile of the latest S issued per query tile
-            bool ok = true;
-            for (int q = 0; ok && q < NQ; ++q) ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
-            for (int i = 0; ok && i < ntile; ++i) {
-                const int s = i % NSTAGE;
-                const uint32_t ph = (i / NSTAGE) & 1;
-                bool any = false;
-                for (int q = 0; ok && q < NQ; ++q) {  // S_q(i), unless issued ahead
-                    if (!nd[q](i, npt)) continue;
-                    any = true;
-                    if (s_at[q] == i) continue;
-                    ok = wait_or_fail(&bars[B_KFULL + s], ph, fail, a.status);
-                    if (ok && npv[q] > 0) ok = wait_or_fail(&bars[B_ODONE + q], (npv[q] - 1) & 1, fail, a.status);
-                    if (ok) { issue_s(q, i); s_at[q] = i; }
-                }
-                if (!ok) break;
-                // the stage's data must have landed before it is released
-                ok = wait_or_fail(&bars[B_VFULL + s], ph, fail, a.status);
-                if (ok && !any) ok = wait_or_fail(&bars[B_KFULL + s], ph, fail, a.status);
-                for (int q = 0; ok && any && q < NQ; ++q) {
-                    if (!nd[q](i, npt)) continue;
-                    ok = wait_or_fail(&bars[B_PFULL + q], npv[q] & 1, fail, a.status);
-                    if (!ok) break;
-                    issue_pv(q, i, npv[q] > 0);
-                    ++npv[q];
-                    const int n = i + 1;
-                    if (n < ntile && nd[q](n, npt)) {  // S_q(i+1) as soon as P_q(i) is consumed
-                        ok = wait_or_fail(&bars[B_KFULL + n % NSTAGE], (n / NSTAGE) & 1, fail, a.status);
-                        if (ok) ok = wait_or_fail(&bars[B_ODONE + q], (npv[q] - 1) & 1, fail, a.status);
-                        if (ok) { issue_s(q, n); s_at[q] = n; }
-                    }
-                }
-                if (ok) tc_commit(&bars[B_KVEMPTY + s]);
+                if (prev >= 0) issue_pv(prev, k - 1);
+                prev = i;
+                ++k;
             }
+            if (ok && prev >= 0) issue_pv(prev, k - 1);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------- softmax
@@ -265,8 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int lo = Pq * a.m;
         const uint32_t lane_f = (uint32_t)(32 * (warp & 3)) << 16;
         const int half = a.rho / 2;
-        const uint32_t tS = tbase + 256 * q + lane_f;
-        const uint32_t tO = tS + 128;
+        const uint32_t tS = tbase + 256 * q + lane_f + T_S;
+        const uint32_t tP = tbase + 256 * q + lane_f + T_P;
+        const uint32_t tO = tbase + 256 * q + lane_f + T_O;
         uint8_t* sQ = smem + OFF_Q + q * QTILE;
 
         // this query row's cos/sin, fetched in one batch while Q lands
@@ -306,7 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const bool pooled = i < npt;
             const int base = pooled ? i * BN : s_lo + (i - npt) * BN;
             ok = warp_wait(&bars[B_SFULL + q], k & 1, fail, a.status);
-            ++k;
             if (!ok) break;
             tc_fence_after();
             float s[BN];
@@ -315,9 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 float v[32];
                 tmem_ld32(tS + 32 * c, v);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) s[32 * c + k] = v[k];
+                for (int e = 0; e < 32; ++e) s[32 * c + e] = v[e];
             }
             tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars[B_SFREE + q]);  // S may be overwritten by the next tile's S
 
             // visible columns of this row in this tile: [c_lo, c_hi)
             int c_lo, c_hi;
@@ -325,15 +340,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             else { c_lo = max(0, lo - base); c_hi = min(BN, t - base + 1); }
             if (!valid) c_hi = 0;
             c_hi = max(c_hi, c_lo);  // an empty range masks every column
-            if (c_lo > 0 || c_hi < BN) {
+            float mxv[8];
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
+            for (int e = 0; e < 8; ++e) mxv[e] = kNegInf;
+            if (__any_sync(0xffffffffu, c_lo > 0 || c_hi < BN)) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
                     if ((unsigned)(c - c_lo) >= (unsigned)(c_hi - c_lo)) s[c] = kNegInf;
-            }
-            float mx0 = kNegInf, mx1 = kNegInf;
+                    mxv[c & 7] = fmaxf(mxv[c & 7], s[c]);
+                }
+            } else {
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) { mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); }
-            const float mx = fmaxf(mx0, mx1);
+                for (int c = 0; c < BN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], s[c]);
+            }
+            const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                                   fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
             // lazy rescale: only when the row max grows by more than 2^8 in probability
             float alpha = 1.f;
             bool rescale = false;
@@ -343,43 +364,46 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 m_ref = mx;
             }
             const float mneg = m_ref == kNegInf ? 0.f : -m_ref * sc;
-            float ps0 = 0.f, ps1 = 0.f;
-            // P as fp16 pairs, written over S in two halves of 32 columns (64 entries)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[32];
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int c = 64 * hh + 2 * k;
-                    const float p0 = ex2(fmaf(s[c], sc, mneg));
-                    const float p1 = ex2(fmaf(s[c + 1], sc, mneg));
-                    ps0 += p0;
-                    ps1 += p1;
-                    v[k] = __uint_as_float(pack_f16x2(p0, p1));
-                }
-                tmem_st32(tS + 32 * hh, v);  // columns [32 hh, 32 hh + 32) of S_q: already read
-            }
-            l = l * alpha + (ps0 + ps1);
-            // PV_q(i-1) finished before S_q(i) was issued: O is quiet, rescale it if needed
             if (__any_sync(0xffffffffu, rescale)) {
+                // O must be quiet: every P V issued so far (up to tile k-1) has completed
+                if (k > 0) ok = warp_wait(&bars[B_PVDONE + 2 * q + ((k - 1) & 1)], ((k - 1) >> 1) & 1, fail, a.status);
+                if (!ok) break;
+                tc_fence_after();
                 const float f = rescale ? alpha : 1.f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < HD / 32; ++c) {
                     float v[32];
                     tmem_ld32(tO + 32 * c, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] *= f;
+                    for (int e = 0; e < 32; ++e) v[e] *= f;
                     tmem_st32(tO + 32 * c, v);
                 }
             }
+            // P buffer k & 1 is free once the P V of tile k-2 has read it
+            if (k >= 2) ok = warp_wait(&bars[B_PVDONE + 2 * q + (k & 1)], ((k >> 1) - 1) & 1, fail, a.status);
+            if (!ok) break;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            float pk[32];
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) {  // one exponential in four on the FMA pipe
+                const float p0 = ex2(fmaf(s[2 * e], sc, mneg));
+                const float x1 = fmaf(s[2 * e + 1], sc, mneg);
+                const float p1 = (e & 1) ? exp2_fma(x1) : ex2(x1);
+                ps[e & 3] += p0 + p1;
+                pk[e] = __uint_as_float(pack_f16x2(p0, p1));
+            }
+            tc_fence_after();
+            tmem_st32(tP + 32 * (k & 1), pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + q]);
+            l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            ++k;
         }
         // ---- epilogue: normalise the O row into this query tile's shared memory
         // (free: the last S MMA that read Q is complete), then TMA-store the tile
-        if (ok && k > 0) ok = warp_wait(&bars[B_ODONE + q], (k - 1) & 1, fail, a.status);
+        if (ok && k > 0) ok = warp_wait(&bars[B_PVDONE + 2 * q + ((k - 1) & 1)], ((k - 1) >> 1) & 1, fail, a.status);
         tc_fence_after();
         float den = l;
         if (a.sink) den += m_ref == kNegInf ? 1.f : ex2(a.sink[h] * kLog2e - m_ref * sc);

@@ -67,9 +67,8 @@ constexpr uint64_t kWaitNs = 500ull * 1000 * 1000;
 // barrier slots
 constexpr int B_QFULL = 0;
 constexpr int B_QROT = 1;                      // [NQ] softmax warpgroup q has rotated its Q rows
-constexpr int B_KFULL = B_QROT + NQ;           // [NSTAGE]
-constexpr int B_VFULL = B_KFULL + NSTAGE;      // [NSTAGE]
-constexpr int B_KVEMPTY = B_VFULL + NSTAGE;    // [NSTAGE] both issuers are done with the stage
+constexpr int B_KVFULL = B_QROT + NQ;          // [NSTAGE] the stage's K and V tiles have landed
+constexpr int B_KVEMPTY = B_KVFULL + NSTAGE;   // [NSTAGE] both issuers are done with the stage
 constexpr int B_SFULL = B_KVEMPTY + NSTAGE;    // [NQ] S_q computed
 constexpr int B_SFREE = B_SFULL + NQ;          // [NQ] S_q read by the softmax
 constexpr int B_PFULL = B_SFREE + NQ;          // [NQ] P_q written
@@ -188,23 +187,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     break;
                 uint8_t* kd = smem + OFF_K + s * KTILE;
                 uint8_t* vd = smem + OFF_V + s * KTILE;
-                mbar_arrive_expect_tx(&bars[B_KFULL + s], KTILE);
-                mbar_arrive_expect_tx(&bars[B_VFULL + s], KTILE);
+                mbar_arrive_expect_tx(&bars[B_KVFULL + s], 2 * KTILE);
                 if (i < npt) {
                     const int j0 = i * BN;
-                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.tpk, 64 * rg, j0, g, b, &bars[B_KFULL + s]);
-                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.tpv, 64 * rg, j0, g, b, &bars[B_VFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.tpk, 64 * rg, j0, g, b, &bars[B_KVFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.tpv, 64 * rg, j0, g, b, &bars[B_KVFULL + s]);
                 } else {
                     const int s0 = s_lo + (i - npt) * BN;
-                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.trk, 64 * rg, g, s0, b, &bars[B_KFULL + s]);
-                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.trv, 64 * rg, g, s0, b, &bars[B_VFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(kd + rg * KREG, &a.trk, 64 * rg, g, s0, b, &bars[B_KVFULL + s]);
+                    for (int rg = 0; rg < 2; ++rg) tma_load_4d(vd + rg * KREG, &a.trv, 64 * rg, g, s0, b, &bars[B_KVFULL + s]);
                 }
                 issued = i + 1;
             }
             // drain: never leave copies in flight into shared memory (bounded)
             for (int i = max(0, issued - NSTAGE); i < issued; ++i) {
-                mbar_wait(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, kWaitNs);
-                mbar_wait(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, kWaitNs);
+                mbar_wait(&bars[B_KVFULL + i % NSTAGE], (i / NSTAGE) & 1, kWaitNs);
             }
             mbar_wait(&bars[B_QFULL], 0, kWaitNs);
         }
@@ -221,22 +218,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (lane == 0) {
             const uint32_t idS = idesc_f16_f32(BM, BN, false);
             const uint32_t idP = idesc_f16_f32(BM, HD, true);
-            const uint32_t sq = smem_addr(smem + OFF_Q + q * QTILE);
             const uint32_t tq = tbase + 256 * q;
+            // descriptors of each operand's first 16-column step; later steps add their
+            // byte offset >> 4 to the start-address field (no carry: shared addresses < 2^18)
+            const uint64_t dq = smem_desc_sw128(smem_addr(smem + OFF_Q + q * QTILE), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_addr(smem + OFF_K), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(smem + OFF_V), KREG, 1024);
             const Need nd = need_of(a, q, t0, s_lo, nrt);
             bool ok = wait_or_fail(&bars[B_QROT + q], 0, fail, a.status);
             int k = 0;      // needed tiles whose S has been issued
             int prev = -1;  // tile whose P V is still to be issued (the (k-1)-th needed one)
             auto issue_pv = [&](int i, int kk) {  // P V of tile i, the kk-th needed tile of q
-                ok = wait_or_fail(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
-                if (ok) ok = wait_or_fail(&bars[B_PFULL + q], kk & 1, fail, a.status);
+                ok = wait_or_fail(&bars[B_PFULL + q], kk & 1, fail, a.status);  // (its data landed before S(i))
                 if (!ok) return;
-                const uint32_t sv = smem_addr(smem + OFF_V + (i % NSTAGE) * KTILE);
+                const uint64_t dvs = dv + (((i % NSTAGE) * KTILE) >> 4);
                 tc_fence_after();
 #pragma unroll
                 for (int e = 0; e < BN / 16; ++e)  // A = P (16 entries = 8 fp16-pair columns)
-                    tc_mma_ts(tq + T_O, tq + T_P + 32 * (kk & 1) + 8 * e, smem_desc_sw128(sv + e * 2048, KREG, 1024),
-                              idP, (kk > 0 || e > 0) ? 1u : 0u);
+                    tc_mma_ts(tq + T_O, tq + T_P + 32 * (kk & 1) + 8 * e, dvs + ((e * 2048) >> 4), idP,
+                              (kk > 0 || e > 0) ? 1u : 0u);
                 tc_commit(&bars[B_PVDONE + 2 * q + (kk & 1)]);
                 tc_commit(&bars[B_KVEMPTY + i % NSTAGE]);
             };
@@ -247,20 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     if (!ok) break;
                 }
                 if (!nd(i, npt)) {
-                    ok = wait_or_fail(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status) &&
-                         wait_or_fail(&bars[B_VFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
+                    ok = wait_or_fail(&bars[B_KVFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
                     if (ok) tc_commit(&bars[B_KVEMPTY + i % NSTAGE]);
                     continue;
                 }
-                ok = wait_or_fail(&bars[B_KFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
+                ok = wait_or_fail(&bars[B_KVFULL + i % NSTAGE], (i / NSTAGE) & 1, fail, a.status);
                 if (ok && k > 0) ok = wait_or_fail(&bars[B_SFREE + q], (k - 1) & 1, fail, a.status);
                 if (!ok) break;
-                const uint32_t sk = smem_addr(smem + OFF_K + (i % NSTAGE) * KTILE);
+                const uint64_t dks = dk + (((i % NSTAGE) * KTILE) >> 4);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    tc_mma_bf16(tq + T_S, smem_desc_sw128(sq + (kk >> 2) * QREG + (kk & 3) * 32, 16, 1024),
-                                smem_desc_sw128(sk + (kk >> 2) * KREG + (kk & 3) * 32, 16, 1024), idS, kk > 0);
+                    tc_mma_bf16(tq + T_S, dq + (((kk >> 2) * QREG + (kk & 3) * 32) >> 4),
+                                dks + (((kk >> 2) * KREG + (kk & 3) * 32) >> 4), idS, kk > 0);
                 tc_commit(&bars[B_SFULL + q]);
                 if (prev >= 0) issue_pv(prev, k - 1);
                 prev = i;

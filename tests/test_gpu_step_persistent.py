@@ -82,3 +82,23 @@ def test_persistent_step_full_size_sampled(L):
     want = oracle_decode(w, inp, 2, seqs)
     assert_close(f64(got)[seqs], want, "bf16", "persistent full size")
     assert int(run.status.item()) == 0
+
+
+def test_persistent_step_reports_contexts_beyond_max_ctx(L):
+    """A workspace sized for a smaller max_ctx than a sequence reaches: the
+    step reports LBCA_ERR_CAPACITY on the status word instead of writing past
+    the partials it was given; other sequences are unaffected in shape."""
+    w = synth.scaled(W["ragged_gqa_decode_append"], ctx=(100, 200), batch=16, steps=1)
+    lens = synth.contexts(w)
+    lens[3] = 20000  # far beyond the max_ctx below
+    inp = synth.make(w, lens=lens)
+    run = DecodeRun(L, w, inp)
+    small = 300
+    assert L.lbca_decode_step_form(run.cfg, run.B, small) == L.LBCA_STEP_PERSISTENT
+    run.max_ctx = small
+    run.step_ws = torch.zeros(L.lbca_decode_step_workspace_bytes(run.cfg, run.B, small), dtype=torch.uint8,
+                              device="cuda")
+    got = fused_step(run)
+    torch.cuda.synchronize()
+    assert int(run.status.item()) == L.LBCA_ERR_CAPACITY
+    assert got.shape == (16, w.n_q_heads, w.head_dim)

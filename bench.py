@@ -341,7 +341,9 @@ def run_ours(args, w, rank, world):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src,
                      "kernel": ({L.LBCA_STEP_CLUSTER: "decode_step_kernel (cluster form)",
-                                 L.LBCA_STEP_PERSISTENT: "decode_flat_kernel (persistent evenly split form)"}
+                                 L.LBCA_STEP_PERSISTENT: "decode_flat_kernel (persistent evenly split form)",
+                                 L.LBCA_STEP_SHARED_TC: "decode_mqa_tc_kernel (shared-entry tensor-core form, "
+                                                        "append fused)"}
                                 .get(bench.form, "the decode launch of the step (timed alone over the same replicas)")),
                      "bytes_per_launch": nbytes / K, "launch_us": kernel_ms * 1e3,
                      "traffic": load_traffic(w_.name)},

@@ -113,6 +113,32 @@ lbca_status check_kv(const lbca_config* c, const void* k, const void* v, const v
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Decode arguments common to every decode launch (no workspace, no split plan).
+DecodeArgs decode_args(const lbca_config* cfg, const void* q, const lbca_cache* cache, const float* sink,
+                       const void* gamma_q, void* out, int32_t* d_status) {
+    DecodeArgs a{};
+    a.dtype = cfg->dtype;
+    a.q = q;
+    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
+    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
+    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    a.status = d_status;
+    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
+    a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
+    a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
+    return a;
+}
+
+// The serving step of the shared-entry form on the tensor-core kernel with the
+// append fused in: bf16, one kv head and a raw window (so an entry finished
+// by this step's token is not yet visible to its query).  Shape tests only.
+bool step_mqa_fused(const lbca_config* c, int batch, int max_ctx) {
+    return c->n_kv_heads == 1 && c->n_win >= 1 &&
+           mqa_tc_shape_ok(c->dtype, batch, c->n_q_heads, c->n_kv_heads, c->head_dim, c->block_m, c->n_win,
+                           c->shared_kv, max_ctx);
+}
+
 // The decode launch: the tensor-core kernel for the shared-entry form where it
 // applies (it needs no workspace), else the CUDA-core split-KV kernel.
 lbca_status run_decode(const lbca_config* cfg, DecodeArgs& a, int32_t max_ctx, cudaStream_t s) {
@@ -221,26 +247,17 @@ lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache*
     if (workspace_bytes < decode_workspace_bytes(p)) return LBCA_ERR_CAPACITY;
     LBCA_TRY(check_device());
     char* ws = static_cast<char*>(workspace);
-    DecodeArgs a{};
-    a.dtype = cfg->dtype;
-    a.q = q;
-    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
-    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
-    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, out, d_status);
     a.part_o = reinterpret_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float*>(ws + align256(p.part_o_elems * 4));
     a.counters = reinterpret_cast<uint32_t*>(ws + align256(p.part_o_elems * 4) + align256(p.part_ml_elems * 4));
-    a.status = d_status;
-    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
-    a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
-    a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
-    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
     return run_decode(cfg, a, max_ctx, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t lbca_decode_step_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
     if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return 0;
+    if (step_mqa_fused(cfg, batch, max_ctx)) return 256;  // the fused tensor-core step uses none
     StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
                             cfg->n_win, cfg->shared_kv, max_ctx);
     if (sp.ok) return step_workspace_bytes(sp);
@@ -251,14 +268,16 @@ int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch, int32_t
     if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return -1;
     const StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
                                   cfg->n_win, cfg->shared_kv, max_ctx);
-    return sp.ok ? 1 : 2;
+    return (step_mqa_fused(cfg, batch, max_ctx) || sp.ok) ? 1 : 2;
 }
 
 int32_t lbca_decode_step_form(const lbca_config* cfg, int32_t batch, int32_t max_ctx) {
     if (check_cfg(cfg) != LBCA_OK || batch < 0 || max_ctx < 1) return -1;
     const StepPlan sp = plan_step(cfg->dtype, batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
                                   cfg->n_win, cfg->shared_kv, max_ctx);
-    return !sp.ok ? LBCA_STEP_TWO_CALLS : sp.flat ? LBCA_STEP_PERSISTENT : LBCA_STEP_CLUSTER;
+    if (step_mqa_fused(cfg, batch, max_ctx)) return LBCA_STEP_SHARED_TC;
+    if (!sp.ok) return LBCA_STEP_TWO_CALLS;
+    return sp.flat ? LBCA_STEP_PERSISTENT : LBCA_STEP_CLUSTER;
 }
 
 lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* v, const void* zk, const void* zv,
@@ -276,9 +295,21 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
         const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
         max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
     }
+    if (step_mqa_fused(cfg, cache->batch, max_ctx)) {  // shared-entry tensor-core decode, append fused
+        LBCA_TRY(check_device());
+        const MqaTcPlan tp = plan_decode_mqa_tc(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads,
+                                                cfg->head_dim, cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+        if (tp.cs == 0) return LBCA_ERR_UNSUPPORTED;  // no cluster of the kernel fits this device
+        DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, out, d_status);
+        a.app_k = k; a.app_z = zk; a.app_bp = b_pos_k; a.gamma_kv = gamma_kv;
+        a.ring_w = cache->ring_k; a.pooled_w = cache->pooled_k; a.state = cache->pool_state;
+        a.lens_w = cache->seq_lens;
+        a.tc_cs = tp.cs; a.chunk = tp.rows;
+        return cuda_status(launch_decode_mqa_tc(a, reinterpret_cast<cudaStream_t>(stream)));
+    }
     StepPlan sp = plan_step(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
                             cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
-    if (!sp.ok) {  // shapes the fused kernel does not take: the two-launch path
+    if (!sp.ok) {  // shapes no fused kernel takes: the two-launch path
         LBCA_TRY(lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache, d_status, stream));
         return lbca_decode(cfg, q, cache, sink, gamma_q, max_ctx, out, workspace, workspace_bytes, d_status,
                            stream);

@@ -46,6 +46,18 @@
 //      rotated dims back by -t and writes bf16.
 // A sequence whose whole visible list fits one chunk skips the exchange: its
 // first CTA takes every entry and writes the output straight from TMEM.
+//
+// Serving step (append fused, one kv head): the new token is cached first and
+// the query attends at the new length L = cached + 1 (mSeek README, "How LBCA
+// works", steps 2-4).  Its finalised raw entry is the last visible row, so the
+// CTA whose chunk ends the list appends it with one warp while the other rows'
+// copies are in flight: running per-channel softmax of the open block (and the
+// finished pooled entry when the token closes a block), RMSNorm and RoPE at t,
+// the bf16 row to the ring and straight into its own staged tile.  With a
+// window (n_win > 0) a block closed at this step is not yet visible, so no
+// other CTA needs what the append writes.  The arithmetic and its order are
+// those of the stand-alone append kernel, so the cache and the output are
+// bit-identical to append followed by decode.
 #include <algorithm>
 
 #include "common.cuh"
@@ -144,6 +156,162 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
     return __half22float2(h);
 }
 
+// Sequential sum over the warp of each lane's CPL values, in chunk order
+// (chunk c * 32 + lane holds v[c]): the order of the stand-alone append's
+// per-head sum, so both give the same bits.
+template <int CPL>
+__device__ __forceinline__ float chunk_order_sum(const float (&v)[CPL]) {
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c)
+#pragma unroll
+        for (int src = 0; src < 32; ++src) s += __shfl_sync(0xffffffffu, v[c], src);
+    return s;
+}
+
+// RMSNorm (when on) and RoPE of one lane's chunks of a finished entry; cos/sin
+// from `cs` (pairs from dim D - rho on) or, when it is null, at position `rpos`.
+template <int D, int CPL>
+__device__ __forceinline__ void finalise_row(const DecodeArgs& a, float (&e)[CPL][8], int lane, const float2* cs,
+                                             int64_t rpos) {
+    if (a.rmsnorm) {
+        float v[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            v[c] = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[c] += e[c][k] * e[c][k];
+        }
+        const float ss = chunk_order_sum<CPL>(v);
+        const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+        const __nv_bfloat16* gm = static_cast<const __nv_bfloat16*>(a.gamma_kv);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            float gam[8];
+            if (gm) {
+                ld16(gm + (c * 32 + lane) * 8, gam);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) gam[k] = 1.0f;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) e[c][k] *= inv * gam[k];
+        }
+    }
+    if (a.rho) {
+        const int base = D - a.rho;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+                const int d = (c * 32 + lane) * 8 + k;
+                if (d >= base) {
+                    const int kk = (d - base) >> 1;
+                    rotate_pair(e[c][k], e[c][k + 1], cs ? cs[kk] : rope_cs(rpos, kk, a.rope_step));
+                }
+            }
+    }
+}
+
+// The fused append of the new token at `pos` for (sequence b, kv head g), by
+// one warp: lane l owns the 16-byte chunks l, l + 32, ... of the D-dim row.
+// The running per-channel softmax of the open block (max, sum and weighted
+// sum in the log2 domain, the B_pos row of the token's offset) is advanced;
+// a token that closes block j finishes entry j (weighted sum / sum, RMSNorm,
+// RoPE at the block start j m) into pooled_k, otherwise the state is stored
+// back; the raw token (RMSNorm, RoPE at pos, from `cs_t`) goes to its ring
+// slot and, when `row` >= 0, to that row of the staged bf16 entry tile.
+template <int D>
+__device__ __forceinline__ void append_token(const DecodeArgs& a, int b, int g, int pos, const float2* cs_t,
+                                             uint8_t* sE, uint32_t ereg, int row, int lane) {
+    constexpr int CPL = D / 256;
+    const int GD = a.G * D;
+    const int i = pos % a.m, jb = pos / a.m;
+    const size_t tok = ((size_t)b * a.G + g) * D;
+    const __nv_bfloat16* xk = static_cast<const __nv_bfloat16*>(a.app_k) + tok;
+    const __nv_bfloat16* zk = static_cast<const __nv_bfloat16*>(a.app_z) + tok;
+    const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(a.app_bp) + (size_t)i * GD + (size_t)g * D;
+    float* st = a.state + (size_t)b * 3 * GD + (size_t)g * D;
+    float x[CPL][8], mx[CPL][8], l[CPL][8], acc[CPL][8];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int d0 = (c * 32 + lane) * 8;
+        float z[8], bpv[8];
+        ld16(xk + d0, x[c]);
+        ld16(zk + d0, z);
+        ld16(bp + d0, bpv);
+        float m0[8], l0[8], a0[8];
+        if (i > 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 u = *reinterpret_cast<const float4*>(st + d0 + 4 * h);
+                const float4 w = *reinterpret_cast<const float4*>(st + GD + d0 + 4 * h);
+                const float4 y = *reinterpret_cast<const float4*>(st + 2 * GD + d0 + 4 * h);
+                m0[4 * h] = u.x; m0[4 * h + 1] = u.y; m0[4 * h + 2] = u.z; m0[4 * h + 3] = u.w;
+                l0[4 * h] = w.x; l0[4 * h + 1] = w.y; l0[4 * h + 2] = w.z; l0[4 * h + 3] = w.w;
+                a0[4 * h] = y.x; a0[4 * h + 1] = y.y; a0[4 * h + 2] = y.z; a0[4 * h + 3] = y.w;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float av = (z[e] + bpv[e]) * kLog2e;
+            if (i == 0) {
+                mx[c][e] = av; l[c][e] = 1.f; acc[c][e] = x[c][e];
+            } else {
+                const float mn = fmaxf(m0[e], av);
+                const float r = ex2(m0[e] - mn), p = ex2(av - mn);
+                mx[c][e] = mn;
+                l[c][e] = l0[e] * r + p;
+                acc[c][e] = fmaf(p, x[c][e], a0[e] * r);
+            }
+        }
+    }
+    if (i == a.m - 1) {  // the token closes block jb
+        float e[CPL][8];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) e[c][k] = acc[c][k] / l[c][k];
+        finalise_row<D, CPL>(a, e, lane, nullptr, (int64_t)jb * a.m);
+        if (jb < a.max_blocks) {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.pooled_w) + (((size_t)b * a.G + g) * a.max_blocks + jb) * D;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) st16(o + (c * 32 + lane) * 8, e[c]);
+        } else if (lane == 0) {
+            set_status(a.status, LBCA_ERR_CAPACITY);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int d0 = (c * 32 + lane) * 8;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                *reinterpret_cast<float4*>(st + d0 + 4 * h) =
+                    make_float4(mx[c][4 * h], mx[c][4 * h + 1], mx[c][4 * h + 2], mx[c][4 * h + 3]);
+                *reinterpret_cast<float4*>(st + GD + d0 + 4 * h) =
+                    make_float4(l[c][4 * h], l[c][4 * h + 1], l[c][4 * h + 2], l[c][4 * h + 3]);
+                *reinterpret_cast<float4*>(st + 2 * GD + d0 + 4 * h) =
+                    make_float4(acc[c][4 * h], acc[c][4 * h + 1], acc[c][4 * h + 2], acc[c][4 * h + 3]);
+            }
+        }
+    }
+    finalise_row<D, CPL>(a, x, lane, cs_t, 0);
+    __nv_bfloat16* ring = static_cast<__nv_bfloat16*>(a.ring_w) + (((size_t)b * a.G + g) * a.R + pos % a.R) * D;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int ch = c * 32 + lane;
+        uint4 u;
+        u.x = pack_bf16x2(x[c][0], x[c][1]);
+        u.y = pack_bf16x2(x[c][2], x[c][3]);
+        u.z = pack_bf16x2(x[c][4], x[c][5]);
+        u.w = pack_bf16x2(x[c][6], x[c][7]);
+        *reinterpret_cast<uint4*>(ring + ch * 8) = u;
+        if (row >= 0)
+            *reinterpret_cast<uint4*>(sE + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+                                      (uint32_t)(ch >> 3) * ereg + ((uint32_t)((ch & 7) ^ (row & 7)) << 4)) = u;
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const DecodeArgs a) {
     constexpr int CPR = D / 8;    // 16-byte chunks per entry row
@@ -171,7 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     const int SW = owned_dims(D, CS);
 
     // ---- visible set of this sequence (block-aligned partition) and this CTA's chunk ----
-    const int L = a.seq_lens[b];
+    const bool fuse = a.app_k != nullptr;
+    const int pos = a.seq_lens[b];  // cached tokens (fused: the new token's position)
+    const int L = fuse ? pos + 1 : pos;
     const int t = L - 1;
     const int P = visible_blocks(L, a.m, a.w);
     const int s0 = P * a.m;
@@ -185,6 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     const int e0 = single ? 0 : rank * chunk;
     const int n = single ? (rank == 0 ? n_vis : 0) : max(0, min(n_vis, e0 + chunk) - e0);
     const int n16 = (n + 15) & ~15;
+    // fused append: the CTA holding the last visible row (the new token), the
+    // warp that would have copied that row; row -1 when nothing is visible
+    const int app_rank = (n_vis == 0 || single) ? 0 : (n_vis - 1) / chunk;
+    const bool appender = fuse && rank == app_rank;
+    const int app_row = (appender && n_vis > 0) ? n_vis - 1 - e0 : -1;
+    const int app_warp = app_row >= 0 ? app_row % kWarps : 0;
 
     // query groups this CTA prepares for the whole cluster
     const int preppers = CS >= 8 ? 8 : (CS >= 4 ? 4 : (CS >= 2 ? 2 : 1));
@@ -212,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     const __nv_bfloat16* pk = static_cast<const __nv_bfloat16*>(a.pooled_k);
     const __nv_bfloat16* rk = static_cast<const __nv_bfloat16*>(a.ring_k);
     for (int row = warp; row < n16; row += kWarps) {
+        if (row == app_row) continue;  // the new token: written below by this warp
         const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.q);  // any valid address (zero fill)
         uint32_t bytes = 0;
         if (row < n) {
@@ -286,8 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
         }
         fence_async_smem();
     }
+    if (appender && warp == app_warp) append_token<D>(a, b, g, pos, cs, smem + lay.OFF_E, lay.EREG, app_row, lane);
     __syncthreads();
-    cluster_wait_acquire();  // every CTA's barriers exist
+    cluster_wait_acquire();  // every CTA's barriers exist; every CTA has read seq_lens[b]
+    if (appender && tid == 0) a.lens_w[b] = pos + 1;
     const bool q_sender = prepper && tid < CS && tid != rank;
     if (q_sender) {  // this CTA's query groups to CTA `tid`
         for (int G = rank * gpc; G < rank * gpc + gpc; ++G) {
@@ -587,19 +766,36 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+namespace {
+// Entry rows per CTA for cs CTAs per cluster over at most max_vis visible entries.
+int rows_for(long long max_vis, int cs) {
+    return std::max<int>(16, (int)(((max_vis + cs - 1) / cs + 15) / 16 * 16));
+}
+long long max_visible(int m, int w, int max_ctx) {
+    const long long P = max_ctx - w > 0 ? (long long)(max_ctx - w) / m : 0;
+    return std::min<long long>(max_ctx, P + w + m - 1);
+}
+}  // namespace
+
+bool mqa_tc_shape_ok(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
+    if (dtype != LBCA_BF16 || !shared || G < 1 || Hq != NH * G || (D != 256 && D != 512)) return false;
+    if (B < 1 || max_ctx < 1) return false;
+    const long long max_vis = max_visible(m, w, max_ctx);
+    for (int cs = (int)std::max<long long>(1, (max_vis + 127) / 128); cs <= kMaxCS; ++cs)
+        if (MqaLayout(D, rows_for(max_vis, cs), cs).SMEM <= 227u * 1024u) return true;
+    return false;
+}
+
 MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
     MqaTcPlan p{0, 0};
-    if (dtype != LBCA_BF16 || !shared || G < 1 || Hq != NH * G || (D != 256 && D != 512)) return p;
-    if (B < 1 || max_ctx < 1) return p;
-    const long long P = max_ctx - w > 0 ? (long long)(max_ctx - w) / m : 0;
-    const long long max_vis = std::min<long long>(max_ctx, P + w + m - 1);
+    if (!mqa_tc_shape_ok(dtype, B, Hq, G, D, m, w, shared, max_ctx)) return p;
+    const long long max_vis = max_visible(m, w, max_ctx);
     const int cs_min = (int)std::max<long long>(1, (max_vis + 127) / 128);
-    if (cs_min > kMaxCS) return p;
     // fewest waves of clusters first, then the widest cluster (the most SMs streaming)
     const long long groups = (long long)B * G;
     long long best_waves = 0;
     for (int cs = kMaxCS; cs >= cs_min; --cs) {
-        const int rows = std::max<int>(16, (int)(((max_vis + cs - 1) / cs + 15) / 16 * 16));
+        const int rows = rows_for(max_vis, cs);
         const MqaLayout lay(D, rows, cs);
         if (lay.SMEM > 227u * 1024u) continue;
         const int act = D == 512 ? max_active_clusters<512>(cs, lay.SMEM) : max_active_clusters<256>(cs, lay.SMEM);

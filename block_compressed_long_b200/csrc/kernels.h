@@ -81,6 +81,13 @@ struct DecodeArgs {
     int tc_cs;         // tensor-core shared-entry path: CTAs per cluster (0 = CUDA-core path)
     float eps, scale;
     double rope_step;  // theta^(-2/rho)
+    // Append fused into the tensor-core shared-entry kernel (app_k == nullptr:
+    // none; one kv head only).  The new token [B, G, D] and its Z logits join
+    // the cache first, then the query at the new length attends.
+    const void* app_k; const void* app_z; const void* app_bp; const void* gamma_kv;
+    void* ring_w; void* pooled_w;                    // the cache's ring_k / pooled_k, written
+    float* state;                                    // [B, 1, 3, G, D]
+    int32_t* lens_w;                                 // seq_lens, advanced by one
 };
 // Chooses heads per CTA, chunk and split count for a decode call.
 struct DecodePlan {
@@ -100,6 +107,8 @@ struct MqaTcPlan {
     int cs, rows;
 };
 MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+// The shape tests of plan_decode_mqa_tc alone (host-only, no device query).
+bool mqa_tc_shape_ok(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
 cudaError_t launch_decode_mqa_tc(const DecodeArgs& a, cudaStream_t s);
 
 // One serving step (append + decode) in one cluster launch.

@@ -207,7 +207,7 @@ def lbca_decode_step_launches(cfg: lbca_config, batch: int, max_ctx: int) -> int
     return int(_lib.lbca_decode_step_launches(ctypes.byref(cfg), batch, max_ctx))
 
 
-LBCA_STEP_TWO_CALLS, LBCA_STEP_CLUSTER, LBCA_STEP_PERSISTENT = range(3)
+LBCA_STEP_TWO_CALLS, LBCA_STEP_CLUSTER, LBCA_STEP_PERSISTENT, LBCA_STEP_SHARED_TC = range(4)
 
 
 def lbca_decode_step_form(cfg: lbca_config, batch: int, max_ctx: int) -> int:

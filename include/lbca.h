@@ -212,7 +212,10 @@ LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lb
  * (sequence, head group) pairs a cluster kernel that splits each pair's
  * entries over the CTAs of a cluster, for many pairs (96 or more) a
  * persistent kernel whose CTAs each take an equal share of all the step's
- * entries, whatever the mix of context lengths.  Other shapes run lbca_append
+ * entries, whatever the mix of context lengths.  The shared-entry form on
+ * the tensor-core decode (bf16, 64 query heads per kv head, D in {256, 512})
+ * with one kv head and n_win >= 1 also runs as one kernel: the CTA that holds
+ * the newest visible row appends the token.  Other shapes run lbca_append
  * then lbca_decode.  Results equal those of the two calls.  A sequence longer
  * than max_ctx sets d_status to LBCA_ERR_CAPACITY.
  */
@@ -225,7 +228,8 @@ LBCA_API int32_t lbca_decode_step_launches(const lbca_config* cfg, int32_t batch
 typedef enum {
     LBCA_STEP_TWO_CALLS = 0,   /* lbca_append, then lbca_decode */
     LBCA_STEP_CLUSTER = 1,     /* one cluster kernel */
-    LBCA_STEP_PERSISTENT = 2   /* one persistent, evenly split kernel */
+    LBCA_STEP_PERSISTENT = 2,  /* one persistent, evenly split kernel */
+    LBCA_STEP_SHARED_TC = 3    /* one tensor-core shared-entry kernel, append fused */
 } lbca_step_form;
 /* Returns an lbca_step_form, or -1 for an invalid configuration. */
 LBCA_API int32_t lbca_decode_step_form(const lbca_config* cfg, int32_t batch, int32_t max_ctx);

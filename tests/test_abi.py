@@ -115,12 +115,15 @@ def test_cache_and_decode_checks(L):
 
 
 def test_decode_step_launches(L):
-    """One fused kernel for the GQA step shapes, append + decode for the
-    shared-entry D = 512 form (and for no window); -1 for a bad config."""
+    """One fused kernel for the GQA step shapes and for the shared-entry
+    D = 512 form with one kv head; append + decode for two kv heads of that
+    form and for no window; -1 for a bad config."""
     assert L.lbca_decode_step_launches(_cfg(L), 1, 32769) == 1
     assert L.lbca_decode_step_launches(_cfg(L, n_win=0), 1, 32769) == 2
     hca = _cfg(L, n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128, rope_dims=64)
-    assert L.lbca_decode_step_launches(hca, 8, 131073) == 2
+    assert L.lbca_decode_step_launches(hca, 8, 131073) == 1
+    assert L.lbca_decode_step_launches(_cfg(L, n_q_heads=128, n_kv_heads=2, head_dim=512, shared_kv=True,
+                                            block_m=128, rope_dims=64), 8, 131073) == 2
     assert L.lbca_decode_step_launches(_cfg(L, block_m=0), 1, 100) == -1
 
 
@@ -132,6 +135,10 @@ def test_decode_step_form(L):
     assert L.lbca_decode_step_form(cfg, 1, 32769) == L.LBCA_STEP_CLUSTER
     assert L.lbca_decode_step_form(cfg, 32, 65600) == L.LBCA_STEP_PERSISTENT
     assert L.lbca_decode_step_form(_cfg(L, n_win=0), 32, 65600) == L.LBCA_STEP_TWO_CALLS
+    hca = _cfg(L, n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128, rope_dims=64)
+    assert L.lbca_decode_step_form(hca, 8, 131073) == L.LBCA_STEP_SHARED_TC
+    assert L.lbca_decode_step_form(_cfg(L, n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128,
+                                        rope_dims=64, n_win=0), 8, 131073) == L.LBCA_STEP_TWO_CALLS
     assert L.lbca_decode_step_form(_cfg(L, block_m=0), 32, 100) == -1
     small = L.lbca_decode_step_workspace_bytes(cfg, 32, 4096)
     big = L.lbca_decode_step_workspace_bytes(cfg, 32, 65600)

@@ -97,10 +97,23 @@ def test_empty_sequence_gives_zeros(L):
     assert int(run.status.item()) == 0
 
 
-def test_step_entry_point_equals_append_then_decode(L):
-    """lbca_decode_step on this form runs append then the tensor-core decode:
-    bit-identical to the two calls."""
-    w, inp = _inputs(W, [300, 1500, 40], 3)
+def _cache_equal(x, y, what):
+    for name in ("pooled_k", "ring_k", "pool_state", "seq_lens"):
+        assert torch.equal(getattr(x.cache, name), getattr(y.cache, name)), f"{what}: {name}"
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(head_dim=256, rmsnorm=False, sink="none")], ids=["hca", "d256"])
+def test_step_entry_point_equals_append_then_decode(L, kw):
+    """lbca_decode_step on this form is one launch, the append done by the CTA
+    that holds the newest visible row: output, ring, pooled entries, running
+    pool state and lengths bit-identical to lbca_append then lbca_decode.  The
+    lengths put steps on a block's last token (an entry finishes), on a block's
+    first token (the running state restarts), in a one-CTA list and in lists
+    split over the cluster."""
+    w = synth.scaled(W, **kw)
+    assert L.lbca_decode_step_launches(L.config(**_cfg_kw(w)), 5, 3000) == 1
+    assert L.lbca_decode_step_form(L.config(**_cfg_kw(w)), 5, 3000) == L.LBCA_STEP_SHARED_TC
+    w, inp = _inputs(w, [383, 1500, 40, 255, 2900], 3)
     a = DecodeRun(L, w, inp, steps=3)
     b = DecodeRun(L, w, inp, steps=3)
     for s in range(3):
@@ -108,5 +121,25 @@ def test_step_entry_point_equals_append_then_decode(L):
         y = fused_step(b)
         torch.cuda.synchronize()
         assert torch.equal(x, y), f"step {s}"
+        _cache_equal(a, b, f"step {s}")
         assert_close(f64(y), oracle_decode(w, inp, s), "bf16", f"step {s}")
     assert int(a.status.item()) == 0 and int(b.status.item()) == 0
+
+
+def _cfg_kw(w):
+    return dict(n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, shared_kv=w.shared_kv,
+                block_m=w.block_m, n_win=w.n_win, rope_dims=w.rope_dims, rmsnorm=w.rmsnorm)
+
+
+def test_step_with_two_kv_heads_takes_two_calls(L):
+    """Two kv heads of the shared form: the step runs append then decode and
+    still matches the oracle."""
+    w = synth.scaled(W, n_kv_heads=2, n_q_heads=128)
+    assert L.lbca_decode_step_launches(L.config(**_cfg_kw(w)), 2, 3000) == 2
+    w, inp = _inputs(w, [383, 700], 2)
+    run = DecodeRun(L, w, inp, steps=2)
+    for s in range(2):
+        y = fused_step(run)
+        torch.cuda.synchronize()
+        assert_close(f64(y), oracle_decode(w, inp, s), "bf16", f"step {s}")
+    assert int(run.status.item()) == 0

@@ -101,18 +101,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* f
     return __all_sync(0xffffffffu, wait_or_fail(bar, parity, fail, status));
 }
 
-// 2^x on the FMA pipe, after Cody and Waite's range reduction: x = n + f with
-// n = rint(x) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial (a weighted
-// least-squares fit of 2^f on that interval, relative error below 7.5e-5, under
-// half an fp16 ulp, the precision P is kept in); 2^n added to the exponent
-// field.  Inputs below -125 (masked scores are -inf) give 2^-125, which is 0 in
-// fp16; inputs are at most 8 here (the lazy rescale bounds them).
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
-    const float f = x - (t - 12582912.0f);
-    const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// 2^x for a pair of values on the FMA pipe (packed f32x2), after Cody and
+// Waite's range reduction: x = n + f with n = rint(x) and f in [-1/2, 1/2]; 2^f
+// from a degree-3 polynomial (a weighted least-squares fit of 2^f on that
+// interval, relative error below 7.5e-5, under half an fp16 ulp, the precision
+// P is kept in); 2^n added to the exponent field.  Inputs below -125 (masked
+// scores are -inf) give 2^-125, which is 0 in fp16; inputs are at most 8 here
+// (the lazy rescale bounds them).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = fadd2(x, make_float2(kShift, kShift));
+    const float2 n = fadd2(t, make_float2(-kShift, -kShift));
+    const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
+    float2 p = ffma2(make_float2(0.0551716648f, 0.0551716648f), f, make_float2(0.2426111251f, 0.2426111251f));
+    p = ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+    p = ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // The K/V tiles of a CTA run over the pooled entries [0, npt BN) and then the
@@ -339,21 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             else { c_lo = max(0, lo - base); c_hi = min(BN, t - base + 1); }
             if (!valid) c_hi = 0;
             c_hi = max(c_hi, c_lo);  // an empty range masks every column
-            float mxv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mxv[e] = kNegInf;
             if (__any_sync(0xffffffffu, c_lo > 0 || c_hi < BN)) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
+                for (int c = 0; c < BN; ++c)
                     if ((unsigned)(c - c_lo) >= (unsigned)(c_hi - c_lo)) s[c] = kNegInf;
-                    mxv[c & 7] = fmaxf(mxv[c & 7], s[c]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) mxv[c & 7] = fmaxf(mxv[c & 7], s[c]);
             }
-            const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
-                                   fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
+            float mxv[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+            for (int c = 0; c < BN / 2; ++c) mxv[c & 3] = fmax3(mxv[c & 3], s[2 * c], s[2 * c + 1]);
+            const float mx = fmax3(fmaxf(mxv[0], mxv[1]), mxv[2], mxv[3]);
             // lazy rescale: only when the row max grows by more than 2^8 in probability
             float alpha = 1.f;
             bool rescale = false;
@@ -382,22 +383,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             // P buffer k & 1 is free once the P V of tile k-2 has read it
             if (k >= 2) ok = warp_wait(&bars[B_PVDONE + 2 * q + (k & 1)], ((k >> 1) - 1) & 1, fail, a.status);
             if (!ok) break;
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            // exponentials in pairs: pairs 1, 4 and 6 of every 8 on the FMA pipe
+            // (packed polynomial), the rest on the SFU, which 3/8 relieves enough
+            // for the two warps sharing each SFU to keep pace with the FMA pipe
+            float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             float pk[32];
+            const float2 sc2 = make_float2(sc, sc), mn2 = make_float2(mneg, mneg);
 #pragma unroll
-            for (int e = 0; e < BN / 2; ++e) {  // one exponential in four on the FMA pipe
-                const float p0 = ex2(fmaf(s[2 * e], sc, mneg));
-                const float x1 = fmaf(s[2 * e + 1], sc, mneg);
-                const float p1 = (e & 1) ? exp2_fma(x1) : ex2(x1);
-                ps[e & 3] += p0 + p1;
-                pk[e] = __uint_as_float(pack_f16x2(p0, p1));
+            for (int e = 0; e < BN / 2; ++e) {
+                const float2 x = ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, mn2);
+                float2 p;
+                if ((0x52u >> (e & 7)) & 1u) {
+                    p = exp2_fma2(x);
+                } else {
+                    p.x = ex2(x.x);
+                    p.y = ex2(x.y);
+                }
+                ps[e & 1] = fadd2(ps[e & 1], p);
+                pk[e] = __uint_as_float(pack_f16x2(p.x, p.y));
             }
             tc_fence_after();
             tmem_st32(tP + 32 * (k & 1), pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + q]);
-            l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            l = l * alpha + ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y));
             ++k;
         }
         // ---- epilogue: normalise the O row into this query tile's shared memory

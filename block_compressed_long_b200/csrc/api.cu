@@ -387,6 +387,17 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
         pooled_bytes = align256(one) * (cfg->shared_kv ? 1 : 2);
     }
     char* tc_scratch = static_cast<char*>(workspace) + pooled_bytes;
+    PrefillArgs pa{};
+    pa.dtype = cfg->dtype;
+    pa.q = q; pa.k = k; pa.v = v; pa.pooled_k = pk; pa.pooled_v = cfg->shared_kv ? pk : pv;
+    pa.pool_stride = stride; pa.sink = sink; pa.gamma_q = gamma_q; pa.gamma_kv = gamma_kv; pa.out = out;
+    pa.B = batch; pa.T = T; pa.Hq = cfg->n_q_heads; pa.G = cfg->n_kv_heads; pa.D = cfg->head_dim;
+    pa.m = m; pa.w = cfg->n_win; pa.rho = cfg->rope_dims; pa.rmsnorm = cfg->rmsnorm;
+    pa.shared = cfg->shared_kv; pa.eps = cfg->rms_eps; pa.scale = scale_of(cfg); pa.rope_step = rope_step_of(cfg);
+    // the tensor-core path: cos/sin table first, so that the pool pass can leave
+    // fp16 copies of the raw keys (rotated) and values as it streams them
+    if (use_tc) LBCA_TRY(cuda_status(launch_prefill_tc_table(pa, tc_scratch, s)));
+    const PrefillRawF16 raw16 = use_tc ? prefill_tc_raw_f16(pa, tc_scratch) : PrefillRawF16{nullptr, nullptr, nullptr};
     for (int series = 0; series < (cfg->shared_kv ? 1 : 2); ++series) {
         PoolArgs a{};
         a.dtype = cfg->dtype;
@@ -405,6 +416,8 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
                                           : prefill_tc_pooled_v_f16_offset(batch, T, cfg->n_kv_heads,
                                                                            cfg->rope_dims, m));
             a.out_f16_blocks = NB;
+            a.raw_f16 = series == 0 ? raw16.keys : raw16.vals;
+            a.tab = raw16.tab;
         }
         LBCA_TRY(cuda_status(launch_pool(a, s)));
     }
@@ -421,17 +434,10 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
     }
     // 3. attention
     if (out) {
-        PrefillArgs a{};
-        a.dtype = cfg->dtype;
-        a.q = q; a.k = k; a.v = v; a.pooled_k = pk; a.pooled_v = cfg->shared_kv ? pk : pv;
-        a.pool_stride = stride; a.sink = sink; a.gamma_q = gamma_q; a.gamma_kv = gamma_kv; a.out = out;
-        a.B = batch; a.T = T; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
-        a.m = m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
-        a.shared = cfg->shared_kv; a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
         if (use_tc) {
-            LBCA_TRY(cuda_status(launch_prefill_tc(a, tc_scratch, d_status, s)));
+            LBCA_TRY(cuda_status(launch_prefill_tc(pa, tc_scratch, d_status, s)));
         } else {
-            LBCA_TRY(cuda_status(launch_prefill_simt(a, s)));
+            LBCA_TRY(cuda_status(launch_prefill_simt(pa, s)));
         }
     }
     return LBCA_OK;

@@ -26,6 +26,11 @@ struct PoolArgs {
     int S, series;
     void* out_f16;         // optional fp16 copy [B, G, out_f16_blocks, D] (bf16 input only)
     int out_f16_blocks;
+    // optional fp16 copy of every token of each complete block, [B, T, G, D]
+    // (bf16 input only); key series rotated at their position s with cos/sin
+    // from `tab` ([rho/2][T], pair-major)
+    void* raw_f16;
+    const float2* tab;
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 
@@ -171,6 +176,15 @@ size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m);
 // where, inside that scratch, the pool pass leaves the fp16 copy of the pooled keys
 size_t prefill_tc_pooled_f16_offset(int B, int T, int G, int rho);
 size_t prefill_tc_pooled_v_f16_offset(int B, int T, int G, int rho, int m);
+// The parts of that scratch the pool pass fills for the tensor-core kernel: fp16
+// raw keys (rotated) and values of every complete block, from the cos/sin table.
+struct PrefillRawF16 {
+    void* keys; void* vals; const float2* tab;
+};
+PrefillRawF16 prefill_tc_raw_f16(const PrefillArgs& a, void* scratch);
+// 1. the cos/sin table (before the pool pass); 2. the tail tokens past the last
+// complete block, then the attention kernel (after it).
+cudaError_t launch_prefill_tc_table(const PrefillArgs& a, void* scratch, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, void* scratch, int32_t* status, cudaStream_t s);
 bool prefill_simt_supported(int D);
 

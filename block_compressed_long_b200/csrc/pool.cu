@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     float mx[VEC], l[VEC], acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) { mx[e] = kNegInf; l[e] = 0.f; acc[e] = 0.f; }
+    const int g = cv / NVH, d0 = (cv % NVH) * VEC;
+    const bool raw_copy = VEC == 8 && a.raw_f16 && full;  // uniform per CTA
 
     if (active) {
         // U tokens per step: their X, Z and B_pos vectors are loaded together
@@ -112,6 +114,24 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
                     cz[u] = __ldcs(zp + (size_t)(i0 + u) * rstride);
                     cb[u] = __ldg(bp + (size_t)(i0 + u) * rstride);
                 }
+            if constexpr (VEC == 8) {
+                if (raw_copy) {  // these tokens' fp16 copy; keys turned at their position
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        if (i0 + u < n_tok) {
+                            float xf[VEC];
+                            unpack<T>(cx[u], xf);
+                            const int s_tok = j * a.m + i0 + u;
+                            const int dr = d0 - (a.D - a.rho);
+                            if (a.key && a.rho)
+#pragma unroll
+                                for (int e = 0; e < VEC; e += 2)
+                                    if (dr + e >= 0)
+                                        rotate_pair(xf[e], xf[e + 1], a.tab[(size_t)((dr + e) >> 1) * a.T + s_tok]);
+                            st16_f16(static_cast<__half*>(a.raw_f16) + row0 + (size_t)(i0 + u) * GD, xf);
+                        }
+                }
+            }
             float cmax[VEC];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) cmax[e] = mx[e];
@@ -150,7 +170,6 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
         }
     }
 
-    const int g = cv / NVH, d0 = (cv % NVH) * VEC;
     if (full) {
         float e[VEC];
 #pragma unroll

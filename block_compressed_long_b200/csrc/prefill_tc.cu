@@ -462,13 +462,16 @@ __global__ void rope_table_kernel(float2* tab, int T, int half, double step) {
         tab[i] = rope_cs(i % T, (int)(i / T), step);
 }
 
-// Finalised raw keys (RoPE at s applied once) and raw values, both widened to
-// fp16, the operand type of the tensor-core MMAs; same [B, T, G, D] layout.
+// Finalised raw keys (RoPE at s applied once) and raw values of tokens
+// [s_begin, T), both widened to fp16, the operand type of the tensor-core MMAs;
+// same [B, T, G, D] layout.  (The pool pass writes those of complete blocks.)
 __global__ void finalise_kv_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                                    __half* __restrict__ ko, __half* __restrict__ vo, const float2* __restrict__ tab,
-                                   int64_t n_vec, int G, int T, int rho) {
-    const int half = rho / 2;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec; i += (int64_t)gridDim.x * blockDim.x) {
+                                   int64_t n_vec, int G, int T, int s_begin, int rho) {
+    const int64_t per_b = (int64_t)(T - s_begin) * G * (HD / 8);  // vectors of one sequence's tail
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < n_vec; j += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = j / per_b;
+        const int64_t i = (b * T + s_begin) * G * (HD / 8) + j % per_b;  // vector index in [B, T, G, D / 8]
         const int d0 = (int)(i % (HD / 8)) * 8;
         const int64_t row = i / (HD / 8);            // (b, s, g)
         const int s = (int)((row / G) % T);
@@ -531,25 +534,39 @@ size_t prefill_tc_scratch_bytes(int B, int T, int G, int rho, int m) {
     return prefill_tc_pooled_v_f16_offset(B, T, G, rho, m) + a256((size_t)B * G * (T / m) * HD * 2);
 }
 
+PrefillRawF16 prefill_tc_raw_f16(const PrefillArgs& p, void* scratch) {
+    const size_t raw_bytes = a256((size_t)p.B * p.T * p.G * HD * 2);
+    PrefillRawF16 r;
+    r.keys = scratch;
+    r.vals = static_cast<char*>(scratch) + raw_bytes;
+    r.tab = reinterpret_cast<const float2*>(static_cast<char*>(scratch) + 2 * raw_bytes);
+    return r;
+}
+
+cudaError_t launch_prefill_tc_table(const PrefillArgs& p, void* scratch, cudaStream_t s) {
+    const int half = p.rho / 2;
+    if (p.B == 0 || p.T == 0 || half == 0) return cudaSuccess;
+    float2* tab = const_cast<float2*>(prefill_tc_raw_f16(p, scratch).tab);
+    const int64_t n = (int64_t)p.T * half;
+    rope_table_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 148 * 16), 256, 0, s>>>(tab, p.T, half, p.rope_step);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* status, cudaStream_t s) {
     if (p.B == 0 || p.T == 0) return cudaSuccess;
     const int G = p.G, T = p.T, B = p.B, Hq = p.Hq;
-    const size_t raw_bytes = a256((size_t)B * T * G * HD * 2);
-    __half* keys = static_cast<__half*>(scratch);
-    __half* vals = reinterpret_cast<__half*>(static_cast<char*>(scratch) + raw_bytes);
-    float2* tab = reinterpret_cast<float2*>(static_cast<char*>(scratch) + 2 * raw_bytes);
+    const PrefillRawF16 raw = prefill_tc_raw_f16(p, scratch);
+    __half* keys = static_cast<__half*>(raw.keys);
+    __half* vals = static_cast<__half*>(raw.vals);
+    const float2* tab = raw.tab;
     const void* pooled_k16 = static_cast<char*>(scratch) + prefill_tc_pooled_f16_offset(B, T, G, p.rho);
     const void* pooled_v16 = static_cast<char*>(scratch) + prefill_tc_pooled_v_f16_offset(B, T, G, p.rho, p.m);
-    const int half = p.rho / 2;
-    if (half > 0) {
-        const int64_t n = (int64_t)T * half;
-        rope_table_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 148 * 16), 256, 0, s>>>(tab, T, half, p.rope_step);
-    }
-    {
-        const int64_t nv = (int64_t)B * T * G * (HD / 8);
+    const int s_begin = T / p.m * p.m;  // tokens of complete blocks came from the pool pass
+    if (s_begin < T) {
+        const int64_t nv = (int64_t)B * (T - s_begin) * G * (HD / 8);
         finalise_kv_kernel<<<(int)std::min<int64_t>((nv + 255) / 256, 148 * 32), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v), keys, vals, tab, nv, G, T,
-            p.rho);
+            s_begin, p.rho);
     }
     TcArgs a;
     memset(&a, 0, sizeof(a));

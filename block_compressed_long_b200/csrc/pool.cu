@@ -68,8 +68,10 @@ __device__ __forceinline__ void finalise_key(float (&e)[VEC], int d0, int D, boo
     }
 }
 
-// CTA = (block j, sequence b, slice of whole kv heads); <= 256 threads.
-template <typename T>
+// CTA = (block j, sequence b, slice of whole kv heads); <= 256 threads.  RAW:
+// also the fp16 copy of every token (the tensor-core prefill's operands), in
+// an instantiation of its own so that plain pooling carries none of it.
+template <typename T, bool RAW>
 __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     constexpr int VEC = Vec<T>::N;
     constexpr int U = 4;  // tokens per online-softmax step
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) { mx[e] = kNegInf; l[e] = 0.f; acc[e] = 0.f; }
     const int g = cv / NVH, d0 = (cv % NVH) * VEC;
-    const bool raw_copy = VEC == 8 && a.raw_f16 && full;  // uniform per CTA
+    const bool raw_copy = RAW && VEC == 8 && full;  // uniform per CTA
 
     if (active) {
         // U tokens per step: their X, Z and B_pos vectors are loaded together
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
                     cz[u] = __ldcs(zp + (size_t)(i0 + u) * rstride);
                     cb[u] = __ldg(bp + (size_t)(i0 + u) * rstride);
                 }
-            if constexpr (VEC == 8) {
+            if constexpr (RAW && VEC == 8) {
                 if (raw_copy) {  // these tokens' fp16 copy; keys turned at their position
 #pragma unroll
                     for (int u = 0; u < U; ++u)
@@ -374,10 +376,14 @@ cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s) {
     const int threads = round32(hpc * nvh);
     const size_t smem = (size_t)a.rho * 4 + (size_t)threads * 4;
     dim3 grid(nblk, a.B, (a.G + hpc - 1) / hpc);
-    if (a.dtype == LBCA_BF16)
-        pool_kernel<__nv_bfloat16><<<grid, threads, smem, s>>>(a);
-    else
-        pool_kernel<float><<<grid, threads, smem, s>>>(a);
+    if (a.dtype == LBCA_BF16) {
+        if (a.raw_f16)
+            pool_kernel<__nv_bfloat16, true><<<grid, threads, smem, s>>>(a);
+        else
+            pool_kernel<__nv_bfloat16, false><<<grid, threads, smem, s>>>(a);
+    } else {
+        pool_kernel<float, false><<<grid, threads, smem, s>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -281,7 +281,10 @@ def run_ours(args, w, rank, world):
     # ---- end to end through the public API: pinned host inputs and output ----
     # each step's inputs (q and the new token's k, v, z_k, z_v) sit packed in
     # one pinned host buffer and cross with one copy; the output comes back
-    # with one copy
+    # with one copy.  As in a serving loop, the copies run on streams of their
+    # own beside the kernels: step i+1's upload overlaps step i's kernel and
+    # step i's download overlaps step i+1's (two staging slots; every step
+    # waits for its own upload, every download for its own step).
     parts = [bench.q] + [t for t in (bench.tk, bench.tv, bench.tzk, bench.tzv) if t is not None]
     sizes = [t[0].numel() * t[0].element_size() for t in parts]
     offs = np.cumsum([0] + sizes)
@@ -289,25 +292,56 @@ def run_ours(args, w, rank, world):
     hstage = torch.empty(nloc, int(offs[-1]), dtype=torch.uint8).pin_memory()
     for pi, t in enumerate(parts):
         hstage[:, offs[pi]:offs[pi + 1]] = t.cpu().contiguous().view(nloc, -1).view(torch.uint8)
-    dstage = torch.empty(int(offs[-1]), dtype=torch.uint8, device="cuda")
-    views = [dstage[offs[pi]:offs[pi + 1]].view(parts[pi].dtype).view(parts[pi][0].shape) for pi in range(len(parts))]
-    dq = views[0]
-    it = iter(views[1:])
-    dtok = [None if t is None else next(it) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)]
-    hout = torch.empty(bench.outs[0].shape, dtype=bench.outs[0].dtype).pin_memory()
+    NS = 2  # staging slots
+    dstage = [torch.empty(int(offs[-1]), dtype=torch.uint8, device="cuda") for _ in range(NS)]
+    dq, dtok = [], []
+    for sl in range(NS):
+        views = [dstage[sl][offs[pi]:offs[pi + 1]].view(parts[pi].dtype).view(parts[pi][0].shape)
+                 for pi in range(len(parts))]
+        it = iter(views[1:])
+        dq.append(views[0])
+        dtok.append([None if t is None else next(it) for t in (bench.tk, bench.tv, bench.tzk, bench.tzv)])
+    hout = [torch.empty(bench.outs[0].shape, dtype=bench.outs[0].dtype).pin_memory() for _ in range(NS)]
     h2d = int(offs[-1])
-    d2h = hout.numel() * hout.element_size()
+    d2h = hout[0].numel() * hout[0].element_size()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(NS)]        # slot's upload done
+    ev_run = [torch.cuda.Event() for _ in range(NS)]       # the step that read the slot is done
+    ev_down = [torch.cuda.Event() for _ in range(bench.NR)]  # download of an output replica done
 
-    def e2e_body(i):
-        dstage.copy_(hstage[i // bench.NR], non_blocking=True)
-        bench.launch(i, q=dq, tok=dtok)
-        hout.copy_(bench.outs[i % bench.NR], non_blocking=True)
+    def e2e_steps(first, n):
+        cur = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cur)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
+        for j, i in enumerate(range(first, first + n)):
+            sl, rep = j % NS, i % bench.NR
+            if j >= NS:
+                s_in.wait_event(ev_run[sl])       # the step two back has read this slot
+            with torch.cuda.stream(s_in):
+                dstage[sl].copy_(hstage[i // bench.NR], non_blocking=True)
+                ev_in[sl].record(s_in)
+            cur.wait_event(ev_in[sl])
+            if j >= bench.NR:
+                cur.wait_event(ev_down[rep])     # this output replica has been read back
+            bench.launch(i, q=dq[sl], tok=dtok[sl])
+            ev_run[sl].record(cur)
+            s_out.wait_event(ev_run[sl])
+            with torch.cuda.stream(s_out):
+                hout[sl].copy_(bench.outs[rep], non_blocking=True)
+                ev_down[rep].record(s_out)
+        for st in (s_in, s_out):  # join both copy streams back
+            ev = torch.cuda.Event()
+            ev.record(st)
+            cur.wait_event(ev)
 
-    for _ in range(W):
-        e2e_body(bench.i)
-        bench.i += 1
+    e2e_steps(bench.i, W)
+    bench.i += W
     torch.cuda.synchronize()
-    g_e2e = graph_of(bench.i, K, e2e_body)
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=cap):
+        e2e_steps(bench.i, K)
     torch.cuda.synchronize()
     e0.record()
     g_e2e.replay()
@@ -337,7 +371,9 @@ def run_ours(args, w, rank, world):
                    "l2": (f"inputs larger than L2: steps rotate over {bench.NR} cache replicas "
                           f"(>= 3x L2 of data in total), each step's data cold"),
                    "launch": (f"K steps of lbca_decode_step ({bench.launches} kernel launch"
-                              f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph")},
+                              f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph; "
+                              "e2e: each step's upload and download on copy streams beside the kernels "
+                              "(uploads one step ahead, downloads one step behind), all inside the timed graph")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src,
                      "kernel": ({L.LBCA_STEP_CLUSTER: "decode_step_kernel (cluster form)",

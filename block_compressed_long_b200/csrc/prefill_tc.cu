@@ -28,8 +28,9 @@
 //              fp16 into the free P buffer, and finally normalises its O row
 //              (plus the sink) into shared memory, from where one thread
 //              TMA-stores the tile.
-// Raw keys arrive already rotated and, like the values, in fp16 (a pre-pass
-// writes them once instead of every query tile converting them again); Q is
+// Raw keys arrive already rotated and, like the values, in fp16 (the pool pass
+// writes them while it streams K and V, instead of every query tile converting
+// them again); Q is
 // rotated in shared memory from a per-position cos/sin table.  Rows past a tensor's valid extent
 // are zero-filled by TMA, so masked products never meet garbage.
 #include <cudaTypedefs.h>

@@ -145,6 +145,23 @@ def test_decode_step_form(L):
     assert 0 < small < big
 
 
+def test_shared_entry_step_forms(L):
+    """The fused tensor-core step takes the shared-entry form with 64 query
+    heads per kv head, one kv head, D 256 or 512, bf16 and a raw window;
+    other shared-entry shapes keep the CUDA-core forms or the two calls.  Its
+    workspace query returns a small positive size (it uses none)."""
+    hca = dict(n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128, rope_dims=64, n_win=128)
+    assert L.lbca_decode_step_form(_cfg(L, **hca), 8, 131073) == L.LBCA_STEP_SHARED_TC
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, head_dim=256)), 8, 131073) == L.LBCA_STEP_SHARED_TC
+    assert 0 < L.lbca_decode_step_workspace_bytes(_cfg(L, **hca), 8, 131073) <= 4096
+    # not the tensor-core shape: 48 heads per kv head, f32, D = 128
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, n_q_heads=48)), 8, 131073) != L.LBCA_STEP_SHARED_TC
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, dtype="f32")), 8, 131073) != L.LBCA_STEP_SHARED_TC
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, head_dim=128)), 8, 131073) != L.LBCA_STEP_SHARED_TC
+    # a list longer than 16 CTAs x 128 rows can hold: no tensor-core plan at all
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, block_m=16)), 1, 131073) != L.LBCA_STEP_SHARED_TC
+
+
 def test_status_strings(L):
     for s in range(7):
         assert L.lbca_status_string(s)

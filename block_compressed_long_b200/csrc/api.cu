@@ -115,13 +115,13 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Decode arguments common to every decode launch (no workspace, no split plan).
 DecodeArgs decode_args(const lbca_config* cfg, const void* q, const lbca_cache* cache, const float* sink,
-                       const void* gamma_q, void* out, int32_t* d_status) {
+                       const void* gamma_q, const void* gamma_kv, void* out, int32_t* d_status) {
     DecodeArgs a{};
     a.dtype = cfg->dtype;
     a.q = q;
     a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
     a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
-    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.gamma_kv = gamma_kv; a.out = out;
     a.status = d_status;
     a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
     a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
@@ -231,12 +231,13 @@ lbca_status lbca_append(const lbca_config* cfg, const void* k, const void* v, co
 }
 
 lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache* cache, const float* sink,
-                        const void* gamma_q, int32_t max_ctx, void* out, void* workspace,
+                        const void* gamma_q, const void* gamma_kv, int32_t max_ctx, void* out, void* workspace,
                         size_t workspace_bytes, int32_t* d_status, lbca_stream_t stream) {
     LBCA_TRY(check_cfg(cfg));
     LBCA_TRY(check_cache(cfg, cache));
     if (!q || !out || !workspace) return LBCA_ERR_ARG;
-    if (!al16(q) || !al16(out) || !al16(workspace) || !al16n(gamma_q) || !al16n(sink)) return LBCA_ERR_ALIGN;
+    if (!al16(q) || !al16(out) || !al16(workspace) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink))
+        return LBCA_ERR_ALIGN;
     if (max_ctx <= 0) {
         const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
         max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
@@ -247,7 +248,7 @@ lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache*
     if (workspace_bytes < decode_workspace_bytes(p)) return LBCA_ERR_CAPACITY;
     LBCA_TRY(check_device());
     char* ws = static_cast<char*>(workspace);
-    DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, out, d_status);
+    DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, gamma_kv, out, d_status);
     a.part_o = reinterpret_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float*>(ws + align256(p.part_o_elems * 4));
     a.counters = reinterpret_cast<uint32_t*>(ws + align256(p.part_o_elems * 4) + align256(p.part_ml_elems * 4));
@@ -300,8 +301,8 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
         const MqaTcPlan tp = plan_decode_mqa_tc(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads,
                                                 cfg->head_dim, cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
         if (tp.cs == 0) return LBCA_ERR_UNSUPPORTED;  // no cluster of the kernel fits this device
-        DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, out, d_status);
-        a.app_k = k; a.app_z = zk; a.app_bp = b_pos_k; a.gamma_kv = gamma_kv;
+        DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, gamma_kv, out, d_status);
+        a.app_k = k; a.app_z = zk; a.app_bp = b_pos_k;
         a.ring_w = cache->ring_k; a.pooled_w = cache->pooled_k; a.state = cache->pool_state;
         a.lens_w = cache->seq_lens;
         a.tc_cs = tp.cs; a.chunk = tp.rows;
@@ -311,8 +312,8 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
                             cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
     if (!sp.ok) {  // shapes no fused kernel takes: the two-launch path
         LBCA_TRY(lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache, d_status, stream));
-        return lbca_decode(cfg, q, cache, sink, gamma_q, max_ctx, out, workspace, workspace_bytes, d_status,
-                           stream);
+        return lbca_decode(cfg, q, cache, sink, gamma_q, gamma_kv, max_ctx, out, workspace, workspace_bytes,
+                           d_status, stream);
     }
     if (workspace_bytes < step_workspace_bytes(sp)) return LBCA_ERR_CAPACITY;
     LBCA_TRY(check_device());
@@ -418,6 +419,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
             a.out_f16_blocks = NB;
             a.raw_f16 = series == 0 ? raw16.keys : raw16.vals;
             a.tab = raw16.tab;
+            a.status = d_status;
         }
         LBCA_TRY(cuda_status(launch_pool(a, s)));
     }
@@ -474,15 +476,30 @@ lbca_status scratch_for_current_device(void** addr) {
 }  // namespace
 
 lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbca_cache* cache,
-                                const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
-                                int32_t* d_status, lbca_stream_t stream) {
+                                const float* sink, const void* gamma_q, const void* gamma_kv, int32_t max_ctx,
+                                void* out, int32_t* d_status, lbca_stream_t stream) {
     LBCA_TRY(check_cfg(cfg));
     LBCA_TRY(check_cache(cfg, cache));
     if (!q || !out) return LBCA_ERR_ARG;
-    if (!al16(q) || !al16(out) || !al16n(gamma_q) || !al16n(sink)) return LBCA_ERR_ALIGN;
+    if (!al16(q) || !al16(out) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink)) return LBCA_ERR_ALIGN;
     if (max_ctx <= 0) {
         const long long cap = (long long)cache->max_blocks * cfg->block_m + cache->ring_slots;
         max_ctx = cap > INT32_MAX ? INT32_MAX : (int32_t)(cap < 1 ? 1 : cap);
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the tensor-core kernel of the shared-entry form merges inside its cluster
+    // and needs no scratch at all: no capacity check, no counters to clear
+    if (mqa_tc_shape_ok(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->block_m,
+                        cfg->n_win, cfg->shared_kv, max_ctx)) {
+        LBCA_TRY(check_device());
+        DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, gamma_kv, out, d_status);
+        const MqaTcPlan tc = plan_decode_mqa_tc(cfg->dtype, a.B, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
+                                                cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
+        if (tc.cs > 0) {
+            a.tc_cs = tc.cs;
+            a.chunk = tc.rows;
+            return cuda_status(launch_decode_mqa_tc(a, s));
+        }
     }
     DecodePlan p = plan_decode(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
                                cfg->block_m, cfg->n_win, cfg->shared_kv, max_ctx);
@@ -491,27 +508,16 @@ lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbc
     LBCA_TRY(check_device());
     void* scratch = nullptr;
     LBCA_TRY(scratch_for_current_device(&scratch));
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(scratch);
     const size_t ctr_off = align256(p.part_o_elems * 4) + align256(p.part_ml_elems * 4);
     // the scratch keeps whatever the previous call left: the merge counters must start at zero
     if (cudaMemsetAsync(ws + ctr_off, 0, p.counter_elems * 4, s) != cudaSuccess) return LBCA_ERR_CUDA;
-    DecodeArgs a{};
-    a.dtype = cfg->dtype;
-    a.q = q;
-    a.pooled_k = cache->pooled_k; a.pooled_v = cache->pooled_v;
-    a.ring_k = cache->ring_k; a.ring_v = cache->ring_v;
-    a.seq_lens = cache->seq_lens; a.sink = sink; a.gamma_q = gamma_q; a.out = out;
+    DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, gamma_kv, out, d_status);
     a.part_o = reinterpret_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float*>(ws + align256(p.part_o_elems * 4));
     a.counters = reinterpret_cast<uint32_t*>(ws + ctr_off);
-    a.status = d_status;
-    a.B = cache->batch; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim;
-    a.m = cfg->block_m; a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm;
-    a.shared = cfg->shared_kv; a.max_blocks = cache->max_blocks; a.R = cache->ring_slots;
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
-    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
-    return run_decode(cfg, a, max_ctx, s);
+    return cuda_status(launch_decode(a, s));
 }
 
 const char* lbca_status_string(lbca_status status) {

@@ -71,6 +71,12 @@ __device__ __forceinline__ void st16_f16(__half* p, const float (&o)[8]) {
     v.w = pack_f16x2(o[6], o[7]);
     *reinterpret_cast<uint4*>(p) = v;
 }
+// The same, flagging any value beyond the fp16 range (it would become inf).
+__device__ __forceinline__ void st16_f16_checked(__half* p, const float (&o)[8], bool& ovf) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ovf |= fabsf(o[i]) > 65504.f;
+    st16_f16(p, o);
+}
 __device__ __forceinline__ void st16(float* p, const float (&o)[4]) {
     *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
 }

@@ -58,6 +58,43 @@ template <> __device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16*
     *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
 }
 
+// Shared form: a raw window row, held as 16 dims per lane over the LG lanes of
+// an entry group (lane gl holds dims (c LG + gl) VEC + i), is finalised as it
+// is read -- RMSNorm over the whole row (when on), then RoPE of the rotated
+// dims at the token's position `pos` -- in f32, so that the entry the output
+// averages carries no rounding beyond its input's.  Every lane of the warp
+// calls it (the row sum crosses lanes); `raw` is uniform per entry group.
+template <typename T, int D, int LG, int VEC>
+__device__ __forceinline__ void finalise_raw16(float (&x)[16], bool raw, int64_t pos, int gl, const DecodeArgs& a) {
+    constexpr int NCH = 16 / VEC;
+    if (a.rmsnorm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+        for (int off = LG / 2; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if (raw) {
+            const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+            const T* gm = static_cast<const T*>(a.gamma_kv);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int i = 0; i < VEC; ++i)
+                    x[c * VEC + i] *= inv * (gm ? to_f<T>(gm[(c * LG + gl) * VEC + i]) : 1.0f);
+        }
+    }
+    if (raw && a.rho) {
+        const int base = D - a.rho;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+#pragma unroll
+            for (int i = 0; i < VEC; i += 2) {
+                const int d = (c * LG + gl) * VEC + i;
+                if (d >= base) rotate_pair(x[c * VEC + i], x[c * VEC + i + 1], rope_cs(pos, (d - base) >> 1, a.rope_step));
+            }
+    }
+}
+
 template <typename T, int D, int R>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
     constexpr int VEC = Vec<T>::N;
@@ -211,6 +248,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
 #pragma unroll
             for (int i = 0; i < VEC; ++i) { kfa[c * VEC + i] = t0[i]; kfb[c * VEC + i] = t1[i]; }
         }
+        if (a.shared) {  // rows past the pooled ones are raw window entries
+            const int ia = e0 + ea, ib = e0 + ebb;
+            finalise_raw16<T, D, LG, VEC>(kfa, va && ia >= P, (int64_t)s0 + (ia - P), gl, a);
+            finalise_raw16<T, D, LG, VEC>(kfb, vb && ib >= P, (int64_t)s0 + (ib - P), gl, a);
+        }
         float sa[R], sb[R];
 #pragma unroll
         for (int h = 0; h < R; ++h) {
@@ -228,16 +270,21 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
                 sb[h] += __shfl_xor_sync(0xffffffffu, sb[h], off);
             }
         if (!va) continue;  // no shuffles below
-        const T* vra = vbuf + (size_t)ea * D;
-        const T* vrb = vbuf + (size_t)(vb ? ebb : ea) * D;
         float vfa[16], vfb[16];
+        if (a.shared) {  // the (finalised) entry is its own value
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            float t0[VEC], t1[VEC];
-            ld16(vra + (c * LG + gl) * VEC, t0);
-            ld16(vrb + (c * LG + gl) * VEC, t1);
+            for (int i = 0; i < 16; ++i) { vfa[i] = kfa[i]; vfb[i] = kfb[i]; }
+        } else {
+            const T* vra = vbuf + (size_t)ea * D;
+            const T* vrb = vbuf + (size_t)(vb ? ebb : ea) * D;
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) { vfa[c * VEC + i] = t0[i]; vfb[c * VEC + i] = t1[i]; }
+            for (int c = 0; c < NCH; ++c) {
+                float t0[VEC], t1[VEC];
+                ld16(vra + (c * LG + gl) * VEC, t0);
+                ld16(vrb + (c * LG + gl) * VEC, t1);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { vfa[c * VEC + i] = t0[i]; vfb[c * VEC + i] = t1[i]; }
+            }
         }
 #pragma unroll
         for (int h = 0; h < R; ++h) {

@@ -29,7 +29,10 @@
 // CTAs of a cluster share one (sequence, kv head):
 //   1. Each CTA copies its chunk of the visible list (<= C rows: pooled rows,
 //      then ring rows) into 128-byte-swizzled shared memory with 16-byte
-//      cp.async and widens it to fp16 in place.  Meanwhile up to 8 CTAs each
+//      cp.async and widens it to fp16 in place.  The ring holds the raw
+//      entries as appended; a warp finalises each of them (RMSNorm, RoPE at
+//      the token's position) in f32 before its one fp16 rounding, so a window
+//      row that is also the value carries no bf16 rounding of its own.  Meanwhile up to 8 CTAs each
 //      prepare a share of the queries (RMSNorm, RoPE at t, fp16) and
 //      bulk-copy it into every other CTA's query tile (shared memory to
 //      shared memory across the cluster, one destination per copy).
@@ -49,13 +52,13 @@
 //
 // Serving step (append fused, one kv head): the new token is cached first and
 // the query attends at the new length L = cached + 1 (mSeek README, "How LBCA
-// works", steps 2-4).  Its finalised raw entry is the last visible row, so the
-// CTA whose chunk ends the list appends it with one warp while the other rows'
+// works", steps 2-4).  Its raw entry is the last visible row, so the CTA
+// whose chunk ends the list appends it with one warp while the other rows'
 // copies are in flight: running per-channel softmax of the open block (and the
-// finished pooled entry when the token closes a block), RMSNorm and RoPE at t,
-// the bf16 row to the ring and straight into its own staged tile.  With a
-// window (n_win > 0) a block closed at this step is not yet visible, so no
-// other CTA needs what the append writes.  The arithmetic and its order are
+// finished pooled entry when the token closes a block), the raw row to the
+// ring and straight into its own staged tile, where it is finalised with the
+// other window rows.  With a window (n_win > 0) a block closed at this step is
+// not yet visible, so no other CTA needs what the append writes.  The arithmetic and its order are
 // those of the stand-alone append kernel, so the cache and the output are
 // bit-identical to append followed by decode.
 #include <algorithm>
@@ -220,10 +223,11 @@ __device__ __forceinline__ void finalise_row(const DecodeArgs& a, float (&e)[CPL
 // a token that closes block j finishes entry j (weighted sum / sum, RMSNorm,
 // RoPE at the block start j m) into pooled_k, otherwise the state is stored
 // back; the raw token (RMSNorm, RoPE at pos, from `cs_t`) goes to its ring
-// slot and, when `row` >= 0, to that row of the staged bf16 entry tile.
+// slot and, when `row` >= 0, to that row of the staged bf16 entry tile, as
+// given: window rows are finalised when the tile is widened.
 template <int D>
-__device__ __forceinline__ void append_token(const DecodeArgs& a, int b, int g, int pos, const float2* cs_t,
-                                             uint8_t* sE, uint32_t ereg, int row, int lane) {
+__device__ __forceinline__ void append_token(const DecodeArgs& a, int b, int g, int pos, uint8_t* sE, uint32_t ereg,
+                                             int row, int lane) {
     constexpr int CPL = D / 256;
     const int GD = a.G * D;
     const int i = pos % a.m, jb = pos / a.m;
@@ -295,7 +299,8 @@ __device__ __forceinline__ void append_token(const DecodeArgs& a, int b, int g, 
             }
         }
     }
-    finalise_row<D, CPL>(a, x, lane, cs_t, 0);
+    // the raw entry as given joins the window (ring slot and staged tile row);
+    // like every window row it is finalised when the tile is widened
     __nv_bfloat16* ring = static_cast<__nv_bfloat16*>(a.ring_w) + (((size_t)b * a.G + g) * a.R + pos % a.R) * D;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
@@ -463,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
         }
         fence_async_smem();
     }
-    if (appender && warp == app_warp) append_token<D>(a, b, g, pos, cs, smem + lay.OFF_E, lay.EREG, app_row, lane);
+    if (appender && warp == app_warp) append_token<D>(a, b, g, pos, smem + lay.OFF_E, lay.EREG, app_row, lane);
     __syncthreads();
     cluster_wait_acquire();  // every CTA's barriers exist; every CTA has read seq_lens[b]
     if (appender && tid == 0) a.lens_w[b] = pos + 1;
@@ -476,10 +481,70 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
         bulk_commit();
     }
 
-    // ---- this thread's entry copies have landed: widen them to fp16 in place ----
+    // ---- this thread's entry copies have landed: widen them to fp16 in place.
+    // Pooled rows are finalised entries; window rows are the raw entries as
+    // appended and are finalised here, in f32 (RMSNorm over the row held by
+    // this warp, RoPE at the token's position), before their one fp16 rounding.
     cp_async_wait_all();
     for (int row = warp; row < n16; row += kWarps) {
         uint8_t* rbase = smem + lay.OFF_E + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
+        const int idx = e0 + row;
+        if (row < n && idx >= P) {  // uniform per warp: a window row
+            float x[CPR / 32][8];
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPR / 32; ++j) {
+                const int ch = j * 32 + lane;
+                const uint4 u = *reinterpret_cast<const uint4*>(rbase + (uint32_t)(ch >> 3) * lay.EREG +
+                                                                ((uint32_t)((ch & 7) ^ (row & 7)) << 4));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    x[j][2 * i] = __uint_as_float(w[i] << 16);
+                    x[j][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss = fmaf(x[j][i], x[j][i], ss);
+            }
+            if (a.rmsnorm) {
+#pragma unroll
+                for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
+                const __nv_bfloat16* gm = static_cast<const __nv_bfloat16*>(a.gamma_kv);
+#pragma unroll
+                for (int j = 0; j < CPR / 32; ++j) {
+                    float gam[8];
+                    if (gm) {
+                        ld16(gm + (j * 32 + lane) * 8, gam);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) gam[i] = 1.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[j][i] *= inv * gam[i];
+                }
+            }
+            const int64_t spos = (int64_t)s0 + (idx - P);
+            const int rope0 = D - a.rho;
+#pragma unroll
+            for (int j = 0; j < CPR / 32; ++j) {
+                const int ch = j * 32 + lane;
+#pragma unroll
+                for (int i = 0; i < 8; i += 2)
+                    if (a.rho > 0 && ch * 8 + i >= rope0)
+                        rotate_pair(x[j][i], x[j][i + 1], rope_cs(spos, (ch * 8 + i - rope0) >> 1, a.rope_step));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ovf |= fabsf(x[j][i]) > kF16Max;
+                uint4 o;
+                o.x = pack_f16x2(x[j][0], x[j][1]);
+                o.y = pack_f16x2(x[j][2], x[j][3]);
+                o.z = pack_f16x2(x[j][4], x[j][5]);
+                o.w = pack_f16x2(x[j][6], x[j][7]);
+                *reinterpret_cast<uint4*>(rbase + (uint32_t)(ch >> 3) * lay.EREG +
+                                          ((uint32_t)((ch & 7) ^ (row & 7)) << 4)) = o;
+            }
+            continue;
+        }
 #pragma unroll
         for (int j = 0; j < CPR / 32; ++j) {
             const int ch = j * 32 + lane;

@@ -604,7 +604,10 @@ cudaError_t step_dispatch(const StepArgs& a, size_t smem, cudaStream_t s) {
 StepPlan plan_step(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
     StepPlan p{};
     p.ok = false;
-    if ((D != 64 && D != 128 && D != 256) || w < 1) return p;
+    // GQA form only: the shared form's window rows are raw entries finalised
+    // by the decode kernels that read them (lbca_append then lbca_decode, or
+    // the tensor-core shared-entry step)
+    if ((D != 64 && D != 128 && D != 256) || w < 1 || shared) return p;
     const int r = Hq / G;
     int R = 1;
     for (int c : {4, 3, 2, 1})

@@ -31,6 +31,9 @@ struct PoolArgs {
     // from `tab` ([rho/2][T], pair-major)
     void* raw_f16;
     const float2* tab;
+    // device status word for the fp16 copies: a value beyond the fp16 range
+    // sets LBCA_ERR_UNSUPPORTED (nullable)
+    int32_t* status;
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     for (int e = 0; e < VEC; ++e) { mx[e] = kNegInf; l[e] = 0.f; acc[e] = 0.f; }
     const int g = cv / NVH, d0 = (cv % NVH) * VEC;
     const bool raw_copy = RAW && VEC == 8 && full;  // uniform per CTA
+    bool f16_ovf = false;                           // an fp16 copy left the fp16 range
 
     if (active) {
         // U tokens per step: their X, Z and B_pos vectors are loaded together
@@ -130,7 +131,8 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
                                 for (int e = 0; e < VEC; e += 2)
                                     if (dr + e >= 0)
                                         rotate_pair(xf[e], xf[e + 1], a.tab[(size_t)((dr + e) >> 1) * a.T + s_tok]);
-                            st16_f16(static_cast<__half*>(a.raw_f16) + row0 + (size_t)(i0 + u) * GD, xf);
+                            st16_f16_checked(static_cast<__half*>(a.raw_f16) + row0 + (size_t)(i0 + u) * GD, xf,
+                                             f16_ovf);
                         }
                 }
             }
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
             if constexpr (VEC == 8) {
                 if (a.out_f16) {  // the f32 value, rounded once to fp16
                     const size_t oi16 = (((size_t)b * a.G + g) * a.out_f16_blocks + a.blk_off + j) * a.D + d0;
-                    st16_f16(static_cast<__half*>(a.out_f16) + oi16, tmp);
+                    st16_f16_checked(static_cast<__half*>(a.out_f16) + oi16, tmp, f16_ovf);
                 }
             }
         }
@@ -208,6 +210,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
             st[2 * GD + i] = acc[i];
         }
     }
+    if (f16_ovf) set_status(a.status, LBCA_ERR_UNSUPPORTED);
 }
 
 template <typename T>
@@ -233,14 +236,18 @@ __global__ void __launch_bounds__(1024) ring_fill_kernel(const RingFillArgs a) {
     else
 #pragma unroll
         for (int i = 0; i < VEC; ++i) e[i] = 0.f;
-    float ss = 0.f;
-    if (a.rmsnorm) {
-        float v = 0.f;
+    // GQA form: the finalised key.  Shared form (no value series): the raw
+    // entry as given, finalised by the decode kernels when they read it.
+    if (a.v) {
+        float ss = 0.f;
+        if (a.rmsnorm) {
+            float v = 0.f;
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) v += e[i] * e[i];
-        ss = head_sum(part, v, active ? tid - (cv % NVH) : 0, NVH);
+            for (int i = 0; i < VEC; ++i) v += e[i] * e[i];
+            ss = head_sum(part, v, active ? tid - (cv % NVH) : 0, NVH);
+        }
+        finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma), a.rho, cs);
     }
-    finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma), a.rho, cs);
     if (active) {
         st16(static_cast<T*>(a.ring_k) + dst, e);
         if (a.v) {
@@ -339,21 +346,25 @@ __global__ void __launch_bounds__(1024) append_kernel(const AppendArgs a) {
         }
     }
 
-    // the raw token joins the window: finalised key, or the value as is
+    // the raw token joins the window: the finalised key (GQA form), the value
+    // as is, or -- in the shared form, where the row is also the value -- the
+    // raw entry as given, finalised in f32 by the decode kernels when read
     float r[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; ++k) r[k] = x[k];
-    float ss = 0.f;
-    if (a.rmsnorm) {
-        float v = 0.f;
-        if (key)
+    if (a.S == 2) {  // uniform across the CTA
+        float ss = 0.f;
+        if (a.rmsnorm) {
+            float v = 0.f;
+            if (key)
 #pragma unroll
-            for (int k = 0; k < VEC; ++k) v += r[k] * r[k];
-        ss = head_sum(part, v, active ? tid - (cv % NVH) : 0, NVH);
+                for (int k = 0; k < VEC; ++k) v += r[k] * r[k];
+            ss = head_sum(part, v, active ? tid - (cv % NVH) : 0, NVH);
+        }
+        if (key)
+            finalise_key<T, VEC>(r, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma), a.rho,
+                                 cs_raw);
     }
-    if (key)
-        finalise_key<T, VEC>(r, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma), a.rho,
-                             cs_raw);
     if (active) {
         T* o = static_cast<T*>(key ? a.ring_k : a.ring_v) +
                (((size_t)b * a.G + g) * a.R + (pos % a.R)) * a.D + d0;

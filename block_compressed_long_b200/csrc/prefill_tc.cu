@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         bool ok = warp_wait(&bars[B_QFULL], 0, fail, a.status);
         if (ok) {  // this query row, in place: bf16 -> f32, RoPE at t, -> fp16 (QK^T runs in fp16)
+            bool ovf = false;  // a value beyond the fp16 range would become inf
 #pragma unroll
             for (int c8 = 0; c8 < HD / 8; ++c8) {
                 uint4* p = reinterpret_cast<uint4*>(sQ + sw128_off(r, 8 * c8, QREG));
@@ -310,10 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 for (int e = 0; e < 4; ++e) {
                     float x = __uint_as_float(wv[e] << 16), y = __uint_as_float(wv[e] & 0xffff0000u);
                     rotate_pair(x, y, cs_row[4 * c8 + e]);
+                    ovf |= fabsf(x) > 65504.f || fabsf(y) > 65504.f;
                     wv[e] = pack_f16x2(x, y);
                 }
                 *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
+            if (ovf) set_status(a.status, LBCA_ERR_UNSUPPORTED);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&bars[B_QROT + q]);
@@ -468,7 +471,8 @@ __global__ void rope_table_kernel(float2* tab, int T, int half, double step) {
 // same [B, T, G, D] layout.  (The pool pass writes those of complete blocks.)
 __global__ void finalise_kv_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                                    __half* __restrict__ ko, __half* __restrict__ vo, const float2* __restrict__ tab,
-                                   int64_t n_vec, int G, int T, int s_begin, int rho) {
+                                   int64_t n_vec, int G, int T, int s_begin, int rho, int32_t* status) {
+    bool ovf = false;  // a value beyond the fp16 range would become inf
     const int64_t per_b = (int64_t)(T - s_begin) * G * (HD / 8);  // vectors of one sequence's tail
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < n_vec; j += (int64_t)gridDim.x * blockDim.x) {
         const int64_t b = j / per_b;
@@ -484,9 +488,10 @@ __global__ void finalise_kv_kernel(const __nv_bfloat16* __restrict__ k, const __
             const int d = d0 + e;
             if (d >= HD - rho) rotate_pair(x[e], x[e + 1], tab[(size_t)((d - (HD - rho)) >> 1) * T + s]);
         }
-        st16_f16(ko + i * 8, x);
-        st16_f16(vo + i * 8, y);
+        st16_f16_checked(ko + i * 8, x, ovf);
+        st16_f16_checked(vo + i * 8, y, ovf);
     }
+    if (ovf) set_status(status, LBCA_ERR_UNSUPPORTED);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -567,7 +572,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
         const int64_t nv = (int64_t)B * (T - s_begin) * G * (HD / 8);
         finalise_kv_kernel<<<(int)std::min<int64_t>((nv + 255) / 256, 148 * 32), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v), keys, vals, tab, nv, G, T,
-            s_begin, p.rho);
+            s_begin, p.rho, status);
     }
     TcArgs a;
     memset(&a, 0, sizeof(a));

@@ -64,7 +64,7 @@ _lib.lbca_pool.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp,
 _lib.lbca_pool.restype = ctypes.c_int
 _lib.lbca_append.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp]
 _lib.lbca_append.restype = ctypes.c_int
-_lib.lbca_decode.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _sz, _vp, _vp]
+_lib.lbca_decode.argtypes = [_CP, _vp, _KP, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp, _vp]
 _lib.lbca_decode.restype = ctypes.c_int
 _lib.lbca_prefill.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
                               _KP, _vp, _sz, _vp, _vp]
@@ -78,7 +78,7 @@ _lib.lbca_decode_step_launches.argtypes = [_CP, _i32, _i32]
 _lib.lbca_decode_step_launches.restype = _i32
 _lib.lbca_decode_step_form.argtypes = [_CP, _i32, _i32]
 _lib.lbca_decode_step_form.restype = _i32
-_lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _i32, _vp, _vp, _vp]
+_lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
 _lib.lbca_decode_noalloc.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
 _lib.lbca_status_string.restype = ctypes.c_char_p
@@ -190,11 +190,12 @@ def lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache: Cache, d_s
                                            _ptr(d_status), _stream(stream)))
 
 
-def lbca_decode(cfg, q, cache: Cache, sink, gamma_q, out, workspace, max_ctx=0, d_status=None, stream=None):
+def lbca_decode(cfg, q, cache: Cache, sink, gamma_q, gamma_kv, out, workspace, max_ctx=0, d_status=None,
+                stream=None):
     """q, out [B, Hq, D]; workspace a zero-filled uint8 tensor."""
     cc = cache.c()
     _check("lbca_decode", _lib.lbca_decode(ctypes.byref(cfg), _ptr(q), ctypes.byref(cc), _ptr(sink),
-                                           _ptr(gamma_q), max_ctx, _ptr(out), _ptr(workspace),
+                                           _ptr(gamma_q), _ptr(gamma_kv), max_ctx, _ptr(out), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), _ptr(d_status),
                                            _stream(stream)))
 
@@ -238,11 +239,13 @@ def lbca_prefill(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv
                                              _ptr(workspace), wb, _ptr(d_status), _stream(stream)))
 
 
-def lbca_decode_noalloc(cfg, q, cache: Cache, sink, gamma_q, out, max_ctx=0, d_status=None, stream=None):
+def lbca_decode_noalloc(cfg, q, cache: Cache, sink, gamma_q, gamma_kv, out, max_ctx=0, d_status=None,
+                        stream=None):
     """lbca_decode without a workspace, for callers that may not allocate device
     memory: the library's own static scratch holds the split partials.  Calls
     that overlap on the GPU race on that scratch."""
     cc = cache.c()
     _check("lbca_decode_noalloc", _lib.lbca_decode_noalloc(ctypes.byref(cfg), _ptr(q), ctypes.byref(cc), _ptr(sink),
-                                                           _ptr(gamma_q), max_ctx, _ptr(out), _ptr(d_status),
+                                                           _ptr(gamma_q), _ptr(gamma_kv), max_ctx, _ptr(out),
+                                                           _ptr(d_status),
                                                            _stream(stream)))

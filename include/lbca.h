@@ -95,7 +95,11 @@ typedef struct {
  *   pooled_k   [B, G, max_blocks, D] finalised pooled key entries (shared form:
  *              the entries, used as key and value)
  *   pooled_v   [B, G, max_blocks, D] pooled values; NULL in the shared form
- *   ring_k     [B, G, ring_slots, D] finalised raw keys; token s in slot s % ring_slots
+ *   ring_k     [B, G, ring_slots, D] raw window; token s in slot s % ring_slots.  GQA
+ *              form: the finalised keys (RMSNorm when enabled, RoPE at s).  Shared
+ *              form: the raw entries C exactly as appended, finalised (RMSNorm,
+ *              RoPE at s) in f32 by the decode kernels when read -- there the
+ *              row also serves as the value, so it is not rounded a second time
  *   ring_v     [B, G, ring_slots, D] raw values; NULL in the shared form
  *   pool_state [B, S, 3, G, D] f32 running (max, sum, weighted sum) of the
  *              open block's pooling softmax, S = 2 (K then V) or 1 (shared)
@@ -183,6 +187,8 @@ LBCA_API lbca_status lbca_append(const lbca_config* cfg, const void* k, const vo
  *              t = seq_lens[b] - 1 (call lbca_append for the token first)
  *   sink       device [Hq] f32 sink logits or NULL
  *   gamma_q    device [D] query RMSNorm gain or NULL
+ *   gamma_kv   device [D] key RMSNorm gain or NULL: the one given to lbca_append
+ *              and lbca_prefill (the shared form finalises its raw window here)
  *   max_ctx    upper bound of seq_lens (sizes the split grid); <= 0 derives it
  *              from the cache capacity
  *   out        device [B, Hq, D]
@@ -191,11 +197,14 @@ LBCA_API lbca_status lbca_append(const lbca_config* cfg, const void* k, const vo
  * The visible entries are split into chunks processed by separate CTAs; the
  * last CTA of each (sequence, head group) merges the partial softmaxes.
  * A sequence with no tokens yields zeros.  A sequence longer than max_ctx sets
- * d_status to LBCA_ERR_CAPACITY (its output is then incomplete).
+ * d_status to LBCA_ERR_CAPACITY (its output is then incomplete).  The
+ * shared-entry form on the tensor cores (bf16, 64 query heads per kv head,
+ * D 256 or 512) multiplies in fp16: an entry or query beyond the fp16 range
+ * sets d_status to LBCA_ERR_UNSUPPORTED.
  * Calls that share a workspace must not overlap on the GPU.
  */
 LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lbca_cache* cache,
-                        const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                        const float* sink, const void* gamma_q, const void* gamma_kv, int32_t max_ctx, void* out,
                         void* workspace, size_t workspace_bytes, int32_t* d_status,
                         lbca_stream_t stream);
 
@@ -205,9 +214,9 @@ LBCA_API lbca_status lbca_decode(const lbca_config* cfg, const void* q, const lb
  * (mSeek README, repository layout: generation through the LBCA cache; "How
  * LBCA works", steps 2-5.)  Arguments as in lbca_append and lbca_decode;
  * `workspace` (zero-filled before first use, left zero-filled) must hold
- * lbca_decode_step_workspace_bytes(cfg, B, max_ctx) bytes.  With n_win >= 1,
- * D in {64, 128, 256} and up to 4 query heads per kv head per CTA group, the
- * step runs as one kernel (the appended token's block cannot be visible to
+ * lbca_decode_step_workspace_bytes(cfg, B, max_ctx) bytes.  In the GQA form
+ * with n_win >= 1, D in {64, 128, 256} and up to 4 query heads per kv head per
+ * CTA group, the step runs as one kernel (the appended token's block cannot be visible to
  * the same query, so appending and attending are independent): for a few
  * (sequence, head group) pairs a cluster kernel that splits each pair's
  * entries over the CTAs of a cluster, for many pairs (96 or more) a
@@ -254,7 +263,10 @@ LBCA_API lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, con
  *                that lbca_append / lbca_decode continue the sequences
  *   workspace    device, lbca_prefill_workspace_bytes(cfg, B, T, cache_out != NULL)
  *   d_status     nullable device word for device-side conditions (a bounded
- *                wait of the tensor-core kernel giving up: LBCA_ERR_TIMEOUT)
+ *                wait of the tensor-core kernel giving up: LBCA_ERR_TIMEOUT; a
+ *                query, key or value beyond the fp16 range of its tensor-core
+ *                operands, |x| > 65504 after RoPE: LBCA_ERR_UNSUPPORTED, the
+ *                output then not valid)
  * bf16 I/O with D = 128, no RMSNorm and separate K/V runs QK^T and PV on the
  * tensor cores (tcgen05, TMEM accumulators, TMA-fed tiles); every other
  * shape runs the f32 CUDA-core kernel (no TF32).
@@ -291,7 +303,8 @@ LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const v
  */
 #define LBCA_NOALLOC_SCRATCH_BYTES (8u << 20)
 LBCA_API lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbca_cache* cache,
-                                         const float* sink, const void* gamma_q, int32_t max_ctx, void* out,
+                                         const float* sink, const void* gamma_q, const void* gamma_kv,
+                                         int32_t max_ctx, void* out,
                                          int32_t* d_status, lbca_stream_t stream);
 
 /* Static text for a status code. */

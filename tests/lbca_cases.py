@@ -68,50 +68,6 @@ def assert_close_stored(got, want, dtype: str, what: str = ""):
     assert d.mean() <= mean_bound, f"{what}: mean-abs {d.mean():.3e} > {mean_bound:.3e}"
 
 
-def assert_close_few_entries(got, want, emax, what: str = ""):
-    """bf16 check of decode outputs that lean on a handful of stored entries
-    (a visible list of fewer than 32 entries).  The cache keeps every
-    finalised entry in the I/O dtype, so each entry carries a bf16 rounding
-    of up to 2^-8 of its magnitude, and the output adds its own; an output
-    built from few entries inherits them instead of averaging them out.  An
-    element may then be off by max(1e-2, 2^-8 (max_j |E_j,d| + |o_d|)), with
-    E_j the oracle's visible entries (emax [n_seq, D] = max_j |E_j,d|), and
-    the mean by 1e-3 plus 2^-9 mean(max_j |E_j,d|).  Outputs averaged over
-    more entries keep the plain bound (assert_close)."""
-    got = np.asarray(got, dtype=np.float64)
-    want = np.asarray(want, dtype=np.float64)
-    assert got.shape == want.shape and np.all(np.isfinite(got)), what
-    d = np.abs(got - want)
-    bound = np.maximum(1e-2, 2.0 ** -8 * (emax[:, None, :] + np.abs(want)))
-    worst = float((d / bound).max())
-    assert worst <= 1.0, f"{what}: error {worst:.2f}x the entry-rounding bound"
-    mean_bound = 1e-3 + 2.0 ** -9 * float(emax.mean())
-    assert d.mean() <= mean_bound, f"{what}: mean-abs {d.mean():.3e} > {mean_bound:.3e}"
-
-
-def entry_magnitudes(w, inp, step, seqs):
-    """max_j |E_j,d| over the visible entries of each listed sequence at decode
-    step `step` (shared-entry form): pooled entries from the oracle's pooling,
-    raw entries as the oracle's finalisation of single tokens (m = 1, zero
-    logits and bias: pooling is then the identity)."""
-    assert w.shared_kv
-    c = ocfg(w)
-    c1 = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, True, 1, w.n_win, w.rope_dims, w.rmsnorm, w.rope_theta)
-    out = []
-    for b in seqs:
-        L = int(inp.lens[b]) + step + 1
-        P = max(0, (L - w.n_win) // w.block_m)
-        x = f64(inp.k[b:b + 1, :L])
-        rows = []
-        if P:
-            rows.append(orc.pool(c, 0, x[:, :P * w.block_m], f64(inp.zk[b:b + 1, :P * w.block_m]),
-                                 f64(inp.bpos_k))[0, :, 0])
-        raw = orc.pool(c1, 0, x, np.zeros_like(x), np.zeros((1, w.n_kv_heads * w.head_dim)))[0, P * w.block_m:, 0]
-        rows.append(raw)
-        out.append(np.abs(np.concatenate(rows)).max(axis=0))
-    return np.stack(out)
-
-
 def visible_entries(w, L):
     """Size of the visible list at length L (block-aligned partition)."""
     P = max(0, (L - w.n_win) // w.block_m)
@@ -190,7 +146,7 @@ class DecodeRun:
         L.lbca_append(self.cfg, self.token(self.k), self.token(self.v), self.token(self.zk), self.token(self.zv),
                       self.bpk, self.bpv, None, self.cache, self.status)
         out = torch.empty(self.B, self.w.n_q_heads, self.w.head_dim, dtype=L.torch_dtype(self.cfg), device="cuda")
-        L.lbca_decode(self.cfg, self.q[self.step_i], self.cache, self.sink, None, out, self.ws, self.max_ctx,
+        L.lbca_decode(self.cfg, self.q[self.step_i], self.cache, self.sink, None, None, out, self.ws, self.max_ctx,
                       self.status)
         self.pos += 1
         self.step_i += 1

@@ -98,7 +98,7 @@ def test_cache_and_decode_checks(L):
     shared_bad = L.lbca_cache(A, None, A, None, A, A, 1, 600, 192, 0)
     ws = L.lbca_decode_workspace_bytes(cfg, 1, 32769)
     assert ws > 0
-    dec = lambda c, wsb: L._lib.lbca_decode(ctypes.byref(cfg), A, ctypes.byref(c), None, None, 32769,  # noqa
+    dec = lambda c, wsb: L._lib.lbca_decode(ctypes.byref(cfg), A, ctypes.byref(c), None, None, None, 32769,  # noqa
                                             A, A, wsb, None, None)
     assert dec(small, ws) == L.LBCA_ERR_CAPACITY          # ring too small for the window
     assert dec(shared_bad, ws) == L.LBCA_ERR_ARG          # GQA needs pooled_v / ring_v
@@ -148,8 +148,9 @@ def test_decode_step_form(L):
 def test_shared_entry_step_forms(L):
     """The fused tensor-core step takes the shared-entry form with 64 query
     heads per kv head, one kv head, D 256 or 512, bf16 and a raw window;
-    other shared-entry shapes keep the CUDA-core forms or the two calls.  Its
-    workspace query returns a small positive size (it uses none)."""
+    other shared-entry shapes run the two calls (the CUDA-core fused forms
+    serve the GQA form only).  Its workspace query returns a small positive
+    size (it uses none)."""
     hca = dict(n_q_heads=64, n_kv_heads=1, head_dim=512, shared_kv=True, block_m=128, rope_dims=64, n_win=128)
     assert L.lbca_decode_step_form(_cfg(L, **hca), 8, 131073) == L.LBCA_STEP_SHARED_TC
     assert L.lbca_decode_step_form(_cfg(L, **dict(hca, head_dim=256)), 8, 131073) == L.LBCA_STEP_SHARED_TC
@@ -157,7 +158,8 @@ def test_shared_entry_step_forms(L):
     # not the tensor-core shape: 48 heads per kv head, f32, D = 128
     assert L.lbca_decode_step_form(_cfg(L, **dict(hca, n_q_heads=48)), 8, 131073) != L.LBCA_STEP_SHARED_TC
     assert L.lbca_decode_step_form(_cfg(L, **dict(hca, dtype="f32")), 8, 131073) != L.LBCA_STEP_SHARED_TC
-    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, head_dim=128)), 8, 131073) != L.LBCA_STEP_SHARED_TC
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, head_dim=128)), 8, 131073) == L.LBCA_STEP_TWO_CALLS
+    assert L.lbca_decode_step_form(_cfg(L, **dict(hca, n_q_heads=4, head_dim=128)), 32, 4096) == L.LBCA_STEP_TWO_CALLS
     # a list longer than 16 CTAs x 128 rows can hold: no tensor-core plan at all
     assert L.lbca_decode_step_form(_cfg(L, **dict(hca, block_m=16)), 1, 131073) != L.LBCA_STEP_SHARED_TC
 

@@ -161,7 +161,7 @@ def test_decode_empty_sequence_gives_zeros(L):
     run = DecodeRun(L, w, inp, steps=1)
     run.cache.seq_lens.zero_()
     out = torch.full((2, w.n_q_heads, w.head_dim), 3.0, dtype=torch.bfloat16, device="cuda")
-    L.lbca_decode(run.cfg, run.q[0], run.cache, None, None, out, run.ws, 1, run.status)
+    L.lbca_decode(run.cfg, run.q[0], run.cache, None, None, None, out, run.ws, 1, run.status)
     torch.cuda.synchronize()
     assert torch.all(out == 0)
 
@@ -177,3 +177,35 @@ def test_append_beyond_capacity_sets_status(L):
         run.pos += 1
     torch.cuda.synchronize()
     assert int(run.status.item()) == L.LBCA_ERR_CAPACITY
+
+
+# ----------------------------------------------------- fp16 operand range ----
+@pytest.mark.parametrize("where", ["none", "query", "key_in_block", "value_in_tail"])
+def test_prefill_fp16_range_sets_status(L, where):
+    """The tensor-core prefill multiplies in fp16: a bf16 input beyond the fp16
+    range (|x| > 65504) would silently become inf, so it sets the status word
+    to LBCA_ERR_UNSUPPORTED -- a query (widened in the kernel), a key of a
+    complete block (fp16 copy made by the pool pass), a value past the last
+    complete block (fp16 copy of the tail).  In-range inputs leave it zero."""
+    w = synth.scaled(W["gqa_prefill_16k"], seq_len=16 * 18 + 7)
+    inp = synth.make(w)
+    big = 1.0e5  # after any rotation one of its pair's components stays above 65504
+    if where == "query":
+        inp.q[0, 100, 5, 17] = big
+    elif where == "key_in_block":
+        inp.k[0, 40, 3, 120] = -big
+    elif where == "value_in_tail":
+        inp.v[0, 16 * 18 + 3, 6, 2] = big
+    cfg = lcfg(L, w)
+    B, T = 1, w.seq_len
+    out = torch.empty(B, T, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(L.lbca_prefill_workspace_bytes(cfg, B, T, False), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    d = lambda t: None if t is None else t.cuda()  # noqa: E731
+    L.lbca_prefill(cfg, d(inp.q), d(inp.k), d(inp.v), d(inp.zk), d(inp.zv), d(inp.bpos_k), d(inp.bpos_v), None,
+                   None, None, out, None, ws, d_status=st)
+    torch.cuda.synchronize()
+    want = 0 if where == "none" else L.LBCA_ERR_UNSUPPORTED
+    assert int(st.item()) == want
+    if where == "none":
+        assert_close(f64(out), oracle_prefill(w, inp), "bf16", "in-range prefill")

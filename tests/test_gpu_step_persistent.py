@@ -25,7 +25,7 @@ CASES = [
     ("ragged_gqa_decode_append", dict(ctx=(0, 2500), batch=16), 66),
     # one long sequence among short ones: its segments are cut between many CTAs
     ("ragged_gqa_decode_append", dict(ctx=(20, 200), batch=13, block_m=16), 20),
-    # shared-entry form on CUDA cores: RMSNorm, partial RoPE, sink, -t output rotation
+    # shared-entry form on CUDA cores (append then decode): RMSNorm, partial RoPE, sink, -t output rotation
     ("hca_mqa_decode_128k", dict(ctx=(100, 900), batch=8, n_q_heads=48, head_dim=128, rope_dims=32, block_m=16),
      20),
     # f32 I/O, 4 query heads on one shared entry, sink logit 0
@@ -43,7 +43,10 @@ def test_persistent_step_matches_oracle(L, name, kw, steps):
         lens[[3, 40]] = 0  # sequences with no cached tokens
     inp = synth.make(w, lens=lens)
     run = DecodeRun(L, w, inp)
-    assert L.lbca_decode_step_form(run.cfg, run.B, run.max_ctx) == L.LBCA_STEP_PERSISTENT
+    # the CUDA-core fused forms serve the GQA form; the shared form's raw window
+    # is finalised by the decode kernels, so its steps run append then decode
+    want_form = L.LBCA_STEP_TWO_CALLS if w.shared_kv else L.LBCA_STEP_PERSISTENT
+    assert L.lbca_decode_step_form(run.cfg, run.B, run.max_ctx) == want_form
     for s in range(steps):
         got = fused_step(run)
         if s % 6 == 0 or s == steps - 1:

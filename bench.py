@@ -46,11 +46,16 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gqa_decode_32k")
+    ap.add_argument("--workload", default="ragged_gqa_decode_append",
+                    help="the decode workload of the headline line (default: the largest single-GPU one)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--leg", default="decode", choices=["decode", "prefill", "pool"],
-                    help="decode: the decode-step benchmark (default, with the prefill and pool legs appended); "
-                         "prefill / pool: that leg alone (one JSON line)")
+                    help="decode: the decode-step benchmark (default, with the other decode workloads, the "
+                         "prefill and the pool legs appended under 'also' at one GPU); prefill / pool: that leg "
+                         "alone (one JSON line)")
+    ap.add_argument("--prefill", default="gqa_prefill_16k", help="workload of --leg prefill")
+    ap.add_argument("--pool", default=next(iter(POOL_CASES)), choices=list(POOL_CASES), help="case of --leg pool")
+    ap.add_argument("--no-also", action="store_true", help="the headline line alone")
     return ap.parse_args()
 
 
@@ -204,7 +209,7 @@ class DecodeBench:
         that runs as append + decode."""
         L = self.L
         rep, j = i % self.NR, i // self.NR
-        L.lbca_decode(self.cfg, self.q[j], self.caches[rep], self.sink, None, self.outs[rep], self.dec_ws[rep],
+        L.lbca_decode(self.cfg, self.q[j], self.caches[rep], self.sink, None, None, self.outs[rep], self.dec_ws[rep],
                       self.max_ctx, self.status)
 
     def launch(self, i, q=None, tok=None):
@@ -218,14 +223,20 @@ class DecodeBench:
                            self.outs[rep], self.step_ws[rep], self.max_ctx, self.status)
 
 
-def run_ours(args, w, rank, world):
+def run_ours(args, w, rank, world, reps=3):
+    """Decode steps of workload `w` on this GPU: W warm-up steps, then K steps
+    replayed back to back from one CUDA graph, `reps` times (median taken, the
+    clock sampler running throughout); then the end-to-end loop (e2e_loop).
+    Returns (JSON line, bench)."""
     import torch
     import torch.distributed as dist
 
     from block_compressed_long_b200 import ranks
 
     K, W = args.steps, args.warmup
-    bench = DecodeBench(w, rank, 2 * (W + K))
+    # steps each replica must hold: warm-up, reps graph replays, decode-only
+    # timing of a two-launch step, e2e warm-up and steps
+    bench = DecodeBench(w, rank, W + reps * K + (W + K) + (W + K))
     L = bench.L
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     cap = torch.cuda.Stream()
@@ -251,17 +262,20 @@ def run_ours(args, w, rank, world):
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
-    e0, e1 = E(), E()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0.record()
-    g_main.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    step_ms = e0.elapsed_time(e1) / K
+    times = []
+    for _ in range(reps):  # each replay appends K more tokens per replica: the cache holds them
+        e0, e1 = E(), E()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record()
+        g_main.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        times.append(e0.elapsed_time(e1) / K)
+    step_ms = statistics.median(times)
     bench.i += K
     del g_main
     kernel_ms = step_ms  # one fused kernel per step: the step is the kernel
@@ -271,20 +285,70 @@ def run_ours(args, w, rank, world):
             bench.launch_decode(i)
         g_dec = graph_of(bench.i, K, bench.launch_decode)
         torch.cuda.synchronize()
+        e0, e1 = E(), E()
         e0.record()
         g_dec.replay()
         e1.record()
         torch.cuda.synchronize()
         kernel_ms = e0.elapsed_time(e1) / K
         del g_dec
+    e2e_ms, h2d, d2h = e2e_loop(bench, K, W)
+    clocks = sampler.stop()
+    status = int(bench.status.item())
+    if status:
+        raise RuntimeError(f"device status {L.lbca_status_string(status)}")
 
-    # ---- end to end through the public API: pinned host inputs and output ----
-    # each step's inputs (q and the new token's k, v, z_k, z_v) sit packed in
-    # one pinned host buffer and cross with one copy; the output comes back
-    # with one copy.  As in a serving loop, the copies run on streams of their
-    # own beside the kernels: step i+1's upload overlaps step i's kernel and
-    # step i's download overlaps step i+1's (two staging slots; every step
-    # waits for its own upload, every download for its own step).
+    step_ms, e2e_ms, kernel_ms = ranks.max_over_ranks([step_ms, e2e_ms, kernel_ms], device="cuda")
+    hbm, src = peaks()
+    achieved = nbytes / K / (kernel_ms * 1e-3) / 1e9
+    w_ = bench.w
+    line = {
+        "metric": METRIC, "value": ranks.job_us_per_token(step_ms, bench.B, world), "unit": "µs/token",
+        "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
+        "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
+                   "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
+                   "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
+                   "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
+                   "l2": (f"inputs larger than L2: steps rotate over {bench.NR} cache replicas "
+                          f"(>= 3x L2 of data in total), each step's data cold"),
+                   "launch": (f"K steps of lbca_decode_step ({bench.launches} kernel launch"
+                              f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph, "
+                              f"median of {reps} replays; e2e: an eager host loop of lbca_decode_step calls "
+                              "(host-side validation and launch every step), each step's inputs uploaded from "
+                              "pinned host memory and its output read back on copy streams beside the kernels, "
+                              "timed as the longer of the device events and the host wall clock")},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": src,
+                     "kernel": ({L.LBCA_STEP_CLUSTER: "decode_step_kernel (cluster form)",
+                                 L.LBCA_STEP_PERSISTENT: "decode_flat_kernel (persistent evenly split form)",
+                                 L.LBCA_STEP_SHARED_TC: "decode_mqa_tc_kernel (shared-entry tensor-core form, "
+                                                        "append fused)"}
+                                .get(bench.form, "the decode launch of the step (timed alone over the same replicas)")),
+                     "bytes_per_launch": nbytes / K, "launch_us": kernel_ms * 1e3,
+                     "traffic": load_traffic(w_.name)},
+        "e2e": {"value": ranks.job_us_per_token(e2e_ms, bench.B, world), "unit": "µs/token",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * bench.launches,
+        "clocks": clocks,
+    }
+    return line, bench
+
+
+def e2e_loop(bench, K, W):
+    """The decode steps end to end through the public API, eagerly: each step
+    is one lbca_decode_step call from the host (argument validation and launch
+    included), its inputs (q and the new token's k, v, z_k, z_v, packed in one
+    pinned host buffer) cross with one copy and its output comes back with one
+    copy.  As in a serving loop the copies run on streams of their own beside
+    the kernels (step i+1's upload overlaps step i's kernel, step i's download
+    overlaps step i+1's; two staging slots; every step waits for its own
+    upload, every download for its own step).  Returns (ms per step = the
+    longer of the device-event span and the host wall clock, H2D bytes and D2H
+    bytes per step)."""
+    import torch
+
     parts = [bench.q] + [t for t in (bench.tk, bench.tv, bench.tzk, bench.tzv) if t is not None]
     sizes = [t[0].numel() * t[0].element_size() for t in parts]
     offs = np.cumsum([0] + sizes)
@@ -308,13 +372,9 @@ def run_ours(args, w, rank, world):
     ev_in = [torch.cuda.Event() for _ in range(NS)]        # slot's upload done
     ev_run = [torch.cuda.Event() for _ in range(NS)]       # the step that read the slot is done
     ev_down = [torch.cuda.Event() for _ in range(bench.NR)]  # download of an output replica done
+    cur = torch.cuda.current_stream()
 
-    def e2e_steps(first, n):
-        cur = torch.cuda.current_stream()
-        fork = torch.cuda.Event()
-        fork.record(cur)
-        s_in.wait_event(fork)
-        s_out.wait_event(fork)
+    def steps(first, n):
         for j, i in enumerate(range(first, first + n)):
             sl, rep = j % NS, i % bench.NR
             if j >= NS:
@@ -336,60 +396,38 @@ def run_ours(args, w, rank, world):
             ev.record(st)
             cur.wait_event(ev)
 
-    e2e_steps(bench.i, W)
+    steps(bench.i, W)
     bench.i += W
     torch.cuda.synchronize()
-    g_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_e2e, stream=cap):
-        e2e_steps(bench.i, K)
-    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     e0.record()
-    g_e2e.replay()
+    steps(bench.i, K)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / K
+    wall_ms = (time.perf_counter() - t0) * 1e3
     bench.i += K
-    del g_e2e
-    clocks = sampler.stop()
-    status = int(bench.status.item())
-    if status:
-        raise RuntimeError(f"device status {L.lbca_status_string(status)}")
+    return max(e0.elapsed_time(e1), wall_ms) / K, h2d, d2h
 
-    step_ms, e2e_ms, kernel_ms = ranks.max_over_ranks([step_ms, e2e_ms, kernel_ms], device="cuda")
-    hbm, src = peaks()
-    achieved = nbytes / K / (kernel_ms * 1e-3) / 1e9
-    w_ = bench.w
-    line = {
-        "metric": METRIC, "value": ranks.job_us_per_token(step_ms, bench.B, world), "unit": "µs/token",
-        "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
-        "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
-                   "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
-                   "block_m": w_.block_m, "n_win": w_.n_win, "rope_dims": w_.rope_dims,
-                   "shared_kv": w_.shared_kv, "parallelism": f"dp{world}",
-                   "l2": (f"inputs larger than L2: steps rotate over {bench.NR} cache replicas "
-                          f"(>= 3x L2 of data in total), each step's data cold"),
-                   "launch": (f"K steps of lbca_decode_step ({bench.launches} kernel launch"
-                              f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph; "
-                              "e2e: each step's upload and download on copy streams beside the kernels "
-                              "(uploads one step ahead, downloads one step behind), all inside the timed graph")},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src,
-                     "kernel": ({L.LBCA_STEP_CLUSTER: "decode_step_kernel (cluster form)",
-                                 L.LBCA_STEP_PERSISTENT: "decode_flat_kernel (persistent evenly split form)",
-                                 L.LBCA_STEP_SHARED_TC: "decode_mqa_tc_kernel (shared-entry tensor-core form, "
-                                                        "append fused)"}
-                                .get(bench.form, "the decode launch of the step (timed alone over the same replicas)")),
-                     "bytes_per_launch": nbytes / K, "launch_us": kernel_ms * 1e3,
-                     "traffic": load_traffic(w_.name)},
-        "e2e": {"value": ranks.job_us_per_token(e2e_ms, bench.B, world), "unit": "µs/token",
-                "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * bench.launches,
-        "clocks": clocks,
-    }
-    return line, bench
+
+def decode_also(args, name):
+    """One more decode workload at N = 1 (its own line under "also"), with the
+    oracle beside it."""
+    import gc
+
+    import torch
+
+    from block_compressed_long_b200 import synth
+    line, bench = run_ours(args, synth.WORKLOADS[name], 0, 1)
+    del bench
+    gc.collect()
+    torch.cuda.empty_cache()
+    for k in ("n_gpus", "steps", "warmup", "scaling", "vs_baseline", "data"):
+        line.pop(k, None)
+    line = {"workload": name, **line}
+    us, n, cores, desc = oracle_decode_timing(synth.WORKLOADS[name])
+    line["cpu_baseline"] = {"value": us, "unit": "µs/token", "cores": cores, "kind": "oracle", "sample": desc}
+    return line
 
 
 def peak_tflops():
@@ -400,92 +438,142 @@ def peak_tflops():
         return 1590.0, "fallback"
 
 
-def prefill_flops(w):
-    """Algorithmic FLOPs: 4 D Hq per visible (query, entry) pair."""
-    T, m, n = w.seq_len, w.block_m, w.n_win
+# FP32 CUDA-core peak of one B200: 148 SMs x 128 FP32 lanes x 2 flops per FMA x
+# 1965 MHz (the SM clock the machine's GPUs run at under load) = 74.4 TFLOP/s.
+F32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def prefill_pairs(w, rows=None):
+    """Visible (query, entry) pairs of the rows (all T by default), per head
+    and sequence."""
+    m, n = w.block_m, w.n_win
+    rows = range(w.seq_len) if rows is None else rows
     pairs = 0
-    for L in range(1, T + 1):
+    for t in rows:
+        L = t + 1
         P = max(0, (L - n) // m)
         pairs += P + (L - P * m)
-    return 4.0 * w.head_dim * w.n_q_heads * pairs * w.batch
+    return pairs
 
 
-def extra_prefill(reps=10, warm=3):
-    """lbca_prefill of the 16K-token GQA layer (pool pass, RoPE table, finalised
-    keys, tensor-core attention), inputs resident (> L2), CUDA events."""
+def prefill_flops(w, rows=None):
+    """Algorithmic FLOPs: 4 D Hq per visible (query, entry) pair."""
+    return 4.0 * w.head_dim * w.n_q_heads * prefill_pairs(w, rows) * w.batch
+
+
+def timed(run, reps, warm, uuid=None):
+    """Median over `reps` CUDA-event-timed calls of run() (ms), after `warm`
+    untimed calls, with the clock sampler running."""
+    import torch
+    for _ in range(warm):
+        run()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts), sampler.stop()
+
+
+def prefill_leg(name="gqa_prefill_16k", reps=10, warm=3, baseline=True):
+    """lbca_prefill of a prefill workload (pool pass, RoPE table, finalised
+    keys, attention), inputs resident in HBM (larger than L2 for the 16K
+    layer), CUDA events; the oracle on a bounded sample beside it."""
     import torch
 
     from block_compressed_long_b200 import lbca as L
     from block_compressed_long_b200 import synth
-    w = synth.WORKLOADS["gqa_prefill_16k"]
+    w = synth.WORKLOADS[name]
     inp = synth.make(w)
     cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
                    w.rmsnorm, w.rope_theta, dtype=w.dtype)
     d = lambda t: None if t is None else t.cuda()  # noqa: E731
-    q, k, v, zk, zv, bpk, bpv = (d(t) for t in (inp.q, inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v))
+    q, k, v, zk, zv, bpk, bpv, sink = (d(t) for t in (inp.q, inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v,
+                                                      inp.sink))
     out = torch.empty_like(q)
-    ws = torch.zeros(L.lbca_prefill_workspace_bytes(cfg, w.batch, w.seq_len, False), dtype=torch.uint8,
+    ws = torch.zeros(max(L.lbca_prefill_workspace_bytes(cfg, w.batch, w.seq_len, False), 16), dtype=torch.uint8,
                      device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for _ in range(warm):
-        L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, out, None, ws, d_status=st)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, out, None, ws, d_status=st)
-    e1.record()
-    torch.cuda.synchronize()
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    ms, clocks = timed(lambda: L.lbca_prefill(cfg, q, k, v, zk, zv, bpk, bpv, sink, None, None, out, None, ws,
+                                              d_status=st), reps, warm, uuid)
     if int(st.item()):
         raise RuntimeError(f"prefill device status {L.lbca_status_string(int(st.item()))}")
-    ms = e0.elapsed_time(e1) / reps
     fl = prefill_flops(w)
     tf = fl / (ms * 1e-3) / 1e12
-    pk, src = peak_tflops()
-    return {"workload": w.name, "metric": "prefill TFLOP/s", "value": tf, "unit": "TFLOP/s", "ms_per_call": ms,
-            "dtype": "bf16 I/O, fp16 tensor-core operands, f32 accumulate",
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
-                         "peak_source": src, "kernel": "prefill_tc_kernel (whole lbca_prefill call timed)",
-                         "flops_per_call": fl}}
+    if w.dtype == "bf16":
+        pk, src = peak_tflops()
+        roof = {"bound": "tensor", "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+                "peak_source": src, "kernel": "prefill_tc_kernel (whole lbca_prefill call timed)"}
+        dt = "bf16 I/O, fp16 tensor-core operands, f32 accumulate"
+    else:
+        roof = {"bound": "alu", "achieved": tf, "peak": F32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": tf / F32_ALU_TFLOPS, "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+                "kernel": "prefill_simt_kernel (whole lbca_prefill call timed)"}
+        dt = "f32 I/O and arithmetic (CUDA cores, no TF32)"
+    roof["flops_per_call"] = fl
+    line = {"workload": name, "metric": "prefill TFLOP/s", "value": tf, "unit": "TFLOP/s", "ms_per_call": ms,
+            "dtype": dt, "roofline": roof, "clocks": clocks}
+    del q, k, v, zk, zv, out, ws
+    torch.cuda.empty_cache()
+    if baseline:
+        line["cpu_baseline"] = oracle_prefill_timing(w, inp)
+    return line
 
 
-def extra_pool(reps=10, warm=3):
-    """lbca_pool of both series of the 32K-token GQA prefix (HBM-bound)."""
+POOL_CASES = {
+    # name: (workload, tokens, batch, series)
+    "gqa_decode_32k prefix (32768 tokens, K and V series)": ("gqa_decode_32k", 32768, 1, (0, 1)),
+    "gqa_prefill_16k (16384 tokens, m = 16, K and V series)": ("gqa_prefill_16k", 16384, 1, (0, 1)),
+    "hca_mqa_decode_128k (8 x 131072 tokens, D = 512, shared entries: RMSNorm and RoPE epilogue)":
+        ("hca_mqa_decode_128k", 131072, 8, (0,)),
+}
+
+
+def pool_leg(label, reps=10, warm=3, baseline=True):
+    """lbca_pool of every complete block of a workload's raw K/V (or C), each
+    series once per call (HBM-bound: X and Z read once, entries written)."""
     import torch
 
     from block_compressed_long_b200 import lbca as L
     from block_compressed_long_b200 import synth
-    w = synth.scaled(synth.WORKLOADS["gqa_decode_32k"], kind="prefill", seq_len=32768)
+    name, T, B, series = POOL_CASES[label]
+    w = synth.scaled(synth.WORKLOADS[name], kind="prefill", seq_len=T, batch=B, steps=1)
     inp = synth.make(w)
     cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
-                   dtype=w.dtype)
-    d = lambda t: t.cuda()  # noqa: E731
-    k, v, zk, zv, bpk, bpv = (d(t) for t in (inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v))
-    nb = w.seq_len // w.block_m
-    ok_ = torch.empty(1, w.n_kv_heads, nb, w.head_dim, dtype=torch.bfloat16, device="cuda")
-    ov_ = torch.empty_like(ok_)
+                   w.rmsnorm, w.rope_theta, dtype=w.dtype)
+    d = lambda t: None if t is None else t.cuda()  # noqa: E731
+    srcs = [(d(inp.k), d(inp.zk), d(inp.bpos_k))] + ([] if w.shared_kv else [(d(inp.v), d(inp.zv), d(inp.bpos_v))])
+    nb = T // w.block_m
+    outs = [torch.empty(B, w.n_kv_heads, nb, w.head_dim, dtype=L.torch_dtype(cfg), device="cuda") for _ in srcs]
 
     def run():
-        L.lbca_pool(cfg, L.LBCA_KEY, k, zk, bpk, None, ok_)
-        L.lbca_pool(cfg, L.LBCA_VALUE, v, zv, bpv, None, ov_)
+        for s, (x, z, bp) in zip(series, srcs):
+            L.lbca_pool(cfg, s, x, z, bp, None, outs[s])
 
-    for _ in range(warm):
-        run()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        run()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
-    nbytes = 2 * (2 * k.numel() * 2 + ok_.numel() * 2)  # K and V series: read X and Z, write entries
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    ms, clocks = timed(run, reps, warm, uuid)
+    esz = 2 if w.dtype == "bf16" else 4
+    nbytes = sum(2 * x.numel() * esz + o.numel() * esz for (x, _, _), o in zip(srcs, outs))
     gbs = nbytes / (ms * 1e-3) / 1e9
     hbm, src = peaks()
-    return {"workload": "gqa_decode_32k prefix (32768 tokens, K and V series)", "metric": "pool GB/s", "value": gbs,
-            "unit": "GB/s", "ms_per_call": ms,
+    line = {"workload": label, "metric": "pool GB/s", "value": gbs, "unit": "GB/s", "ms_per_call": ms,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "peak_source": src, "kernel": "pool_kernel", "bytes_per_call": nbytes}}
+                         "peak_source": src, "kernel": "pool_kernel", "bytes_per_call": nbytes,
+                         "launches_per_call": len(srcs)},
+            "clocks": clocks}
+    del srcs, outs
+    torch.cuda.empty_cache()
+    if baseline:
+        line["cpu_baseline"] = oracle_pool_timing(w, inp, series)
+    return line
 
 
 def load_traffic(workload):
@@ -502,19 +590,29 @@ def load_traffic(workload):
 
 
 # ----------------------------------------------------- oracle (CPU) timing ----
+def _cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
 def oracle_decode_timing(w, budget_s=12.0, max_steps=None):
     """The fp64 oracle as it stands, driven step by step on the host cores:
     each step appends one token per sequence (pooling a block when it
-    completes) and attends its query.  Returns (µs/token, steps, cores, desc)."""
+    completes) and attends its query.  Each step is timed on its own and the
+    median step is reported (a few steps that pool a block take longer).
+    Returns (µs/token, tokens, cores, description)."""
     from block_compressed_long_b200 import synth
     from oracle import oracle as orc
     f64 = synth.f64
     nb = max_steps or 64
-    ws = synth.scaled(w, steps=nb)
-    inp = synth.make(ws)
+    # a bounded sample: the workload's first (at most) 4 sequences, drawn alone
+    # (every sequence has its own random streams, so they equal those of the
+    # whole batch)
+    nseq = min(w.batch, 4)
+    ws = synth.scaled(w, steps=nb, batch=nseq)
+    inp = synth.make(ws, lens=synth.contexts(w)[:nseq])
     c = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
                    w.rmsnorm, w.rope_theta)
-    seqs = list(range(min(ws.batch, 4)))  # bounded sample of sequences
+    seqs = list(range(nseq))
     streams = []
     for b in seqs:
         Lb = int(inp.lens[b])
@@ -523,21 +621,78 @@ def oracle_decode_timing(w, budget_s=12.0, max_steps=None):
                   None if w.shared_kv else f64(inp.zv[b, :Lb]))
         streams.append(st)
     sink = f64(inp.sink)
-    t0 = time.perf_counter()
+    t_start = time.perf_counter()
+    per_step = []
     n = 0
-    while n < nb and (time.perf_counter() - t0) < budget_s:
+    while n < nb and (time.perf_counter() - t_start) < budget_s:
+        t0 = time.perf_counter()
         for st, b in zip(streams, seqs):
             p = int(inp.lens[b]) + n
             st.extend(f64(inp.k[b, p:p + 1]), f64(inp.zk[b, p:p + 1]),
                       None if w.shared_kv else f64(inp.v[b, p:p + 1]),
                       None if w.shared_kv else f64(inp.zv[b, p:p + 1]))
             st.query(f64(inp.q[n, b]), sink)
+        per_step.append(time.perf_counter() - t0)
         n += 1
-    dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    med = statistics.median(per_step)
     desc = (f"{n} decode steps of {len(seqs)} sequence(s) of {w.name} (contexts "
-            f"{[int(inp.lens[b]) for b in seqs]}), fp64 C oracle, cache of pooled entries kept between steps")
-    return dt * 1e6 / (n * len(seqs)), n * len(seqs), cores, desc
+            f"{[int(inp.lens[b]) for b in seqs]}), fp64 C oracle, cache of pooled entries kept between steps; "
+            f"median step {med * 1e3:.2f} ms (min {min(per_step) * 1e3:.2f}, max {max(per_step) * 1e3:.2f})")
+    return med * 1e6 / len(seqs), n * len(seqs), _cores(), desc
+
+
+def oracle_prefill_timing(w, inp, n_rows=48):
+    """The fp64 oracle's prefill of the same inputs on the host cores: the
+    pooling of every complete block timed in full, the attention of a bounded
+    sample of query rows (spread over the sequence) timed and scaled to all T
+    rows by their share of the visible pairs.  Returns a cpu_baseline record
+    in the leg's unit (TFLOP/s of the algorithmic flops)."""
+    from block_compressed_long_b200 import synth
+    from oracle import oracle as orc
+    f64 = synth.f64
+    c = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta)
+    T = w.seq_len
+    k, v, zk, zv = f64(inp.k), f64(inp.v), f64(inp.zk), f64(inp.zv)
+    t0 = time.perf_counter()
+    nbk = T // w.block_m * w.block_m
+    ek = orc.pool(c, orc.KEY, k[:, :nbk], zk[:, :nbk], f64(inp.bpos_k))
+    ev = None if w.shared_kv else orc.pool(c, orc.VALUE, v[:, :nbk], zv[:, :nbk], f64(inp.bpos_v))
+    t_pool = time.perf_counter() - t0
+    rows = np.unique(np.linspace(0, T - 1, min(n_rows, T)).astype(np.int64))
+    q = f64(inp.q[:, rows])
+    t0 = time.perf_counter()
+    orc.attend(c, q, np.broadcast_to(rows, (w.batch, len(rows))), ek, ev, k, None if w.shared_kv else v,
+               np.full(w.batch, T), f64(inp.sink))
+    t_att = time.perf_counter() - t0
+    t_total = t_pool + t_att * prefill_pairs(w) / max(1, prefill_pairs(w, rows))
+    return {"value": prefill_flops(w) / t_total / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": (f"{w.name}: fp64 C oracle, pooling of all {T // w.block_m} blocks timed ({t_pool:.2f} s), "
+                       f"attention of {len(rows)} of {T} query rows timed ({t_att:.2f} s) and scaled by visible "
+                       f"pairs to all rows: {t_total:.1f} s per prefill")}
+
+
+def oracle_pool_timing(w, inp, series, max_tokens=8192):
+    """The fp64 oracle's pooling of a bounded sample (the first blocks, at most
+    max_tokens tokens of every sequence) on the host cores, in GB/s of the same
+    algorithmic bytes the GPU leg counts."""
+    from block_compressed_long_b200 import synth
+    from oracle import oracle as orc
+    f64 = synth.f64
+    c = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta)
+    n = min(w.seq_len, max_tokens) // w.block_m * w.block_m
+    srcs = [(orc.KEY, inp.k, inp.zk, inp.bpos_k)] + ([] if w.shared_kv else [(orc.VALUE, inp.v, inp.zv, inp.bpos_v)])
+    xs = [(s, f64(x[:, :n]), f64(z[:, :n]), f64(bp)) for s, x, z, bp in srcs]
+    t0 = time.perf_counter()
+    for s, x, z, bp in xs:
+        orc.pool(c, s, x, z, bp)
+    dt = time.perf_counter() - t0
+    esz = 2 if w.dtype == "bf16" else 4
+    nbytes = len(xs) * w.batch * n * w.n_kv_heads * w.head_dim * esz * (2 + 1.0 / w.block_m)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+            "sample": (f"fp64 C oracle pooling the first {n} tokens of each of {w.batch} sequence(s), "
+                       f"{len(xs)} series ({dt:.2f} s)")}
 
 
 def main():
@@ -551,7 +706,8 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        us, n, cores, desc = oracle_decode_timing(w, budget_s=max(5.0, 0.5 * args.steps), max_steps=args.warmup + args.steps)
+        budget = min(60.0, max(5.0, 0.5 * (args.warmup + args.steps)))
+        us, n, cores, desc = oracle_decode_timing(w, budget_s=budget, max_steps=args.warmup + args.steps)
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": us, "unit": "µs/token", "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
                           "dtype": "f64", "data": "synthetic", "config": {"workload": w.name},
@@ -573,12 +729,22 @@ def main():
     __graft_entry__.build()
     if args.leg != "decode":  # one leg alone, on this GPU
         if rank == 0:
-            leg = extra_prefill if args.leg == "prefill" else extra_pool
-            print(json.dumps(leg(reps=args.steps, warm=args.warmup)), flush=True)
+            if args.leg == "prefill":
+                out = prefill_leg(args.prefill, reps=args.steps, warm=args.warmup, baseline=False)
+            else:
+                out = pool_leg(args.pool, reps=args.steps, warm=args.warmup, baseline=False)
+            print(json.dumps(out), flush=True)
         return
-    line, _ = run_ours(args, w, rank, world)
-    if world == 1 and args.workload == "gqa_decode_32k":
-        line["also"] = [extra_prefill(), extra_pool()]
+    line, bench = run_ours(args, w, rank, world)
+    del bench
+    if world == 1 and not args.no_also:
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        also = [decode_also(args, n) for n in ("gqa_decode_32k", "hca_mqa_decode_128k") if n != w.name]
+        also += [prefill_leg("gqa_prefill_16k"), prefill_leg("tiny_f32_prefill")]
+        also += [pool_leg(label) for label in POOL_CASES]
+        line["also"] = also
     if rank == 0 and world == 1:
         us, n, cores, desc = oracle_decode_timing(w)
         line["cpu_baseline"] = {"value": us, "unit": "µs/token", "cores": cores, "kind": "oracle", "sample": desc}

@@ -107,3 +107,63 @@ def attention(q, k, v, zk, zv, bpk, bpv, *, m, w, shared_kv, rope_dims=0, theta=
                 o = _rot(o, -t, rope_dims, theta)
             out[t, h] = o
     return out
+
+
+# ---- CSA form (CSA page, "What is implemented": Eqs 9-12, 13-17, 18-19, 27) ----
+def pool_dual_series(xa, za, xb, zb, bpa, bpb, m):
+    """Dual overlapped pooling, one sequence: x*, z* [T, G, D]; bp* [m, G*D] ->
+    [T//m, G, D].  Entry i stacks block i of the a-series and block i-1 of the
+    b-series along one axis and takes scipy's softmax over all of it (block 0:
+    the a-series block alone)."""
+    T, G, D = xa.shape
+    nb = T // m
+    out = np.zeros((nb, G, D))
+    for i in range(nb):
+        la = za[i * m:(i + 1) * m] + bpa.reshape(m, G, D)
+        va = xa[i * m:(i + 1) * m]
+        if i > 0:
+            lb = zb[(i - 1) * m:i * m] + bpb.reshape(m, G, D)
+            logits = np.concatenate([la, lb], axis=0)
+            vals = np.concatenate([va, xb[(i - 1) * m:i * m]], axis=0)
+        else:
+            logits, vals = la, va
+        out[i] = (softmax(logits, axis=0) * vals).sum(axis=0)
+    return out
+
+
+def indexer(q, w, kx, nvis):
+    """q [HI, DI], w [HI], kx [NB, DI] -> scores of the first nvis blocks."""
+    dots = kx[:nvis] @ q.T                      # [nvis, HI]
+    return np.maximum(dots, 0.0) @ w
+
+
+def topk(scores, k):
+    """Indices of the k largest scores (ties: lower index first), by sorting."""
+    order = sorted(range(len(scores)), key=lambda j: (-scores[j], j))
+    return order[:k]
+
+
+def attention_sparse(q, entries, sel, c_hist, t, *, w, rope_dims=0, theta=10000.0, rmsnorm=False, eps=1e-6,
+                     sink=None, gamma_q=None, gamma_kv=None, scale=None):
+    """One query q [Hq, D] at position t over entries[sel] ([NB, D] finalised)
+    plus the raw window c_hist[max(0, t+1-w) .. t] ([T, D], finalised here)
+    and the sink; output rotated back by -t.  [Hq, D]."""
+    Hq, D = q.shape
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    win = list(range(max(0, t + 1 - w), t + 1))
+    raw = c_hist[win]
+    if rmsnorm:
+        raw = _rms(raw, gamma_kv, eps)
+    raw = _rot(raw, np.asarray(win, dtype=np.float64), rope_dims, theta)
+    rows = np.concatenate([entries[[j for j in sel if j >= 0]], raw], axis=0)
+    qn = _rms(q, gamma_q, eps) if rmsnorm else q
+    qr = _rot(qn, np.full(Hq, float(t)), rope_dims, theta)
+    out = np.zeros((Hq, D))
+    for h in range(Hq):
+        logits = rows @ qr[h] * scale
+        vals = rows
+        if sink is not None:
+            logits = np.append(logits, sink[h])
+            vals = np.concatenate([vals, np.zeros((1, D))], axis=0)
+        out[h] = _rot(softmax(logits) @ vals, -t, rope_dims, theta)
+    return out

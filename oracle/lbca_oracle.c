@@ -279,3 +279,186 @@ int orc_attend(const orc_config* c, int B, int nq, const long* qpos,
     }
     return err ? -1 : 0;
 }
+
+/* ===================================================================== *
+ * CSA form: dual overlapped pooling, lightning-indexer relevance, sparse *
+ * attention over the selected entries and an overlapping raw window.    *
+ * (CSA page, section "What is implemented": dual overlapped compression *
+ * Eqs 9-12, lightning indexer Eqs 13-17, shared-KV MQA core attention   *
+ * Eqs 18-19 with the sliding-window branch, sink Eq 27.)                *
+ * ===================================================================== */
+
+/*
+ * Dual overlapped pooling of the floor(T/m) complete blocks.  Two series,
+ * a and b, each with raw values x and content logits z ([B, T, G, D]) and a
+ * positional bias ([m, G*D], by in-block offset).  Entry i pools, per
+ * channel, its own block i from the a-series and the preceding block i-1 from
+ * the b-series under ONE softmax over the 2m logits (block 0 has no preceding
+ * block: its softmax runs over its m a-series logits alone):
+ *     w = softmax( [z_a[i m + r] + B_a[r]]_r , [z_b[(i-1) m + r] + B_b[r]]_r )
+ *     entry_i = sum_r w_a[r] x_a[i m + r] + sum_r w_b[r] x_b[(i-1) m + r]
+ * series ORC_KEY then finalises (RMSNorm when on, RoPE at the entry's own
+ * block start i*m); ORC_VALUE keeps the pooled value.  out [B, T/m, G, D].
+ */
+int orc_pool_dual(const orc_config* c, int series, int B, long T,
+                  const double* xa, const double* za, const double* xb, const double* zb,
+                  const double* bpos_a, const double* bpos_b, const double* gamma, double* out)
+{
+    if (!cfg_ok(c) || B < 0 || T < 0 || !xa || !za || !xb || !zb || !bpos_a || !bpos_b || !out) return -1;
+    const int m = c->block_m, G = c->n_kv_heads, D = c->head_dim;
+    const long NB = T / m;
+    const long ts = (long)G * D;
+    long total = (long)B * NB * G;
+#pragma omp parallel for schedule(static)
+    for (long idx = 0; idx < total; ++idx) {
+        const int g = (int)(idx % G);
+        const long i = (idx / G) % NB;
+        const long b = idx / ((long)G * NB);
+        double* e = out + ((b * NB + i) * G + g) * (long)D;
+        for (int ch = 0; ch < D; ++ch) {
+            const long col = (long)g * D + ch;
+            /* the joint list of logits: own block (a), then the preceding one (b) */
+            double amax = -INFINITY;
+            for (int r = 0; r < m; ++r) {
+                double a = za[(b * T + i * m + r) * ts + col] + bpos_a[r * ts + col];
+                if (a > amax) amax = a;
+            }
+            if (i > 0)
+                for (int r = 0; r < m; ++r) {
+                    double a = zb[(b * T + (i - 1) * m + r) * ts + col] + bpos_b[r * ts + col];
+                    if (a > amax) amax = a;
+                }
+            double den = 0.0, num = 0.0;
+            for (int r = 0; r < m; ++r) {
+                double p = exp(za[(b * T + i * m + r) * ts + col] + bpos_a[r * ts + col] - amax);
+                den += p;
+                num += p * xa[(b * T + i * m + r) * ts + col];
+            }
+            if (i > 0)
+                for (int r = 0; r < m; ++r) {
+                    double p = exp(zb[(b * T + (i - 1) * m + r) * ts + col] + bpos_b[r * ts + col] - amax);
+                    den += p;
+                    num += p * xb[(b * T + (i - 1) * m + r) * ts + col];
+                }
+            e[ch] = num / den;
+        }
+        if (series == ORC_KEY) finalise_key(c, e, gamma, (double)(i * m));
+    }
+    return 0;
+}
+
+/*
+ * Lightning-indexer relevance of every complete entry to one query per
+ * sequence: I_j = sum_h w_h * ReLU(q_h . k_j) over the indexer heads h, for
+ * the entries j < nvis[b] (the complete blocks the query can see); the rest
+ * of the row is -infinity.
+ *   q [B, HI, DI] indexer queries, w [B, HI] head weights,
+ *   kx [B, NB, DI] compressed indexer keys, out [B, NB].
+ */
+int orc_indexer_scores(int B, long NB, int HI, int DI, const double* q, const double* w,
+                       const double* kx, const long* nvis, double* out)
+{
+    if (B < 0 || NB < 0 || HI < 1 || DI < 1 || !q || !w || !kx || !nvis || !out) return -1;
+    for (int b = 0; b < B; ++b)
+        if (nvis[b] < 0 || nvis[b] > NB) return -1;
+    long total = (long)B * NB;
+#pragma omp parallel for schedule(static)
+    for (long idx = 0; idx < total; ++idx) {
+        const long j = idx % NB, b = idx / NB;
+        if (j >= nvis[b]) {
+            out[idx] = -INFINITY;
+            continue;
+        }
+        double s = 0.0;
+        for (int h = 0; h < HI; ++h) {
+            double dot = 0.0;
+            for (int d = 0; d < DI; ++d) dot += q[((long)b * HI + h) * DI + d] * kx[(b * NB + j) * DI + d];
+            s += w[(long)b * HI + h] * (dot > 0.0 ? dot : 0.0);
+        }
+        out[idx] = s;
+    }
+    return 0;
+}
+
+/*
+ * Sparse core attention of the shared-KV form for one query per sequence at
+ * position t = lens[b] - 1: one softmax over the selected entries (finalised
+ * compressed entries, sel[b, i] >= 0; -1 entries are unused) and the raw
+ * window of the last n_win tokens s in [max(0, lens - n_win), t] (finalised
+ * at s), plus the sink; the output's RoPE dims turn back by -t.
+ *   q [B, Hq, D]; ek [B, NB, 1, D]; sel [B, K]; k [B, T_hist, 1, D] raw history;
+ *   sink [Hq] or NULL; gq, gkv [D] or NULL; out [B, Hq, D].
+ * The window may cover tokens that a selected entry also summarises (the
+ * two branches overlap).
+ */
+int orc_attend_sparse(const orc_config* c, int B, const double* q, const double* ek, long NB,
+                      const long* sel, int K, const double* k, long T_hist, const long* lens,
+                      const double* sink, const double* gq, const double* gkv, double* out)
+{
+    if (!cfg_ok(c) || !c->shared_kv || c->n_kv_heads != 1 || B < 0 || K < 0 || !q || !k || !lens || !out)
+        return -1;
+    if (K > 0 && (!sel || !ek)) return -1;
+    const int Hq = c->n_q_heads, D = c->head_dim, w = c->n_win;
+    const double scale = c->softmax_scale > 0 ? c->softmax_scale : 1.0 / sqrt((double)D);
+    for (int b = 0; b < B; ++b) {
+        if (lens[b] < 1 || lens[b] > T_hist) return -1;
+        for (int i = 0; i < K; ++i)
+            if (sel[(long)b * K + i] >= NB) return -1;
+    }
+    int err = 0;
+    long total = (long)B * Hq;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long idx = 0; idx < total; ++idx) {
+        const int h = (int)(idx % Hq);
+        const long b = idx / Hq;
+        const long t = lens[b] - 1;
+        const long s0 = lens[b] - w > 0 ? lens[b] - w : 0;
+        const long n = K + (t - s0 + 1);
+        double* qt = malloc(sizeof(double) * D);
+        double* rows = malloc(sizeof(double) * D * (size_t)(n > 0 ? n : 1));
+        double* sc = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        char* use = malloc((size_t)(n > 0 ? n : 1));
+        double* o = out + (b * Hq + h) * (long)D;
+        if (!qt || !rows || !sc || !use) {
+            free(qt); free(rows); free(sc); free(use);
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        memcpy(qt, q + (b * Hq + h) * (long)D, sizeof(double) * D);
+        if (c->rmsnorm) rmsnorm(qt, D, gq, c->rms_eps);
+        if (c->rope_dims) rope(qt, D, c->rope_dims, c->rope_theta, (double)t);
+        /* the visible rows: selected entries, then the window */
+        for (int i = 0; i < K; ++i) {
+            long j = sel[b * K + i];
+            use[i] = j >= 0;
+            if (j >= 0) memcpy(rows + (long)i * D, ek + (b * NB + j) * (long)D, sizeof(double) * D);
+        }
+        for (long s = s0; s <= t; ++s) {
+            double* r = rows + (K + (s - s0)) * (long)D;
+            memcpy(r, k + (b * T_hist + s) * (long)D, sizeof(double) * D);
+            finalise_key(c, r, gkv, (double)s);
+            use[K + (s - s0)] = 1;
+        }
+        double smax = sink ? sink[h] : -INFINITY;
+        for (long e = 0; e < n; ++e) {
+            if (!use[e]) continue;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += qt[d] * rows[e * D + d];
+            sc[e] = acc * scale;
+            if (sc[e] > smax) smax = sc[e];
+        }
+        double den = sink ? exp(sink[h] - smax) : 0.0;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (long e = 0; e < n; ++e) {
+            if (!use[e]) continue;
+            double p = exp(sc[e] - smax);
+            den += p;
+            for (int d = 0; d < D; ++d) o[d] += p * rows[e * D + d];
+        }
+        for (int d = 0; d < D; ++d) o[d] /= den;
+        if (c->rope_dims) rope(o, D, c->rope_dims, c->rope_theta, -(double)t);
+        free(qt); free(rows); free(sc); free(use);
+    }
+    return err ? -1 : 0;
+}

@@ -18,6 +18,17 @@ Functions and the passages they follow:
   * ``Stream``    -- the same definition driven token by token, pooling each
                      block when it completes ("mSeek" README, repository
                      layout: generation through the LBCA cache).
+  * ``pool_dual``  -- CSA dual overlapped pooling: entry i pools its own block
+                     (a-series) and the preceding block (b-series) under one
+                     joint softmax (CSA page, "What is implemented", Eqs 9-12).
+  * ``indexer_scores`` / ``topk_blocks`` -- lightning-indexer relevance
+                     sum_h w_h ReLU(q_h . k_j) over the complete blocks, and
+                     the top-k of them (CSA page, "What is implemented",
+                     Eqs 13-17).
+  * ``attend_sparse`` -- shared-KV core attention over the selected entries
+                     plus the overlapping window of the last n_win raw tokens
+                     and the sink (CSA page, "What is implemented", Eqs 18-19,
+                     Eq 27, -i rotation).
   * ``visible_blocks`` -- P(L) of the block-aligned visibility reading.
   * ``cache_entries`` / ``kv_cache_bytes`` -- analytic cache accounting
                      ("mSeek" README, "Results").
@@ -93,6 +104,15 @@ def _load():
         lib.orc_attend.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int, lp, dp, dp, dp,
                                    ctypes.c_long, dp, dp, ctypes.c_long, lp, dp, dp, dp, dp]
         lib.orc_attend.restype = ctypes.c_int
+        lib.orc_pool_dual.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int, ctypes.c_long,
+                                      dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.orc_pool_dual.restype = ctypes.c_int
+        lib.orc_indexer_scores.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int, dp, dp, dp,
+                                           lp, dp]
+        lib.orc_indexer_scores.restype = ctypes.c_int
+        lib.orc_attend_sparse.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, dp, dp, ctypes.c_long, lp,
+                                          ctypes.c_int, dp, ctypes.c_long, lp, dp, dp, dp, dp]
+        lib.orc_attend_sparse.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -253,6 +273,96 @@ class Stream:
                       None if ek is None else ek[None], None if ev is None else ev[None],
                       self._arr("k", L)[None], None if shared else self._arr("v", L)[None],
                       np.array([L]), sink, gamma_q, self.gamma_kv)[0, 0]
+
+
+def pool_dual(cfg: Config, series: int, xa, za, xb, zb, bpos_a, bpos_b, gamma=None):
+    """Dual overlapped pooling of the T//m complete blocks: [B, T//m, G, D] fp64.
+    Entry i: one softmax over block i's a-series logits and block i-1's
+    b-series logits (block 0: its a-series alone); ORC KEY entries then take
+    RMSNorm (when on) and RoPE at i*m."""
+    xa, xap = _d(xa)
+    za, zap = _d(za)
+    xb, xbp = _d(xb)
+    zb, zbp = _d(zb)
+    bpos_a, bap = _d(bpos_a)
+    bpos_b, bbp = _d(bpos_b)
+    gamma, gp = _d(gamma)
+    B, T, G, D = xa.shape
+    assert za.shape == xb.shape == zb.shape == xa.shape and G == cfg.n_kv_heads and D == cfg.head_dim
+    assert bpos_a.shape == bpos_b.shape == (cfg.block_m, G * D)
+    out = np.zeros((B, T // cfg.block_m, G, D))
+    rc = _load().orc_pool_dual(ctypes.byref(cfg.c()), series, B, T, xap, zap, xbp, zbp, bap, bbp, gp,
+                               out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc:
+        raise ValueError("orc_pool_dual rejected its arguments")
+    return out
+
+
+def complete_blocks(L: int, m: int) -> int:
+    """Blocks of m tokens complete within the first L tokens: the compressed
+    entries a query that sees L tokens may select (the CSA form's entries are
+    visible once complete; its raw window overlaps them)."""
+    return int(L) // int(m)
+
+
+def indexer_scores(q, w, kx, nvis):
+    """I[b, j] = sum_h w[b, h] ReLU(q[b, h] . kx[b, j]) for j < nvis[b], -inf after.
+    q [B, HI, DI], w [B, HI], kx [B, NB, DI]."""
+    q, qp = _d(q)
+    w, wp = _d(w)
+    kx, kp = _d(kx)
+    B, HI, DI = q.shape
+    NB = kx.shape[1]
+    assert w.shape == (B, HI) and kx.shape == (B, NB, DI)
+    nvis = np.ascontiguousarray(nvis, dtype=np.int64).reshape(B)
+    out = np.zeros((B, NB))
+    rc = _load().orc_indexer_scores(B, NB, HI, DI, qp, wp, kp,
+                                    nvis.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
+                                    out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc:
+        raise ValueError("orc_indexer_scores rejected its arguments")
+    return out
+
+
+def topk_blocks(scores, nvis, k: int):
+    """The k highest-scoring visible blocks per row, highest first (equal
+    scores: lower index first), padded with -1 when fewer than k are visible:
+    [B, k] int64."""
+    scores = np.asarray(scores, dtype=np.float64)
+    B, NB = scores.shape
+    out = np.full((B, k), -1, dtype=np.int64)
+    for b in range(B):
+        n = int(nvis[b])
+        idx = np.arange(n)
+        order = np.lexsort((idx, -scores[b, :n]))  # by score descending, then index
+        take = order[:k]
+        out[b, :len(take)] = take
+    return out
+
+
+def attend_sparse(cfg: Config, q, ek, sel, k, lens, sink=None, gamma_q=None, gamma_kv=None):
+    """Shared-KV attention of one query per sequence (at lens[b] - 1) over the
+    selected entries ek[b, sel[b, i]] (sel -1: unused) plus the raw window of
+    the last n_win tokens and the sink: [B, Hq, D]."""
+    q, qp = _d(q)
+    B, Hq, D = q.shape
+    ek, ekp = _d(ek)
+    sel = np.ascontiguousarray(sel, dtype=np.int64)
+    K = sel.shape[1] if sel.ndim == 2 else 0
+    k, kp = _d(k)
+    lens = np.ascontiguousarray(lens, dtype=np.int64).reshape(B)
+    sink, sp = _d(sink)
+    gamma_q, gqp = _d(gamma_q)
+    gamma_kv, gkp = _d(gamma_kv)
+    out = np.zeros((B, Hq, D))
+    lp = ctypes.POINTER(ctypes.c_long)
+    rc = _load().orc_attend_sparse(ctypes.byref(cfg.c()), B, qp, ekp, 0 if ek is None else ek.shape[1],
+                                   sel.ctypes.data_as(lp) if K else None, K, kp, k.shape[1],
+                                   lens.ctypes.data_as(lp), sp, gqp, gkp,
+                                   out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc:
+        raise ValueError("orc_attend_sparse rejected its arguments")
+    return out
 
 
 def cache_entries(T: int, m: int, w: int) -> int:

@@ -462,3 +462,231 @@ int orc_attend_sparse(const orc_config* c, int B, const double* q, const double*
     }
     return err ? -1 : 0;
 }
+
+/* ===================================================================== *
+ * Backward of the prefill (pooling + attention), for training.          *
+ * ("mSeek" README, "Experiment at a glance": the LBCA layers are trained *
+ * by continued pretraining, so gradients flow through the pooling       *
+ * weights Z, the positional bias B_pos, the raw keys and values, and the *
+ * queries.)  Plain reverse-mode differentiation of orc_pool + orc_attend *
+ * as written above, in fp64.                                            *
+ * ===================================================================== */
+
+/* dx of y = x * r * gamma, r = 1/sqrt(mean(x^2) + eps), given dy (all [D]). */
+static void rmsnorm_bwd(const double* x, const double* dy, int D, const double* gamma, double eps, double* dx)
+{
+    double ss = 0.0, dot = 0.0;
+    for (int d = 0; d < D; ++d) ss += x[d] * x[d];
+    const double r = 1.0 / sqrt(ss / D + eps);
+    for (int d = 0; d < D; ++d) dot += (gamma ? gamma[d] : 1.0) * dy[d] * x[d];
+    for (int d = 0; d < D; ++d) dx[d] = r * (gamma ? gamma[d] : 1.0) * dy[d] - x[d] * r * r * r * dot / D;
+}
+
+/* d(input of the key finalisation) from d(finalised), at position pos. */
+static void finalise_key_bwd(const orc_config* c, const double* raw, const double* dfin, const double* gamma,
+                             double pos, double* dx)
+{
+    const int D = c->head_dim;
+    double* t = malloc(sizeof(double) * D);
+    memcpy(t, dfin, sizeof(double) * D);
+    if (c->rope_dims) rope(t, D, c->rope_dims, c->rope_theta, -pos);  /* rotations are orthogonal */
+    if (c->rmsnorm) rmsnorm_bwd(raw, t, D, gamma, c->rms_eps, dx);
+    else memcpy(dx, t, sizeof(double) * D);
+    free(t);
+}
+
+/*
+ * Gradients of sum(dout * out) for out = the prefill of every row (all T
+ * queries of each sequence), with respect to every input.
+ *   q [B, T, Hq, D]; k, v, zk, zv [B, T, G, D] (v, zv NULL in the shared form);
+ *   bpk, bpv [m, G*D]; sink [Hq] or NULL; gq, gkv [D] or NULL; dout [B, T, Hq, D].
+ * Outputs (zeroed here; any may be NULL except dq): dq, dk, dv, dzk, dzv like
+ * their inputs, dbk, dbv [m, G*D], dsink [Hq].  Gains are not differentiated.
+ */
+int orc_prefill_backward(const orc_config* c, int B, long T, const double* q, const double* k, const double* v,
+                         const double* zk, const double* zv, const double* bpk, const double* bpv,
+                         const double* sink, const double* gq, const double* gkv, const double* dout,
+                         double* dq, double* dk, double* dv, double* dzk, double* dzv, double* dbk,
+                         double* dbv, double* dsink)
+{
+    if (!cfg_ok(c) || B < 0 || T < 0 || !q || !k || !zk || !bpk || !dout || !dq) return -1;
+    if (!c->shared_kv && (!v || !zv || !bpv)) return -1;
+    const int Hq = c->n_q_heads, G = c->n_kv_heads, D = c->head_dim, m = c->block_m, w = c->n_win;
+    const int r = Hq / G, S = c->shared_kv ? 1 : 2;
+    const long NB = T / m, ts = (long)G * D;
+    const double scale = c->softmax_scale > 0 ? c->softmax_scale : 1.0 / sqrt((double)D);
+    const long nx = (long)B * T * ts;
+    memset(dq, 0, sizeof(double) * (size_t)B * T * Hq * D);
+    double* dX[2] = {dk, dv};
+    double* dZ[2] = {dzk, dzv};
+    double* dBp[2] = {dbk, dbv};
+    /* scratch: the pooled and finalised entries, their gradients, the raw
+       finalised keys and their gradients, the pooling weights */
+    double* P = calloc((size_t)S * B * NB * ts + 1, sizeof(double));    /* pooled, before finalisation */
+    double* E = calloc((size_t)S * B * NB * ts + 1, sizeof(double));    /* keys finalised; values as pooled */
+    double* dE = calloc((size_t)S * B * NB * ts + 1, sizeof(double));
+    double* Kf = calloc((size_t)nx + 1, sizeof(double));                /* raw keys finalised */
+    double* dKf = calloc((size_t)nx + 1, sizeof(double));
+    double* dVr = calloc((size_t)nx + 1, sizeof(double));               /* raw values (GQA) */
+    double* Wt = calloc((size_t)S * B * NB * m * ts + 1, sizeof(double)); /* pooling weights [S][B][NB][m][G][D] */
+    double* gX = calloc((size_t)S * nx + 1, sizeof(double));            /* d raw x of each series */
+    double* gZ = calloc((size_t)S * nx + 1, sizeof(double));
+    double* gB = calloc((size_t)S * m * ts + 1, sizeof(double));
+    double* ds = calloc((size_t)Hq + 1, sizeof(double));
+    double* qt = malloc(sizeof(double) * D);
+    double* dqt = malloc(sizeof(double) * D);
+    double* dof = malloc(sizeof(double) * D);
+    double* o = malloc(sizeof(double) * D);
+    double* sc = malloc(sizeof(double) * (size_t)(NB + T + 1));
+    double* tmp = malloc(sizeof(double) * D);
+    if (!P || !E || !dE || !Kf || !dKf || !dVr || !Wt || !gX || !gZ || !gB || !ds || !qt || !dqt || !dof || !o ||
+        !sc || !tmp) {
+        free(P); free(E); free(dE); free(Kf); free(dKf); free(dVr); free(Wt); free(gX); free(gZ); free(gB);
+        free(ds); free(qt); free(dqt); free(dof); free(o); free(sc); free(tmp);
+        return -1;
+    }
+    /* ---- forward: pooling weights, pooled and finalised entries, finalised raw keys ---- */
+    for (int sr = 0; sr < S; ++sr) {
+        const double* x = sr ? v : k;
+        const double* z = sr ? zv : zk;
+        const double* bp = sr ? bpv : bpk;
+        for (int b = 0; b < B; ++b)
+            for (long j = 0; j < NB; ++j)
+                for (int g = 0; g < G; ++g)
+                    for (int ch = 0; ch < D; ++ch) {
+                        const long col = (long)g * D + ch;
+                        double amax = -INFINITY;
+                        for (int i = 0; i < m; ++i) {
+                            double a = z[(b * T + j * m + i) * ts + col] + bp[i * ts + col];
+                            if (a > amax) amax = a;
+                        }
+                        double den = 0.0, num = 0.0;
+                        for (int i = 0; i < m; ++i)
+                            den += exp(z[(b * T + j * m + i) * ts + col] + bp[i * ts + col] - amax);
+                        for (int i = 0; i < m; ++i) {
+                            double wi = exp(z[(b * T + j * m + i) * ts + col] + bp[i * ts + col] - amax) / den;
+                            Wt[((((long)sr * B + b) * NB + j) * m + i) * ts + col] = wi;
+                            num += wi * x[(b * T + j * m + i) * ts + col];
+                        }
+                        P[(((long)sr * B + b) * NB + j) * ts + col] = num;
+                    }
+        for (int b = 0; b < B; ++b)
+            for (long j = 0; j < NB; ++j)
+                for (int g = 0; g < G; ++g) {
+                    const long o_ = (((long)sr * B + b) * NB + j) * ts + (long)g * D;
+                    memcpy(E + o_, P + o_, sizeof(double) * D);
+                    if (sr == 0) finalise_key(c, E + o_, gkv, (double)(j * m));
+                }
+    }
+    for (long idx = 0; idx < (long)B * T * G; ++idx) {
+        memcpy(Kf + idx * D, k + idx * D, sizeof(double) * D);
+        finalise_key(c, Kf + idx * D, gkv, (double)((idx / G) % T));
+    }
+    /* ---- attention backward, row by row ---- */
+    for (int b = 0; b < B; ++b)
+        for (long t = 0; t < T; ++t)
+            for (int h = 0; h < Hq; ++h) {
+                const int g = h / r;
+                const long L = t + 1, Pv = orc_visible_blocks(L, m, w), s0 = Pv * m;
+                const long n = Pv + (t - s0 + 1);
+                memcpy(qt, q + ((b * T + t) * Hq + h) * (long)D, sizeof(double) * D);
+                if (c->rmsnorm) rmsnorm(qt, D, gq, c->rms_eps);
+                if (c->rope_dims) rope(qt, D, c->rope_dims, c->rope_theta, (double)t);
+                /* keys and values of the visible list, entry e */
+#define KEY(e) ((e) < Pv ? E + (((long)0 * B + b) * NB + (e)) * ts + (long)g * D \
+                         : Kf + (b * T + s0 + ((e) - Pv)) * ts + (long)g * D)
+#define VAL(e) (c->shared_kv ? KEY(e) : ((e) < Pv ? E + (((long)1 * B + b) * NB + (e)) * ts + (long)g * D \
+                                                  : v + (b * T + s0 + ((e) - Pv)) * ts + (long)g * D))
+                double smax = sink ? sink[h] : -INFINITY;
+                for (long e = 0; e < n; ++e) {
+                    const double* kk = KEY(e);
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += qt[d] * kk[d];
+                    sc[e] = acc * scale;
+                    if (sc[e] > smax) smax = sc[e];
+                }
+                double den = sink ? exp(sink[h] - smax) : 0.0;
+                for (long e = 0; e < n; ++e) {
+                    sc[e] = exp(sc[e] - smax);
+                    den += sc[e];
+                }
+                for (long e = 0; e < n; ++e) sc[e] /= den;                     /* p_e */
+                const double psink = sink ? exp(sink[h] - smax) / den : 0.0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (long e = 0; e < n; ++e) {
+                    const double* vv = VAL(e);
+                    for (int d = 0; d < D; ++d) o[d] += sc[e] * vv[d];
+                }
+                /* d of o: the output of the shared form was turned back by -t */
+                memcpy(dof, dout + ((b * T + t) * Hq + h) * (long)D, sizeof(double) * D);
+                if (c->shared_kv && c->rope_dims) rope(dof, D, c->rope_dims, c->rope_theta, (double)t);
+                double Dsum = 0.0;
+                for (int d = 0; d < D; ++d) Dsum += dof[d] * o[d];
+                for (int d = 0; d < D; ++d) dqt[d] = 0.0;
+                for (long e = 0; e < n; ++e) {
+                    const double* kk = KEY(e);
+                    const double* vv = VAL(e);
+                    double dp = 0.0;
+                    for (int d = 0; d < D; ++d) dp += dof[d] * vv[d];
+                    const double dS = sc[e] * (dp - Dsum);
+                    double* dkey = e < Pv ? dE + (((long)0 * B + b) * NB + e) * ts + (long)g * D
+                                          : dKf + (b * T + s0 + (e - Pv)) * ts + (long)g * D;
+                    double* dval = c->shared_kv ? dkey
+                                                : (e < Pv ? dE + (((long)1 * B + b) * NB + e) * ts + (long)g * D
+                                                          : dVr + (b * T + s0 + (e - Pv)) * ts + (long)g * D);
+                    for (int d = 0; d < D; ++d) {
+                        dqt[d] += scale * dS * kk[d];
+                        dkey[d] += scale * dS * qt[d];
+                        dval[d] += sc[e] * dof[d];
+                    }
+                }
+#undef KEY
+#undef VAL
+                ds[h] += -psink * Dsum;
+                /* back through the query's RoPE at t and RMSNorm */
+                double* dqo = dq + ((b * T + t) * Hq + h) * (long)D;
+                const double* qraw = q + ((b * T + t) * Hq + h) * (long)D;
+                if (c->rope_dims) rope(dqt, D, c->rope_dims, c->rope_theta, -(double)t);
+                if (c->rmsnorm) rmsnorm_bwd(qraw, dqt, D, gq, c->rms_eps, dqo);
+                else memcpy(dqo, dqt, sizeof(double) * D);
+            }
+    /* ---- raw keys and values: their own gradient, through the key finalisation ---- */
+    for (long idx = 0; idx < (long)B * T * G; ++idx) {
+        finalise_key_bwd(c, k + idx * D, dKf + idx * D, gkv, (double)((idx / G) % T), tmp);
+        for (int d = 0; d < D; ++d) gX[idx * D + d] = tmp[d];
+        if (!c->shared_kv)
+            for (int d = 0; d < D; ++d) gX[nx + idx * D + d] = dVr[idx * D + d];
+    }
+    /* ---- pooled entries: through the finalisation, then the pooling softmax ---- */
+    for (int sr = 0; sr < S; ++sr) {
+        const double* x = sr ? v : k;
+        for (int b = 0; b < B; ++b)
+            for (long j = 0; j < NB; ++j)
+                for (int g = 0; g < G; ++g) {
+                    const long o_ = (((long)sr * B + b) * NB + j) * ts + (long)g * D;
+                    if (sr == 0) finalise_key_bwd(c, P + o_, dE + o_, gkv, (double)(j * m), tmp);
+                    else memcpy(tmp, dE + o_, sizeof(double) * D);
+                    for (int ch = 0; ch < D; ++ch) {
+                        const long col = (long)g * D + ch;
+                        const double dPc = tmp[ch], Pc = P[o_ + ch];
+                        for (int i = 0; i < m; ++i) {
+                            const long tok = (b * T + j * m + i) * ts + col;
+                            const double wi = Wt[((((long)sr * B + b) * NB + j) * m + i) * ts + col];
+                            const double da = wi * (x[tok] - Pc) * dPc;
+                            gX[(long)sr * nx + tok] += wi * dPc;
+                            gZ[(long)sr * nx + tok] += da;
+                            gB[((long)sr * m + i) * ts + col] += da;
+                        }
+                    }
+                }
+    }
+    for (int sr = 0; sr < S; ++sr) {
+        if (dX[sr]) memcpy(dX[sr], gX + (long)sr * nx, sizeof(double) * (size_t)nx);
+        if (dZ[sr]) memcpy(dZ[sr], gZ + (long)sr * nx, sizeof(double) * (size_t)nx);
+        if (dBp[sr]) memcpy(dBp[sr], gB + (long)sr * m * ts, sizeof(double) * (size_t)m * ts);
+    }
+    if (dsink) memcpy(dsink, ds, sizeof(double) * Hq);
+    free(P); free(E); free(dE); free(Kf); free(dKf); free(dVr); free(Wt); free(gX); free(gZ); free(gB);
+    free(ds); free(qt); free(dqt); free(dof); free(o); free(sc); free(tmp);
+    return 0;
+}

@@ -29,6 +29,11 @@ Functions and the passages they follow:
                      plus the overlapping window of the last n_win raw tokens
                      and the sink (CSA page, "What is implemented", Eqs 18-19,
                      Eq 27, -i rotation).
+  * ``prefill_backward`` -- gradients of sum(dout * prefill output) with
+                     respect to the queries, raw keys and values, the pooling
+                     logits, the positional biases and the sink: reverse-mode
+                     differentiation of ``pool`` + ``attend`` ("mSeek" README,
+                     "Experiment at a glance": the LBCA layers are trained).
   * ``visible_blocks`` -- P(L) of the block-aligned visibility reading.
   * ``cache_entries`` / ``kv_cache_bytes`` -- analytic cache accounting
                      ("mSeek" README, "Results").
@@ -113,6 +118,8 @@ def _load():
         lib.orc_attend_sparse.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, dp, dp, ctypes.c_long, lp,
                                           ctypes.c_int, dp, ctypes.c_long, lp, dp, dp, dp, dp]
         lib.orc_attend_sparse.restype = ctypes.c_int
+        lib.orc_prefill_backward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_long] + [dp] * 19
+        lib.orc_prefill_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -362,6 +369,34 @@ def attend_sparse(cfg: Config, q, ek, sel, k, lens, sink=None, gamma_q=None, gam
                                    out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc:
         raise ValueError("orc_attend_sparse rejected its arguments")
+    return out
+
+
+def prefill_backward(cfg: Config, q, k, v, zk, zv, bpos_k, bpos_v, dout, sink=None, gamma_q=None, gamma_kv=None):
+    """Gradients of sum(dout * forward(...)) over every row: a dict with dq,
+    dk, dzk, dbk, dsink and (GQA) dv, dzv, dbv, fp64 in the inputs' shapes."""
+    q, qp = _d(q)
+    k, kp = _d(k)
+    v, vp = _d(v)
+    zk, zkp = _d(zk)
+    zv, zvp = _d(zv)
+    bpos_k, bkp = _d(bpos_k)
+    bpos_v, bvp = _d(bpos_v)
+    dout, dop = _d(dout)
+    sink, sp = _d(sink)
+    gamma_q, gqp = _d(gamma_q)
+    gamma_kv, gkp = _d(gamma_kv)
+    B, T = q.shape[:2]
+    out = {"dq": np.zeros(q.shape), "dk": np.zeros(k.shape), "dzk": np.zeros(k.shape),
+           "dbk": np.zeros(bpos_k.shape), "dsink": np.zeros(cfg.n_q_heads)}
+    if not cfg.shared_kv:
+        out.update(dv=np.zeros(k.shape), dzv=np.zeros(k.shape), dbv=np.zeros(bpos_k.shape))
+    ptr = lambda name: out[name].ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if name in out else None  # noqa
+    rc = _load().orc_prefill_backward(ctypes.byref(cfg.c()), B, T, qp, kp, vp, zkp, zvp, bkp, bvp, sp, gqp, gkp,
+                                      dop, ptr("dq"), ptr("dk"), ptr("dv"), ptr("dzk"), ptr("dzv"), ptr("dbk"),
+                                      ptr("dbv"), ptr("dsink"))
+    if rc:
+        raise ValueError("orc_prefill_backward rejected its arguments")
     return out
 
 

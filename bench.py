@@ -529,6 +529,8 @@ def prefill_leg(name="gqa_prefill_16k", reps=10, warm=3, baseline=True):
 
 
 POOL_CASES = {
+    "csa_sparse_decode_64k (4 x 65536 tokens, D = 512, m = 4, dual overlapped a/b series: RMSNorm and RoPE "
+    "epilogue)": ("csa_sparse_decode_64k", 65536, 4, (0,)),
     # name: (workload, tokens, batch, series)
     "gqa_decode_32k prefix (32768 tokens, K and V series)": ("gqa_decode_32k", 32768, 1, (0, 1)),
     "gqa_prefill_16k (16384 tokens, m = 16, K and V series)": ("gqa_prefill_16k", 16384, 1, (0, 1)),
@@ -545,7 +547,8 @@ def pool_leg(label, reps=10, warm=3, baseline=True):
     from block_compressed_long_b200 import lbca as L
     from block_compressed_long_b200 import synth
     name, T, B, series = POOL_CASES[label]
-    w = synth.scaled(synth.WORKLOADS[name], kind="prefill", seq_len=T, batch=B, steps=1)
+    # the raw series of T tokens per sequence (no queries are drawn: steps = 0)
+    w = synth.scaled(synth.WORKLOADS[name], kind="decode", ctx=(T, T), seq_len=T, batch=B, steps=0, index_heads=0)
     inp = synth.make(w)
     cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
                    w.rmsnorm, w.rope_theta, dtype=w.dtype)
@@ -554,26 +557,322 @@ def pool_leg(label, reps=10, warm=3, baseline=True):
     nb = T // w.block_m
     outs = [torch.empty(B, w.n_kv_heads, nb, w.head_dim, dtype=L.torch_dtype(cfg), device="cuda") for _ in srcs]
 
+    dual = w.dual
+    if dual:  # the b-series of the dual overlapped form
+        xb, zb, bpb = d(inp.csa["kb"]), d(inp.csa["zkb"]), d(inp.csa["bpos_kb"])
+
     def run():
         for s, (x, z, bp) in zip(series, srcs):
-            L.lbca_pool(cfg, s, x, z, bp, None, outs[s])
+            if dual:
+                L.lbca_pool_dual(cfg, s, x, z, xb, zb, bp, bpb, None, outs[s])
+            else:
+                L.lbca_pool(cfg, s, x, z, bp, None, outs[s])
 
     uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
     ms, clocks = timed(run, reps, warm, uuid)
     esz = 2 if w.dtype == "bf16" else 4
-    nbytes = sum(2 * x.numel() * esz + o.numel() * esz for (x, _, _), o in zip(srcs, outs))
+    nbytes = sum((4 if dual else 2) * x.numel() * esz + o.numel() * esz for (x, _, _), o in zip(srcs, outs))
     gbs = nbytes / (ms * 1e-3) / 1e9
     hbm, src = peaks()
     line = {"workload": label, "metric": "pool GB/s", "value": gbs, "unit": "GB/s", "ms_per_call": ms,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "peak_source": src, "kernel": "pool_kernel", "bytes_per_call": nbytes,
+                         "peak_source": src, "kernel": "pool_kernel" + (" (dual overlapped form)" if dual else ""),
+                         "bytes_per_call": nbytes,
                          "launches_per_call": len(srcs)},
             "clocks": clocks}
     del srcs, outs
+    if dual:
+        del xb, zb, bpb
     torch.cuda.empty_cache()
     if baseline:
         line["cpu_baseline"] = oracle_pool_timing(w, inp, series)
     return line
+
+
+def layer_chain_leg(NL=14, K=20, W=3, reps=3):
+    """One token through NL LBCA layers of the 32K GQA shape (the README's
+    retrofit replaces 14 of the 3B model's 28 layers): layer l's query is layer
+    l-1's output, so the steps form a true dependency chain, each layer with
+    its own cache, K tokens back to back from one CUDA graph.  Timed twice:
+    with the caches flagged LBCA_CACHE_OVERLAP_PREV (each layer's step starts
+    and reads its cache while the previous layer's kernel drains; programmatic
+    dependent launch) and without.  Chains rotate over replicas holding more
+    than 3x the L2 of cache, so every step reads cold data."""
+    import gc
+
+    import torch
+
+    from block_compressed_long_b200 import lbca as L
+    from block_compressed_long_b200 import synth
+    w = synth.WORKLOADS["gqa_decode_32k"]
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    lens0 = synth.contexts(w)
+    per_layer = bytes_per_decode(w, lens0 + 1)
+    NR = max(1, -(-3 * l2 // (per_layer * NL)))
+    total_steps = W + 2 * reps * K + W
+    local = -(-total_steps // NR) + 1
+    ws_ = synth.scaled(w, steps=local)
+    inp = synth.make(ws_)
+    cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta, dtype=w.dtype)
+    max_ctx = int(inp.lens.max()) + local
+    c0 = L.Cache.allocate(cfg, 1, max_ctx)
+    d = lambda t: None if t is None else t.cuda()  # noqa: E731
+    n0 = int(inp.lens[0])
+    L.lbca_prefill(cfg, None, d(inp.k[:, :n0]), d(inp.v[:, :n0]), d(inp.zk[:, :n0]), d(inp.zv[:, :n0]),
+                   d(inp.bpos_k), d(inp.bpos_v), None, None, None, None, c0,
+                   torch.zeros(16, dtype=torch.uint8, device="cuda"), batch=1, T=n0)
+    cl = lambda t: None if t is None else t.clone()  # noqa: E731
+    chains = [[L.Cache(cfg, 1, c0.max_blocks, c0.ring_slots, cl(c0.pooled_k), cl(c0.pooled_v), cl(c0.ring_k),
+                       cl(c0.ring_v), cl(c0.pool_state), cl(c0.seq_lens)) for _ in range(NL)] for _ in range(NR)]
+    del c0
+    wsb = max(L.lbca_decode_step_workspace_bytes(cfg, 1, max_ctx), 16)
+    wss = [[torch.zeros(wsb, dtype=torch.uint8, device="cuda") for _ in range(NL)] for _ in range(NR)]
+    outs = [[torch.empty(1, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda") for _ in range(NL)]
+            for _ in range(NR)]
+    tok = [d(t[:, n0:n0 + local].transpose(0, 1).contiguous()) for t in (inp.k, inp.v, inp.zk, inp.zv)]
+    q0 = d(inp.q[:, 0].contiguous())
+    bpk, bpv = d(inp.bpos_k), d(inp.bpos_v)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    launches = L.lbca_decode_step_launches(cfg, 1, max_ctx)
+
+    def token(i, flags):
+        r, j = i % NR, (i // NR) % local
+        q = q0[j]
+        for layer in range(NL):
+            c = chains[r][layer]
+            c.flags = flags
+            L.lbca_decode_step(cfg, tok[0][j], tok[1][j], tok[2][j], tok[3][j], bpk, bpv, None, q, c, None, None,
+                               outs[r][layer], wss[r][layer], max_ctx, status)
+            q = outs[r][layer]  # the next layer attends with this layer's output
+
+    i = 0
+    for _ in range(W):
+        token(i, 0)
+        i += 1
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    res = {}
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    for name, flags in (("overlap", L.LBCA_CACHE_OVERLAP_PREV), ("serial", 0)):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap):
+            for ii in range(i, i + K):
+                token(ii, flags)
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) / K)
+        i += K
+        res[name] = statistics.median(ts)
+        del gr
+    clocks = sampler.stop()
+    st = int(status.item())
+    if st:
+        raise RuntimeError(f"layer chain device status {L.lbca_status_string(st)}")
+    ms = res["overlap"]
+    hbm, src = peaks()
+    nbytes = NL * per_layer
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del chains, wss, outs, tok
+    gc.collect()
+    torch.cuda.empty_cache()
+    return {"workload": f"layer chain: {NL} LBCA layers of gqa_decode_32k, one token, each layer's query the "
+                        "previous layer's output", "metric": "decode µs/token (all layers)", "value": ms * 1e3,
+            "unit": "µs/token", "serial_us_per_token": res["serial"] * 1e3, "per_layer_us": ms * 1e3 / NL,
+            "config": {"layers": NL, "launches_per_layer": launches,
+                       "l2": f"chains rotate over {NR} replicas of {NL} caches (>= 3x L2), each step's data cold",
+                       "launch": (f"{K} tokens x {NL} lbca_decode_step calls back to back from one CUDA graph, "
+                                  f"median of {reps}; caches flagged LBCA_CACHE_OVERLAP_PREV (programmatic "
+                                  "dependent launch); serial_us_per_token: the same graph without the flag")},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_source": src, "bytes_per_token": nbytes,
+                         "kernel": "decode_step_kernel (cluster form) x layers"},
+            "gpu_launches": K * NL * launches, "clocks": clocks}
+
+
+class CsaBench:
+    """The CSA workload's decode state on one GPU, built through the C ABI:
+    dual-pooled finalised entries, dual-pooled indexer keys, the raw window
+    and the lengths, cloned into NR replicas that together hold more than 3x
+    the L2 so that every step reads cold data.  A step, for every sequence:
+    lightning-indexer relevance and top-k (lbca_indexer_topk), then the
+    sparse attention over the selected entries and the window
+    (lbca_decode_sparse); the cache is not advanced (no append)."""
+
+    def __init__(self, w, steps):
+        import torch
+
+        from block_compressed_long_b200 import lbca as L
+        from block_compressed_long_b200 import synth
+        self.L, self.w = L, w
+        ws = synth.scaled(w, steps=steps)
+        inp = synth.make(ws)
+        self.inp = inp
+        B = w.batch
+        self.cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                            w.rmsnorm, w.rope_theta, dtype=w.dtype)
+        icfg = L.config(1, 1, w.index_dim, True, w.block_m, w.n_win, 0, False, dtype=w.dtype)
+        lens = np.asarray(inp.lens, dtype=np.int64)
+        c0 = L.Cache.allocate(self.cfg, B, int(lens.max()) + 1)
+        nb = c0.max_blocks
+        kidx = torch.zeros(B, 1, nb, w.index_dim, dtype=torch.bfloat16, device="cuda")
+        c = inp.csa
+        d = lambda t: t.contiguous().cuda()  # noqa: E731
+        for b in range(B):
+            n = int(lens[b])
+            sl = lambda t: d(t[b:b + 1, :n])  # noqa: E731
+            L.lbca_pool_dual(self.cfg, L.LBCA_KEY, sl(inp.k), sl(inp.zk), sl(c["kb"]), sl(c["zkb"]), d(inp.bpos_k),
+                             d(c["bpos_kb"]), None, c0.pooled_k[b:b + 1], nb)
+            L.lbca_pool_dual(icfg, L.LBCA_VALUE, sl(c["ika"]), sl(c["izka"]), sl(c["ikb"]), sl(c["izkb"]),
+                             d(c["ibpa"]), d(c["ibpb"]), None, kidx[b:b + 1], nb)
+            R = c0.ring_slots
+            rows = torch.arange(max(0, n - R), n)
+            c0.ring_k[b, 0, rows % R] = inp.k[b, rows, 0].cuda()
+        c0.seq_lens.copy_(torch.as_tensor(lens, dtype=torch.int32))
+        kidx = kidx[:, 0].contiguous()
+        torch.cuda.synchronize()
+        self.nvis = np.minimum(lens // w.block_m, nb)
+        self.step_bytes = self.bytes_per_step()
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        self.NR = max(1, -(-3 * l2 // self.step_bytes))
+        cl = lambda t: None if t is None else t.clone()  # noqa: E731
+        self.caches = [c0] + [L.Cache(self.cfg, B, nb, c0.ring_slots, cl(c0.pooled_k), None, cl(c0.ring_k), None,
+                                      cl(c0.pool_state), cl(c0.seq_lens)) for _ in range(self.NR - 1)]
+        self.kidx = [kidx] + [kidx.clone() for _ in range(self.NR - 1)]
+        self.iq = c["iq"].cuda()
+        self.iw = c["iw"].cuda()
+        self.q = inp.q.cuda()
+        self.sink = inp.sink.cuda()
+        self.sel = [torch.empty(B, w.top_k, dtype=torch.int32, device="cuda") for _ in range(self.NR)]
+        self.outs = [torch.empty(B, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+                     for _ in range(self.NR)]
+        self.ws = torch.zeros(L.lbca_indexer_workspace_bytes(B, nb), dtype=torch.uint8, device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.steps = steps
+
+    def bytes_per_step(self):
+        """Algorithmic HBM bytes of one step: the visible indexer keys, the
+        indexer queries and weights, the selected entries and the window rows,
+        the queries and the outputs, each once."""
+        w = self.w
+        nsel = np.minimum(self.nvis, w.top_k)
+        nwin = np.minimum(np.asarray(self.inp.lens), w.n_win)
+        b = int(self.nvis.sum()) * w.index_dim * 2 + w.batch * w.index_heads * (w.index_dim * 2 + 4)
+        b += int((nsel + nwin).sum()) * w.head_dim * 2 + 2 * w.batch * w.n_q_heads * w.head_dim * 2
+        return b
+
+    def flops_per_step(self):
+        w = self.w
+        nsel = np.minimum(self.nvis, w.top_k)
+        nwin = np.minimum(np.asarray(self.inp.lens), w.n_win)
+        return (2.0 * int(self.nvis.sum()) * w.index_heads * w.index_dim +
+                4.0 * int((nsel + nwin).sum()) * w.n_q_heads * w.head_dim)
+
+    def launch(self, i):
+        L, rep, j = self.L, i % self.NR, (i // self.NR) % self.steps
+        L.lbca_indexer_topk(self.iq[j], self.iw[j], self.kidx[rep], self.caches[rep].seq_lens, self.w.block_m,
+                            self.sel[rep], None, self.ws, self.status)
+        L.lbca_decode_sparse(self.cfg, self.q[j], self.caches[rep], self.sel[rep], self.sink, None, None,
+                             self.outs[rep], self.status)
+
+
+def csa_leg(K=20, W=5, reps=3):
+    """The CSA sparse decode step (indexer relevance + top-k + sparse
+    attention) of the 4 x 64K workload, K steps replayed from one CUDA graph,
+    median of `reps` replays; the oracle on one sequence beside it."""
+    import gc
+
+    import torch
+
+    from block_compressed_long_b200 import synth
+    w = synth.WORKLOADS["csa_sparse_decode_64k"]
+    bench = CsaBench(w, steps=8)
+    for i in range(W):
+        bench.launch(i)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=cap):
+        for i in range(W, W + K):
+            bench.launch(i)
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / K)
+    clocks = sampler.stop()
+    st = int(bench.status.item())
+    if st:
+        raise RuntimeError(f"CSA step device status {bench.L.lbca_status_string(st)}")
+    ms = statistics.median(ts)
+    hbm, src = peaks()
+    gbs = bench.step_bytes / (ms * 1e-3) / 1e9
+    line = {"workload": w.name, "metric": METRIC, "value": ms * 1e3 / w.batch, "unit": "µs/token",
+            "ms_per_step": ms, "dtype": "bf16 I/O; indexer bf16 tensor-core products, f32 accumulate; "
+                                        "attention fp16 tensor-core operands",
+            "config": {"batch": w.batch, "context": w.ctx[0], "block_m": w.block_m, "n_win": w.n_win,
+                       "n_q_heads": w.n_q_heads, "head_dim": w.head_dim, "index_heads": w.index_heads,
+                       "index_dim": w.index_dim, "top_k": w.top_k,
+                       "l2": f"steps rotate over {bench.NR} cache replicas (>= 3x L2), each step's data cold",
+                       "launch": f"{K} steps (3 kernels each) back to back from one CUDA graph, median of {reps}"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_source": src, "bytes_per_step": bench.step_bytes,
+                         "flops_per_step": bench.flops_per_step(),
+                         "kernel": "indexer_score_kernel + topk_kernel + decode_mqa_tc_kernel (whole step timed)"},
+            "gpu_launches": 3 * K, "clocks": clocks}
+    inp = bench.inp
+    del bench, gr
+    gc.collect()
+    torch.cuda.empty_cache()
+    line["cpu_baseline"] = oracle_csa_timing(w, inp)
+    return line
+
+
+def oracle_csa_timing(w, inp):
+    """The fp64 oracle's CSA decode step for the first sequence (indexer
+    relevance over its complete blocks, top-k, sparse attention), the
+    sequence's pooled entries and indexer keys computed beforehand (untimed,
+    as the GPU leg's cache is built beforehand)."""
+    from block_compressed_long_b200 import synth
+    from oracle import oracle as orc
+    f64 = synth.f64
+    c = inp.csa
+    n = int(inp.lens[0])
+    oc = orc.Config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                    w.rmsnorm, w.rope_theta)
+    ic = orc.Config(1, 1, w.index_dim, True, w.block_m, w.n_win)
+    ek = orc.pool_dual(oc, orc.KEY, f64(inp.k[:1, :n]), f64(inp.zk[:1, :n]), f64(c["kb"][:1, :n]),
+                       f64(c["zkb"][:1, :n]), f64(inp.bpos_k), f64(c["bpos_kb"]))
+    kx = orc.pool_dual(ic, orc.VALUE, *(f64(c[t][:1, :n]) for t in ("ika", "izka", "ikb", "izkb")),
+                       f64(c["ibpa"]), f64(c["ibpb"]))[:, :, 0]
+    hist = f64(inp.k[:1, :n])
+    per = []
+    for j in range(3):
+        t0 = time.perf_counter()
+        sc = orc.indexer_scores(f64(c["iq"][j, :1]), f64(c["iw"][j, :1]), kx, [kx.shape[1]])
+        sel = orc.topk_blocks(sc, [kx.shape[1]], w.top_k)
+        orc.attend_sparse(oc, f64(inp.q[j, :1]), ek, sel, hist, [n], f64(inp.sink))
+        per.append(time.perf_counter() - t0)
+    med = statistics.median(per)
+    return {"value": med * 1e6, "unit": "µs/token", "cores": _cores(), "kind": "oracle",
+            "sample": f"3 decode steps of sequence 0 of {w.name} (context {n}), fp64 C oracle; median step"}
 
 
 def load_traffic(workload):
@@ -684,12 +983,17 @@ def oracle_pool_timing(w, inp, series, max_tokens=8192):
     n = min(w.seq_len, max_tokens) // w.block_m * w.block_m
     srcs = [(orc.KEY, inp.k, inp.zk, inp.bpos_k)] + ([] if w.shared_kv else [(orc.VALUE, inp.v, inp.zv, inp.bpos_v)])
     xs = [(s, f64(x[:, :n]), f64(z[:, :n]), f64(bp)) for s, x, z, bp in srcs]
+    if w.dual:
+        xb, zb, bpb = f64(inp.csa["kb"][:, :n]), f64(inp.csa["zkb"][:, :n]), f64(inp.csa["bpos_kb"])
     t0 = time.perf_counter()
     for s, x, z, bp in xs:
-        orc.pool(c, s, x, z, bp)
+        if w.dual:
+            orc.pool_dual(c, s, x, z, xb, zb, bp, bpb)
+        else:
+            orc.pool(c, s, x, z, bp)
     dt = time.perf_counter() - t0
     esz = 2 if w.dtype == "bf16" else 4
-    nbytes = len(xs) * w.batch * n * w.n_kv_heads * w.head_dim * esz * (2 + 1.0 / w.block_m)
+    nbytes = len(xs) * w.batch * n * w.n_kv_heads * w.head_dim * esz * ((4 if w.dual else 2) + 1.0 / w.block_m)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": _cores(), "kind": "oracle",
             "sample": (f"fp64 C oracle pooling the first {n} tokens of each of {w.batch} sequence(s), "
                        f"{len(xs)} series ({dt:.2f} s)")}
@@ -742,6 +1046,7 @@ def main():
         gc.collect()
         torch.cuda.empty_cache()
         also = [decode_also(args, n) for n in ("gqa_decode_32k", "hca_mqa_decode_128k") if n != w.name]
+        also += [layer_chain_leg(), csa_leg()]
         also += [prefill_leg("gqa_prefill_16k"), prefill_leg("tiny_f32_prefill")]
         also += [pool_leg(label) for label in POOL_CASES]
         line["also"] = also

@@ -75,7 +75,7 @@ lbca_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LBCA_OK : LBC
 
 lbca_status check_cache(const lbca_config* c, const lbca_cache* k) {
     if (!k) return LBCA_ERR_ARG;
-    if (k->batch < 0 || k->max_blocks < 0 || k->reserved != 0) return LBCA_ERR_ARG;
+    if (k->batch < 0 || k->max_blocks < 0 || (k->flags & ~LBCA_CACHE_OVERLAP_PREV) != 0) return LBCA_ERR_ARG;
     const int rmin = ring_min(c);
     if (rmin < 0 || k->ring_slots < rmin) return LBCA_ERR_CAPACITY;
     const bool pooled = k->max_blocks > 0;  // a cache with no block capacity needs no pooled arrays
@@ -200,13 +200,40 @@ lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, con
     LBCA_TRY(check_device());
     PoolArgs a{};
     a.dtype = cfg->dtype;
-    a.x = x; a.z = z; a.bpos = b_pos; a.gamma = gamma;
-    a.out = out; a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
+    a.nser = 1;
+    a.ser[0].x = x; a.ser[0].z = z; a.ser[0].bpos = b_pos; a.ser[0].gamma = gamma; a.ser[0].out = out;
+    a.ser[0].key = series == LBCA_KEY; a.ser[0].state_series = 0;
+    a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
     a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
     a.pos0 = pos0;
-    a.key = series == LBCA_KEY; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
+    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
     a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
-    a.state = nullptr; a.S = 1; a.series = 0;
+    a.state = nullptr; a.S = 1;
+    return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lbca_status lbca_pool_dual(const lbca_config* cfg, int32_t series, const void* xa, const void* za, const void* xb,
+                           const void* zb, const void* b_pos_a, const void* b_pos_b, const void* gamma, int32_t batch,
+                           int32_t T, void* out, int32_t out_blocks, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    if (series != LBCA_KEY && series != LBCA_VALUE) return LBCA_ERR_ARG;
+    if (!xa || !za || !xb || !zb || !b_pos_a || !b_pos_b || !out) return LBCA_ERR_ARG;
+    if (batch < 0 || T < 0 || out_blocks < 0 || T / cfg->block_m > out_blocks) return LBCA_ERR_ARG;
+    if (!al16(xa) || !al16(za) || !al16(xb) || !al16(zb) || !al16(b_pos_a) || !al16(b_pos_b) || !al16(out) ||
+        !al16n(gamma))
+        return LBCA_ERR_ALIGN;
+    LBCA_TRY(check_device());
+    PoolArgs a{};
+    a.dtype = cfg->dtype;
+    a.nser = 1;
+    a.dual = 1;
+    PoolSeries& sr = a.ser[0];
+    sr.x = xa; sr.z = za; sr.bpos = b_pos_a; sr.xb = xb; sr.zb = zb; sr.bposb = b_pos_b;
+    sr.gamma = gamma; sr.out = out; sr.key = series == LBCA_KEY;
+    a.out_blocks = out_blocks; a.blk_off = 0;
+    a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m; a.pos0 = 0;
+    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims; a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
+    a.S = 1;
     return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -306,6 +333,7 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
         a.ring_w = cache->ring_k; a.pooled_w = cache->pooled_k; a.state = cache->pool_state;
         a.lens_w = cache->seq_lens;
         a.tc_cs = tp.cs; a.chunk = tp.rows;
+        a.pdl = (cache->flags & LBCA_CACHE_OVERLAP_PREV) != 0;
         return cuda_status(launch_decode_mqa_tc(a, reinterpret_cast<cudaStream_t>(stream)));
     }
     StepPlan sp = plan_step(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim,
@@ -328,6 +356,7 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
     a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm; a.shared = cfg->shared_kv;
     a.max_blocks = cache->max_blocks; a.R = cache->ring_slots; a.S = cfg->shared_kv ? 1 : 2;
     a.CS = sp.CS; a.SE = sp.SE; a.heads_per_cta = sp.heads_per_cta;
+    a.pdl = (cache->flags & LBCA_CACHE_OVERLAP_PREV) != 0 && !sp.flat;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
     if (sp.flat) {
         for (int kk = 0; kk < cfg->rope_dims / 2 && kk < 128; ++kk) a.rope_f[kk] = rope_turns(kk, a.rope_step);  // workspace: [arrival counter][segment counters][partial max, sum][partial outputs]
@@ -399,28 +428,33 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
     // fp16 copies of the raw keys (rotated) and values as it streams them
     if (use_tc) LBCA_TRY(cuda_status(launch_prefill_tc_table(pa, tc_scratch, s)));
     const PrefillRawF16 raw16 = use_tc ? prefill_tc_raw_f16(pa, tc_scratch) : PrefillRawF16{nullptr, nullptr, nullptr};
-    for (int series = 0; series < (cfg->shared_kv ? 1 : 2); ++series) {
+    {   // both series (or the shared entries) in one launch
         PoolArgs a{};
         a.dtype = cfg->dtype;
-        a.x = series ? v : k; a.z = series ? zv : zk; a.bpos = series ? b_pos_v : b_pos_k;
-        a.gamma = series ? nullptr : gamma_kv;
-        a.out = series ? pv : pk; a.out_blocks = stride; a.blk_off = 0;
+        a.nser = cfg->shared_kv ? 1 : 2;
+        for (int series = 0; series < a.nser; ++series) {
+            PoolSeries& sr = a.ser[series];
+            sr.x = series ? v : k; sr.z = series ? zv : zk; sr.bpos = series ? b_pos_v : b_pos_k;
+            sr.gamma = series ? nullptr : gamma_kv;
+            sr.out = series ? pv : pk;
+            sr.key = series == 0; sr.state_series = series;
+            if (use_tc) {
+                // the tensor-core MMAs read dense fp16 copies of the pooled keys and values, [B, G, NB, D]
+                sr.out_f16 = tc_scratch + (series == 0
+                                               ? prefill_tc_pooled_f16_offset(batch, T, cfg->n_kv_heads, cfg->rope_dims)
+                                               : prefill_tc_pooled_v_f16_offset(batch, T, cfg->n_kv_heads,
+                                                                                cfg->rope_dims, m));
+                sr.raw_f16 = series == 0 ? raw16.keys : raw16.vals;
+            }
+        }
+        a.out_blocks = stride; a.blk_off = 0; a.out_f16_blocks = NB;
         a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = m; a.pos0 = 0;
-        a.key = series == 0; a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
+        a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
         a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
         a.state = cache_out ? cache_out->pool_state : nullptr;
-        a.S = cfg->shared_kv ? 1 : 2; a.series = series;
-        if (use_tc) {
-            // the tensor-core MMAs read dense fp16 copies of the pooled keys and values, [B, G, NB, D]
-            a.out_f16 = tc_scratch + (series == 0
-                                          ? prefill_tc_pooled_f16_offset(batch, T, cfg->n_kv_heads, cfg->rope_dims)
-                                          : prefill_tc_pooled_v_f16_offset(batch, T, cfg->n_kv_heads,
-                                                                           cfg->rope_dims, m));
-            a.out_f16_blocks = NB;
-            a.raw_f16 = series == 0 ? raw16.keys : raw16.vals;
-            a.tab = raw16.tab;
-            a.status = d_status;
-        }
+        a.S = cfg->shared_kv ? 1 : 2;
+        a.tab = use_tc ? raw16.tab : nullptr;
+        a.status = d_status;
         LBCA_TRY(cuda_status(launch_pool(a, s)));
     }
     // 2. the raw window and the lengths, so decode can continue from T
@@ -518,6 +552,100 @@ lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbc
     a.counters = reinterpret_cast<uint32_t*>(ws + ctr_off);
     a.n_split = p.n_split; a.chunk = p.chunk; a.heads_per_cta = p.heads_per_cta;
     return cuda_status(launch_decode(a, s));
+}
+
+lbca_status lbca_decode_sparse(const lbca_config* cfg, const void* q, const lbca_cache* cache, const int32_t* sel,
+                               int32_t top_k, const float* sink, const void* gamma_q, const void* gamma_kv, void* out,
+                               int32_t* d_status, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    LBCA_TRY(check_cache(cfg, cache));
+    if (!q || !out || !sel || top_k < 1) return LBCA_ERR_ARG;
+    if (!al16(q) || !al16(out) || !al16n(gamma_q) || !al16n(gamma_kv) || !al16n(sink)) return LBCA_ERR_ALIGN;
+    if (!cfg->shared_kv) return LBCA_ERR_UNSUPPORTED;
+    if (cache->ring_slots < cfg->n_win) return LBCA_ERR_CAPACITY;
+    const MqaTcPlan tc = plan_decode_mqa_tc_vis(cfg->dtype, cache->batch, cfg->n_q_heads, cfg->n_kv_heads,
+                                                cfg->head_dim, cfg->shared_kv, (long long)top_k + cfg->n_win);
+    if (tc.cs == 0) return cache->batch == 0 ? LBCA_OK : LBCA_ERR_UNSUPPORTED;
+    LBCA_TRY(check_device());
+    DecodeArgs a = decode_args(cfg, q, cache, sink, gamma_q, gamma_kv, out, d_status);
+    a.sel = sel; a.sel_k = top_k;
+    a.tc_cs = tc.cs; a.chunk = tc.rows;
+    return cuda_status(launch_decode_mqa_tc(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t lbca_prefill_backward_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t T) {
+    if (check_cfg(cfg) != LBCA_OK || batch < 0 || T < 0) return (size_t)-1;
+    return align256(backward_scratch_floats(cfg->shared_kv ? 1 : 2, batch, T, cfg->n_q_heads, cfg->n_kv_heads,
+                                            cfg->head_dim, cfg->block_m) * 4) + 256 * 10;
+}
+
+lbca_status lbca_prefill_backward(const lbca_config* cfg, const void* q, const void* k, const void* v, const void* zk,
+                                  const void* zv, const void* b_pos_k, const void* b_pos_v, const float* sink,
+                                  const void* gamma_q, const void* gamma_kv, const void* dout, int32_t batch, int32_t T, float* dq, float* dk, float* dv, float* dzk, float* dzv,
+                                  float* db_pos_k, float* db_pos_v, float* dsink, void* workspace,
+                                  size_t workspace_bytes, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    if (batch < 0 || T < 0) return LBCA_ERR_ARG;
+    const bool any = batch > 0 && T > 0;
+    LBCA_TRY(check_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v, any));
+    if (any && (!q || !dout || !dq || !dk || !dzk || !db_pos_k || !workspace)) return LBCA_ERR_ARG;
+    if (any && !cfg->shared_kv && (!dv || !dzv || !db_pos_v)) return LBCA_ERR_ARG;
+    if (any && sink && !dsink) return LBCA_ERR_ARG;
+    if (!al16n(q) || !al16n(dout) || !al16n(workspace) || !al16n(gamma_q) || !al16n(gamma_kv))
+        return LBCA_ERR_ALIGN;
+    if (!backward_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
+    if (workspace_bytes < lbca_prefill_backward_workspace_bytes(cfg, batch, T)) return LBCA_ERR_CAPACITY;
+    if (!any) return LBCA_OK;
+    LBCA_TRY(check_device());
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    BwdArgs a{};
+    a.dtype = cfg->dtype;
+    a.q = q; a.k = k; a.v = v; a.zk = zk; a.zv = zv; a.bpk = b_pos_k; a.bpv = b_pos_v; a.sink = sink;
+    a.gamma_q = gamma_q; a.gamma_kv = gamma_kv; a.dout = dout;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dzk = dzk; a.dzv = dzv; a.dbk = db_pos_k; a.dbv = db_pos_v; a.dsink = dsink;
+    a.B = batch; a.T = T; a.Hq = cfg->n_q_heads; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
+    a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm; a.shared = cfg->shared_kv;
+    a.S = cfg->shared_kv ? 1 : 2; a.NB = T / cfg->block_m;
+    a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
+    const size_t pooled = (size_t)a.S * batch * a.NB * a.G * a.D, raw = (size_t)batch * T * a.G * a.D;
+    const size_t rows = (size_t)batch * T * a.Hq;
+    float* f = static_cast<float*>(workspace);
+    auto take = [&](size_t n) { float* p = f; f += (n + 63) / 64 * 64; return p; };
+    a.Ef = take(pooled); a.dE = take(pooled); a.Pk = take((size_t)batch * a.NB * a.G * a.D);
+    a.Kf = take(raw); a.dKf = take(raw); a.vf = a.shared ? nullptr : take(raw);
+    a.qf = take(rows * a.D); a.dof = take(rows * a.D); a.lse = take(rows); a.dsum = take(rows);
+    // the gradients that are accumulated, or written for complete blocks only, start at zero
+    const size_t gd = (size_t)a.G * a.D;
+    if (cudaMemsetAsync(dzk, 0, raw * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(db_pos_k, 0, (size_t)a.m * gd * 4, s) != cudaSuccess)
+        return LBCA_ERR_CUDA;
+    if (!cfg->shared_kv && (cudaMemsetAsync(dzv, 0, raw * 4, s) != cudaSuccess ||
+                            cudaMemsetAsync(db_pos_v, 0, (size_t)a.m * gd * 4, s) != cudaSuccess))
+        return LBCA_ERR_CUDA;
+    if (sink && cudaMemsetAsync(dsink, 0, (size_t)a.Hq * 4, s) != cudaSuccess) return LBCA_ERR_CUDA;
+    return cuda_status(launch_backward(a, s));
+}
+
+size_t lbca_indexer_workspace_bytes(int32_t batch, int32_t max_blocks) {
+    if (batch < 0 || max_blocks < 0) return 0;
+    return align256((size_t)batch * max_blocks * 4);
+}
+
+lbca_status lbca_indexer_topk(int32_t batch, int32_t n_heads, int32_t head_dim, int32_t block_m, int32_t top_k,
+                              const void* q_idx, const float* w_idx, const void* k_idx, int32_t max_blocks,
+                              const int32_t* seq_lens, int32_t* sel, float* sel_scores, void* workspace,
+                              size_t workspace_bytes, int32_t* d_status, lbca_stream_t stream) {
+    if (batch < 0 || block_m < 1 || top_k < 1 || max_blocks < 0) return LBCA_ERR_ARG;
+    if (!q_idx || !w_idx || !k_idx || !seq_lens || !sel || !workspace) return LBCA_ERR_ARG;
+    if (!indexer_shape_ok(n_heads, head_dim)) return LBCA_ERR_UNSUPPORTED;
+    if (!al16(q_idx) || !al16(k_idx) || !al16(workspace)) return LBCA_ERR_ALIGN;
+    if (workspace_bytes < lbca_indexer_workspace_bytes(batch, max_blocks)) return LBCA_ERR_CAPACITY;
+    LBCA_TRY(check_device());
+    IndexerArgs a{};
+    a.q_idx = q_idx; a.w_idx = w_idx; a.k_idx = k_idx; a.seq_lens = seq_lens;
+    a.scores = static_cast<float*>(workspace); a.sel = sel; a.sel_scores = sel_scores; a.status = d_status;
+    a.B = batch; a.HI = n_heads; a.DI = head_dim; a.m = block_m; a.max_blocks = max_blocks; a.top_k = top_k;
+    return cuda_status(launch_indexer_topk(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* lbca_status_string(lbca_status status) {

@@ -141,6 +141,15 @@ __device__ __forceinline__ void rotate_pair(float& a, float& b, float2 cs) {
     b = __fmaf_rn(x, cs.y, __fmul_rn(y, cs.x));
 }
 
+// ---- programmatic dependent launch --------------------------------------------------
+// Launched with programmatic stream serialisation, a kernel may start while the
+// preceding kernel on its stream drains: work before griddep_wait() must not
+// read what that kernel writes.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- status -------------------------------------------------------------------------
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
     if (st) atomicCAS(st, 0, code);

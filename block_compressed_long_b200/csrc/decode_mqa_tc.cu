@@ -84,7 +84,7 @@ __host__ __device__ inline int owned_dims(int D, int CS) { return ((D + CS - 1) 
 // and CS CTAs per cluster.
 struct MqaLayout {
     uint32_t EREG, GS, SLICE;
-    uint32_t OFF_E, OFF_Q, OFF_P, OFF_MALL, OFF_LRECV, OFF_CS, OFF_RED, OFF_MH, OFF_LLOC, OFF_DEN, OFF_BAR;
+    uint32_t OFF_E, OFF_Q, OFF_P, OFF_MALL, OFF_LRECV, OFF_CS, OFF_TURN, OFF_RED, OFF_MH, OFF_LLOC, OFF_DEN, OFF_BAR;
     uint32_t TOTAL, SMEM;
     __host__ __device__ MqaLayout(int D, int C, int CS) {
         EREG = (uint32_t)C * 128u;                          // one 64-dim column region of E
@@ -99,7 +99,8 @@ struct MqaLayout {
         OFF_MALL = OFF_P + (uint32_t)C * 128u;              // [kMaxCS][NH] f32 pushed maxima
         OFF_LRECV = OFF_MALL + kMaxCS * NH * 4u;            // [kMaxCS][NH] f32 pushed sums
         OFF_CS = OFF_LRECV + kMaxCS * NH * 4u;              // [D/2] float2 cos/sin at t
-        OFF_RED = OFF_CS + (uint32_t)(D / 2) * 8u;          // [4][NH] warp partials
+        OFF_TURN = OFF_CS + (uint32_t)(D / 2) * 8u;         // [D/2] u64 fixed-point turns per position
+        OFF_RED = OFF_TURN + (uint32_t)(D / 2) * 8u;        // [4][NH] warp partials
         OFF_MH = OFF_RED + 4u * NH * 4u;                    // [NH] reference max
         OFF_LLOC = OFF_MH + NH * 4u;                        // [NH] this CTA's sums
         OFF_DEN = OFF_LLOC + NH * 4u;                       // [NH] denominators
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.OFF_BAR);  // S done, O done, Q in, slices in
     uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(smem + lay.OFF_BAR + 32);
     float2* cs = reinterpret_cast<float2*>(smem + lay.OFF_CS);
+    uint64_t* turns = reinterpret_cast<uint64_t*>(smem + lay.OFF_TURN);
     float* red = reinterpret_cast<float*>(smem + lay.OFF_RED);
     float* mh = reinterpret_cast<float*>(smem + lay.OFF_MH);
     float* lloc = reinterpret_cast<float*>(smem + lay.OFF_LLOC);
@@ -348,12 +350,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     const int pos = a.seq_lens[b];  // cached tokens (fused: the new token's position)
     const int L = fuse ? pos + 1 : pos;
     const int t = L - 1;
-    const int P = visible_blocks(L, a.m, a.w);
-    const int s0 = P * a.m;
-    int n_vis = L > 0 ? P + (L - s0) : 0;
-    if (P > a.max_blocks || L - s0 > a.R || n_vis > C * CS) {  // cache or split grid cannot hold it
-        if (rank == 0 && g == 0 && tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
-        n_vis = 0;
+    // the visible list: P pooled entries, then the raw window tokens [s0, t]
+    // (block-aligned partition); with a selection (CSA form) the selected
+    // entries, then the window of the last n_win tokens, which may cover
+    // tokens a selected entry also summarises
+    int P, s0, n_vis;
+    if (a.sel) {
+        P = L > 0 ? min(a.sel_k, min(L / a.m, a.max_blocks)) : 0;
+        const int nw = min(L, a.w);
+        s0 = L - nw;
+        n_vis = L > 0 ? P + nw : 0;
+        if (nw > a.R || n_vis > C * CS) {
+            if (rank == 0 && g == 0 && tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
+            n_vis = 0;
+        }
+    } else {
+        P = visible_blocks(L, a.m, a.w);
+        s0 = P * a.m;
+        n_vis = L > 0 ? P + (L - s0) : 0;
+        if (P > a.max_blocks || L - s0 > a.R || n_vis > C * CS) {  // cache or split grid cannot hold it
+            if (rank == 0 && g == 0 && tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
+            n_vis = 0;
+        }
     }
     const bool single = n_vis <= C;  // one CTA takes the whole list: no exchange (uniform per cluster)
     const int chunk = single ? n_vis : (n_vis + CS - 1) / CS;
@@ -398,8 +416,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
         uint32_t bytes = 0;
         if (row < n) {
             const int idx = e0 + row;
-            src = idx < P ? pk + (pool_head + idx) * D : rk + (ring_head + (s0 + (idx - P)) % a.R) * D;
             bytes = 16;
+            if (idx < P) {
+                int j = idx;
+                if (a.sel) {  // a selected entry: its index must name a stored block
+                    j = a.sel[(size_t)b * a.sel_k + idx];
+                    if (j < 0 || j >= a.max_blocks) {
+                        if (lane == 0) set_status(a.status, LBCA_ERR_ARG);
+                        j = 0;
+                        bytes = 0;  // zero row
+                    }
+                }
+                src = pk + (pool_head + j) * D;
+            } else {
+                src = rk + (ring_head + (s0 + (idx - P)) % a.R) * D;
+            }
         }
         const uint32_t rbase = sE + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;
 #pragma unroll
@@ -411,7 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     }
 
     // ---- cos/sin at t; this CTA's query groups: RMSNorm, RoPE, fp16, group-major swizzled ----
-    for (int k = tid; k < a.rho / 2; k += kThreads) cs[k] = rope_cs((int64_t)t, k, a.rope_step);
+    for (int k = tid; k < a.rho / 2; k += kThreads) {
+        const uint64_t F = rope_turns(k, a.rope_step);
+        turns[k] = F;
+        cs[k] = rope_cs_turns((int64_t)t, F);
+    }
+    // the query and the new token may come from the preceding kernel (programmatic
+    // dependent launch): everything above reads only this cache
+    griddep_wait();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_sh;
@@ -524,15 +562,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
                     for (int i = 0; i < 8; ++i) x[j][i] *= inv * gam[i];
                 }
             }
+            // RoPE at the token's position: lane l forms cos/sin of pair kb + l
+            // (one sincos per lane for 32 pairs), the lanes holding a pair's
+            // dims take it by shuffle
             const int64_t spos = (int64_t)s0 + (idx - P);
             const int rope0 = D - a.rho;
+            for (int kb = 0; kb < a.rho / 2; kb += 32) {
+                const int k = kb + lane;
+                const float2 mine = k < a.rho / 2 ? rope_cs_turns(spos, turns[k]) : make_float2(1.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < CPR / 32; ++j) {
+                    const int ch = j * 32 + lane;
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2) {
+                        const int kk = (ch * 8 + i - rope0) >> 1;  // this lane's pair (negative: not rotated)
+                        const bool here = ch * 8 + i >= rope0 && kk >= kb && kk < kb + 32;
+                        const int src = here ? kk - kb : lane;
+                        const float2 c = make_float2(__shfl_sync(0xffffffffu, mine.x, src),
+                                                     __shfl_sync(0xffffffffu, mine.y, src));
+                        if (here) rotate_pair(x[j][i], x[j][i + 1], c);
+                    }
+                }
+            }
 #pragma unroll
             for (int j = 0; j < CPR / 32; ++j) {
                 const int ch = j * 32 + lane;
-#pragma unroll
-                for (int i = 0; i < 8; i += 2)
-                    if (a.rho > 0 && ch * 8 + i >= rope0)
-                        rotate_pair(x[j][i], x[j][i + 1], rope_cs(spos, (ch * 8 + i - rope0) >> 1, a.rope_step));
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ovf |= fabsf(x[j][i]) > kF16Max;
                 uint4 o;
@@ -659,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
     ok2 = __syncthreads_and(ok2);
     if (!ok2 && tid == 0) set_status(a.status, LBCA_ERR_TIMEOUT);
     const bool have_o = live && ok2;
+    griddep_launch_dependents();  // the next kernel on the stream may start its cache reads
     tc_fence_after();
 
     const int rope0 = D - a.rho;
@@ -815,17 +870,19 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
     auto fn = decode_mqa_tc_kernel<D>;
     const MqaLayout lay(D, a.chunk, a.tc_cs);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = a.tc_cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(a.tc_cs, a.G, a.B);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = lay.SMEM;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = (a.pdl && !a.sel) ? 2 : 1;  // a selection comes from the preceding kernel: no early start
     return cudaLaunchKernelEx(&cfg, fn, a);
 }
 
@@ -852,9 +909,14 @@ bool mqa_tc_shape_ok(int dtype, int B, int Hq, int G, int D, int m, int w, int s
 }
 
 MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx) {
+    if (!mqa_tc_shape_ok(dtype, B, Hq, G, D, m, w, shared, max_ctx)) return MqaTcPlan{0, 0};
+    return plan_decode_mqa_tc_vis(dtype, B, Hq, G, D, shared, max_visible(m, w, max_ctx));
+}
+
+MqaTcPlan plan_decode_mqa_tc_vis(int dtype, int B, int Hq, int G, int D, int shared, long long max_vis) {
     MqaTcPlan p{0, 0};
-    if (!mqa_tc_shape_ok(dtype, B, Hq, G, D, m, w, shared, max_ctx)) return p;
-    const long long max_vis = max_visible(m, w, max_ctx);
+    if (dtype != LBCA_BF16 || !shared || G < 1 || Hq != NH * G || (D != 256 && D != 512)) return p;
+    if (B < 1 || max_vis < 1) return p;
     const int cs_min = (int)std::max<long long>(1, (max_vis + 127) / 128);
     // fewest waves of clusters first, then the widest cluster (the most SMs streaming)
     const long long groups = (long long)B * G;

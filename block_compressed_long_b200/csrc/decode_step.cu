@@ -110,34 +110,23 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     const int GD = a.G * D;
     const int DS = D / CS;  // dims this CTA finalises
 
-    // ---- loads that do not depend on the length go out first ----
+    // ---- the open block's running pooling state (this cache's; read before the
+    // preceding kernel completes when launched with programmatic dependence) ----
     const bool app = rank == 0 && h0 % r == 0;  // the CTA that appends for (sequence, kv head)
     const bool pair_owner = tid < D / 2;
     constexpr int QV = (R * D / VEC + kThreads - 1) / kThreads;
     uint4 qv[QV];
-#pragma unroll
-    for (int j = 0; j < QV; ++j) {
-        const int idx = tid + j * kThreads;
-        if (idx < R * D / VEC)
-            qv[j] = *reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((size_t)b * a.Hq + h0 + idx / (D / VEC)) * D +
-                                                    (idx % (D / VEC)) * VEC);
-    }
     const size_t tok = (size_t)b * GD + (size_t)g * D + 2 * tid;  // this thread's pair of the new token
     typename Pair<T>::Raw kraw{}, vraw{}, zraw[2]{};
     float2 am[2], al_[2], aa[2];  // running pooling state of the open block
-    if (pair_owner) {
-        kraw = Pair<T>::load(static_cast<const T*>(a.k) + tok);
-        if (!a.shared) vraw = Pair<T>::load(static_cast<const T*>(a.v) + tok);
-        if (app) {
+    if (pair_owner && app) {
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {  // series: key (or shared entry), value
-                if (s >= a.S) break;
-                zraw[s] = Pair<T>::load(static_cast<const T*>(s == 0 ? a.zk : a.zv) + tok);
-                const float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
-                am[s] = *reinterpret_cast<const float2*>(st);
-                al_[s] = *reinterpret_cast<const float2*>(st + GD);
-                aa[s] = *reinterpret_cast<const float2*>(st + 2 * GD);
-            }
+        for (int s = 0; s < 2; ++s) {  // series: key (or shared entry), value
+            if (s >= a.S) break;
+            const float* st = a.state + (((size_t)b * a.S + s) * 3) * GD + (size_t)g * D + 2 * tid;
+            am[s] = *reinterpret_cast<const float2*>(st);
+            al_[s] = *reinterpret_cast<const float2*>(st + GD);
+            aa[s] = *reinterpret_cast<const float2*>(st + 2 * GD);
         }
     }
 
@@ -199,6 +188,12 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
     if (tid == 0) {
         if (nst > 0) issue(0);
         if (nst > 1) issue(1);
+    }
+
+    // ---- the step's own inputs (the query and the new token) may come from the
+    // preceding kernel: everything above reads only this cache ----
+    griddep_wait();
+    if (tid == 0) {
         // Every CTA of the sequence has read its length once it has arrived
         // here, so the last to arrive may advance it (latency hidden behind
         // the copies).
@@ -206,6 +201,24 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         if (atomicAdd(&a.arrive[b], 1u) == total - 1) {
             a.seq_lens[b] = L;
             a.arrive[b] = 0u;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < QV; ++j) {
+        const int idx = tid + j * kThreads;
+        if (idx < R * D / VEC)
+            qv[j] = *reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((size_t)b * a.Hq + h0 + idx / (D / VEC)) * D +
+                                                    (idx % (D / VEC)) * VEC);
+    }
+    if (pair_owner) {
+        kraw = Pair<T>::load(static_cast<const T*>(a.k) + tok);
+        if (!a.shared) vraw = Pair<T>::load(static_cast<const T*>(a.v) + tok);
+        if (app) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                if (s >= a.S) break;
+                zraw[s] = Pair<T>::load(static_cast<const T*>(s == 0 ? a.zk : a.zv) + tok);
+            }
         }
     }
 
@@ -447,6 +460,8 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         }
     }
 
+    griddep_launch_dependents();  // the next kernel on the stream may start its cache reads
+
     // ---- merge the entry groups of each warp with shuffles, then the warps ----
 #pragma unroll
     for (int off = LG; off < 32; off <<= 1)
@@ -558,10 +573,12 @@ cudaError_t launch_step_one(const StepArgs& a, size_t smem, cudaStream_t s) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (b.CS > 8) {
@@ -576,6 +593,7 @@ cudaError_t launch_step_one(const StepArgs& a, size_t smem, cudaStream_t s) {
     }
     cfg.gridDim = dim3(b.CS, b.Hq / R, b.B);
     attr[0].val.clusterDim.x = b.CS;
+    cfg.numAttrs = b.pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, fn, b);
 }
 template <typename T, int D>

@@ -1,0 +1,289 @@
+// indexer.cu -- lightning-indexer relevance and top-k block selection (the
+// CSA form; CSA page, "What is implemented": low-rank indexer queries,
+// per-head ReLU-scored relevance against compressed indexer keys, learned
+// head weights, top-k selection restricted to causally visible blocks,
+// Eqs 13-17).
+//
+// For one query per sequence with indexer heads q_h [HI, DI] and head
+// weights w_h, the relevance of complete block j is
+//     I_j = sum_h w_h ReLU(q_h . k_j),     j < floor(L / m),
+// and the k highest-relevance blocks are selected.
+//
+// B200 mapping.
+//   Relevance: the heads' dot products with a tile of 128 compressed keys are
+//   one small dense contraction, S^T = K . Q^T (M = 128 key rows, N = HI
+//   heads, K = DI), run on tcgen05 with bf16 operands and the f32 result in
+//   TMEM; the epilogue thread of TMEM lane r reads its row's HI scores and
+//   forms sum_h w_h ReLU(s_h).  A CTA (128 threads) owns one (sequence, tile):
+//   the tile and the queries are staged with 16-byte cp.async into
+//   128-byte-swizzled shared memory, so each key crosses HBM once.  Several
+//   CTAs per SM overlap one tile's copies with another's MMA and epilogue.
+//   Top-k: one CTA per sequence selects the k largest relevances by a radix
+//   select over order-preserving 32-bit keys (four 8-bit passes with a
+//   shared-memory histogram), then writes the selected block indices in
+//   increasing index order (equal relevances: lower index first) followed by
+//   -1 padding when fewer than k blocks are visible.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace lbca {
+namespace {
+
+constexpr int kRows = 128;       // compressed keys per tile (M of the MMA)
+constexpr int kThreads = 128;    // one thread per TMEM lane / key row
+constexpr uint64_t kWaitNs = 200ull * 1000 * 1000;
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Relevance of the visible blocks of one 128-row tile.  DI: indexer head dim
+// (64 or 128), HI: indexer heads (32, 64 or 128).
+template <int DI, int HI>
+__global__ void __launch_bounds__(kThreads) indexer_score_kernel(const IndexerArgs a) {
+    constexpr int REG_K = kRows * 128;   // one 64-dim column region of the key tile (bytes)
+    constexpr int REG_Q = HI * 128;      // one 64-dim column region of the query tile
+    constexpr int NREG = DI / 64;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sK = smem;                                   // [NREG][128 rows x 128 B]
+    uint8_t* sQ = sK + NREG * REG_K;                      // [NREG][HI rows x 128 B]
+    float* sw = reinterpret_cast<float*>(sQ + NREG * REG_Q);  // [HI] head weights
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sw + HI);
+    uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(bar + 1);
+
+    const int tile = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = a.seq_lens[b];
+    const int nvis = min(max(L, 0) / a.m, a.max_blocks);
+    const int r0 = tile * kRows;
+    if (r0 >= nvis) return;  // uniform per CTA: nothing of this tile is visible
+    const int nrows = min(kRows, nvis - r0);
+
+    if (warp == 0) tmem_alloc(tmem_sh, HI < 32 ? 32 : HI);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
+    // ---- stage the key tile (rows past nrows zero) and the queries, 128B-swizzled ----
+    const __nv_bfloat16* kx = static_cast<const __nv_bfloat16*>(a.k_idx) + ((size_t)b * a.max_blocks + r0) * DI;
+    const __nv_bfloat16* qx = static_cast<const __nv_bfloat16*>(a.q_idx) + (size_t)b * HI * DI;
+    const uint32_t sKa = smem_addr(sK), sQa = smem_addr(sQ);
+    for (int c = tid; c < kRows * (DI / 8); c += kThreads) {
+        const int r = c / (DI / 8), ch = c % (DI / 8);
+        const uint32_t dst = sKa + (uint32_t)(ch >> 3) * REG_K + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
+                             ((uint32_t)((ch & 7) ^ (r & 7)) << 4);
+        const bool ok = r < nrows;
+        cp16(dst, ok ? kx + (size_t)r * DI + ch * 8 : kx, ok ? 16u : 0u);
+    }
+    for (int c = tid; c < HI * (DI / 8); c += kThreads) {
+        const int r = c / (DI / 8), ch = c % (DI / 8);
+        const uint32_t dst = sQa + (uint32_t)(ch >> 3) * REG_Q + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u +
+                             ((uint32_t)((ch & 7) ^ (r & 7)) << 4);
+        cp16(dst, qx + (size_t)r * DI + ch * 8, 16u);
+    }
+    for (int h = tid; h < HI; h += kThreads) sw[h] = a.w_idx[(size_t)b * HI + h];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes -> tensor core reads
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_sh;
+
+    // ---- S^T = K . Q^T: M = 128 key rows, N = HI heads, K = DI, bf16 in, f32 in TMEM ----
+    if (tid == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(kRows, HI, false);
+#pragma unroll
+        for (int kk = 0; kk < DI / 16; ++kk)
+            tc_mma_bf16(tbase, smem_desc_sw128(sKa + (kk >> 2) * REG_K + (kk & 3) * 32, 16, 1024),
+                        smem_desc_sw128(sQa + (kk >> 2) * REG_Q + (kk & 3) * 32, 16, 1024), idesc, kk > 0);
+        tc_commit(bar);
+    }
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait(bar, 0, kWaitNs);
+    ok = __syncthreads_and(ok);
+    if (!ok) {
+        if (tid == 0) set_status(a.status, LBCA_ERR_TIMEOUT);
+    } else {
+        // ---- epilogue: TMEM lane = key row; sum_h w_h ReLU(s_h) ----
+        tc_fence_after();
+        const int row = 32 * warp + lane;
+        float acc = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < HI; c0 += 32) {
+            float s[32];
+            tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc = fmaf(sw[c0 + i], fmaxf(s[i], 0.f), acc);
+        }
+        if (row < nrows) a.scores[(size_t)b * a.max_blocks + r0 + row] = acc;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, HI < 32 ? 32 : HI);
+}
+
+// Order-preserving key of an f32: larger float -> larger unsigned key.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kSelThreads = 1024;
+
+// Exclusive prefix sum over the CTA of one value per thread; *total gets the sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kSelThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_sums[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+    *total = warp_sums[kSelThreads / 32 - 1];
+    __syncthreads();
+    return before;
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) {
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_sums[32];
+    __shared__ uint32_t sh_prefix;
+    __shared__ int sh_krem, sh_gt;
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int L = a.seq_lens[b];
+    const int nvis = min(max(L, 0) / a.m, a.max_blocks);
+    const int K = a.top_k;
+    const float* sc = a.scores + (size_t)b * a.max_blocks;
+    int32_t* sel = a.sel + (size_t)b * K;
+    float* selv = a.sel_scores ? a.sel_scores + (size_t)b * K : nullptr;
+    const int chunk = (nvis + kSelThreads - 1) / kSelThreads;  // contiguous indices per thread
+    const int i0 = tid * chunk, i1 = min(nvis, i0 + chunk);
+
+    if (nvis <= K) {  // every visible block is selected
+        for (int i = tid; i < K; i += kSelThreads) {
+            sel[i] = i < nvis ? i : -1;
+            if (selv) selv[i] = i < nvis ? sc[i] : kNegInf;
+        }
+        return;
+    }
+    // ---- radix select of the K-th largest key, 8 bits per pass, most significant first ----
+    if (tid == 0) {
+        sh_prefix = 0u;
+        sh_krem = K;
+        sh_gt = 0;
+    }
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
+        __syncthreads();
+        const uint32_t prefix = sh_prefix;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t k = order_key(sc[i]);
+            if (pass == 0 || (k >> (shift + 8)) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int need = sh_krem, above = 0, d = 255;
+            for (; d > 0; --d) {
+                if (above + (int)hist[d] >= need) break;
+                above += (int)hist[d];
+            }
+            sh_prefix = (prefix << 8) | (uint32_t)d;
+            sh_krem = need - above;
+            sh_gt += above;
+        }
+        __syncthreads();
+    }
+    const uint32_t thr = sh_prefix;  // the K-th largest key
+    const int ties_needed = sh_krem;
+    // ---- selection in index order: every key above thr, and the first ties_needed equal to it ----
+    int my_gt = 0, my_tie = 0;
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t k = order_key(sc[i]);
+        my_gt += k > thr;
+        my_tie += k == thr;
+    }
+    int total;
+    const int tie_before = block_exclusive_scan(my_tie, warp_sums, &total);
+    const int my_take = my_gt + max(0, min(my_tie, ties_needed - tie_before));
+    const int pos0 = block_exclusive_scan(my_take, warp_sums, &total);
+    int pos = pos0, tie_rank = tie_before;
+    for (int i = i0; i < i1; ++i) {
+        const float f = sc[i];
+        const uint32_t k = order_key(f);
+        bool take = k > thr;
+        if (k == thr) take = tie_rank++ < ties_needed;
+        if (take) {
+            if (pos < K) {
+                sel[pos] = i;
+                if (selv) selv[pos] = f;
+            }
+            ++pos;
+        }
+    }
+    if (tid == 0 && total != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
+}
+
+template <int DI, int HI>
+size_t score_smem() {
+    return (size_t)DI / 64 * (kRows + HI) * 128 + HI * 4 + 64 + 1024;
+}
+
+template <int DI, int HI>
+cudaError_t launch_score(const IndexerArgs& a, cudaStream_t s) {
+    const size_t smem = score_smem<DI, HI>();
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(indexer_score_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid((a.max_blocks + kRows - 1) / kRows, a.B);
+    indexer_score_kernel<DI, HI><<<grid, kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool indexer_shape_ok(int HI, int DI) {
+    return (DI == 64 || DI == 128) && (HI == 32 || HI == 64 || HI == 128);
+}
+
+cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s) {
+    if (a.B == 0) return cudaSuccess;
+    if (a.B > 65535) return cudaErrorInvalidValue;
+    cudaError_t e = cudaSuccess;
+    if (a.max_blocks > 0) {
+        if (a.DI == 64) {
+            e = a.HI == 32 ? launch_score<64, 32>(a, s) : a.HI == 64 ? launch_score<64, 64>(a, s)
+                                                                      : launch_score<64, 128>(a, s);
+        } else {
+            e = a.HI == 32 ? launch_score<128, 32>(a, s) : a.HI == 64 ? launch_score<128, 64>(a, s)
+                                                                       : launch_score<128, 128>(a, s);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    topk_kernel<<<a.B, kSelThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace lbca

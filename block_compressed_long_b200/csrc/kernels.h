@@ -8,32 +8,49 @@
 
 namespace lbca {
 
-// Pool complete blocks (and optionally record the open block's running state).
-struct PoolArgs {
-    int dtype;
+// One pooled series of a pool launch.
+struct PoolSeries {
     const void* x;         // [B, T, G, D]
     const void* z;         // [B, T, G, D]
     const void* bpos;      // [m, G*D]
-    const void* gamma;     // [D] or null
+    const void* gamma;     // [D] or null (key series with RMSNorm)
     void* out;             // [B, G, out_blocks, D]; block j at blk_off + j
-    int out_blocks, blk_off;
+    void* out_f16;         // optional fp16 copy [B, G, out_f16_blocks, D] (bf16 input only)
+    // optional fp16 copy of every token of each complete block, [B, T, G, D]
+    // (bf16 input only); key series rotated at their position s with cos/sin
+    // from PoolArgs::tab ([rho/2][T], pair-major)
+    void* raw_f16;
+    int key;               // 1: key series (RMSNorm when on, RoPE at the block start)
+    int state_series;      // index of this series in the pooling state
+    // dual overlapped pooling (CSA form): the b-series [B, T, G, D] and its
+    // bias [m, G*D]; entry j pools block j of (x, z) and block j - 1 of
+    // (xb, zb) under one softmax.  Null for single-series pooling.
+    const void* xb;
+    const void* zb;
+    const void* bposb;
+};
+// Pool complete blocks of one or two series in one launch (and optionally
+// record the open block's running state).
+struct PoolArgs {
+    int dtype;
+    PoolSeries ser[2];
+    int nser;
+    int out_blocks, blk_off, out_f16_blocks;
     int B, T, G, D, m;
     int64_t pos0;          // absolute position of token 0 of x
-    int key, rmsnorm, rho;
+    int rmsnorm, rho;
     double rope_step;  // theta^(-2/rho)
     float eps;
     float* state;          // [B, S, 3, G, D] or null: running state of the partial block
-    int S, series;
-    void* out_f16;         // optional fp16 copy [B, G, out_f16_blocks, D] (bf16 input only)
-    int out_f16_blocks;
-    // optional fp16 copy of every token of each complete block, [B, T, G, D]
-    // (bf16 input only); key series rotated at their position s with cos/sin
-    // from `tab` ([rho/2][T], pair-major)
-    void* raw_f16;
+    int S;
     const float2* tab;
     // device status word for the fp16 copies: a value beyond the fp16 range
     // sets LBCA_ERR_UNSUPPORTED (nullable)
     int32_t* status;
+    // launch geometry (set by launch_pool): blocks per series and sequence,
+    // head slices, blocks per CTA
+    int nblk, gz, bpc;
+    int dual;              // 1: every series is pooled in the dual overlapped form
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);
 
@@ -96,6 +113,12 @@ struct DecodeArgs {
     void* ring_w; void* pooled_w;                    // the cache's ring_k / pooled_k, written
     float* state;                                    // [B, 1, 3, G, D]
     int32_t* lens_w;                                 // seq_lens, advanced by one
+    // CSA form (tensor-core shared-entry decode only): the selected entries
+    // [B, sel_k] (block indices, valid ones first) replace the pooled prefix,
+    // and the raw window is the last n_win tokens; null: block-aligned partition
+    const int32_t* sel;
+    int sel_k;
+    int pdl;           // launch with programmatic dependence on the preceding kernel (cache reads first)
 };
 // Chooses heads per CTA, chunk and split count for a decode call.
 struct DecodePlan {
@@ -115,6 +138,9 @@ struct MqaTcPlan {
     int cs, rows;
 };
 MqaTcPlan plan_decode_mqa_tc(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
+// The same plan for a visible list of at most max_vis entries (the CSA form:
+// top_k selected entries plus n_win window tokens).
+MqaTcPlan plan_decode_mqa_tc_vis(int dtype, int B, int Hq, int G, int D, int shared, long long max_vis);
 // The shape tests of plan_decode_mqa_tc alone (host-only, no device query).
 bool mqa_tc_shape_ok(int dtype, int B, int Hq, int G, int D, int m, int w, int shared, int max_ctx);
 cudaError_t launch_decode_mqa_tc(const DecodeArgs& a, cudaStream_t s);
@@ -140,6 +166,7 @@ struct StepArgs {
     uint32_t* seg_count;                                           // [segments], zeroed
     int C, grid, maxc;
     uint64_t rope_f[128];  // persistent form: fixed-point turns per position of each RoPE pair (rope_turns)
+    int pdl;               // launch with programmatic dependence on the preceding kernel (cache reads first)
 };
 struct StepPlan {
     int heads_per_cta, CS, SE;
@@ -157,6 +184,38 @@ size_t flat_smem_bytes(int dtype, int B, int D, int R, int C, int shared);
 cudaError_t launch_decode_flat(const StepArgs& a, cudaStream_t s);
 // CTAs of the persistent grid on the current device (every SM filled).
 cudaError_t flat_grid(int* grid, int dtype, int D, int R, size_t smem);
+
+// Lightning-indexer relevance and top-k selection (CSA form): one query per
+// sequence, bf16 queries [B, HI, DI] and compressed keys [B, max_blocks, DI].
+struct IndexerArgs {
+    const void* q_idx; const float* w_idx; const void* k_idx; const int32_t* seq_lens;
+    float* scores;                                   // [B, max_blocks] workspace
+    int32_t* sel;                                    // [B, top_k]
+    float* sel_scores;                               // [B, top_k] or null
+    int32_t* status;
+    int B, HI, DI, m, max_blocks, top_k;
+};
+bool indexer_shape_ok(int HI, int DI);
+cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s);
+
+// Backward of the prefill (pooling + attention): f32 gradients and scratch.
+struct BwdArgs {
+    int dtype;
+    const void* q; const void* k; const void* v; const void* zk; const void* zv;
+    const void* bpk; const void* bpv; const float* sink; const void* gamma_q; const void* gamma_kv;
+    const void* dout;                                  // gradient of the forward's output [B, T, Hq, D]
+    float* dq; float* dk; float* dv; float* dzk; float* dzv; float* dbk; float* dbv; float* dsink;
+    // scratch: Ef, dE [S][B][NB][G][D]; Pk [B][NB][G][D]; Kf, dKf, vf [B][T][G][D];
+    // qf, dof [B][T][Hq][D]; lse, dsum [B][T][Hq]
+    float* Ef; float* dE; float* Pk; float* Kf; float* dKf; float* vf; float* qf; float* dof; float* lse;
+    float* dsum;
+    int B, T, Hq, G, D, m, w, rho, rmsnorm, shared, S, NB;
+    float eps, scale;
+    double rope_step;
+};
+bool backward_supported(int D);
+size_t backward_scratch_floats(int S, int B, int T, int Hq, int G, int D, int m);
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
 
 struct PrefillArgs {
     int dtype;

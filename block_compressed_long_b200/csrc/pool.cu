@@ -68,71 +68,72 @@ __device__ __forceinline__ void finalise_key(float (&e)[VEC], int d0, int D, boo
     }
 }
 
-// CTA = (block j, sequence b, slice of whole kv heads); <= 256 threads.  RAW:
-// also the fp16 copy of every token (the tensor-core prefill's operands), in
-// an instantiation of its own so that plain pooling carries none of it.
-template <typename T, bool RAW>
+// CTA = (block j, sequence b, slice of whole kv heads, series); <= 256
+// threads.  RAW: also the fp16 copy of every token of a complete block (the
+// tensor-core prefill's operands), in an instantiation of its own so that
+// plain pooling carries none of it.  DUAL: dual overlapped pooling (CSA page,
+// "What is implemented", Eqs 9-12): entry j folds block j - 1 of the b-series
+// (none for j = 0) and then block j of the a-series into one online softmax.
+template <typename T, bool RAW, bool DUAL>
 __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     constexpr int VEC = Vec<T>::N;
     constexpr int U = 4;  // tokens per online-softmax step
     extern __shared__ __align__(16) float smem[];
+    const PoolSeries& sr = a.ser[blockIdx.z / a.gz];
     const int GD = a.G * a.D, NVH = a.D / VEC;
     const int hpc = blockDim.x / NVH;  // heads per CTA
+    const int hs = blockIdx.z % a.gz;
     const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const bool active = tid < hpc * NVH && (int)blockIdx.z * hpc + tid / NVH < a.G;
-    const int cv = active ? blockIdx.z * hpc * NVH + tid : 0;  // vector index within the G*D row
+    const bool active = tid < hpc * NVH && hs * hpc + tid / NVH < a.G;
+    const int cv = active ? hs * hpc * NVH + tid : 0;  // vector index within the G*D row
     const int n_tok = min(a.m, a.T - j * a.m);
     const bool full = n_tok == a.m;
     float2* cs = reinterpret_cast<float2*>(smem);
     float* part = smem + a.rho;
-    if (full && a.key && a.rho)
+    if (full && sr.key && a.rho)
         for (int k = tid; k < a.rho / 2; k += blockDim.x)
             cs[k] = rope_cs(a.pos0 + (int64_t)j * a.m, k, a.rope_step);
     __syncthreads();
 
-    const size_t row0 = ((size_t)b * a.T + (size_t)j * a.m) * GD + (size_t)cv * VEC;
-    const uint4* xp = reinterpret_cast<const uint4*>(static_cast<const T*>(a.x) + row0);
-    const uint4* zp = reinterpret_cast<const uint4*>(static_cast<const T*>(a.z) + row0);
-    const uint4* bp = reinterpret_cast<const uint4*>(static_cast<const T*>(a.bpos) + (size_t)cv * VEC);
     const int rstride = GD / VEC;  // uint4 per token row
-
     float mx[VEC], l[VEC], acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) { mx[e] = kNegInf; l[e] = 0.f; acc[e] = 0.f; }
     const int g = cv / NVH, d0 = (cv % NVH) * VEC;
-    const bool raw_copy = RAW && VEC == 8 && full;  // uniform per CTA
-    bool f16_ovf = false;                           // an fp16 copy left the fp16 range
+    bool f16_ovf = false;  // an fp16 copy left the fp16 range
 
-    if (active) {
-        // U tokens per step: their X, Z and B_pos vectors are loaded together
-        // (12 x 16 bytes in flight per thread), then one rescale and U
-        // accumulations.  Memory parallelism comes from many resident warps
-        // (few registers per thread) rather than from a register prefetch.
-        for (int i0 = 0; i0 < n_tok; i0 += U) {
+    // Fold the n tokens of one block of one series (raw rows from xs, zs, the
+    // bias rows from bs) into the running softmax.  U tokens per step: their
+    // X, Z and B_pos vectors are loaded together (12 x 16 bytes in flight per
+    // thread), then one rescale and U accumulations.  Memory parallelism comes
+    // from many resident warps (few registers per thread).
+    auto fold = [&](const uint4* xp, const uint4* zp, const uint4* bp, int n, int blk, bool raw_copy) {
+        for (int i0 = 0; i0 < n; i0 += U) {
             uint4 cx[U], cz[U], cb[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (i0 + u < n_tok) {
+                if (i0 + u < n) {
                     cx[u] = __ldcs(xp + (size_t)(i0 + u) * rstride);
                     cz[u] = __ldcs(zp + (size_t)(i0 + u) * rstride);
                     cb[u] = __ldg(bp + (size_t)(i0 + u) * rstride);
                 }
-            if constexpr (RAW && VEC == 8) {
+            if constexpr (RAW && !DUAL && VEC == 8) {
                 if (raw_copy) {  // these tokens' fp16 copy; keys turned at their position
 #pragma unroll
                     for (int u = 0; u < U; ++u)
-                        if (i0 + u < n_tok) {
+                        if (i0 + u < n) {
                             float xf[VEC];
                             unpack<T>(cx[u], xf);
-                            const int s_tok = j * a.m + i0 + u;
+                            const int s_tok = blk * a.m + i0 + u;
                             const int dr = d0 - (a.D - a.rho);
-                            if (a.key && a.rho)
+                            if (sr.key && a.rho)
 #pragma unroll
                                 for (int e = 0; e < VEC; e += 2)
                                     if (dr + e >= 0)
                                         rotate_pair(xf[e], xf[e + 1], a.tab[(size_t)((dr + e) >> 1) * a.T + s_tok]);
-                            st16_f16_checked(static_cast<__half*>(a.raw_f16) + row0 + (size_t)(i0 + u) * GD, xf,
-                                             f16_ovf);
+                            st16_f16_checked(static_cast<__half*>(sr.raw_f16) +
+                                                 ((size_t)b * a.T + s_tok) * GD + (size_t)cv * VEC,
+                                             xf, f16_ovf);
                         }
                 }
             }
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
             for (int e = 0; e < VEC; ++e) cmax[e] = mx[e];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (i0 + u < n_tok) {
+                if (i0 + u < n) {
                     float zf[VEC], bf[VEC];
                     unpack<T>(cz[u], zf);
                     unpack<T>(cb[u], bf);
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (i0 + u < n_tok) {
+                if (i0 + u < n) {
                     float xf[VEC], zf[VEC], bf[VEC];
                     unpack<T>(cx[u], xf);
                     unpack<T>(cz[u], zf);
@@ -172,6 +173,21 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
                 }
             }
         }
+    };
+    auto series_rows = [&](const void* x, int blk) {
+        return reinterpret_cast<const uint4*>(static_cast<const T*>(x) + ((size_t)b * a.T + (size_t)blk * a.m) * GD +
+                                              (size_t)cv * VEC);
+    };
+    if (active) {
+        if constexpr (DUAL) {
+            if (j > 0)  // the preceding block of the b-series joins the same softmax
+                fold(series_rows(sr.xb, j - 1), series_rows(sr.zb, j - 1),
+                     reinterpret_cast<const uint4*>(static_cast<const T*>(sr.bposb) + (size_t)cv * VEC), a.m, j - 1,
+                     false);
+        }
+        fold(series_rows(sr.x, j), series_rows(sr.z, j),
+             reinterpret_cast<const uint4*>(static_cast<const T*>(sr.bpos) + (size_t)cv * VEC), n_tok, j,
+             full && sr.raw_f16 != nullptr);
     }
 
     if (full) {
@@ -179,30 +195,26 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
 #pragma unroll
         for (int i = 0; i < VEC; ++i) e[i] = active ? acc[i] / l[i] : 0.f;
         float ss = 0.f;
-        if (a.key && a.rmsnorm) {
+        if (sr.key && a.rmsnorm) {
             float v = 0.f;
 #pragma unroll
             for (int i = 0; i < VEC; ++i) v += e[i] * e[i];
             ss = head_sum(part, v, active ? tid - (cv % NVH) : 0, NVH);
         }
-        if (a.key)
-            finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(a.gamma),
-                                 a.rho, cs);
+        if (sr.key)
+            finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(sr.gamma), a.rho, cs);
         if (active) {
             const size_t oi = (((size_t)b * a.G + g) * a.out_blocks + a.blk_off + j) * a.D + d0;
-            float tmp[VEC];
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) tmp[i] = e[i];
-            st16(static_cast<T*>(a.out) + oi, tmp);
+            st16(static_cast<T*>(sr.out) + oi, e);
             if constexpr (VEC == 8) {
-                if (a.out_f16) {  // the f32 value, rounded once to fp16
+                if (sr.out_f16) {  // the f32 value, rounded once to fp16
                     const size_t oi16 = (((size_t)b * a.G + g) * a.out_f16_blocks + a.blk_off + j) * a.D + d0;
-                    st16_f16_checked(static_cast<__half*>(a.out_f16) + oi16, tmp, f16_ovf);
+                    st16_f16_checked(static_cast<__half*>(sr.out_f16) + oi16, e, f16_ovf);
                 }
             }
         }
     } else if (a.state && active) {
-        float* st = a.state + (((size_t)b * a.S + a.series) * 3) * GD + (size_t)cv * VEC;
+        float* st = a.state + (((size_t)b * a.S + sr.state_series) * 3) * GD + (size_t)cv * VEC;
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
             st[i] = mx[i];
@@ -212,6 +224,8 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
     }
     if (f16_ovf) set_status(a.status, LBCA_ERR_UNSUPPORTED);
 }
+
+inline int round32(int n) { return (n + 31) / 32 * 32; }
 
 template <typename T>
 __global__ void __launch_bounds__(1024) ring_fill_kernel(const RingFillArgs a) {
@@ -374,26 +388,34 @@ __global__ void __launch_bounds__(1024) append_kernel(const AppendArgs a) {
     if (tid == 0) a.seq_lens[b] = pos + 1;
 }
 
-inline int round32(int n) { return (n + 31) / 32 * 32; }
 
 }  // namespace
 
-cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s) {
+cudaError_t launch_pool(const PoolArgs& in, cudaStream_t s) {
+    PoolArgs a = in;
     const int vec = a.dtype == LBCA_BF16 ? 8 : 4;
     const int nvh = a.D / vec;                 // <= 128 threads per head
     const int hpc = std::min(a.G, 256 / nvh);  // whole heads per CTA
-    const int nblk = a.T / a.m + ((a.state && (a.T % a.m)) ? 1 : 0);
-    if (nblk == 0 || a.B == 0) return cudaSuccess;
+    a.nblk = a.T / a.m + ((!a.dual && a.state && (a.T % a.m)) ? 1 : 0);
+    if (a.nblk == 0 || a.B == 0 || a.nser < 1) return cudaSuccess;
     const int threads = round32(hpc * nvh);
     const size_t smem = (size_t)a.rho * 4 + (size_t)threads * 4;
-    dim3 grid(nblk, a.B, (a.G + hpc - 1) / hpc);
+    a.gz = (a.G + hpc - 1) / hpc;
+    if (a.B > 65535 || (long long)a.gz * a.nser > 65535) return cudaErrorInvalidValue;
+    dim3 grid(a.nblk, a.B, a.gz * a.nser);
+    const bool raw = a.ser[0].raw_f16 || (a.nser > 1 && a.ser[1].raw_f16);
+    if (a.dual && raw) return cudaErrorInvalidValue;
     if (a.dtype == LBCA_BF16) {
-        if (a.raw_f16)
-            pool_kernel<__nv_bfloat16, true><<<grid, threads, smem, s>>>(a);
+        if (a.dual)
+            pool_kernel<__nv_bfloat16, false, true><<<grid, threads, smem, s>>>(a);
+        else if (raw)
+            pool_kernel<__nv_bfloat16, true, false><<<grid, threads, smem, s>>>(a);
         else
-            pool_kernel<__nv_bfloat16, false><<<grid, threads, smem, s>>>(a);
+            pool_kernel<__nv_bfloat16, false, false><<<grid, threads, smem, s>>>(a);
+    } else if (a.dual) {
+        pool_kernel<float, false, true><<<grid, threads, smem, s>>>(a);
     } else {
-        pool_kernel<float, false><<<grid, threads, smem, s>>>(a);
+        pool_kernel<float, false, false><<<grid, threads, smem, s>>>(a);
     }
     return cudaGetLastError();
 }

@@ -29,7 +29,9 @@ ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspa
                 "lbca_prefill_workspace_bytes", "lbca_pool", "lbca_append", "lbca_decode",
                 "lbca_prefill", "lbca_status_string", "lbca_decode_noalloc",
                 "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches",
-                "lbca_decode_step_form")
+                "lbca_decode_step_form", "lbca_selftest_bounded_wait", "lbca_pool_dual", "lbca_decode_sparse",
+                "lbca_indexer_workspace_bytes", "lbca_indexer_topk", "lbca_prefill_backward_workspace_bytes",
+                "lbca_prefill_backward")
 
 
 class lbca_config(ctypes.Structure):
@@ -47,7 +49,9 @@ class lbca_cache(ctypes.Structure):
                 ("ring_k", ctypes.c_void_p), ("ring_v", ctypes.c_void_p),
                 ("pool_state", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
-                ("ring_slots", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("ring_slots", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+LBCA_CACHE_OVERLAP_PREV = 1
 
 
 _vp, _i32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
@@ -62,6 +66,8 @@ _lib.lbca_prefill_workspace_bytes.argtypes = [_CP, _i32, _i32, _i32]
 _lib.lbca_prefill_workspace_bytes.restype = _sz
 _lib.lbca_pool.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp]
 _lib.lbca_pool.restype = ctypes.c_int
+_lib.lbca_pool_dual.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp]
+_lib.lbca_pool_dual.restype = ctypes.c_int
 _lib.lbca_append.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp]
 _lib.lbca_append.restype = ctypes.c_int
 _lib.lbca_decode.argtypes = [_CP, _vp, _KP, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp, _vp]
@@ -80,6 +86,19 @@ _lib.lbca_decode_step_form.argtypes = [_CP, _i32, _i32]
 _lib.lbca_decode_step_form.restype = _i32
 _lib.lbca_decode_noalloc.argtypes = [_CP, _vp, _KP, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
 _lib.lbca_decode_noalloc.restype = ctypes.c_int
+_lib.lbca_selftest_bounded_wait.argtypes = [_i32, ctypes.c_uint64, _vp, _vp]
+_lib.lbca_selftest_bounded_wait.restype = ctypes.c_int
+_lib.lbca_decode_sparse.argtypes = [_CP, _vp, _KP, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.lbca_decode_sparse.restype = ctypes.c_int
+_lib.lbca_indexer_workspace_bytes.argtypes = [_i32, _i32]
+_lib.lbca_indexer_workspace_bytes.restype = _sz
+_lib.lbca_indexer_topk.argtypes = [_i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp,
+                                   _vp]
+_lib.lbca_indexer_topk.restype = ctypes.c_int
+_lib.lbca_prefill_backward_workspace_bytes.argtypes = [_CP, _i32, _i32]
+_lib.lbca_prefill_backward_workspace_bytes.restype = _sz
+_lib.lbca_prefill_backward.argtypes = [_CP] + [_vp] * 12 + [_i32, _i32] + [_vp] * 9 + [_sz, _vp]
+_lib.lbca_prefill_backward.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
 _lib.lbca_status_string.restype = ctypes.c_char_p
 
@@ -154,6 +173,7 @@ class Cache:
     ring_v: torch.Tensor | None
     pool_state: torch.Tensor
     seq_lens: torch.Tensor
+    flags: int = 0  # LBCA_CACHE_OVERLAP_PREV: steps may read this cache while the preceding kernel drains
 
     @staticmethod
     def allocate(cfg: lbca_config, batch: int, max_ctx: int, device="cuda") -> "Cache":
@@ -171,7 +191,7 @@ class Cache:
     def c(self) -> lbca_cache:
         return lbca_cache(_ptr(self.pooled_k), _ptr(self.pooled_v), _ptr(self.ring_k), _ptr(self.ring_v),
                           _ptr(self.pool_state), _ptr(self.seq_lens), self.batch, self.max_blocks,
-                          self.ring_slots, 0)
+                          self.ring_slots, self.flags)
 
 
 def lbca_pool(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, stream=None):
@@ -180,6 +200,16 @@ def lbca_pool(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, str
     ob = out.shape[2] if out_blocks is None else out_blocks
     _check("lbca_pool", _lib.lbca_pool(ctypes.byref(cfg), series, _ptr(x), _ptr(z), _ptr(b_pos), _ptr(gamma),
                                        B, T, pos0, _ptr(out), ob, _stream(stream)))
+
+
+def lbca_pool_dual(cfg, series, xa, za, xb, zb, b_pos_a, b_pos_b, gamma, out, out_blocks=None, stream=None):
+    """x*, z* [B, T, G, D]; out [B, G, out_blocks, D] (entry j pools block j of
+    the a-series and block j - 1 of the b-series under one softmax)."""
+    B, T = xa.shape[0], xa.shape[1]
+    ob = out.shape[2] if out_blocks is None else out_blocks
+    _check("lbca_pool_dual", _lib.lbca_pool_dual(ctypes.byref(cfg), series, _ptr(xa), _ptr(za), _ptr(xb), _ptr(zb),
+                                                 _ptr(b_pos_a), _ptr(b_pos_b), _ptr(gamma), B, T, _ptr(out), ob,
+                                                 _stream(stream)))
 
 
 def lbca_append(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, cache: Cache, d_status=None, stream=None):
@@ -249,3 +279,50 @@ def lbca_decode_noalloc(cfg, q, cache: Cache, sink, gamma_q, gamma_kv, out, max_
                                                            _ptr(gamma_q), _ptr(gamma_kv), max_ctx, _ptr(out),
                                                            _ptr(d_status),
                                                            _stream(stream)))
+
+
+def lbca_selftest_bounded_wait(arrive: bool, limit_ns: int, d_status, stream=None):
+    """One CTA waits on an mbarrier nothing arrives at (arrive=False) or that it
+    completes itself (arrive=True); a wait that runs out writes
+    LBCA_ERR_TIMEOUT to d_status (an int32 device tensor)."""
+    _check("lbca_selftest_bounded_wait", _lib.lbca_selftest_bounded_wait(int(arrive), int(limit_ns), _ptr(d_status),
+                                                                         _stream(stream)))
+
+
+def lbca_decode_sparse(cfg, q, cache: Cache, sel, sink, gamma_q, gamma_kv, out, d_status=None, stream=None):
+    """q, out [B, Hq, D]; sel [B, top_k] int32 selected block indices."""
+    cc = cache.c()
+    _check("lbca_decode_sparse", _lib.lbca_decode_sparse(ctypes.byref(cfg), _ptr(q), ctypes.byref(cc), _ptr(sel),
+                                                         sel.shape[1], _ptr(sink), _ptr(gamma_q), _ptr(gamma_kv),
+                                                         _ptr(out), _ptr(d_status), _stream(stream)))
+
+
+def lbca_indexer_workspace_bytes(batch: int, max_blocks: int) -> int:
+    return int(_lib.lbca_indexer_workspace_bytes(batch, max_blocks))
+
+
+def lbca_indexer_topk(q_idx, w_idx, k_idx, seq_lens, block_m, sel, sel_scores, workspace, d_status=None,
+                      stream=None):
+    """q_idx [B, HI, DI] bf16, w_idx [B, HI] f32, k_idx [B, max_blocks, DI] bf16,
+    seq_lens [B] int32; sel [B, top_k] int32 (and sel_scores [B, top_k] f32 or None) out."""
+    B, HI, DI = q_idx.shape
+    _check("lbca_indexer_topk", _lib.lbca_indexer_topk(
+        B, HI, DI, block_m, sel.shape[1], _ptr(q_idx), _ptr(w_idx), _ptr(k_idx), k_idx.shape[1], _ptr(seq_lens),
+        _ptr(sel), _ptr(sel_scores), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(d_status),
+        _stream(stream)))
+
+
+def lbca_prefill_backward_workspace_bytes(cfg: lbca_config, batch: int, T: int) -> int:
+    return int(_lib.lbca_prefill_backward_workspace_bytes(ctypes.byref(cfg), batch, T))
+
+
+def lbca_prefill_backward(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q, gamma_kv, dout, grads: dict,
+                          workspace, stream=None):
+    """Gradients into the f32 tensors of ``grads`` (dq, dk, dzk, dbk and, GQA,
+    dv, dzv, dbv; dsink with a sink)."""
+    B, T = q.shape[0], q.shape[1]
+    g = lambda n: _ptr(grads.get(n))  # noqa: E731
+    _check("lbca_prefill_backward", _lib.lbca_prefill_backward(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv), _ptr(b_pos_k), _ptr(b_pos_v), _ptr(sink),
+        _ptr(gamma_q), _ptr(gamma_kv), _ptr(dout), B, T, g("dq"), g("dk"), g("dv"), g("dzk"), g("dzv"), g("dbk"),
+        g("dbv"), g("dsink"), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

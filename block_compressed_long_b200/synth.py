@@ -46,6 +46,13 @@ class Workload:
     bpos_std: float = 0.02
     seed: int = 0
     rope_theta: float = 10000.0
+    # CSA form: dual overlapped pooling (a second raw series and bias), a
+    # lightning indexer of index_heads x index_dim over its own dual-pooled
+    # keys, and top_k selected entries per query
+    dual: bool = False
+    index_heads: int = 0
+    index_dim: int = 0
+    top_k: int = 0
 
 
 WORKLOADS = {
@@ -61,6 +68,9 @@ WORKLOADS = {
                  seed=1004),
         Workload("ragged_gqa_decode_append", "decode", "bf16", 32, 24, 8, 128, False, 64, 128,
                  rope_dims=128, ctx=(4096, 65536), steps=64, seed=1005),
+        Workload("csa_sparse_decode_64k", "decode", "bf16", 4, 64, 1, 512, True, 4, 128,
+                 rope_dims=64, rmsnorm=True, sink="normal", ctx=(65536, 65536), steps=8, seed=1006,
+                 dual=True, index_heads=64, index_dim=128, top_k=512),
     ]
 }
 
@@ -134,6 +144,10 @@ class Inputs:
     bpos_v: torch.Tensor | None
     sink: torch.Tensor | None         # [Hq] f32
     lens: np.ndarray = field(default_factory=lambda: np.zeros(0, np.int64))  # decode: context per sequence
+    # CSA form: b-series kb, zkb [B,T,G,D] and bias bpos_kb [m, G*D]; indexer
+    # queries iq [steps,B,HI,DI] and head weights iw [steps,B,HI] (f32), its
+    # key series ika, izka, ikb, izkb [B,T,1,DI] and biases ibpa, ibpb [m, DI]
+    csa: dict = field(default_factory=dict)
 
 
 def make(w: Workload, lens: np.ndarray | None = None) -> Inputs:
@@ -162,7 +176,21 @@ def make(w: Workload, lens: np.ndarray | None = None) -> Inputs:
         sink = torch.zeros(Hq, dtype=torch.float32)
     else:
         sink = normal(w.seed, "sink", (Hq,), dtype="f32")
-    return Inputs(q, k, v, zk, zv, bpk, bpv, sink, lens)
+    csa = {}
+    if w.dual:
+        csa["kb"] = normal(w.seed, "kb", (B, T, G, D), dtype=w.dtype, row_len=rl)
+        csa["zkb"] = normal(w.seed, "zkb", (B, T, G, D), dtype=w.dtype, row_len=rl)
+        csa["bpos_kb"] = normal(w.seed, "bpos_kb", (m, G * D), std=w.bpos_std, dtype=w.dtype)
+        if w.index_heads:
+            HI, DI = w.index_heads, w.index_dim
+            lead = (B, T, HI, DI) if w.kind == "prefill" else (w.steps, B, HI, DI)
+            csa["iq"] = normal(w.seed, "iq", lead, dtype=w.dtype)
+            csa["iw"] = normal(w.seed, "iw", lead[:-1], dtype="f32")
+            for tag in ("ika", "izka", "ikb", "izkb"):
+                csa[tag] = normal(w.seed, tag, (B, T, 1, DI), dtype=w.dtype, row_len=rl)
+            csa["ibpa"] = normal(w.seed, "ibpa", (m, DI), std=w.bpos_std, dtype=w.dtype)
+            csa["ibpb"] = normal(w.seed, "ibpb", (m, DI), std=w.bpos_std, dtype=w.dtype)
+    return Inputs(q, k, v, zk, zv, bpk, bpv, sink, lens, csa)
 
 
 def f64(t):

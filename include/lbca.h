@@ -116,8 +116,18 @@ typedef struct {
     int32_t  batch;
     int32_t  max_blocks;
     int32_t  ring_slots;
-    int32_t  reserved;     /* must be 0 */
+    int32_t  flags;        /* 0, or LBCA_CACHE_OVERLAP_PREV */
 } lbca_cache;
+
+/* lbca_cache.flags: the one-launch serving steps (lbca_decode_step in its fused
+ * forms) may start before the preceding work on the stream has finished and
+ * read this cache (lengths, pooling state, entries, window) while it drains
+ * (programmatic dependent launch); the step's own inputs -- the query and the
+ * new token -- are read, and anything is written, only once that work has
+ * completed.  Set it only when the preceding work does not write this cache:
+ * in a model, the other layers' kernels that run between two steps of this
+ * layer.  Two steps of the same cache back to back must not set it. */
+#define LBCA_CACHE_OVERLAP_PREV 1
 
 /* Minimum ring slots: m * ceil((n_win + m - 1) / m), the most raw tokens a
  * query can see rounded up to whole blocks.  -1 on an invalid config. */
@@ -156,6 +166,30 @@ LBCA_API size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t bat
 LBCA_API lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
                       const void* b_pos, const void* gamma, int32_t batch, int32_t T,
                       int32_t pos0, void* out, int32_t out_blocks, lbca_stream_t stream);
+
+/*
+ * lbca_pool_dual -- dual overlapped pooling of the floor(T/m) complete blocks
+ * (the CSA form; CSA page, "What is implemented": dual overlapped
+ * compression, Eqs 9-12; entry RoPE at block starts: "Deviations from paper").
+ *   xa, za      device [B, T, G, D] a-series raw values and content logits
+ *   xb, zb      device [B, T, G, D] b-series raw values and content logits
+ *   b_pos_a/_b  device [m, G*D] positional biases of the two series
+ *   gamma       device [D] RMSNorm gain (key series with rmsnorm) or NULL
+ *   out         device [B, G, out_blocks, D]; entry j at index j < out_blocks
+ * Per (entry j, kv head g, channel c), ONE softmax over the 2m logits of block
+ * j of the a-series and block j - 1 of the b-series (entry 0: its m a-series
+ * logits alone) weights the matching raw values:
+ *   out_j = sum_r w_a[r] xa[j m + r] + sum_r w_b[r] xb[(j - 1) m + r],
+ * then, for LBCA_KEY: RMSNorm (when enabled) and RoPE at position j m.  Each
+ * token of each series is read once.  The CSA form's indexer keys are pooled
+ * the same way with their own series (LBCA_VALUE: no finalisation).
+ * Errors: LBCA_ERR_ARG (null or bad sizes, out_blocks < T / m),
+ * LBCA_ERR_ALIGN, LBCA_ERR_UNSUPPORTED, LBCA_ERR_CUDA.
+ */
+LBCA_API lbca_status lbca_pool_dual(const lbca_config* cfg, int32_t series, const void* xa, const void* za,
+                                    const void* xb, const void* zb, const void* b_pos_a, const void* b_pos_b,
+                                    const void* gamma, int32_t batch, int32_t T, void* out, int32_t out_blocks,
+                                    lbca_stream_t stream);
 
 /*
  * lbca_append -- add one raw token to every sequence of the cache.
@@ -281,6 +315,36 @@ LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const v
                          int32_t* d_status, lbca_stream_t stream);
 
 /*
+ * lbca_prefill_backward -- gradients of the prefill for training (mSeek
+ * README, "Experiment at a glance": the LBCA layers are trained by continued
+ * pretraining; the forward is lbca_prefill's).  Given dout [B, T, Hq, D], the
+ * gradient of a loss with respect to every output row of lbca_prefill on the
+ * same inputs, writes the gradients of that loss with respect to
+ *   dq        [B, T, Hq, D]  the queries
+ *   dk, dv    [B, T, G, D]   the raw keys and values (shared form: dk is the
+ *                            gradient of C, dv NULL)
+ *   dzk, dzv  [B, T, G, D]   the pooling logits (zero for tokens of the open
+ *                            block, which is never pooled)
+ *   db_pos_k/_v [m, G*D]     the positional biases
+ *   dsink     [Hq]           the sink logits (NULL when sink is NULL)
+ * all f32, device, overwritten (RMSNorm gains are not differentiated).  The
+ * inputs are lbca_prefill's (I/O dtype); arithmetic is f32 on the CUDA cores:
+ * the pooled entries, finalised keys and queries and the attention output are
+ * recomputed in f32 in `workspace` (>= lbca_prefill_backward_workspace_bytes
+ * bytes), then dq per query row, dkey and dvalue per entry over the contiguous
+ * range of rows that see it, back through RoPE and RMSNorm, then through the
+ * pooling softmax.  D in {32, 64, 128, 256, 512} (else LBCA_ERR_UNSUPPORTED).
+ */
+LBCA_API size_t lbca_prefill_backward_workspace_bytes(const lbca_config* cfg, int32_t batch, int32_t T);
+LBCA_API lbca_status lbca_prefill_backward(const lbca_config* cfg, const void* q, const void* k, const void* v,
+                                           const void* zk, const void* zv, const void* b_pos_k,
+                                           const void* b_pos_v, const float* sink, const void* gamma_q,
+                                           const void* gamma_kv, const void* dout, int32_t batch, int32_t T,
+                                           float* dq, float* dk, float* dv, float* dzk, float* dzv,
+                                           float* db_pos_k, float* db_pos_v, float* dsink, void* workspace,
+                                           size_t workspace_bytes, lbca_stream_t stream);
+
+/*
  * lbca_decode_noalloc -- lbca_decode for callers that cannot allocate.
  * The pages have no counterpart of this entry point; it exists for callers
  * that are not allowed to allocate device memory at all -- for example code
@@ -306,6 +370,75 @@ LBCA_API lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, 
                                          const float* sink, const void* gamma_q, const void* gamma_kv,
                                          int32_t max_ctx, void* out,
                                          int32_t* d_status, lbca_stream_t stream);
+
+/*
+ * lbca_selftest_bounded_wait -- check of the bounded device-side wait.
+ * The pages have no counterpart; it exists so that the timeout path of the
+ * kernels' waits can be exercised without a fault.  One CTA waits, with the
+ * helper every kernel uses, on an mbarrier that nothing arrives at (arrive =
+ * 0) or that its own thread completes first (arrive = 1, the control); after
+ * limit_ns nanoseconds of wall time (1 .. 2e9) the wait gives up and
+ * LBCA_ERR_TIMEOUT is written to the device word d_status (required).  The
+ * kernel returns normally either way, so the context stays usable.
+ */
+LBCA_API lbca_status lbca_selftest_bounded_wait(int32_t arrive, uint64_t limit_ns, int32_t* d_status,
+                                                lbca_stream_t stream);
+
+/*
+ * lbca_decode_sparse -- core attention of the CSA form for one query per
+ * sequence over the selected compressed entries plus the raw window (CSA page,
+ * "What is implemented": shared-KV MQA core attention, Eqs 18-19, where the
+ * selected compressed entries serve as both key and value, the sliding-window
+ * branch of n_win uncompressed recent tokens, RMSNorm on queries and entries,
+ * partial RoPE with the -i rotation of outputs, attention sink, Eq 27).
+ *   q        device [B, Hq, D] queries at position t = seq_lens[b] - 1
+ *   cache    pooled_k holds the finalised compressed entries (lbca_pool_dual,
+ *            LBCA_KEY); ring_k the raw entries of (at least) the last n_win
+ *            tokens, token s in slot s % ring_slots (ring_slots >= n_win)
+ *   sel      device [B, top_k] int32: the selected block indices (as
+ *            lbca_indexer_topk writes them: valid ones first); the first
+ *            min(top_k, floor(L / m), max_blocks) are used
+ *   out      device [B, Hq, D]
+ * One softmax over the selected entries, the window tokens s in
+ * [max(0, L - n_win), t] (finalised in f32 when read: RMSNorm, RoPE at s) and
+ * the sink; a window token may also be summarised by a selected entry (the
+ * two branches overlap).  The output's RoPE dims turn back by -t.  Runs on the
+ * tensor-core shared-entry kernel: bf16, 64 query heads per kv head, D 256 or
+ * 512, top_k + n_win within its cluster capacity (else LBCA_ERR_UNSUPPORTED).
+ * A selected index outside [0, max_blocks) sets d_status to LBCA_ERR_ARG (its
+ * row counts as zeros).
+ */
+LBCA_API lbca_status lbca_decode_sparse(const lbca_config* cfg, const void* q, const lbca_cache* cache,
+                                        const int32_t* sel, int32_t top_k, const float* sink, const void* gamma_q,
+                                        const void* gamma_kv, void* out, int32_t* d_status, lbca_stream_t stream);
+
+/*
+ * lbca_indexer_topk -- lightning-indexer relevance and top-k block selection
+ * for one query per sequence (the CSA form; CSA page, "What is implemented":
+ * low-rank indexer queries, per-head ReLU-scored relevance against compressed
+ * indexer keys, learned head weights, top-k selection restricted to causally
+ * visible blocks, Eqs 13-17).
+ *   q_idx      device [B, n_heads, head_dim] bf16 indexer queries
+ *   w_idx      device [B, n_heads] f32 head weights
+ *   k_idx      device [B, max_blocks, head_dim] bf16 compressed indexer keys
+ *              (e.g. lbca_pool_dual of the indexer key series, LBCA_VALUE)
+ *   seq_lens   device [B] tokens the query sees (L); blocks j < floor(L /
+ *              block_m), capped at max_blocks, are visible
+ *   sel        device [B, top_k] int32 out: the selected block indices in
+ *              increasing order (equal relevances: lower index first), then
+ *              -1 where fewer than top_k blocks are visible
+ *   sel_scores device [B, top_k] f32 out (nullable): their relevances
+ *   workspace  device, >= lbca_indexer_workspace_bytes(B, max_blocks) bytes
+ * Relevance of block j: I_j = sum_h w_h ReLU(q_h . k_j) (f32 accumulation of
+ * exact bf16 products on the tensor cores).  Shapes: n_heads 32, 64 or 128;
+ * head_dim 64 or 128 (else LBCA_ERR_UNSUPPORTED).
+ */
+LBCA_API size_t lbca_indexer_workspace_bytes(int32_t batch, int32_t max_blocks);
+LBCA_API lbca_status lbca_indexer_topk(int32_t batch, int32_t n_heads, int32_t head_dim, int32_t block_m,
+                                       int32_t top_k, const void* q_idx, const float* w_idx, const void* k_idx,
+                                       int32_t max_blocks, const int32_t* seq_lens, int32_t* sel,
+                                       float* sel_scores, void* workspace, size_t workspace_bytes,
+                                       int32_t* d_status, lbca_stream_t stream);
 
 /* Static text for a status code. */
 LBCA_API const char* lbca_status_string(lbca_status status);

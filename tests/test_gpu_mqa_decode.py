@@ -148,3 +148,18 @@ def test_entry_beyond_fp16_range_sets_status(L):
     run.step()
     torch.cuda.synchronize()
     assert int(run.status.item()) == L.LBCA_ERR_UNSUPPORTED
+
+
+def test_step_full_size_sampled(L):
+    """lbca_decode_step in its fused tensor-core form (the launch the HCA bench
+    times) at the full 8 x 128K size: two steps, outputs of sampled sequences
+    against the oracle."""
+    w = synth.scaled(W, steps=2)
+    inp = synth.make(w)
+    run = DecodeRun(L, w, inp, steps=2)
+    assert L.lbca_decode_step_form(run.cfg, run.B, run.max_ctx) == L.LBCA_STEP_SHARED_TC
+    for s in range(2):
+        got = fused_step(run)
+    torch.cuda.synchronize()
+    assert_close(f64(got)[[0, 3, 7]], oracle_decode(w, inp, 1, [0, 3, 7]), "bf16", "hca step full size")
+    assert int(run.status.item()) == 0

@@ -60,3 +60,58 @@ def test_step_full_size(L):
         got = fused_step(run)
     torch.cuda.synchronize()
     assert_close(f64(got), oracle_decode(w, inp, 2), "bf16", "step full")
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("gqa_decode_32k", dict(ctx=(1000, 1000))),                                  # cluster step
+    ("hca_mqa_decode_128k", dict(ctx=(700, 700), batch=2)),                      # tensor-core shared-entry step
+])
+@pytest.mark.parametrize("graph", [False, True], ids=["eager", "graph"])
+def test_overlap_flag_changes_nothing_but_timing(L, name, kw, graph):
+    """A chain of three layers, each with its own cache, each layer's query the
+    previous layer's output (so every step depends on the kernel before it):
+    with the caches flagged LBCA_CACHE_OVERLAP_PREV the steps launch with
+    programmatic dependence and read their caches while the previous kernel
+    drains; outputs and caches must be bit-identical to the unflagged chain."""
+    NL, steps = 3, 5
+    w = synth.scaled(W[name], steps=steps, **kw)
+    inp = synth.make(w)
+    runs = {f: [DecodeRun(L, w, inp, steps=steps) for _ in range(NL)] for f in (0, L.LBCA_CACHE_OVERLAP_PREV)}
+    outs = {}
+    for flags, chain in runs.items():
+        for run in chain:
+            run.cache.flags = flags
+            run.step_ws = torch.zeros(max(L.lbca_decode_step_workspace_bytes(run.cfg, run.B, run.max_ctx), 16),
+                                      dtype=torch.uint8, device="cuda")
+        o = [[torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda") for _ in range(NL)]
+             for _ in range(steps)]
+
+        def token(s):
+            q = chain[0].q[s]
+            for layer, run in enumerate(chain):
+                L.lbca_decode_step(run.cfg, run.token(run.k), run.token(run.v), run.token(run.zk),
+                                   run.token(run.zv), run.bpk, run.bpv, None, q, run.cache, run.sink, None,
+                                   o[s][layer], run.step_ws, run.max_ctx, run.status)
+                q = o[s][layer]
+            for run in chain:
+                run.pos += 1
+
+        if graph and flags:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for s in range(steps):
+                    token(s)
+            gr.replay()
+        else:
+            for s in range(steps):
+                token(s)
+        torch.cuda.synchronize()
+        outs[flags] = o
+    for s in range(steps):
+        for layer in range(NL):
+            assert torch.equal(outs[0][s][layer], outs[L.LBCA_CACHE_OVERLAP_PREV][s][layer]), (s, layer)
+    for a, b in zip(runs[0], runs[L.LBCA_CACHE_OVERLAP_PREV]):
+        for f in ("pooled_k", "pooled_v", "ring_k", "ring_v", "pool_state", "seq_lens"):
+            x, y = getattr(a.cache, f), getattr(b.cache, f)
+            assert (x is None and y is None) or torch.equal(x, y), f
+        assert int(a.status.item()) == 0 and int(b.status.item()) == 0

@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--workload", default="ragged_gqa_decode_append",
                     help="the decode workload of the headline line (default: the largest single-GPU one)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--leg", default="decode", choices=["decode", "prefill", "pool"],
+    ap.add_argument("--leg", default="decode", choices=["decode", "prefill", "pool", "csa", "backward", "chain"],
                     help="decode: the decode-step benchmark (default, with the other decode workloads, the "
                          "prefill and the pool legs appended under 'also' at one GPU); prefill / pool: that leg "
                          "alone (one JSON line)")
@@ -236,7 +236,7 @@ def run_ours(args, w, rank, world, reps=3):
     K, W = args.steps, args.warmup
     # steps each replica must hold: warm-up, reps graph replays, decode-only
     # timing of a two-launch step, e2e warm-up and steps
-    bench = DecodeBench(w, rank, W + reps * K + (W + K) + (W + K))
+    bench = DecodeBench(w, rank, W + 2 * reps * K + (W + K) + (W + K))
     L = bench.L
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     cap = torch.cuda.Stream()
@@ -254,30 +254,42 @@ def run_ours(args, w, rank, world, reps=3):
         bench.i += 1
     torch.cuda.synchronize()
     nbytes = sum(bytes_per_decode(bench.w, bench.lens_at(i)) for i in range(bench.i, bench.i + K))
-    g_main = graph_of(bench.i, K, bench.launch)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
     uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
-    times = []
-    for _ in range(reps):  # each replay appends K more tokens per replica: the cache holds them
-        e0, e1 = E(), E()
+    # Consecutive steps run on different cache replicas (as a model's layers
+    # follow each other), which is the contract of LBCA_CACHE_OVERLAP_PREV:
+    # timed with the replicas flagged (each step starts and reads its cache
+    # while the previous one drains) and without.
+    medians = {}
+    for flags in (L.LBCA_CACHE_OVERLAP_PREV, 0):
+        for c in bench.caches:
+            c.flags = flags
+        g_main = graph_of(bench.i, K, bench.launch)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        e0.record()
-        g_main.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        times.append(e0.elapsed_time(e1) / K)
-    step_ms = statistics.median(times)
+        times = []
+        for _ in range(reps):  # each replay appends K more tokens per replica: the cache holds them
+            e0, e1 = E(), E()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            e0.record()
+            g_main.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            times.append(e0.elapsed_time(e1) / K)
+        medians[flags] = statistics.median(times)
+        del g_main
+    for c in bench.caches:
+        c.flags = 0
+    step_ms = medians[L.LBCA_CACHE_OVERLAP_PREV]
+    serial_ms = medians[0]
     bench.i += K
-    del g_main
     kernel_ms = step_ms  # one fused kernel per step: the step is the kernel
     if bench.launches == 2:
         # append + decode: time the decode launches alone (same replicas, same rotation)
@@ -298,14 +310,16 @@ def run_ours(args, w, rank, world, reps=3):
     if status:
         raise RuntimeError(f"device status {L.lbca_status_string(status)}")
 
-    step_ms, e2e_ms, kernel_ms = ranks.max_over_ranks([step_ms, e2e_ms, kernel_ms], device="cuda")
+    step_ms, e2e_ms, kernel_ms, serial_ms = ranks.max_over_ranks([step_ms, e2e_ms, kernel_ms, serial_ms],
+                                                                 device="cuda")
     hbm, src = peaks()
     achieved = nbytes / K / (kernel_ms * 1e-3) / 1e9
     w_ = bench.w
     line = {
         "metric": METRIC, "value": ranks.job_us_per_token(step_ms, bench.B, world), "unit": "µs/token",
         "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": step_ms, "higher_is_better": False,
+        "steps": K, "warmup": W, "ms_per_step": step_ms, "serial_ms_per_step": serial_ms,
+        "serial_value": ranks.job_us_per_token(serial_ms, bench.B, world), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": w_.dtype, "data": "synthetic",
         "config": {"workload": w_.name, "batch_per_gpu": w_.batch, "context": [int(w_.ctx[0]), int(w_.ctx[1])],
                    "n_q_heads": w_.n_q_heads, "n_kv_heads": w_.n_kv_heads, "head_dim": w_.head_dim,
@@ -315,7 +329,10 @@ def run_ours(args, w, rank, world, reps=3):
                           f"(>= 3x L2 of data in total), each step's data cold"),
                    "launch": (f"K steps of lbca_decode_step ({bench.launches} kernel launch"
                               f"{'es' if bench.launches > 1 else ''} each), back to back from one CUDA graph, "
-                              f"median of {reps} replays; e2e: an eager host loop of lbca_decode_step calls "
+                              f"median of {reps} replays, the replicas flagged LBCA_CACHE_OVERLAP_PREV (each step "
+                              "reads its cache while the previous step, on another replica, drains); "
+                              "serial_value: the same graph without the flag; "
+                              "e2e: an eager host loop of lbca_decode_step calls "
                               "(host-side validation and launch every step), each step's inputs uploaded from "
                               "pinned host memory and its output read back on copy streams beside the kernels, "
                               "timed as the longer of the device events and the host wall clock")},
@@ -526,6 +543,41 @@ def prefill_leg(name="gqa_prefill_16k", reps=10, warm=3, baseline=True):
     if baseline:
         line["cpu_baseline"] = oracle_prefill_timing(w, inp)
     return line
+
+
+def backward_leg(T=2048, reps=5, warm=2):
+    """lbca_prefill_backward of a T-token GQA layer (the 16K prefill layer's
+    shapes, m = 16): all gradients in f32 on the CUDA cores.  Algorithmic
+    flops: 10 D Hq per visible (query, entry) pair (the scores recomputed, and
+    the products giving dP, dQ, dK and dV)."""
+    import torch
+
+    from block_compressed_long_b200 import lbca as L
+    from block_compressed_long_b200 import synth
+    w = synth.scaled(synth.WORKLOADS["gqa_prefill_16k"], seq_len=T)
+    inp = synth.make(w)
+    cfg = L.config(w.n_q_heads, w.n_kv_heads, w.head_dim, w.shared_kv, w.block_m, w.n_win, w.rope_dims,
+                   w.rmsnorm, w.rope_theta, dtype=w.dtype)
+    d = lambda t: None if t is None else t.cuda()  # noqa: E731
+    q, k, v, zk, zv, bpk, bpv = (d(t) for t in (inp.q, inp.k, inp.v, inp.zk, inp.zv, inp.bpos_k, inp.bpos_v))
+    dout = d(synth.normal(w.seed, "dout", tuple(inp.q.shape), dtype=w.dtype))
+    f = lambda *sh: torch.empty(*sh, dtype=torch.float32, device="cuda")  # noqa: E731
+    G, D, m = w.n_kv_heads, w.head_dim, w.block_m
+    grads = {"dq": f(*q.shape), "dk": f(*k.shape), "dv": f(*k.shape), "dzk": f(*k.shape), "dzv": f(*k.shape),
+             "dbk": f(m, G * D), "dbv": f(m, G * D)}
+    ws = torch.zeros(L.lbca_prefill_backward_workspace_bytes(cfg, w.batch, T), dtype=torch.uint8, device="cuda")
+    uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    ms, clocks = timed(lambda: L.lbca_prefill_backward(cfg, q, k, v, zk, zv, bpk, bpv, None, None, None, dout, grads,
+                                                       ws), reps, warm, uuid)
+    fl = 2.5 * prefill_flops(w)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": f"gqa_prefill_16k shapes, T = {T}: prefill backward", "metric": "backward TFLOP/s",
+            "value": tf, "unit": "TFLOP/s", "ms_per_call": ms, "dtype": "bf16 inputs, f32 arithmetic and gradients",
+            "roofline": {"bound": "alu", "achieved": tf, "peak": F32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tf / F32_ALU_TFLOPS, "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+                         "flops_per_call": fl,
+                         "kernel": "pool_fwd, finalise, row_lse, dq, dkv, key_bwd, pool_bwd kernels (call timed)"},
+            "clocks": clocks}
 
 
 POOL_CASES = {
@@ -1035,8 +1087,14 @@ def main():
         if rank == 0:
             if args.leg == "prefill":
                 out = prefill_leg(args.prefill, reps=args.steps, warm=args.warmup, baseline=False)
-            else:
+            elif args.leg == "pool":
                 out = pool_leg(args.pool, reps=args.steps, warm=args.warmup, baseline=False)
+            elif args.leg == "csa":
+                out = csa_leg(K=args.steps, W=args.warmup)
+            elif args.leg == "backward":
+                out = backward_leg(reps=args.steps, warm=args.warmup)
+            else:
+                out = layer_chain_leg(K=args.steps, W=args.warmup)
             print(json.dumps(out), flush=True)
         return
     line, bench = run_ours(args, w, rank, world)
@@ -1046,7 +1104,7 @@ def main():
         gc.collect()
         torch.cuda.empty_cache()
         also = [decode_also(args, n) for n in ("gqa_decode_32k", "hca_mqa_decode_128k") if n != w.name]
-        also += [layer_chain_leg(), csa_leg()]
+        also += [layer_chain_leg(), csa_leg(), backward_leg()]
         also += [prefill_leg("gqa_prefill_16k"), prefill_leg("tiny_f32_prefill")]
         also += [pool_leg(label) for label in POOL_CASES]
         line["also"] = also

@@ -356,7 +356,7 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
     a.w = cfg->n_win; a.rho = cfg->rope_dims; a.rmsnorm = cfg->rmsnorm; a.shared = cfg->shared_kv;
     a.max_blocks = cache->max_blocks; a.R = cache->ring_slots; a.S = cfg->shared_kv ? 1 : 2;
     a.CS = sp.CS; a.SE = sp.SE; a.heads_per_cta = sp.heads_per_cta;
-    a.pdl = (cache->flags & LBCA_CACHE_OVERLAP_PREV) != 0 && !sp.flat;
+    a.pdl = (cache->flags & LBCA_CACHE_OVERLAP_PREV) != 0;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
     if (sp.flat) {
         for (int kk = 0; kk < cfg->rope_dims / 2 && kk < 128; ++kk) a.rope_f[kk] = rope_turns(kk, a.rope_step);  // workspace: [arrival counter][segment counters][partial max, sum][partial outputs]

@@ -131,9 +131,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         fence_barrier_init();
     }
     __syncthreads();
-    // arrival ticket: taken now, looked at only at the end (its latency hides behind the work)
+    // arrival ticket: taken once the step's inputs may be read (below), looked at
+    // only at the end (its latency hides behind the work)
     unsigned int ticket = 0u;
-    if (tid == 0) ticket = atomicAdd(a.arrive, 1u);
     // exclusive prefix of the step's entries per sequence (HG segments of nvis each)
     {
         const int per = (B + kThreads - 1) / kThreads;
@@ -264,6 +264,15 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
     };
 
     const bool pair_owner = tid < D / 2;
+
+    // Everything above reads only this cache.  Launched with programmatic
+    // dependence on the preceding kernel, the first pieces' copies go out now,
+    // while that kernel drains; otherwise after the first append's few loads
+    // (ahead of the copies in the memory queues).  The step's own inputs (the
+    // new tokens, the queries) and the workspace are touched only after the wait.
+    if (a.pdl) issue_first();
+    griddep_wait();
+    if (tid == 0) ticket = atomicAdd(a.arrive, 1u);
 
     // ---- appends of (sequence, kv head) pairs c, c + N, ... while the copies land ----
     const int kp = pair_owner && a.rho && 2 * tid >= D - a.rho ? (2 * tid - (D - a.rho)) >> 1 : -1;  // RoPE pair
@@ -669,6 +678,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         advance(cur, n);
         ++k;
     }
+    griddep_launch_dependents();  // the next kernel on the stream may start its cache reads
     if (seg_cur >= 0) finish();
     // ---- the last CTA to have read the lengths advances them ----
     if (tid == 0) flags[0] = ticket == gridDim.x - 1;
@@ -698,8 +708,17 @@ template <typename T, int D, int R>
 cudaError_t launch_flat_one(const StepArgs& a, size_t smem, cudaStream_t s) {
     cudaError_t e = flat_attr<T, D, R>();
     if (e != cudaSuccess) return e;
-    decode_flat_kernel<T, D, R><<<a.grid, kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(a.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_flat_kernel<T, D, R>, a);
 }
 // Persistent grid: every SM filled with as many CTAs as fit (cached per device and shape).
 template <typename T, int D, int R>

@@ -195,9 +195,16 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
         __syncthreads();
         const uint32_t prefix = sh_prefix;
-        for (int i = i0; i < i1; ++i) {
+        // strided (coalesced) reads; the lanes of a warp that fall in the same
+        // bin add once (relevances share their top byte: per-element atomics
+        // on one bin would serialise)
+        for (int i = tid; i < nvis; i += kSelThreads) {
             const uint32_t k = order_key(sc[i]);
-            if (pass == 0 || (k >> (shift + 8)) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            const bool in = pass == 0 || (k >> (shift + 8)) == prefix;
+            const uint32_t bin = (k >> shift) & 255u;
+            const unsigned act = __activemask();
+            const unsigned peers = __match_any_sync(act, in ? bin : 256u + (threadIdx.x & 31));
+            if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
         }
         __syncthreads();
         if (tid == 0) {

@@ -97,7 +97,7 @@ _lib.lbca_indexer_topk.argtypes = [_i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, 
 _lib.lbca_indexer_topk.restype = ctypes.c_int
 _lib.lbca_prefill_backward_workspace_bytes.argtypes = [_CP, _i32, _i32]
 _lib.lbca_prefill_backward_workspace_bytes.restype = _sz
-_lib.lbca_prefill_backward.argtypes = [_CP] + [_vp] * 12 + [_i32, _i32] + [_vp] * 9 + [_sz, _vp]
+_lib.lbca_prefill_backward.argtypes = [_CP] + [_vp] * 11 + [_i32, _i32] + [_vp] * 9 + [_sz, _vp]
 _lib.lbca_prefill_backward.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
 _lib.lbca_status_string.restype = ctypes.c_char_p

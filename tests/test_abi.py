@@ -167,3 +167,46 @@ def test_shared_entry_step_forms(L):
 def test_status_strings(L):
     for s in range(7):
         assert L.lbca_status_string(s)
+
+
+def test_every_binding_wrapper_reaches_the_library(L):
+    """Each Python wrapper marshals its arguments into the C entry point it
+    names: called with host tensors (no GPU here) it must come back with a
+    library status, never with a ctypes arity or type error."""
+    import torch
+    cfg = L.config(4, 2, 32, False, 4, 8, rope_dims=8)
+    hca = L.config(64, 1, 256, True, 4, 8, rope_dims=8, rmsnorm=True)
+    q = torch.zeros(1, 8, 4, 32)
+    kv = torch.zeros(1, 8, 2, 32)
+    tok = torch.zeros(1, 2, 32)
+    bp = torch.zeros(4, 64)
+    q1 = torch.zeros(1, 4, 32)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    st = torch.zeros(1, dtype=torch.int32)
+    cache = L.Cache(cfg, 1, 2, L.lbca_ring_slots(cfg), torch.zeros(1, 2, 2, 32), torch.zeros(1, 2, 2, 32),
+                    torch.zeros(1, 2, 12, 32), torch.zeros(1, 2, 12, 32), torch.zeros(L.lbca_pool_state_elems(cfg, 1)),
+                    torch.zeros(1, dtype=torch.int32))
+    hcache = L.Cache(hca, 1, 2, L.lbca_ring_slots(hca), torch.zeros(1, 1, 2, 256), None, torch.zeros(1, 1, 12, 256),
+                     None, torch.zeros(L.lbca_pool_state_elems(hca, 1)), torch.zeros(1, dtype=torch.int32))
+    grads = {n: torch.zeros(1) for n in ("dq", "dk", "dv", "dzk", "dzv", "dbk", "dbv")}
+    bws = torch.zeros(L.lbca_prefill_backward_workspace_bytes(cfg, 1, 8), dtype=torch.uint8)
+    calls = [
+        lambda: L.lbca_pool(cfg, 0, kv, kv, bp, None, torch.zeros(1, 2, 2, 32)),
+        lambda: L.lbca_pool_dual(cfg, 0, kv, kv, kv, kv, bp, bp, None, torch.zeros(1, 2, 2, 32)),
+        lambda: L.lbca_append(cfg, tok, tok, tok, tok, bp, bp, None, cache, st),
+        lambda: L.lbca_decode(cfg, q1, cache, None, None, None, torch.zeros_like(q1), ws, 8, st),
+        lambda: L.lbca_decode_noalloc(cfg, q1, cache, None, None, None, torch.zeros_like(q1), 8, st),
+        lambda: L.lbca_decode_step(cfg, tok, tok, tok, tok, bp, bp, None, q1, cache, None, None,
+                                   torch.zeros_like(q1), ws, 8, st),
+        lambda: L.lbca_prefill(cfg, q, kv, kv, kv, kv, bp, bp, None, None, None, torch.zeros_like(q), None, ws),
+        lambda: L.lbca_prefill_backward(cfg, q, kv, kv, kv, kv, bp, bp, None, None, None, q, grads, bws),
+        lambda: L.lbca_decode_sparse(hca, torch.zeros(1, 64, 256), hcache, torch.zeros(1, 4, dtype=torch.int32),
+                                     None, None, None, torch.zeros(1, 64, 256), st),
+        lambda: L.lbca_indexer_topk(torch.zeros(1, 64, 128), torch.zeros(1, 64), torch.zeros(1, 16, 128),
+                                    torch.zeros(1, dtype=torch.int32), 4, torch.zeros(1, 4, dtype=torch.int32), None,
+                                    torch.zeros(256, dtype=torch.uint8), st),
+        lambda: L.lbca_selftest_bounded_wait(False, 1000, st),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(L.LbcaError):
+            call()

@@ -65,6 +65,7 @@ def test_step_full_size(L):
 @pytest.mark.parametrize("name,kw", [
     ("gqa_decode_32k", dict(ctx=(1000, 1000))),                                  # cluster step
     ("hca_mqa_decode_128k", dict(ctx=(700, 700), batch=2)),                      # tensor-core shared-entry step
+    ("ragged_gqa_decode_append", dict(ctx=(50, 900), batch=16)),                 # persistent step
 ])
 @pytest.mark.parametrize("graph", [False, True], ids=["eager", "graph"])
 def test_overlap_flag_changes_nothing_but_timing(L, name, kw, graph):

@@ -187,21 +187,27 @@ size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32
     return bytes;
 }
 
-lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
-                      const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
-                      void* out, int32_t out_blocks, lbca_stream_t stream) {
+// One series pooled into `out` (the I/O dtype) or `out_f32` (f32 entries).
+static lbca_status pool_single(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                               const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
+                               void* out, float* out_f32, int32_t out_blocks, lbca_stream_t stream) {
     LBCA_TRY(check_cfg(cfg));
+    if (!out && !out_f32) return LBCA_ERR_ARG;
     if (series != LBCA_KEY && series != LBCA_VALUE) return LBCA_ERR_ARG;
     if (cfg->shared_kv && series != LBCA_KEY) return LBCA_ERR_ARG;
-    if (!x || !z || !b_pos || !out) return LBCA_ERR_ARG;
+    if (!x || !z || !b_pos) return LBCA_ERR_ARG;
     if (batch < 0 || T < 0 || pos0 < 0 || pos0 % cfg->block_m || out_blocks < 0) return LBCA_ERR_ARG;
     if ((long long)pos0 / cfg->block_m + T / cfg->block_m > out_blocks) return LBCA_ERR_ARG;
-    if (!al16(x) || !al16(z) || !al16(b_pos) || !al16(out) || !al16n(gamma)) return LBCA_ERR_ALIGN;
+    if (!al16(x) || !al16(z) || !al16(b_pos) || !al16n(out) || !al16n(out_f32) || !al16n(gamma))
+        return LBCA_ERR_ALIGN;
     LBCA_TRY(check_device());
     PoolArgs a{};
     a.dtype = cfg->dtype;
     a.nser = 1;
-    a.ser[0].x = x; a.ser[0].z = z; a.ser[0].bpos = b_pos; a.ser[0].gamma = gamma; a.ser[0].out = out;
+    a.ser[0].x = x; a.ser[0].z = z; a.ser[0].bpos = b_pos; a.ser[0].gamma = gamma;
+    // f32 I/O: the entries are f32 already
+    a.ser[0].out = out ? out : (cfg->dtype == LBCA_F32 ? out_f32 : nullptr);
+    a.ser[0].out_f32 = cfg->dtype == LBCA_F32 ? nullptr : out_f32;
     a.ser[0].key = series == LBCA_KEY; a.ser[0].state_series = 0;
     a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
     a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
@@ -210,6 +216,20 @@ lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, con
     a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
     a.state = nullptr; a.S = 1;
     return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                      const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
+                      void* out, int32_t out_blocks, lbca_stream_t stream) {
+    if (!out) return LBCA_ERR_ARG;
+    return pool_single(cfg, series, x, z, b_pos, gamma, batch, T, pos0, out, nullptr, out_blocks, stream);
+}
+
+lbca_status lbca_pool_f32(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                          const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
+                          float* out, int32_t out_blocks, lbca_stream_t stream) {
+    if (!out) return LBCA_ERR_ARG;
+    return pool_single(cfg, series, x, z, b_pos, gamma, batch, T, pos0, nullptr, out, out_blocks, stream);
 }
 
 lbca_status lbca_pool_dual(const lbca_config* cfg, int32_t series, const void* xa, const void* za, const void* xb,
@@ -424,6 +444,7 @@ lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const void* k, c
     pa.B = batch; pa.T = T; pa.Hq = cfg->n_q_heads; pa.G = cfg->n_kv_heads; pa.D = cfg->head_dim;
     pa.m = m; pa.w = cfg->n_win; pa.rho = cfg->rope_dims; pa.rmsnorm = cfg->rmsnorm;
     pa.shared = cfg->shared_kv; pa.eps = cfg->rms_eps; pa.scale = scale_of(cfg); pa.rope_step = rope_step_of(cfg);
+    pa.t_off = 0; pa.s_off = 0; pa.T_raw = T;
     // the tensor-core path: cos/sin table first, so that the pool pass can leave
     // fp16 copies of the raw keys (rotated) and values as it streams them
     if (use_tc) LBCA_TRY(cuda_status(launch_prefill_tc_table(pa, tc_scratch, s)));
@@ -624,6 +645,37 @@ lbca_status lbca_prefill_backward(const lbca_config* cfg, const void* q, const v
         return LBCA_ERR_CUDA;
     if (sink && cudaMemsetAsync(dsink, 0, (size_t)a.Hq * 4, s) != cudaSuccess) return LBCA_ERR_CUDA;
     return cuda_status(launch_backward(a, s));
+}
+
+lbca_status lbca_prefill_rows(const lbca_config* cfg, const void* q, int32_t row0, int32_t n_rows, const void* k,
+                              const void* v, int32_t raw0, int32_t n_raw, const float* pooled_k, const float* pooled_v,
+                              int32_t pool_stride, const float* sink, const void* gamma_q, const void* gamma_kv,
+                              int32_t batch, void* out, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    if (batch < 0 || n_rows < 0 || n_raw < 0 || row0 < 0 || raw0 < 0 || pool_stride < 0) return LBCA_ERR_ARG;
+    if (batch == 0 || n_rows == 0) return LBCA_OK;
+    if (!q || !out || !k || (!cfg->shared_kv && !v) || (cfg->shared_kv && (v || pooled_v))) return LBCA_ERR_ARG;
+    const int m = cfg->block_m, w = cfg->n_win;
+    const long long last = (long long)row0 + n_rows;   // one past the last row
+    const long long Plast = last - w > 0 ? (last - w) / m : 0;
+    const long long Pfirst = (long long)row0 + 1 - w > 0 ? ((long long)row0 + 1 - w) / m : 0;
+    // the raw rows must end at the last query and reach back to the first row's window
+    if ((long long)raw0 + n_raw != last || raw0 > Pfirst * m) return LBCA_ERR_ARG;
+    if (Plast > pool_stride || (Plast > 0 && (!pooled_k || (!cfg->shared_kv && !pooled_v)))) return LBCA_ERR_ARG;
+    if (!al16(q) || !al16(out) || !al16(k) || !al16n(v) || !al16n(pooled_k) || !al16n(pooled_v) || !al16n(sink) ||
+        !al16n(gamma_q) || !al16n(gamma_kv))
+        return LBCA_ERR_ALIGN;
+    if (!prefill_simt_supported(cfg->head_dim)) return LBCA_ERR_UNSUPPORTED;
+    LBCA_TRY(check_device());
+    PrefillArgs pa{};
+    pa.dtype = cfg->dtype;
+    pa.q = q; pa.k = k; pa.v = v; pa.pooled_k = pooled_k; pa.pooled_v = cfg->shared_kv ? pooled_k : pooled_v;
+    pa.pool_stride = pool_stride; pa.pooled_f32 = 1; pa.sink = sink; pa.gamma_q = gamma_q; pa.gamma_kv = gamma_kv; pa.out = out;
+    pa.B = batch; pa.T = n_rows; pa.Hq = cfg->n_q_heads; pa.G = cfg->n_kv_heads; pa.D = cfg->head_dim;
+    pa.m = m; pa.w = w; pa.rho = cfg->rope_dims; pa.rmsnorm = cfg->rmsnorm; pa.shared = cfg->shared_kv;
+    pa.eps = cfg->rms_eps; pa.scale = scale_of(cfg); pa.rope_step = rope_step_of(cfg);
+    pa.t_off = row0; pa.s_off = raw0; pa.T_raw = n_raw;
+    return cuda_status(launch_prefill_simt(pa, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t lbca_indexer_workspace_bytes(int32_t batch, int32_t max_blocks) {

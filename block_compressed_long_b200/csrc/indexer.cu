@@ -18,9 +18,9 @@
 //   the tile and the queries are staged with 16-byte cp.async into
 //   128-byte-swizzled shared memory, so each key crosses HBM once.  Several
 //   CTAs per SM overlap one tile's copies with another's MMA and epilogue.
-//   Top-k: one CTA per sequence selects the k largest relevances by a radix
-//   select over order-preserving 32-bit keys (four 8-bit passes with a
-//   shared-memory histogram), then writes the selected block indices in
+//   Top-k: one CTA per sequence holds the relevances in registers as
+//   order-preserving 32-bit keys and finds the k-th largest one bit at a time
+//   (CTA-wide counts, no atomics), then writes the selected block indices in
 //   increasing index order (equal relevances: lower index first) followed by
 //   -1 padding when fewer than k blocks are visible.
 #include <algorithm>
@@ -134,9 +134,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kKeysPerThread = 32;  // keys held in registers: up to 32768 visible blocks
 
-// Exclusive prefix sum over the CTA of one value per thread; *total gets the sum.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+// Inclusive prefix sum over the CTA of one value per thread (thread order);
+// warp_sums is kSelWarps ints of shared memory.  Every thread must call it.
+__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_sums) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -147,26 +150,39 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = lane < kSelThreads / 32 ? warp_sums[lane] : 0;
+        int w = warp_sums[lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) w += y;
         }
-        warp_sums[lane] = w;  // inclusive over warps
+        warp_sums[lane] = w;
     }
     __syncthreads();
-    const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
-    *total = warp_sums[kSelThreads / 32 - 1];
-    __syncthreads();
-    return before;
+    const int r = x + (warp > 0 ? warp_sums[warp - 1] : 0);
+    __syncthreads();  // warp_sums may be reused
+    return r;
 }
 
+// Sum over the CTA of one count per thread (every thread gets the total).
+__device__ __forceinline__ int block_count(int c, int* warp_sums) {
+    const int w = __reduce_add_sync(0xffffffffu, c);
+    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = w;
+    __syncthreads();
+    const int total = __reduce_add_sync(0xffffffffu, warp_sums[threadIdx.x & 31]);
+    __syncthreads();  // warp_sums may be reused
+    return total;
+}
+
+// One CTA per sequence.  The visible relevances are read once into registers
+// as order-preserving keys (thread t holds blocks t, t + 1024, ...).  The k-th
+// largest key is found one bit at a time, most significant first: a bit is
+// kept when at least k keys are >= the prefix with that bit set (32 rounds of
+// a compare per key and one CTA-wide count, no atomics).  The selection then
+// walks the keys in block order, one block scan per register slot: every key
+// above the threshold, and the first of those equal to it until k are taken.
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) {
-    __shared__ uint32_t hist[256];
-    __shared__ int warp_sums[32];
-    __shared__ uint32_t sh_prefix;
-    __shared__ int sh_krem, sh_gt;
+    __shared__ int warp_sums[kSelWarps];
     const int b = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int nvis = min(max(L, 0) / a.m, a.max_blocks);
@@ -174,8 +190,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
     const float* sc = a.scores + (size_t)b * a.max_blocks;
     int32_t* sel = a.sel + (size_t)b * K;
     float* selv = a.sel_scores ? a.sel_scores + (size_t)b * K : nullptr;
-    const int chunk = (nvis + kSelThreads - 1) / kSelThreads;  // contiguous indices per thread
-    const int i0 = tid * chunk, i1 = min(nvis, i0 + chunk);
 
     if (nvis <= K) {  // every visible block is selected
         for (int i = tid; i < K; i += kSelThreads) {
@@ -184,69 +198,53 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         }
         return;
     }
-    // ---- radix select of the K-th largest key, 8 bits per pass, most significant first ----
-    if (tid == 0) {
-        sh_prefix = 0u;
-        sh_krem = K;
-        sh_gt = 0;
+    if (nvis > kSelThreads * kKeysPerThread) {  // beyond the register capacity (the host sizes forbid it)
+        if (tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
+        for (int i = tid; i < K; i += kSelThreads) sel[i] = -1;
+        return;
     }
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
-        __syncthreads();
-        const uint32_t prefix = sh_prefix;
-        // strided (coalesced) reads; the lanes of a warp that fall in the same
-        // bin add once (relevances share their top byte: per-element atomics
-        // on one bin would serialise)
-        for (int i = tid; i < nvis; i += kSelThreads) {
-            const uint32_t k = order_key(sc[i]);
-            const bool in = pass == 0 || (k >> (shift + 8)) == prefix;
-            const uint32_t bin = (k >> shift) & 255u;
-            const unsigned act = __activemask();
-            const unsigned peers = __match_any_sync(act, in ? bin : 256u + (threadIdx.x & 31));
-            if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    const int slots = (nvis + kSelThreads - 1) / kSelThreads;  // uniform
+    uint32_t key[kKeysPerThread];
+#pragma unroll
+    for (int s = 0; s < kKeysPerThread; ++s) {
+        const int i = tid + s * kSelThreads;
+        key[s] = (s < slots && i < nvis) ? order_key(sc[i]) : 0u;  // 0: below every real key
+    }
+    // ---- the k-th largest key, bit by bit ----
+    uint32_t thr = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = thr | (1u << bit);
+        int c = 0;
+#pragma unroll
+        for (int s = 0; s < kKeysPerThread; ++s)
+            if (s < slots) c += key[s] >= cand;
+        if (block_count(c, warp_sums) >= K) thr = cand;
+    }
+    int c_gt = 0;
+#pragma unroll
+    for (int s = 0; s < kKeysPerThread; ++s)
+        if (s < slots) c_gt += key[s] > thr;
+    const int ties_needed = K - block_count(c_gt, warp_sums);
+    // ---- selection in block order: every key above thr, the first ties_needed equal to it ----
+    int pos_base = 0, tie_base = 0;
+#pragma unroll
+    for (int s = 0; s < kKeysPerThread; ++s) {
+        if (s >= slots) break;  // uniform
+        const int i = tid + s * kSelThreads;
+        const bool valid = i < nvis;
+        const bool gt = valid && key[s] > thr, tie = valid && key[s] == thr;
+        const int tie_incl = block_inclusive_scan(tie ? 1 : 0, warp_sums);
+        const bool take = gt || (tie && tie_base + tie_incl - 1 < ties_needed);
+        const int pos_incl = block_inclusive_scan(take ? 1 : 0, warp_sums);
+        if (take && pos_base + pos_incl - 1 < K) {
+            sel[pos_base + pos_incl - 1] = i;
+            if (selv) selv[pos_base + pos_incl - 1] = sc[i];
         }
-        __syncthreads();
-        if (tid == 0) {
-            int need = sh_krem, above = 0, d = 255;
-            for (; d > 0; --d) {
-                if (above + (int)hist[d] >= need) break;
-                above += (int)hist[d];
-            }
-            sh_prefix = (prefix << 8) | (uint32_t)d;
-            sh_krem = need - above;
-            sh_gt += above;
-        }
-        __syncthreads();
+        tie_base += block_count(tie ? 1 : 0, warp_sums);
+        pos_base += block_count(take ? 1 : 0, warp_sums);
     }
-    const uint32_t thr = sh_prefix;  // the K-th largest key
-    const int ties_needed = sh_krem;
-    // ---- selection in index order: every key above thr, and the first ties_needed equal to it ----
-    int my_gt = 0, my_tie = 0;
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t k = order_key(sc[i]);
-        my_gt += k > thr;
-        my_tie += k == thr;
-    }
-    int total;
-    const int tie_before = block_exclusive_scan(my_tie, warp_sums, &total);
-    const int my_take = my_gt + max(0, min(my_tie, ties_needed - tie_before));
-    const int pos0 = block_exclusive_scan(my_take, warp_sums, &total);
-    int pos = pos0, tie_rank = tie_before;
-    for (int i = i0; i < i1; ++i) {
-        const float f = sc[i];
-        const uint32_t k = order_key(f);
-        bool take = k > thr;
-        if (k == thr) take = tie_rank++ < ties_needed;
-        if (take) {
-            if (pos < K) {
-                sel[pos] = i;
-                if (selv) selv[pos] = f;
-            }
-            ++pos;
-        }
-    }
-    if (tid == 0 && total != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
+    if (tid == 0 && pos_base != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
 }
 
 template <int DI, int HI>

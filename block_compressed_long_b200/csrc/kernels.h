@@ -14,7 +14,8 @@ struct PoolSeries {
     const void* z;         // [B, T, G, D]
     const void* bpos;      // [m, G*D]
     const void* gamma;     // [D] or null (key series with RMSNorm)
-    void* out;             // [B, G, out_blocks, D]; block j at blk_off + j
+    void* out;             // [B, G, out_blocks, D]; block j at blk_off + j (or null)
+    float* out_f32;        // optional f32 entries, same layout as out
     void* out_f16;         // optional fp16 copy [B, G, out_f16_blocks, D] (bf16 input only)
     // optional fp16 copy of every token of each complete block, [B, T, G, D]
     // (bf16 input only); key series rotated at their position s with cos/sin
@@ -223,12 +224,17 @@ struct PrefillArgs {
     const void* k; const void* v;                    // raw [B, T, G, D]
     const void* pooled_k; const void* pooled_v;      // [B, G, pool_stride, D]
     int pool_stride;
+    int pooled_f32;                                  // 1: pooled entries are f32 (row-range form)
     const float* sink;
     const void* gamma_q; const void* gamma_kv;
     void* out;                                       // [B, T, Hq, D]
     int B, T, Hq, G, D, m, w, rho, rmsnorm, shared;
     float eps, scale;
     double rope_step;  // theta^(-2/rho)
+    // row range (CUDA-core kernel): q / out rows at absolute positions t_off ..
+    // t_off + T - 1; k / v hold T_raw rows from absolute position s_off
+    // (the whole-sequence prefill: 0, 0, T)
+    int t_off, s_off, T_raw;
 };
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 // Tensor-core prefill (bf16, D = 128, GQA form without RMSNorm); `scratch` holds

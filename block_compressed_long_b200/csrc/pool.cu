@@ -205,7 +205,12 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const PoolArgs a) {
             finalise_key<T, VEC>(e, d0, a.D, a.rmsnorm, ss, a.eps, static_cast<const T*>(sr.gamma), a.rho, cs);
         if (active) {
             const size_t oi = (((size_t)b * a.G + g) * a.out_blocks + a.blk_off + j) * a.D + d0;
-            st16(static_cast<T*>(sr.out) + oi, e);
+            if (sr.out) st16(static_cast<T*>(sr.out) + oi, e);
+            if (sr.out_f32) {
+#pragma unroll
+                for (int i = 0; i < VEC; i += 4)
+                    *reinterpret_cast<float4*>(sr.out_f32 + oi + i) = make_float4(e[i], e[i + 1], e[i + 2], e[i + 3]);
+            }
             if constexpr (VEC == 8) {
                 if (sr.out_f16) {  // the f32 value, rounded once to fp16
                     const size_t oi16 = (((size_t)b * a.G + g) * a.out_f16_blocks + a.blk_off + j) * a.D + d0;

@@ -40,14 +40,17 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qi = tid / TPQ, j4 = tid % TPQ;
     const int g = h / (a.Hq / a.G);
-    const int t = qt0 + qi;
-    const bool qvalid = t < a.T;
-    const int t_last = min(qt0 + QT, a.T) - 1;
+    // query rows are local (0 .. T-1) at absolute positions t_off + row; raw
+    // rows of k / v are local (0 .. T_raw-1) at absolute positions s_off + row
+    const int tl = qt0 + qi;
+    const bool qvalid = tl < a.T;
+    const int t = a.t_off + tl;
+    const int t_last = a.t_off + min(qt0 + QT, a.T) - 1;
     const int GD = a.G * a.D;
 
     // ---- query: load own dims, RMSNorm across the 4 lanes, RoPE at t ----
     float q[NC][4], o[NC][4];
-    const T* qrow = static_cast<const T*>(a.q) + (((size_t)b * a.T + (qvalid ? t : 0)) * a.Hq + h) * D;
+    const T* qrow = static_cast<const T*>(a.q) + (((size_t)b * a.T + (qvalid ? tl : 0)) * a.Hq + h) * D;
 #pragma unroll
     for (int c = 0; c < NC; ++c)
 #pragma unroll
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
     const int Pq = visible_blocks(t + 1, a.m, a.w);
     const int raw_lo = Pq * a.m;
     const int Pmax = visible_blocks(t_last + 1, a.m, a.w);
-    const int s_lo = visible_blocks(qt0 + 1, a.m, a.w) * a.m;
+    const int s_lo = visible_blocks(a.t_off + qt0 + 1, a.m, a.w) * a.m;
     float mx = kNegInf, ls = 0.f;
 
     const size_t pool_head = ((size_t)b * a.G + g) * a.pool_stride;
@@ -106,7 +109,15 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
         for (int rrow = warp; rrow < KT; rrow += NT / 32) {
             const int e = base + rrow;
             const bool ok = e < lim;
-            if (pooled) {
+            if (pooled && a.pooled_f32) {
+                const size_t o = (pool_head + (ok ? e : 0)) * D;
+                const float* kr = static_cast<const float*>(a.pooled_k) + o;
+                const float* vr = static_cast<const float*>(a.shared ? a.pooled_k : a.pooled_v) + o;
+                for (int d = lane; d < D; d += 32) {
+                    Ks[rrow][d] = ok ? kr[d] : 0.f;
+                    Vs[rrow][d] = ok ? vr[d] : 0.f;
+                }
+            } else if (pooled) {
                 const T* kr = static_cast<const T*>(a.pooled_k) + (pool_head + (ok ? e : 0)) * D;
                 const T* vr = static_cast<const T*>(a.shared ? a.pooled_k : a.pooled_v) + (pool_head + (ok ? e : 0)) * D;
                 for (int d = lane; d < D; d += 32) {
@@ -114,7 +125,8 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
                     Vs[rrow][d] = ok ? to_f<T>(vr[d]) : 0.f;
                 }
             } else {
-                const size_t src = ((size_t)b * a.T + (ok ? e : 0)) * GD + (size_t)g * D;
+                const bool in_raw = ok && e >= a.s_off && e - a.s_off < a.T_raw;  // the host checks the span
+                const size_t src = ((size_t)b * a.T_raw + (in_raw ? e - a.s_off : 0)) * GD + (size_t)g * D;
                 const T* kr = static_cast<const T*>(a.k) + src;
                 float ss = 0.f;
                 for (int d = lane; d < D; d += 32) {
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
     float den = ls;
     if (a.sink) den += (mx == kNegInf) ? 1.0f : ex2(a.sink[h] * kLog2e - mx);
     const float inv = den > 0.f ? 1.0f / den : 0.f;
-    T* orow = static_cast<T*>(a.out) + (((size_t)b * a.T + t) * a.Hq + h) * D;
+    T* orow = static_cast<T*>(a.out) + (((size_t)b * a.T + tl) * a.Hq + h) * D;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         float v[4];

@@ -31,7 +31,7 @@ ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspa
                 "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches",
                 "lbca_decode_step_form", "lbca_selftest_bounded_wait", "lbca_pool_dual", "lbca_decode_sparse",
                 "lbca_indexer_workspace_bytes", "lbca_indexer_topk", "lbca_prefill_backward_workspace_bytes",
-                "lbca_prefill_backward")
+                "lbca_prefill_backward", "lbca_prefill_rows", "lbca_pool_f32")
 
 
 class lbca_config(ctypes.Structure):
@@ -66,6 +66,8 @@ _lib.lbca_prefill_workspace_bytes.argtypes = [_CP, _i32, _i32, _i32]
 _lib.lbca_prefill_workspace_bytes.restype = _sz
 _lib.lbca_pool.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp]
 _lib.lbca_pool.restype = ctypes.c_int
+_lib.lbca_pool_f32.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp]
+_lib.lbca_pool_f32.restype = ctypes.c_int
 _lib.lbca_pool_dual.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp]
 _lib.lbca_pool_dual.restype = ctypes.c_int
 _lib.lbca_append.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp]
@@ -99,6 +101,9 @@ _lib.lbca_prefill_backward_workspace_bytes.argtypes = [_CP, _i32, _i32]
 _lib.lbca_prefill_backward_workspace_bytes.restype = _sz
 _lib.lbca_prefill_backward.argtypes = [_CP] + [_vp] * 11 + [_i32, _i32] + [_vp] * 9 + [_sz, _vp]
 _lib.lbca_prefill_backward.restype = ctypes.c_int
+_lib.lbca_prefill_rows.argtypes = [_CP, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp,
+                                   _vp]
+_lib.lbca_prefill_rows.restype = ctypes.c_int
 _lib.lbca_status_string.argtypes = [ctypes.c_int]
 _lib.lbca_status_string.restype = ctypes.c_char_p
 
@@ -200,6 +205,16 @@ def lbca_pool(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, str
     ob = out.shape[2] if out_blocks is None else out_blocks
     _check("lbca_pool", _lib.lbca_pool(ctypes.byref(cfg), series, _ptr(x), _ptr(z), _ptr(b_pos), _ptr(gamma),
                                        B, T, pos0, _ptr(out), ob, _stream(stream)))
+
+
+def lbca_pool_f32(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, stream=None):
+    """lbca_pool with f32 entries: out float32 [B, G, out_blocks, D]."""
+    if out.dtype != torch.float32:
+        raise TypeError("lbca_pool_f32 writes float32 entries")
+    B, T = x.shape[0], x.shape[1]
+    ob = out.shape[2] if out_blocks is None else out_blocks
+    _check("lbca_pool_f32", _lib.lbca_pool_f32(ctypes.byref(cfg), series, _ptr(x), _ptr(z), _ptr(b_pos), _ptr(gamma),
+                                               B, T, pos0, _ptr(out), ob, _stream(stream)))
 
 
 def lbca_pool_dual(cfg, series, xa, za, xb, zb, b_pos_a, b_pos_b, gamma, out, out_blocks=None, stream=None):
@@ -326,3 +341,17 @@ def lbca_prefill_backward(cfg, q, k, v, zk, zv, b_pos_k, b_pos_v, sink, gamma_q,
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv), _ptr(b_pos_k), _ptr(b_pos_v), _ptr(sink),
         _ptr(gamma_q), _ptr(gamma_kv), _ptr(dout), B, T, g("dq"), g("dk"), g("dv"), g("dzk"), g("dzv"), g("dbk"),
         g("dbv"), g("dsink"), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def lbca_prefill_rows(cfg, q, row0, k, v, raw0, pooled_k, pooled_v, sink, gamma_q, gamma_kv, out, stream=None):
+    """q, out [B, n_rows, Hq, D] at absolute rows row0..; k, v [B, n_raw, G, D]
+    from absolute position raw0; pooled_k/v float32 [B, G, pool_stride, D]
+    (lbca_pool_f32)."""
+    for p in (pooled_k, pooled_v):
+        if p is not None and p.dtype != torch.float32:
+            raise TypeError("lbca_prefill_rows reads float32 pooled entries")
+    B, n = q.shape[0], q.shape[1]
+    stride = 0 if pooled_k is None else pooled_k.shape[2]
+    _check("lbca_prefill_rows", _lib.lbca_prefill_rows(
+        ctypes.byref(cfg), _ptr(q), row0, n, _ptr(k), _ptr(v), raw0, k.shape[1], _ptr(pooled_k), _ptr(pooled_v),
+        stride, _ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), B, _ptr(out), _stream(stream)))

@@ -168,6 +168,17 @@ LBCA_API lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const voi
                       int32_t pos0, void* out, int32_t out_blocks, lbca_stream_t stream);
 
 /*
+ * lbca_pool_f32 -- lbca_pool with the entries written in f32 (out: device
+ * [B, G, out_blocks, D] float), unrounded: the exchange format of a
+ * context-parallel prefill, whose ranks all-gather their pooled entries and
+ * read them with lbca_prefill_rows at the precision the single-GPU prefill
+ * keeps them.  Same arguments, arithmetic and errors as lbca_pool.
+ */
+LBCA_API lbca_status lbca_pool_f32(const lbca_config* cfg, int32_t series, const void* x, const void* z,
+                                   const void* b_pos, const void* gamma, int32_t batch, int32_t T,
+                                   int32_t pos0, float* out, int32_t out_blocks, lbca_stream_t stream);
+
+/*
  * lbca_pool_dual -- dual overlapped pooling of the floor(T/m) complete blocks
  * (the CSA form; CSA page, "What is implemented": dual overlapped
  * compression, Eqs 9-12; entry RoPE at block starts: "Deviations from paper").
@@ -313,6 +324,33 @@ LBCA_API lbca_status lbca_prefill(const lbca_config* cfg, const void* q, const v
                          const void* gamma_kv, int32_t batch, int32_t T, void* out,
                          const lbca_cache* cache_out, void* workspace, size_t workspace_bytes,
                          int32_t* d_status, lbca_stream_t stream);
+
+/*
+ * lbca_prefill_rows -- the prefill's attention for a range of query rows, from
+ * pooled entries and raw tokens the caller assembles: the building block of a
+ * context-parallel prefill, where each rank owns a block-aligned range of
+ * tokens, pools it (lbca_pool with pos0 = its first token), all-gathers the
+ * pooled entries and receives the previous rank's last n_win + m - 1 raw
+ * tokens (mSeek README, "How LBCA works", steps 4-5; same visible set and
+ * arithmetic as lbca_prefill, on the CUDA cores).
+ *   q, out     device [B, n_rows, Hq, D]: rows at absolute positions row0 ..
+ *              row0 + n_rows - 1
+ *   k, v       device [B, n_raw, G, D] raw keys and values at absolute
+ *              positions raw0 .. raw0 + n_raw - 1, with raw0 + n_raw = row0 +
+ *              n_rows and raw0 <= P(row0 + 1) m (the first row's window start;
+ *              raw0 = max(0, row0 - (n_win + m - 1)) always qualifies);
+ *              shared form: k = C, v = NULL
+ *   pooled_k/v device [B, G, pool_stride, D] f32 finalised pooled entries of
+ *              blocks 0 .. P(row0 + n_rows) - 1 (lbca_pool_f32); shared
+ *              form: pooled_v = NULL
+ * Errors: LBCA_ERR_ARG (a span that does not cover the rows' visible sets),
+ * LBCA_ERR_ALIGN, LBCA_ERR_UNSUPPORTED, LBCA_ERR_CUDA.
+ */
+LBCA_API lbca_status lbca_prefill_rows(const lbca_config* cfg, const void* q, int32_t row0, int32_t n_rows,
+                                       const void* k, const void* v, int32_t raw0, int32_t n_raw,
+                                       const float* pooled_k, const float* pooled_v, int32_t pool_stride,
+                                       const float* sink, const void* gamma_q, const void* gamma_kv, int32_t batch,
+                                       void* out, lbca_stream_t stream);
 
 /*
  * lbca_prefill_backward -- gradients of the prefill for training (mSeek

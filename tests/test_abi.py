@@ -23,7 +23,7 @@ def L():
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(lbca_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(lbca_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -88,6 +88,11 @@ def test_pool_argument_checks(L):
     assert L._lib.lbca_pool(ctypes.byref(shared), 1, A, A, A, None, 1, 64, 0, A, 1, None) == L.LBCA_ERR_ARG
     # a valid call with no GPU present must not succeed: there is no CPU fallback
     assert f(0, A, A, A, None, 1, 64, 0, A, 1, None) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
+    g = lambda *a: L._lib.lbca_pool_f32(ctypes.byref(cfg), *a)  # noqa: E731
+    assert g(0, A, A, A, None, 1, 64, 0, None, 1, None) == L.LBCA_ERR_ARG          # null out
+    assert g(0, A, A, A, None, 1, 640, 0, A, 9, None) == L.LBCA_ERR_ARG            # out_blocks too small
+    assert g(0, A, A, A, None, 1, 64, 0, A + 4, 1, None) == L.LBCA_ERR_ALIGN       # misaligned out
+    assert g(0, A, A, A, None, 1, 64, 0, A, 1, None) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
 
 
 def test_cache_and_decode_checks(L):

@@ -52,6 +52,15 @@ def test_pool_matches_oracle(L, name, kw, pos0_blocks):
         assert_close_stored(got, want, w.dtype, f"{name} series {s}")
         untouched = f64(out[:, :, :pos0_blocks]), f64(out[:, :, pos0_blocks + nb:])
         assert all(np.all(u == 7.0) for u in untouched), "pool wrote outside its blocks"
+        # the f32 form: the same entries before their one rounding to the I/O dtype
+        o32 = torch.full((B, w.n_kv_heads, ob, w.head_dim), 7.0, dtype=torch.float32, device="cuda")
+        L.lbca_pool_f32(cfg, s, x.cuda(), z.cuda(), bp.cuda(), None, o32, pos0=pos0_blocks * m)
+        torch.cuda.synchronize()
+        assert torch.equal(o32.to(out.dtype), out), f"{name} series {s}: f32 entries round to other values"
+        g32 = f64(o32[:, :, pos0_blocks:pos0_blocks + nb]).transpose(0, 2, 1, 3)
+        scale = max(float(np.abs(want).max()), 1e-30)
+        assert np.abs(g32 - want).max() <= 1e-5 * scale, f"{name} series {s}: f32 entries"
+        assert np.all(f64(o32[:, :, pos0_blocks + nb:]) == 7.0) and np.all(f64(o32[:, :, :pos0_blocks]) == 7.0)
 
 
 # ------------------------------------------------------------- prefill ----
@@ -209,3 +218,58 @@ def test_prefill_fp16_range_sets_status(L, where):
     assert int(st.item()) == want
     if where == "none":
         assert_close(f64(out), oracle_prefill(w, inp), "bf16", "in-range prefill")
+
+
+# ---------------------------------------------------------- context parallel ----
+@pytest.mark.parametrize("name,kw,world", [
+    ("gqa_prefill_16k", dict(seq_len=16 * 40 + 7, n_win=48), 3),
+    ("hca_mqa_decode_128k", dict(kind="prefill", seq_len=128 * 5 + 30, block_m=32, n_win=40, batch=2), 2),
+])
+def test_context_parallel_rows_equal_the_whole_prefill(L, name, kw, world):
+    """The ranks' compute of a context-parallel prefill, run one after another
+    on this GPU: each pools its own blocks into their slots of one pooled
+    buffer (the union is what the all-gather delivers), attends its own rows
+    from the pooled prefix and the raw tokens from its halo on
+    (lbca_prefill_rows); the rows together match the oracle, and the
+    whole-sequence call of the same kernel (whose groups of rows per CTA
+    start elsewhere, so the rounding order may differ)."""
+    from block_compressed_long_b200 import context_parallel as cp
+    w = synth.scaled(W[name], **kw)
+    inp = synth.make(w)
+    cfg = lcfg(L, w)
+    B, T = inp.q.shape[:2]
+    p = cp.plan(T, w.block_m, w.n_win, world)
+    d = lambda t: None if t is None else t.contiguous().cuda()  # noqa: E731
+    pk = torch.zeros(B, w.n_kv_heads, p.blocks, w.head_dim, dtype=torch.float32, device="cuda")
+    pv = None if w.shared_kv else torch.zeros_like(pk)
+    for r in range(world):
+        t0, t1 = p.ranges[r]
+        L.lbca_pool_f32(cfg, L.LBCA_KEY, d(inp.k[:, t0:t1]), d(inp.zk[:, t0:t1]), d(inp.bpos_k), None, pk, pos0=t0)
+        if not w.shared_kv:
+            L.lbca_pool_f32(cfg, L.LBCA_VALUE, d(inp.v[:, t0:t1]), d(inp.zv[:, t0:t1]), d(inp.bpos_v), None, pv,
+                            pos0=t0)
+    outs = []
+    for r in range(world):
+        t0, t1 = p.ranges[r]
+        lo, _ = p.halo_range(r)
+        outs.append(cp.attend_rows(L, cfg, d(inp.q[:, t0:t1]), t0, d(inp.k[:, lo:t1]),
+                                   None if w.shared_kv else d(inp.v[:, lo:t1]), lo, pk, pv, d(inp.sink)))
+    torch.cuda.synchronize()
+    got = f64(torch.cat(outs, dim=1))
+    assert_close(got, oracle_prefill(w, inp), w.dtype, f"context parallel {name}")
+    # the same rows from one whole-sequence call of the same CUDA-core kernel
+    whole = torch.empty_like(d(inp.q))
+    L.lbca_prefill_rows(cfg, d(inp.q), 0, d(inp.k), d(inp.v), 0, pk, pv, d(inp.sink), None, None, whole)
+    torch.cuda.synchronize()
+    assert_close(got, f64(whole), w.dtype, f"context parallel {name} vs one call")
+
+
+def test_prefill_rows_rejects_a_window_that_starts_too_late(L):
+    w = synth.scaled(W["gqa_prefill_16k"], seq_len=16 * 10, n_win=32)
+    cfg = lcfg(L, w)
+    q = torch.zeros(1, 16, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, 16, w.n_kv_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    pk = torch.zeros(1, w.n_kv_heads, 10, w.head_dim, dtype=torch.float32, device="cuda")
+    with pytest.raises(L.LbcaError) as e:  # rows 96..111 need raw tokens from 64 on; these start at 96
+        L.lbca_prefill_rows(cfg, q, 96, kv, kv, 96, pk, pk, None, None, None, torch.empty_like(q))
+    assert e.value.status == L.LBCA_ERR_ARG

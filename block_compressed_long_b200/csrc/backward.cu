@@ -405,6 +405,441 @@ __global__ void pool_bwd_kernel(const BwdArgs a) {
     }
 }
 
+// ---- register-tiled passes over (row, entry) pairs, D = 64 or 128 ----
+// The pairs a query row sees form, per tile of RT consecutive rows of one head,
+// a prefix of the pooled entries and a band of raw tokens; per tile of ET
+// entries of one kv head, a range of rows.  Tiles of both sides are staged in
+// shared memory and every thread computes a small block of scores (and of the
+// outputs) in registers, so each K/V and Q/dO row is read once per tile
+// instead of once per pair.
+constexpr int kTT = 256;   // threads of the tiled passes
+constexpr int RT = 64;     // query rows per tile
+constexpr int ET = 32;     // entries per tile
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float dot4(float4 x, float4 y, float acc) {
+    return fmaf(x.w, y.w, fmaf(x.z, y.z, fmaf(x.y, y.y, fmaf(x.x, y.x, acc))));
+}
+__device__ __forceinline__ void axpy4(float a, float4 x, float* y) {
+    y[0] = fmaf(a, x.x, y[0]);
+    y[1] = fmaf(a, x.y, y[1]);
+    y[2] = fmaf(a, x.z, y[2]);
+    y[3] = fmaf(a, x.w, y[3]);
+}
+
+// Entry `idx` (pooled block, or raw token) visible to row t, P = P(t + 1).
+__device__ __forceinline__ bool sees(bool pooled, int idx, int t, int P, int m) {
+    return pooled ? idx < P : (idx >= P * m && idx <= t);
+}
+
+// f32 key and value rows of entry idx of (b, g) into Ks, Vs (row r); zeros past cnt.
+template <int D>
+__device__ __forceinline__ void load_entries(const BwdArgs& a, bool pooled, int base, int cnt, int b, int g, float* Ks,
+                                             float* Vs) {
+    constexpr int LD = D + 4;
+    for (int i = threadIdx.x; i < ET * (D / 4); i += kTT) {
+        const int r = i / (D / 4), c = 4 * (i % (D / 4));
+        float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f), v4 = k4;
+        if (r < cnt) {
+            const int e = base + r;
+            const size_t kr = pooled ? (((size_t)b * a.NB + e) * a.G + g) : (((size_t)b * a.T + e) * a.G + g);
+            const float* kp = (pooled ? a.Ef : a.Kf) + kr * D;
+            const float* vp = a.shared ? kp
+                                       : (pooled ? a.Ef + ((size_t)a.B * a.NB * a.G + kr) * D : a.vf + kr * D);
+            k4 = ld4(kp + c);
+            v4 = ld4(vp + c);
+        }
+        st4(Ks + r * LD + c, k4);
+        st4(Vs + r * LD + c, v4);
+    }
+}
+
+template <int D>
+constexpr size_t row_pass_smem() {
+    return (size_t)(2 * RT * (D + 4) + 2 * ET * (D + 4) + RT * (ET + 1)) * 4 + RT * 4 + 64;
+}
+
+// ---- 3+4 (tiled). Per tile of RT rows of one head: sweep 1 -- log-sum-exp and
+// the output (for dsum = dout . o); sweep 2 -- dS and dq~ = scale sum dS key.
+// dq~ goes to dq; the turn back through RoPE and RMSNorm follows (dq_tail).
+template <int D>
+__global__ void __launch_bounds__(kTT, 2) row_pass_kernel(const BwdArgs a) {
+    constexpr int LD = D + 4, NC = D / 32;
+    extern __shared__ __align__(16) float sm[];
+    float* Qs = sm;
+    float* dOs = Qs + RT * LD;
+    float* Ks = dOs + RT * LD;
+    float* Vs = Ks + ET * LD;
+    float* Ps = Vs + ET * LD;                        // [RT][ET + 1]
+    int* Prow = reinterpret_cast<int*>(Ps + RT * (ET + 1));
+    float* red = reinterpret_cast<float*>(Prow + RT);  // [kTT / 32]
+
+    const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7, lane = tid & 31;
+    const int t0 = blockIdx.x * RT, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.Hq / a.G);
+    const int nrow = min(RT, a.T - t0);
+    for (int i = tid; i < RT * (D / 4); i += kTT) {
+        const int r = i / (D / 4), c = 4 * (i % (D / 4));
+        float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = q4;
+        if (r < nrow) {
+            const size_t row = ((size_t)b * a.T + t0 + r) * a.Hq + h;
+            q4 = ld4(a.qf + row * D + c);
+            q4.x *= a.scale; q4.y *= a.scale; q4.z *= a.scale; q4.w *= a.scale;
+            d4 = ld4(a.dof + row * D + c);
+        }
+        st4(Qs + r * LD + c, q4);
+        st4(dOs + r * LD + c, d4);
+    }
+    for (int r = tid; r < RT; r += kTT) Prow[r] = visible_blocks(t0 + r + 1, a.m, a.w);
+    const int t_last = t0 + nrow - 1;
+    const int Pmax = visible_blocks(t_last + 1, a.m, a.w);
+    const int s_lo = visible_blocks(t0 + 1, a.m, a.w) * a.m;
+    const int npt = (Pmax + ET - 1) / ET, nrt = (t_last - s_lo + 1 + ET - 1) / ET;
+    const int r0 = 2 * ty;
+    const float sink = a.sink ? a.sink[h] : kNegInf;
+
+    float M[2], l[2], o[2][4 * NC];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        M[i] = sink;
+        l[i] = a.sink ? 1.f : 0.f;
+#pragma unroll
+        for (int c = 0; c < 4 * NC; ++c) o[i][c] = 0.f;
+    }
+    // ---- sweep 1 ----
+    for (int tile = 0; tile < npt + nrt; ++tile) {
+        const bool pooled = tile < npt;
+        const int base = pooled ? tile * ET : s_lo + (tile - npt) * ET;
+        const int cnt = min(ET, pooled ? Pmax - base : t_last + 1 - base);
+        __syncthreads();  // the previous tile's K, V, P are consumed
+        load_entries<D>(a, pooled, base, cnt, b, g, Ks, Vs);
+        __syncthreads();
+        float sc[2][4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[i][e] = 0.f;
+#pragma unroll 4
+        for (int d = 0; d < D; d += 4) {
+            const float4 q0 = ld4(Qs + r0 * LD + d), q1 = ld4(Qs + (r0 + 1) * LD + d);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 k4 = ld4(Ks + (tx + 8 * e) * LD + d);
+                sc[0][e] = dot4(q0, k4, sc[0][e]);
+                sc[1][e] = dot4(q1, k4, sc[1][e]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = r0 + i, t = t0 + r;
+            float mx = kNegInf;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int ee = tx + 8 * e;
+                const bool ok = r < nrow && ee < cnt && sees(pooled, base + ee, t, Prow[r], a.m);
+                sc[i][e] = ok ? sc[i][e] : kNegInf;
+                mx = fmaxf(mx, sc[i][e]);
+            }
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float mn = fmaxf(M[i], mx);
+            const float c = mn == kNegInf ? 1.f : expf(M[i] - mn);
+            float ps = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float p = sc[i][e] == kNegInf ? 0.f : expf(sc[i][e] - mn);
+                ps += p;
+                Ps[r * (ET + 1) + tx + 8 * e] = p;
+            }
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+            l[i] = l[i] * c + ps;
+            M[i] = mn;
+#pragma unroll
+            for (int k = 0; k < 4 * NC; ++k) o[i][k] *= c;
+        }
+        __syncthreads();
+        for (int e = 0; e < cnt; ++e) {
+            const float p0 = Ps[r0 * (ET + 1) + e], p1 = Ps[(r0 + 1) * (ET + 1) + e];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const float4 v4 = ld4(Vs + e * LD + 32 * c + 4 * tx);
+                axpy4(p0, v4, &o[0][4 * c]);
+                axpy4(p1, v4, &o[1][4 * c]);
+            }
+        }
+    }
+    // ---- log-sum-exp, dout . o / l; the sink's gradient ----
+    float lse[2], dsum[2], sink_g = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        float dt = 0.f;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const float4 d4 = ld4(dOs + r * LD + 32 * c + 4 * tx);
+            dt = fmaf(d4.x, o[i][4 * c], fmaf(d4.y, o[i][4 * c + 1], fmaf(d4.z, o[i][4 * c + 2], fmaf(d4.w, o[i][4 * c + 3], dt))));
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) dt += __shfl_xor_sync(0xffffffffu, dt, off);
+        lse[i] = M[i] + logf(l[i]);
+        dsum[i] = dt / l[i];
+        if (r < nrow && tx == 0) {
+            const size_t row = ((size_t)b * a.T + t0 + r) * a.Hq + h;
+            a.lse[row] = lse[i];
+            a.dsum[row] = dsum[i];
+            if (a.sink) sink_g -= expf(sink - lse[i]) * dsum[i];
+        }
+    }
+    // ---- sweep 2: dq~ ----
+    float dq[2][4 * NC];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int c = 0; c < 4 * NC; ++c) dq[i][c] = 0.f;
+    for (int tile = 0; tile < npt + nrt; ++tile) {
+        const bool pooled = tile < npt;
+        const int base = pooled ? tile * ET : s_lo + (tile - npt) * ET;
+        const int cnt = min(ET, pooled ? Pmax - base : t_last + 1 - base);
+        __syncthreads();
+        load_entries<D>(a, pooled, base, cnt, b, g, Ks, Vs);
+        __syncthreads();
+        float sc[2][4], dp[2][4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[i][e] = dp[i][e] = 0.f;
+#pragma unroll 2
+        for (int d = 0; d < D; d += 4) {
+            const float4 q0 = ld4(Qs + r0 * LD + d), q1 = ld4(Qs + (r0 + 1) * LD + d);
+            const float4 g0 = ld4(dOs + r0 * LD + d), g1 = ld4(dOs + (r0 + 1) * LD + d);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 k4 = ld4(Ks + (tx + 8 * e) * LD + d);
+                const float4 v4 = ld4(Vs + (tx + 8 * e) * LD + d);
+                sc[0][e] = dot4(q0, k4, sc[0][e]);
+                sc[1][e] = dot4(q1, k4, sc[1][e]);
+                dp[0][e] = dot4(g0, v4, dp[0][e]);
+                dp[1][e] = dot4(g1, v4, dp[1][e]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = r0 + i, t = t0 + r;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int ee = tx + 8 * e;
+                const bool ok = r < nrow && ee < cnt && sees(pooled, base + ee, t, Prow[r], a.m);
+                Ps[r * (ET + 1) + ee] = ok ? expf(sc[i][e] - lse[i]) * (dp[i][e] - dsum[i]) * a.scale : 0.f;
+            }
+        }
+        __syncthreads();
+        for (int e = 0; e < cnt; ++e) {
+            const float s0 = Ps[r0 * (ET + 1) + e], s1 = Ps[(r0 + 1) * (ET + 1) + e];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const float4 k4 = ld4(Ks + e * LD + 32 * c + 4 * tx);
+                axpy4(s0, k4, &dq[0][4 * c]);
+                axpy4(s1, k4, &dq[1][4 * c]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        if (r >= nrow) continue;
+        const size_t row = ((size_t)b * a.T + t0 + r) * a.Hq + h;
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+            st4(a.dq + row * D + 32 * c + 4 * tx,
+                make_float4(dq[i][4 * c], dq[i][4 * c + 1], dq[i][4 * c + 2], dq[i][4 * c + 3]));
+    }
+    if (a.sink) {  // one atomic per CTA
+        float v = sink_g;
+#pragma unroll
+        for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) red[tid >> 5] = v;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.f;
+            for (int w = 0; w < kTT / 32; ++w) s += red[w];
+            atomicAdd(a.dsink + h, s);
+        }
+    }
+}
+
+// dq~ (in dq) back through the query's RoPE at t and RMSNorm, one warp per row.
+template <typename T, int NPL>
+__global__ void dq_tail_kernel(const BwdArgs a) {
+    const int lane = threadIdx.x & 31;
+    const size_t r = blockIdx.x * (size_t)kWarpsPerCta + (threadIdx.x >> 5);
+    if (r >= (size_t)a.B * a.T * a.Hq) return;
+    const int t = (int)((r / a.Hq) % a.T);
+    float acc[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) acc[i] = a.dq[r * a.D + lane + 32 * i];
+    row_rope<NPL>(acc, lane, a.D, a.rho, a.rope_step, -(int64_t)t);
+    if (a.rmsnorm) {
+        float x[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) x[i] = ldf(static_cast<const T*>(a.q) + r * a.D + lane + 32 * i);
+        row_rms_bwd<NPL>(x, acc, lane, a.D, a.eps, static_cast<const T*>(a.gamma_q));
+    }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) a.dq[r * a.D + lane + 32 * i] = acc[i];
+}
+
+template <int D>
+constexpr size_t entry_pass_smem() {
+    return (size_t)(2 * ET * (D + 4) + 2 * RT * (D + 4) + 2 * ET * (RT + 1)) * 4 + 3 * RT * 4;
+}
+
+// ---- 5 (tiled). Per tile of ET entries of one kv head: dkey and dval over the
+// rows (of every head of the group) that can see the tile's entries.
+template <int D>
+__global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
+    constexpr int LD = D + 4, NC = D / 64;
+    extern __shared__ __align__(16) float sm[];
+    float* Ks = sm;
+    float* Vs = Ks + ET * LD;
+    float* Qs = Vs + ET * LD;
+    float* dOs = Qs + RT * LD;
+    float* PT = dOs + RT * LD;              // [ET][RT + 1]
+    float* dST = PT + ET * (RT + 1);         // [ET][RT + 1]
+    float* lse_s = dST + ET * (RT + 1);
+    float* dsum_s = lse_s + RT;
+    int* Prow = reinterpret_cast<int*>(dsum_s + RT);
+
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    const int g = blockIdx.y, b = blockIdx.z, rg = a.Hq / a.G;
+    const int npt = (a.NB + ET - 1) / ET;
+    const bool pooled = (int)blockIdx.x < npt;
+    const int base = pooled ? blockIdx.x * ET : (blockIdx.x - npt) * ET;
+    const int cnt = min(ET, (pooled ? a.NB : a.T) - base);
+    // rows that can see some entry of the tile
+    int t_lo, t_hi;
+    if (pooled) {
+        t_lo = (base + 1) * a.m + a.w - 1;
+        t_hi = a.T - 1;
+    } else {
+        t_lo = base;
+        t_hi = min(a.T - 1, ((base + cnt - 1) / a.m + 1) * a.m + a.w - 2);
+    }
+    load_entries<D>(a, pooled, base, cnt, b, g, Ks, Vs);
+    const int e0 = 2 * ty;
+    float dk[2][4 * NC], dv[2][4 * NC];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4 * NC; ++c) dk[j][c] = dv[j][c] = 0.f;
+
+    for (int hh = 0; hh < rg && t_lo <= t_hi; ++hh) {
+        const int h = g * rg + hh;
+        for (int rt = (t_lo / RT) * RT; rt <= t_hi; rt += RT) {
+            const int nrow = min(RT, a.T - rt);
+            __syncthreads();  // the previous row tile is consumed (and K, V are in place)
+            for (int i = tid; i < RT * (D / 4); i += kTT) {
+                const int r = i / (D / 4), c = 4 * (i % (D / 4));
+                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = q4;
+                if (r < nrow) {
+                    const size_t row = ((size_t)b * a.T + rt + r) * a.Hq + h;
+                    q4 = ld4(a.qf + row * D + c);
+                    q4.x *= a.scale; q4.y *= a.scale; q4.z *= a.scale; q4.w *= a.scale;
+                    d4 = ld4(a.dof + row * D + c);
+                }
+                st4(Qs + r * LD + c, q4);
+                st4(dOs + r * LD + c, d4);
+            }
+            for (int r = tid; r < RT; r += kTT) {
+                const size_t row = ((size_t)b * a.T + rt + r) * a.Hq + h;
+                lse_s[r] = r < nrow ? a.lse[row] : 0.f;
+                dsum_s[r] = r < nrow ? a.dsum[row] : 0.f;
+                Prow[r] = visible_blocks(rt + r + 1, a.m, a.w);
+            }
+            __syncthreads();
+            float sc[2][4], dp[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sc[j][i] = dp[j][i] = 0.f;
+#pragma unroll 2
+            for (int d = 0; d < D; d += 4) {
+                const float4 k0 = ld4(Ks + e0 * LD + d), k1 = ld4(Ks + (e0 + 1) * LD + d);
+                const float4 v0 = ld4(Vs + e0 * LD + d), v1 = ld4(Vs + (e0 + 1) * LD + d);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 q4 = ld4(Qs + (tx + 16 * i) * LD + d);
+                    const float4 d4 = ld4(dOs + (tx + 16 * i) * LD + d);
+                    sc[0][i] = dot4(k0, q4, sc[0][i]);
+                    sc[1][i] = dot4(k1, q4, sc[1][i]);
+                    dp[0][i] = dot4(v0, d4, dp[0][i]);
+                    dp[1][i] = dot4(v1, d4, dp[1][i]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = tx + 16 * i, e = e0 + j;
+                    const bool ok = r < nrow && e < cnt && sees(pooled, base + e, rt + r, Prow[r], a.m);
+                    const float p = ok ? expf(sc[j][i] - lse_s[r]) : 0.f;
+                    PT[e * (RT + 1) + r] = p;
+                    dST[e * (RT + 1) + r] = p * (dp[j][i] - dsum_s[r]);
+                }
+            __syncthreads();
+            for (int r = 0; r < nrow; ++r) {
+                const float p0 = PT[e0 * (RT + 1) + r], p1 = PT[(e0 + 1) * (RT + 1) + r];
+                const float s0 = dST[e0 * (RT + 1) + r], s1 = dST[(e0 + 1) * (RT + 1) + r];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const float4 d4 = ld4(dOs + r * LD + 64 * c + 4 * tx);
+                    const float4 q4 = ld4(Qs + r * LD + 64 * c + 4 * tx);
+                    axpy4(p0, d4, &dv[0][4 * c]);
+                    axpy4(p1, d4, &dv[1][4 * c]);
+                    axpy4(s0, q4, &dk[0][4 * c]);
+                    axpy4(s1, q4, &dk[1][4 * c]);
+                }
+            }
+        }
+    }
+    const size_t npool = (size_t)a.B * a.NB * a.G;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int e = e0 + j;
+        if (e >= cnt) continue;
+        const size_t r = pooled ? (((size_t)b * a.NB + base + e) * a.G + g) : (((size_t)b * a.T + base + e) * a.G + g);
+        float* dko = pooled ? a.dE + r * D : a.dKf + r * D;
+        float* dvo = pooled ? a.dE + (npool + r) * D : a.dv + r * D;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            float4 kv = make_float4(dk[j][4 * c], dk[j][4 * c + 1], dk[j][4 * c + 2], dk[j][4 * c + 3]);
+            const float4 vv = make_float4(dv[j][4 * c], dv[j][4 * c + 1], dv[j][4 * c + 2], dv[j][4 * c + 3]);
+            if (a.shared) {
+                kv.x += vv.x; kv.y += vv.y; kv.z += vv.z; kv.w += vv.w;
+            } else {
+                st4(dvo + 64 * c + 4 * tx, vv);
+            }
+            st4(dko + 64 * c + 4 * tx, kv);
+        }
+    }
+}
+
+template <int D>
+cudaError_t tiled_attr() {
+    static bool set = false;
+    if (!set) {
+        cudaError_t e = cudaFuncSetAttribute(row_pass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)row_pass_smem<D>());
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(entry_pass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)entry_pass_smem<D>());
+        if (e != cudaSuccess) return e;
+        set = true;
+    }
+    return cudaSuccess;
+}
+
 inline unsigned warps_grid(size_t warps) { return (unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta); }
 
 template <typename T, int NPL>
@@ -412,9 +847,19 @@ cudaError_t run_rows(const BwdArgs& a, cudaStream_t s) {
     const size_t nk = (size_t)a.B * a.NB * a.G, nr = (size_t)a.B * a.T * a.G, nq = (size_t)a.B * a.T * a.Hq;
     const dim3 blk(32 * kWarpsPerCta);
     finalise_kernel<T, NPL><<<warps_grid(nk + nr + nq), blk, 0, s>>>(a);
-    row_lse_kernel<NPL><<<warps_grid(nq), blk, 0, s>>>(a);
-    dq_kernel<T, NPL><<<warps_grid(nq), blk, 0, s>>>(a);
-    dkv_kernel<NPL><<<warps_grid(nk + nr), blk, 0, s>>>(a);
+    constexpr int D = 32 * NPL;
+    if constexpr (D == 64 || D == 128) {  // register-tiled passes
+        cudaError_t e = tiled_attr<D>();
+        if (e != cudaSuccess) return e;
+        row_pass_kernel<D><<<dim3((a.T + RT - 1) / RT, a.Hq, a.B), kTT, row_pass_smem<D>(), s>>>(a);
+        dq_tail_kernel<T, NPL><<<warps_grid(nq), blk, 0, s>>>(a);
+        const int tiles = (a.NB + ET - 1) / ET + (a.T + ET - 1) / ET;
+        entry_pass_kernel<D><<<dim3(tiles, a.G, a.B), kTT, entry_pass_smem<D>(), s>>>(a);
+    } else {
+        row_lse_kernel<NPL><<<warps_grid(nq), blk, 0, s>>>(a);
+        dq_kernel<T, NPL><<<warps_grid(nq), blk, 0, s>>>(a);
+        dkv_kernel<NPL><<<warps_grid(nk + nr), blk, 0, s>>>(a);
+    }
     key_bwd_kernel<T, NPL><<<warps_grid(nk + nr), blk, 0, s>>>(a);
     return cudaGetLastError();
 }

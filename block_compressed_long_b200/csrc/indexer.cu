@@ -137,52 +137,53 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kKeysPerThread = 32;  // keys held in registers: up to 32768 visible blocks
 
-// Inclusive prefix sum over the CTA of one value per thread (thread order);
-// warp_sums is kSelWarps ints of shared memory.  Every thread must call it.
-__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_sums) {
+// Sum over the CTA of one count per thread (every thread gets the total).  The
+// caller alternates between two kSelWarps-int arrays on successive calls, so
+// one barrier suffices: an array is rewritten only after the barrier of the
+// call between, which every thread passes after reading it.
+__device__ __forceinline__ int block_count(int c, int* warp_sums) {
+    const int lane = threadIdx.x & 31;
+    const int w = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) warp_sums[threadIdx.x >> 5] = w;
+    __syncthreads();
+    return __reduce_add_sync(0xffffffffu, lane < kSelWarps ? warp_sums[lane] : 0);
+}
+
+// Exclusive prefix sum over the CTA (thread order) of one value per thread;
+// *total receives the sum over the CTA.
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* warp_sums, unsigned* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+    unsigned x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
-    if (warp == 0) {
-        int w = warp_sums[lane];
+    unsigned before = 0u, all = 0u;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        warp_sums[lane] = w;
+    for (int q = 0; q < kSelWarps; ++q) {
+        const unsigned w = warp_sums[q];
+        before += q < warp ? w : 0u;
+        all += w;
     }
-    __syncthreads();
-    const int r = x + (warp > 0 ? warp_sums[warp - 1] : 0);
-    __syncthreads();  // warp_sums may be reused
-    return r;
+    *total = all;
+    return before + x - v;
 }
 
-// Sum over the CTA of one count per thread (every thread gets the total).
-__device__ __forceinline__ int block_count(int c, int* warp_sums) {
-    const int w = __reduce_add_sync(0xffffffffu, c);
-    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = w;
-    __syncthreads();
-    const int total = __reduce_add_sync(0xffffffffu, warp_sums[threadIdx.x & 31]);
-    __syncthreads();  // warp_sums may be reused
-    return total;
-}
-
-// One CTA per sequence.  The visible relevances are read once into registers
-// as order-preserving keys (thread t holds blocks t, t + 1024, ...).  The k-th
+// One CTA per sequence.  Thread t holds, as order-preserving keys in
+// registers, the relevances of the contiguous run of blocks [t S, t S + S)
+// (S = ceil(nvis / threads)), so thread order is block order.  The k-th
 // largest key is found one bit at a time, most significant first: a bit is
 // kept when at least k keys are >= the prefix with that bit set (32 rounds of
-// a compare per key and one CTA-wide count, no atomics).  The selection then
-// walks the keys in block order, one block scan per register slot: every key
-// above the threshold, and the first of those equal to it until k are taken.
+// a compare per key and one CTA-wide count, no atomics).  One CTA-wide scan of
+// each thread's counts above and equal to the threshold then gives every
+// thread the output position of its first taken block: all blocks above the
+// threshold, and those equal to it, in block order, until k are taken.
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) {
-    __shared__ int warp_sums[kSelWarps];
+    __shared__ int warp_sums[2][kSelWarps];
+    __shared__ unsigned scan_sums[kSelWarps];
     const int b = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int nvis = min(max(L, 0) / a.m, a.max_blocks);
@@ -203,12 +204,13 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         for (int i = tid; i < K; i += kSelThreads) sel[i] = -1;
         return;
     }
-    const int slots = (nvis + kSelThreads - 1) / kSelThreads;  // uniform
+    const int S = (nvis + kSelThreads - 1) / kSelThreads;  // uniform
+    const int i0 = tid * S;
     uint32_t key[kKeysPerThread];
 #pragma unroll
     for (int s = 0; s < kKeysPerThread; ++s) {
-        const int i = tid + s * kSelThreads;
-        key[s] = (s < slots && i < nvis) ? order_key(sc[i]) : 0u;  // 0: below every real key
+        const int i = i0 + s;
+        key[s] = (s < S && i < nvis) ? order_key(sc[i]) : 0u;  // 0: below every real key
     }
     // ---- the k-th largest key, bit by bit ----
     uint32_t thr = 0u;
@@ -218,33 +220,38 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         int c = 0;
 #pragma unroll
         for (int s = 0; s < kKeysPerThread; ++s)
-            if (s < slots) c += key[s] >= cand;
-        if (block_count(c, warp_sums) >= K) thr = cand;
+            if (s < S) c += key[s] >= cand;
+        if (block_count(c, warp_sums[bit & 1]) >= K) thr = cand;
     }
-    int c_gt = 0;
+    // ---- counts above and at the threshold, one scan of both (16-bit halves) ----
+    int gt = 0, eq = 0;
 #pragma unroll
     for (int s = 0; s < kKeysPerThread; ++s)
-        if (s < slots) c_gt += key[s] > thr;
-    const int ties_needed = K - block_count(c_gt, warp_sums);
-    // ---- selection in block order: every key above thr, the first ties_needed equal to it ----
-    int pos_base = 0, tie_base = 0;
+        if (s < S) {
+            gt += key[s] > thr;
+            eq += key[s] == thr && i0 + s < nvis;
+        }
+    unsigned all = 0u;  // each half sums at most 32768
+    const unsigned packed = block_exclusive_scan((unsigned)gt | ((unsigned)eq << 16), scan_sums, &all);
+    const int gt_before = (int)(packed & 0xffffu), eq_before = (int)(packed >> 16);
+    const int ties_needed = K - (int)(all & 0xffffu);
+    // ---- this thread's blocks, in order ----
+    int pos = gt_before + min(eq_before, ties_needed);
+    int ties_seen = eq_before;
 #pragma unroll
     for (int s = 0; s < kKeysPerThread; ++s) {
-        if (s >= slots) break;  // uniform
-        const int i = tid + s * kSelThreads;
-        const bool valid = i < nvis;
-        const bool gt = valid && key[s] > thr, tie = valid && key[s] == thr;
-        const int tie_incl = block_inclusive_scan(tie ? 1 : 0, warp_sums);
-        const bool take = gt || (tie && tie_base + tie_incl - 1 < ties_needed);
-        const int pos_incl = block_inclusive_scan(take ? 1 : 0, warp_sums);
-        if (take && pos_base + pos_incl - 1 < K) {
-            sel[pos_base + pos_incl - 1] = i;
-            if (selv) selv[pos_base + pos_incl - 1] = sc[i];
+        const int i = i0 + s;
+        const bool real = s < S && i < nvis;
+        const bool tie = real && key[s] == thr;
+        const bool take = (real && key[s] > thr) || (tie && ties_seen < ties_needed);
+        ties_seen += tie ? 1 : 0;
+        if (take && pos < K) {
+            sel[pos] = i;
+            if (selv) selv[pos] = __uint_as_float(key[s] & 0x80000000u ? key[s] & 0x7fffffffu : ~key[s]);
         }
-        tie_base += block_count(tie ? 1 : 0, warp_sums);
-        pos_base += block_count(take ? 1 : 0, warp_sums);
+        pos += take ? 1 : 0;
     }
-    if (tid == 0 && pos_base != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
+    if (tid == kSelThreads - 1 && pos != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
 }
 
 template <int DI, int HI>

@@ -48,7 +48,9 @@ def _run(L, w, inp, dout, gq=None, gkv=None):
     ("hca_mqa_decode_128k", dict(kind="prefill", seq_len=150, head_dim=128, rmsnorm=False, rope_dims=6, block_m=8,
                                  n_win=16, n_q_heads=4)),
     ("tiny_f32_prefill", dict(seq_len=16 * 6 + 9)),
-], ids=["gqa-m16", "gqa-m64", "hca", "shared-rope6", "tiny-f32"])
+    # more pooled entries than one entry tile and many row tiles, a ragged last row tile
+    ("gqa_prefill_16k", dict(seq_len=16 * 40 + 7, n_win=48)),
+], ids=["gqa-m16", "gqa-m64", "hca", "shared-rope6", "tiny-f32", "gqa-multi-tile"])
 def test_backward_matches_oracle(L, name, kw):
     w = synth.scaled(W[name], **kw)
     inp = synth.make(w)

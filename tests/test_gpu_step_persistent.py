@@ -93,7 +93,7 @@ def test_persistent_step_reports_contexts_beyond_max_ctx(L):
     the partials it was given; other sequences are unaffected in shape."""
     w = synth.scaled(W["ragged_gqa_decode_append"], ctx=(100, 200), batch=16, steps=1)
     lens = synth.contexts(w)
-    lens[3] = 20000  # far beyond the max_ctx below
+    lens[3] = 60000  # far beyond the max_ctx below: its segments span more CTAs than any grid leaves room for
     inp = synth.make(w, lens=lens)
     run = DecodeRun(L, w, inp)
     small = 300

@@ -379,7 +379,8 @@ lbca_status lbca_decode_step(const lbca_config* cfg, const void* k, const void* 
     a.pdl = (cache->flags & LBCA_CACHE_OVERLAP_PREV) != 0;
     a.eps = cfg->rms_eps; a.scale = scale_of(cfg); a.rope_step = rope_step_of(cfg);
     if (sp.flat) {
-        for (int kk = 0; kk < cfg->rope_dims / 2 && kk < 128; ++kk) a.rope_f[kk] = rope_turns(kk, a.rope_step);  // workspace: [arrival counter][segment counters][partial max, sum][partial outputs]
+        for (int kk = 0; kk < cfg->rope_dims / 2 && kk < 128; ++kk) a.rope_f[kk] = rope_turns(kk, a.rope_step);
+        // workspace: [arrival counter][segment counters][partial max, sum][partial outputs]
         char* ws = static_cast<char*>(workspace);
         const size_t o1 = align256(4), o2 = o1 + align256(sp.seg_elems * 4), o3 = o2 + align256(sp.part_ml_elems * 4);
         a.seg_count = reinterpret_cast<uint32_t*>(ws + o1);

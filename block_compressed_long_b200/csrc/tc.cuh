@@ -85,11 +85,6 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// kind::f16 instruction descriptor, bf16 A read MN-major and bf16 B K-major, f32 accumulate.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
 // ---- packed f32 pairs and three-input max (sm_100a FMA pipe) ------------------------
 // One instruction for two lanes of f32 arithmetic: d = a * b + c and d = a + b per
 // component, round to nearest, subnormals flushed (the softmax never meets them).
@@ -178,15 +173,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
         "[%6];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
-        : "memory");
-}
-
-// 2-D tensor load (no multicast) of one box at (c0, c1) into dst (shared::cta address).
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
         : "memory");
 }
 

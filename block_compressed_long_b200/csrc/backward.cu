@@ -696,7 +696,11 @@ constexpr size_t entry_pass_smem() {
 }
 
 // ---- 5 (tiled). Per tile of ET entries of one kv head: dkey and dval over the
-// rows (of every head of the group) that can see the tile's entries.
+// rows (of every head of the group) that can see the tile's entries.  A pooled
+// tile is seen by every later row, so its rows are cut into chunks of kRowChunk
+// row tiles, one CTA each, whose sums are added into the (zeroed) entry
+// gradients; a raw tile's few rows stay with one CTA, which stores its sums.
+constexpr int kRowChunk = 8;
 template <int D>
 __global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
     constexpr int LD = D + 4, NC = D / 64;
@@ -713,15 +717,18 @@ __global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
 
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int g = blockIdx.y, b = blockIdx.z, rg = a.Hq / a.G;
-    const int npt = (a.NB + ET - 1) / ET;
+    const int nchunk = (a.T + RT * kRowChunk - 1) / (RT * kRowChunk);
+    const int npt = (a.NB + ET - 1) / ET * nchunk;
     const bool pooled = (int)blockIdx.x < npt;
-    const int base = pooled ? blockIdx.x * ET : (blockIdx.x - npt) * ET;
+    const int base = pooled ? (blockIdx.x / nchunk) * ET : (blockIdx.x - npt) * ET;
     const int cnt = min(ET, (pooled ? a.NB : a.T) - base);
-    // rows that can see some entry of the tile
+    // rows that can see some entry of the tile (for a pooled tile, within this CTA's chunk)
     int t_lo, t_hi;
     if (pooled) {
-        t_lo = (base + 1) * a.m + a.w - 1;
-        t_hi = a.T - 1;
+        const int c0 = (blockIdx.x % nchunk) * RT * kRowChunk;
+        t_lo = max((base + 1) * a.m + a.w - 1, c0);
+        t_hi = min(a.T - 1, c0 + RT * kRowChunk - 1);
+        if (t_lo > t_hi) return;  // no row of this chunk sees the tile (nothing to add)
     } else {
         t_lo = base;
         t_hi = min(a.T - 1, ((base + cnt - 1) / a.m + 1) * a.m + a.w - 2);
@@ -817,10 +824,18 @@ __global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
             const float4 vv = make_float4(dv[j][4 * c], dv[j][4 * c + 1], dv[j][4 * c + 2], dv[j][4 * c + 3]);
             if (a.shared) {
                 kv.x += vv.x; kv.y += vv.y; kv.z += vv.z; kv.w += vv.w;
-            } else {
-                st4(dvo + 64 * c + 4 * tx, vv);
             }
-            st4(dko + 64 * c + 4 * tx, kv);
+            if (pooled) {  // one chunk's share
+                float* pk = dko + 64 * c + 4 * tx;
+                atomicAdd(pk, kv.x); atomicAdd(pk + 1, kv.y); atomicAdd(pk + 2, kv.z); atomicAdd(pk + 3, kv.w);
+                if (!a.shared) {
+                    float* pv = dvo + 64 * c + 4 * tx;
+                    atomicAdd(pv, vv.x); atomicAdd(pv + 1, vv.y); atomicAdd(pv + 2, vv.z); atomicAdd(pv + 3, vv.w);
+                }
+            } else {
+                if (!a.shared) st4(dvo + 64 * c + 4 * tx, vv);
+                st4(dko + 64 * c + 4 * tx, kv);
+            }
         }
     }
 }
@@ -853,7 +868,11 @@ cudaError_t run_rows(const BwdArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         row_pass_kernel<D><<<dim3((a.T + RT - 1) / RT, a.Hq, a.B), kTT, row_pass_smem<D>(), s>>>(a);
         dq_tail_kernel<T, NPL><<<warps_grid(nq), blk, 0, s>>>(a);
-        const int tiles = (a.NB + ET - 1) / ET + (a.T + ET - 1) / ET;
+        const int nchunk = (a.T + RT * kRowChunk - 1) / (RT * kRowChunk);
+        const int tiles = (a.NB + ET - 1) / ET * nchunk + (a.T + ET - 1) / ET;
+        // the pooled entries' gradients are sums over row chunks
+        const size_t pooled = (size_t)a.S * a.B * a.NB * a.G * D;
+        if (pooled && (e = cudaMemsetAsync(a.dE, 0, pooled * 4, s)) != cudaSuccess) return e;
         entry_pass_kernel<D><<<dim3(tiles, a.G, a.B), kTT, entry_pass_smem<D>(), s>>>(a);
     } else {
         row_lse_kernel<NPL><<<warps_grid(nq), blk, 0, s>>>(a);

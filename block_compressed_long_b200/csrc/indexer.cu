@@ -173,14 +173,17 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* w
 }
 
 // One CTA per sequence.  Thread t holds, as order-preserving keys in
-// registers, the relevances of the contiguous run of blocks [t S, t S + S)
-// (S = ceil(nvis / threads)), so thread order is block order.  The k-th
-// largest key is found one bit at a time, most significant first: a bit is
-// kept when at least k keys are >= the prefix with that bit set (32 rounds of
-// a compare per key and one CTA-wide count, no atomics).  One CTA-wide scan of
-// each thread's counts above and equal to the threshold then gives every
-// thread the output position of its first taken block: all blocks above the
-// threshold, and those equal to it, in block order, until k are taken.
+// registers, the relevances of the contiguous run of blocks [t SLOTS, (t + 1)
+// SLOTS) (zero keys past the visible blocks), so thread order is block order;
+// SLOTS is a compile-time count, so every loop over a thread's keys is exactly
+// its compares.  The k-th largest key is found one bit at a time, most
+// significant first: a bit is kept when at least k keys are >= the prefix
+// with that bit set (32 rounds of a compare per key and one CTA-wide count, no
+// atomics).  One CTA-wide scan of each thread's counts above and equal to the
+// threshold then gives every thread the output position of its first taken
+// block: all blocks above the threshold, and those equal to it, in block order,
+// until k are taken.
+template <int SLOTS>
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) {
     __shared__ int warp_sums[2][kSelWarps];
     __shared__ unsigned scan_sums[kSelWarps];
@@ -199,19 +202,15 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         }
         return;
     }
-    if (nvis > kSelThreads * kKeysPerThread) {  // beyond the register capacity (the host sizes forbid it)
+    if (nvis > kSelThreads * SLOTS) {  // beyond the register capacity (the host sizes forbid it)
         if (tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
         for (int i = tid; i < K; i += kSelThreads) sel[i] = -1;
         return;
     }
-    const int S = (nvis + kSelThreads - 1) / kSelThreads;  // uniform
-    const int i0 = tid * S;
-    uint32_t key[kKeysPerThread];
+    const int i0 = tid * SLOTS;
+    uint32_t key[SLOTS];
 #pragma unroll
-    for (int s = 0; s < kKeysPerThread; ++s) {
-        const int i = i0 + s;
-        key[s] = (s < S && i < nvis) ? order_key(sc[i]) : 0u;  // 0: below every real key
-    }
+    for (int s = 0; s < SLOTS; ++s) key[s] = i0 + s < nvis ? order_key(sc[i0 + s]) : 0u;  // 0: below every real key
     // ---- the k-th largest key, bit by bit ----
     uint32_t thr = 0u;
 #pragma unroll 1
@@ -219,18 +218,16 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         const uint32_t cand = thr | (1u << bit);
         int c = 0;
 #pragma unroll
-        for (int s = 0; s < kKeysPerThread; ++s)
-            if (s < S) c += key[s] >= cand;
+        for (int s = 0; s < SLOTS; ++s) c += key[s] >= cand;
         if (block_count(c, warp_sums[bit & 1]) >= K) thr = cand;
     }
     // ---- counts above and at the threshold, one scan of both (16-bit halves) ----
     int gt = 0, eq = 0;
 #pragma unroll
-    for (int s = 0; s < kKeysPerThread; ++s)
-        if (s < S) {
-            gt += key[s] > thr;
-            eq += key[s] == thr && i0 + s < nvis;
-        }
+    for (int s = 0; s < SLOTS; ++s) {
+        gt += key[s] > thr;
+        eq += key[s] == thr && i0 + s < nvis;
+    }
     unsigned all = 0u;  // each half sums at most 32768
     const unsigned packed = block_exclusive_scan((unsigned)gt | ((unsigned)eq << 16), scan_sums, &all);
     const int gt_before = (int)(packed & 0xffffu), eq_before = (int)(packed >> 16);
@@ -239,11 +236,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
     int pos = gt_before + min(eq_before, ties_needed);
     int ties_seen = eq_before;
 #pragma unroll
-    for (int s = 0; s < kKeysPerThread; ++s) {
+    for (int s = 0; s < SLOTS; ++s) {
         const int i = i0 + s;
-        const bool real = s < S && i < nvis;
-        const bool tie = real && key[s] == thr;
-        const bool take = (real && key[s] > thr) || (tie && ties_seen < ties_needed);
+        const bool tie = i < nvis && key[s] == thr;
+        const bool take = key[s] > thr || (tie && ties_seen < ties_needed);
         ties_seen += tie ? 1 : 0;
         if (take && pos < K) {
             sel[pos] = i;
@@ -294,7 +290,14 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s) {
         }
         if (e != cudaSuccess) return e;
     }
-    topk_kernel<<<a.B, kSelThreads, 0, s>>>(a);
+    // the fewest register slots that hold every visible block of any sequence
+    const int need = (a.max_blocks + kSelThreads - 1) / kSelThreads;
+    if (need <= 1) topk_kernel<1><<<a.B, kSelThreads, 0, s>>>(a);
+    else if (need <= 2) topk_kernel<2><<<a.B, kSelThreads, 0, s>>>(a);
+    else if (need <= 4) topk_kernel<4><<<a.B, kSelThreads, 0, s>>>(a);
+    else if (need <= 8) topk_kernel<8><<<a.B, kSelThreads, 0, s>>>(a);
+    else if (need <= 16) topk_kernel<16><<<a.B, kSelThreads, 0, s>>>(a);
+    else topk_kernel<kKeysPerThread><<<a.B, kSelThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

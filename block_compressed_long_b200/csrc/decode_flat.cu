@@ -38,6 +38,13 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
+// The step's work is split into equal shares of a sequence of entries in which
+// every segment with entries is preceded by kSegCost placeholder entries: a
+// CTA pays, for each segment its range starts, a query setup, a partial
+// publish and shorter pieces (~7 us measured on the ragged 32-sequence batch,
+// about 224 entries of piece work), so ranges that start segments are
+// shortened by that much and the CTAs end together.
+constexpr int kSegCost = 224;
 
 struct FlatLayout {
     size_t args, bars, misc, lens, ecum, qs, cs, newk, newv, wred_o, wred_ml, stage, total;
@@ -134,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
     // arrival ticket: taken once the step's inputs may be read (below), looked at
     // only at the end (its latency hides behind the work)
     unsigned int ticket = 0u;
-    // exclusive prefix of the step's entries per sequence (HG segments of nvis each)
+    // exclusive prefix of the step's entries per sequence (HG segments of kSegCost
+    // placeholders then nvis entries each; none for a sequence without entries)
     {
         const int per = (B + kThreads - 1) / kThreads;
         const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -142,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         for (int b = b0; b < b1; ++b) {
             const int nv = vis_count(lens[b] + 1, a.m, a.w, a.max_blocks, a.R);
             if (nv == 0 && blockIdx.x == 0) set_status(a.status, LBCA_ERR_CAPACITY);
-            sum += (long long)HG * nv;
+            sum += nv ? (long long)HG * (nv + kSegCost) : 0;
         }
         long long incl = sum;  // inclusive scan over the warp
 #pragma unroll
@@ -158,7 +166,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         long long run = base + incl - sum;
         for (int b = b0; b < b1; ++b) {
             ecum[b] = run;
-            run += (long long)HG * vis_count(lens[b] + 1, a.m, a.w, a.max_blocks, a.R);
+            const int nv = vis_count(lens[b] + 1, a.m, a.w, a.max_blocks, a.R);
+            run += nv ? (long long)HG * (nv + kSegCost) : 0;
         }
         if (tid == kThreads - 1) ecum[B] = base + incl;
     }
@@ -166,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
 
     // ---- this CTA's range of the step's entries ----
     const long long E = ecum[B];
-    // active CTAs: each takes at least C entries, so a segment of n entries has
+    // active CTAs: each takes at least C positions, so a segment of n entries has
     // at most n / C + 2 contributors
     const long long NA = std::max<long long>(1, std::min<long long>((long long)gridDim.x, E / C));
     const int cta = blockIdx.x;
@@ -184,10 +193,15 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
     };
 
     // ---- piece cursor: (sequence, head group, entry within the segment) of a
-    // global entry, advanced piece by piece without searching ----
+    // position, advanced piece by piece without searching; placeholders are
+    // skipped (a cursor past e_hi ends the walk) ----
     struct Cursor {
         long long e;
         int b, hg, j, nv, P;
+    };
+    // position of the first entry of segment (b, hg) whose sequence has nv entries
+    auto seg_first = [&](int b, int hg, int nv) {
+        return ecum[b] + (long long)hg * (nv + kSegCost) + kSegCost;
     };
     auto cursor_at = [&](long long e0) {
         Cursor c{e0, 0, 0, 0, 1, 0};
@@ -197,8 +211,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         c.nv = vis_count(L, a.m, a.w, a.max_blocks, a.R);
         c.P = visible_blocks(L, a.m, a.w);
         const int loc = (int)(e0 - ecum[c.b]);
-        c.hg = loc / c.nv;
-        c.j = loc - c.hg * c.nv;
+        c.hg = loc / (c.nv + kSegCost);
+        c.j = loc - c.hg * (c.nv + kSegCost) - kSegCost;
+        if (c.j < 0) {  // a placeholder: the segment's first entry
+            c.e -= c.j;
+            c.j = 0;
+        }
         return c;
     };
     auto piece_len = [&](const Cursor& c) { return (int)std::min<long long>(std::min(c.nv - c.j, C), e_hi - c.e); };
@@ -207,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         c.j += n;
         if (c.j == c.nv && c.e < e_hi) {  // next segment: next head group, or the next sequence with entries
             c.j = 0;
+            c.e += kSegCost;
             if (++c.hg == HG) {
                 c.hg = 0;
                 do {
@@ -460,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         }
         __syncthreads();
         const int seg = seg_cur;
-        const long long es = ecum[b_cur] + (long long)hg_cur * nv_cur, ee = es + nv_cur;
+        const long long es = seg_first(b_cur, hg_cur, nv_cur), ee = es + nv_cur;
         const int c_first = ctaof(es), ncon = ctaof(ee - 1) - c_first + 1;
         if (ncon > a.maxc) {  // more contributors than the workspace was sized for (max_ctx too small)
             if (tid == 0) set_status(a.status, LBCA_ERR_CAPACITY);
@@ -540,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
 #pragma unroll
                 for (int i = 0; i < VEC; ++i) qs[h * D + c * VEC + i] = v[i];
             }
-            const bool ends_here = ecum[b] + (long long)hg * nv + nv - 1 < e_hi;  // uniform
+            const bool ends_here = seg_first(b, hg, nv) + nv - 1 < e_hi;  // uniform
             float2 kx = make_float2(0.f, 0.f), vx = kx;
             if (ends_here && pair_owner) {
                 const size_t tok = (size_t)b * GD + (size_t)g * D + 2 * tid;

@@ -353,6 +353,53 @@ def run_ours(args, w, rank, world, reps=3):
     return line, bench
 
 
+class _Driver:
+    """The few CUDA driver calls the end-to-end loop issues per step (one
+    asynchronous copy each way, event record and stream wait), called through
+    ctypes: a fraction of the host time of the same operations through the
+    torch dispatcher.  Streams are torch's (their handles are driver streams)."""
+
+    def __init__(self):
+        import ctypes
+        d = ctypes.CDLL("libcuda.so.1")
+        u64, vp, sz = ctypes.c_uint64, ctypes.c_void_p, ctypes.c_size_t
+        d.cuMemcpyHtoDAsync_v2.argtypes = [u64, vp, sz, vp]
+        d.cuMemcpyDtoHAsync_v2.argtypes = [vp, u64, sz, vp]
+        d.cuEventCreate.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+        d.cuEventRecord.argtypes = [vp, vp]
+        d.cuStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+        d.cuEventDestroy_v2.argtypes = [vp]
+        self.d, self.ct = d, ctypes
+        self.events = []
+
+    def _ok(self, r, what):
+        if r != 0:
+            raise RuntimeError(f"{what} failed with CUresult {r}")
+
+    def event(self):
+        ev = self.ct.c_void_p()
+        self._ok(self.d.cuEventCreate(self.ct.byref(ev), 2), "cuEventCreate")  # CU_EVENT_DISABLE_TIMING
+        self.events.append(ev)
+        return ev
+
+    def h2d(self, dst, src, n, stream):
+        self._ok(self.d.cuMemcpyHtoDAsync_v2(dst, src, n, stream), "cuMemcpyHtoDAsync")
+
+    def d2h(self, dst, src, n, stream):
+        self._ok(self.d.cuMemcpyDtoHAsync_v2(dst, src, n, stream), "cuMemcpyDtoHAsync")
+
+    def record(self, ev, stream):
+        self._ok(self.d.cuEventRecord(ev, stream), "cuEventRecord")
+
+    def wait(self, stream, ev):
+        self._ok(self.d.cuStreamWaitEvent(stream, ev, 0), "cuStreamWaitEvent")
+
+    def close(self):
+        for ev in self.events:
+            self.d.cuEventDestroy_v2(ev)
+        self.events = []
+
+
 def e2e_loop(bench, K, W):
     """The decode steps end to end through the public API, eagerly: each step
     is one lbca_decode_step call from the host (argument validation and launch
@@ -361,9 +408,10 @@ def e2e_loop(bench, K, W):
     copy.  As in a serving loop the copies run on streams of their own beside
     the kernels (step i+1's upload overlaps step i's kernel, step i's download
     overlaps step i+1's; two staging slots; every step waits for its own
-    upload, every download for its own step).  Returns (ms per step = the
-    longer of the device-event span and the host wall clock, H2D bytes and D2H
-    bytes per step)."""
+    upload, every download for its own step); copies and events go to the
+    driver directly (`_Driver`).  Returns (ms per step = the longer of the
+    device-event span and the host wall clock, H2D bytes and D2H bytes per
+    step)."""
     import torch
 
     parts = [bench.q] + [t for t in (bench.tk, bench.tv, bench.tzk, bench.tzv) if t is not None]
@@ -385,33 +433,37 @@ def e2e_loop(bench, K, W):
     hout = [torch.empty(bench.outs[0].shape, dtype=bench.outs[0].dtype).pin_memory() for _ in range(NS)]
     h2d = int(offs[-1])
     d2h = hout[0].numel() * hout[0].element_size()
+    drv = _Driver()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(NS)]        # slot's upload done
-    ev_run = [torch.cuda.Event() for _ in range(NS)]       # the step that read the slot is done
-    ev_down = [torch.cuda.Event() for _ in range(bench.NR)]  # download of an output replica done
-    cur = torch.cuda.current_stream()
+    h_in, h_out, h_cur = s_in.cuda_stream, s_out.cuda_stream, torch.cuda.current_stream().cuda_stream
+    ev_in = [drv.event() for _ in range(NS)]          # slot's upload done
+    ev_run = [drv.event() for _ in range(NS)]         # the step that read the slot is done
+    ev_down = [drv.event() for _ in range(bench.NR)]  # download of an output replica done
+    ev_join = drv.event()
+    dst_in = [t.data_ptr() for t in dstage]
+    src_out = [t.data_ptr() for t in bench.outs]
+    dst_out = [t.data_ptr() for t in hout]
+    row = hstage.stride(0)
 
     def steps(first, n):
+        base = hstage.data_ptr()
         for j, i in enumerate(range(first, first + n)):
             sl, rep = j % NS, i % bench.NR
             if j >= NS:
-                s_in.wait_event(ev_run[sl])       # the step two back has read this slot
-            with torch.cuda.stream(s_in):
-                dstage[sl].copy_(hstage[i // bench.NR], non_blocking=True)
-                ev_in[sl].record(s_in)
-            cur.wait_event(ev_in[sl])
+                drv.wait(h_in, ev_run[sl])       # the step two back has read this slot
+            drv.h2d(dst_in[sl], base + (i // bench.NR) * row, h2d, h_in)
+            drv.record(ev_in[sl], h_in)
+            drv.wait(h_cur, ev_in[sl])
             if j >= bench.NR:
-                cur.wait_event(ev_down[rep])     # this output replica has been read back
+                drv.wait(h_cur, ev_down[rep])    # this output replica has been read back
             bench.launch(i, q=dq[sl], tok=dtok[sl])
-            ev_run[sl].record(cur)
-            s_out.wait_event(ev_run[sl])
-            with torch.cuda.stream(s_out):
-                hout[sl].copy_(bench.outs[rep], non_blocking=True)
-                ev_down[rep].record(s_out)
-        for st in (s_in, s_out):  # join both copy streams back
-            ev = torch.cuda.Event()
-            ev.record(st)
-            cur.wait_event(ev)
+            drv.record(ev_run[sl], h_cur)
+            drv.wait(h_out, ev_run[sl])
+            drv.d2h(dst_out[sl], src_out[rep], d2h, h_out)
+            drv.record(ev_down[rep], h_out)
+        for h in (h_in, h_out):  # join both copy streams back
+            drv.record(ev_join, h)
+            drv.wait(h_cur, ev_join)
 
     steps(bench.i, W)
     bench.i += W
@@ -424,6 +476,7 @@ def e2e_loop(bench, K, W):
     torch.cuda.synchronize()
     wall_ms = (time.perf_counter() - t0) * 1e3
     bench.i += K
+    drv.close()
     return max(e0.elapsed_time(e1), wall_ms) / K, h2d, d2h
 
 

@@ -842,15 +842,16 @@ __global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
 
 template <int D>
 cudaError_t tiled_attr() {
-    static bool set = false;
-    if (!set) {
+    static bool set[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !set[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(row_pass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)row_pass_smem<D>());
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(entry_pass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)entry_pass_smem<D>());
         if (e != cudaSuccess) return e;
-        set = true;
+        if (dev_ >= 0) set[dev_] = true;
     }
     return cudaSuccess;
 }

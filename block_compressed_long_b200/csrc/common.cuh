@@ -209,6 +209,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     return true;
 }
 
+// The current device ordinal, or -1 (beyond 64 devices, or no device): kernel
+// attributes are set once per device, since a process may drive several.
+inline int current_device() {
+    int d = 0;
+    return cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < 64 ? d : -1;
+}
+
 __device__ __forceinline__ int visible_blocks(int L, int m, int w) {
     int p = L - w;
     return p > 0 ? p / m : 0;

@@ -408,12 +408,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
 
 template <typename T, int D, int R>
 cudaError_t launch_one(const DecodeArgs& a, size_t smem, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static bool attr_set[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr_set[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D, R>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (dev_ >= 0) attr_set[dev_] = true;
     }
     dim3 grid(a.n_split, a.Hq / R, a.B);
     decode_kernel<T, D, R><<<grid, kThreads, smem, s>>>(a);

@@ -714,12 +714,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
 
 template <typename T, int D, int R>
 cudaError_t flat_attr() {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static bool attr_set[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr_set[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(decode_flat_kernel<T, D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              200 * 1024);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (dev_ >= 0) attr_set[dev_] = true;
     }
     return cudaSuccess;
 }

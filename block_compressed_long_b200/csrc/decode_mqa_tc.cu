@@ -821,14 +821,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
 template <int D>
 int max_active_clusters(int cs, uint32_t smem) {
     auto fn = decode_mqa_tc_kernel<D>;
-    static bool attr = false;
-    if (!attr) {
+    static bool attr[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr[dev_]) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess ||
             cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
-        attr = true;
+        if (dev_ >= 0) attr[dev_] = true;
     }
     static uint32_t key[kMaxCS + 1];
     static int val[kMaxCS + 1];

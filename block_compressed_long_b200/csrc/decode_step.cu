@@ -558,13 +558,14 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
 
 template <typename T, int D, int R>
 cudaError_t launch_step_one(const StepArgs& a, size_t smem, cudaStream_t s) {
-    static bool attr_set = false;
+    static bool attr_set[64] = {};  // per device
+    const int dev_ = current_device();
     auto fn = decode_step_kernel<T, D, R>;
-    if (!attr_set) {
+    if (dev_ < 0 || !attr_set[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (dev_ >= 0) attr_set[dev_] = true;
     }
     // 16-CTA clusters are non-portable: fall back to 8 if none fits on this device
     static int max16 = -1;

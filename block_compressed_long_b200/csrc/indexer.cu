@@ -258,12 +258,13 @@ size_t score_smem() {
 template <int DI, int HI>
 cudaError_t launch_score(const IndexerArgs& a, cudaStream_t s) {
     const size_t smem = score_smem<DI, HI>();
-    static bool attr = false;
-    if (!attr) {
+    static bool attr[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(indexer_score_kernel<DI, HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        attr = true;
+        if (dev_ >= 0) attr[dev_] = true;
     }
     dim3 grid((a.max_blocks + kRows - 1) / kRows, a.B);
     indexer_score_kernel<DI, HI><<<grid, kThreads, smem, s>>>(a);

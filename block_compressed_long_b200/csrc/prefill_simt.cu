@@ -230,12 +230,13 @@ __global__ void __launch_bounds__(NT) prefill_simt_kernel(const PrefillArgs a) {
 
 template <typename T, int D>
 cudaError_t launch_d(const PrefillArgs& a, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static bool attr_set[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr_set[dev_]) {
         cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<T, D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<D>::smem);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (dev_ >= 0) attr_set[dev_] = true;
     }
     dim3 grid((a.T + Shape<D>::QT - 1) / Shape<D>::QT, a.Hq, a.B);
     prefill_simt_kernel<T, D><<<grid, NT, Shape<D>::smem, s>>>(a);

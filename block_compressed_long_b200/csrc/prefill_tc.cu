@@ -608,12 +608,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& p, void* scratch, int32_t* stat
     a.T = T; a.Hq = Hq; a.G = G; a.m = p.m; a.w = p.w; a.rho = p.rho;
     a.n_ctiles = (T + NQ * BM - 1) / (NQ * BM);
     a.scale = p.scale;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static bool attr_set[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr_set[dev_]) {
         cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)SMEM_BYTES);
         if (err != cudaSuccess) return err;
-        attr_set = true;
+        if (dev_ >= 0) attr_set[dev_] = true;
     }
     dim3 grid(Hq, a.n_ctiles, B);
     prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(a);

@@ -402,6 +402,10 @@ LBCA_API lbca_status lbca_prefill_backward(const lbca_config* cfg, const void* q
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents: calls that overlap on the GPU (other streams, other host
  *     threads) race and corrupt each other's results.
+ *   - The looked-up address, like the kernel attributes every entry point sets
+ *     once per device, belongs to the device's current context: after a
+ *     cudaDeviceReset the process must not call the library on that device
+ *     again (the cached address and attributes are stale).
  */
 #define LBCA_NOALLOC_SCRATCH_BYTES (8u << 20)
 LBCA_API lbca_status lbca_decode_noalloc(const lbca_config* cfg, const void* q, const lbca_cache* cache,

@@ -193,10 +193,21 @@ class Cache:
                      z(lbca_pool_state_elems(cfg, batch), dtype=torch.float32),
                      z(batch, dtype=torch.int32))
 
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        if name != "_c":
+            object.__setattr__(self, "_c", None)  # any field change rebuilds the C struct
+
     def c(self) -> lbca_cache:
-        return lbca_cache(_ptr(self.pooled_k), _ptr(self.pooled_v), _ptr(self.ring_k), _ptr(self.ring_v),
-                          _ptr(self.pool_state), _ptr(self.seq_lens), self.batch, self.max_blocks,
-                          self.ring_slots, self.flags)
+        """The C struct (built once, rebuilt after any field change: a decode loop
+        pays the marshalling of its cache once)."""
+        cc = self.__dict__.get("_c")
+        if cc is None:
+            cc = lbca_cache(_ptr(self.pooled_k), _ptr(self.pooled_v), _ptr(self.ring_k), _ptr(self.ring_v),
+                            _ptr(self.pool_state), _ptr(self.seq_lens), self.batch, self.max_blocks,
+                            self.ring_slots, self.flags)
+            object.__setattr__(self, "_c", cc)
+        return cc
 
 
 def lbca_pool(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None, stream=None):

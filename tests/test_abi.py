@@ -215,3 +215,21 @@ def test_every_binding_wrapper_reaches_the_library(L):
     for i, call in enumerate(calls):
         with pytest.raises(L.LbcaError):
             call()
+
+
+def test_cache_struct_follows_field_changes(L):
+    """The C struct of a Cache is built once and rebuilt after any field
+    change (a decode loop marshals its cache once; a flag or tensor swap is
+    still seen by the next call)."""
+    import torch
+    cfg = _cfg(L)
+    t = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)  # noqa: E731
+    c = L.Cache(cfg, 1, 4, 192, t(1, 2, 4, 32), t(1, 2, 4, 32), t(1, 2, 192, 32), t(1, 2, 192, 32),
+                torch.zeros(16), torch.zeros(1, dtype=torch.int32))
+    first = c.c()
+    assert c.c() is first
+    c.flags = L.LBCA_CACHE_OVERLAP_PREV
+    assert c.c().flags == L.LBCA_CACHE_OVERLAP_PREV
+    other = t(1, 2, 4, 32)
+    c.pooled_k = other
+    assert c.c().pooled_k == other.data_ptr()

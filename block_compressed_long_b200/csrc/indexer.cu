@@ -137,18 +137,6 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kKeysPerThread = 32;  // keys held in registers: up to 32768 visible blocks
 
-// Sum over the CTA of one count per thread (every thread gets the total).  The
-// caller alternates between two kSelWarps-int arrays on successive calls, so
-// one barrier suffices: an array is rewritten only after the barrier of the
-// call between, which every thread passes after reading it.
-__device__ __forceinline__ int block_count(int c, int* warp_sums) {
-    const int lane = threadIdx.x & 31;
-    const int w = __reduce_add_sync(0xffffffffu, c);
-    if (lane == 0) warp_sums[threadIdx.x >> 5] = w;
-    __syncthreads();
-    return __reduce_add_sync(0xffffffffu, lane < kSelWarps ? warp_sums[lane] : 0);
-}
-
 // Exclusive prefix sum over the CTA (thread order) of one value per thread;
 // *total receives the sum over the CTA.
 __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* warp_sums, unsigned* total) {
@@ -176,17 +164,17 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* w
 // registers, the relevances of the contiguous run of blocks [t SLOTS, (t + 1)
 // SLOTS) (zero keys past the visible blocks), so thread order is block order;
 // SLOTS is a compile-time count, so every loop over a thread's keys is exactly
-// its compares.  The k-th largest key is found one bit at a time, most
-// significant first: a bit is kept when at least k keys are >= the prefix
-// with that bit set (32 rounds of a compare per key and one CTA-wide count, no
-// atomics).  One CTA-wide scan of each thread's counts above and equal to the
-// threshold then gives every thread the output position of its first taken
-// block: all blocks above the threshold, and those equal to it, in block order,
-// until k are taken.
+// its keys.  The k-th largest key is found eight bits at a time, most
+// significant first (four rounds of a 256-bin histogram of the keys that match
+// the digits chosen so far, and one scan of it).  One CTA-wide scan of each
+// thread's counts above and equal to the threshold then gives every thread the
+// output position of its first taken block: all blocks above the threshold,
+// and those equal to it, in block order, until k are taken.
 template <int SLOTS>
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) {
-    __shared__ int warp_sums[2][kSelWarps];
     __shared__ unsigned scan_sums[kSelWarps];
+    __shared__ uint32_t hist[256];
+    __shared__ int sel_round[2];
     const int b = blockIdx.x, tid = threadIdx.x;
     const int L = a.seq_lens[b];
     const int nvis = min(max(L, 0) / a.m, a.max_blocks);
@@ -207,19 +195,61 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         for (int i = tid; i < K; i += kSelThreads) sel[i] = -1;
         return;
     }
+    // the relevances pass through shared memory: read from global in block order
+    // (coalesced), then each thread takes its contiguous run (one padding word
+    // per run keeps the runs on different banks)
+    extern __shared__ float stage[];  // kSelThreads runs of SLOTS + 1 words
+    for (int i = tid; i < nvis; i += kSelThreads) stage[i + i / SLOTS] = sc[i];
+    __syncthreads();
     const int i0 = tid * SLOTS;
     uint32_t key[SLOTS];
 #pragma unroll
-    for (int s = 0; s < SLOTS; ++s) key[s] = i0 + s < nvis ? order_key(sc[i0 + s]) : 0u;  // 0: below every real key
-    // ---- the k-th largest key, bit by bit ----
-    uint32_t thr = 0u;
+    for (int s = 0; s < SLOTS; ++s)
+        key[s] = i0 + s < nvis ? order_key(stage[tid * (SLOTS + 1) + s]) : 0u;  // 0: below every real key
+    // ---- the k-th largest key, eight bits at a time ----
+    // Round r histograms digit r (most significant first) of the keys that match
+    // the digits chosen so far; lanes of a warp holding the same digit add once
+    // (__match_any_sync), so keys that share their top bits do not serialise the
+    // shared-memory adds.  The digit whose bin holds the k-th largest of those
+    // keys is kept, and k is reduced by the keys in the bins above it.
+    uint32_t thr = 0u, tmask = 0u;
+    int need = K;
+    const int lane = tid & 31;
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = thr | (1u << bit);
-        int c = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
+        if (tid == 0) sel_round[0] = sel_round[1] = 0;
+        __syncthreads();
 #pragma unroll
-        for (int s = 0; s < SLOTS; ++s) c += key[s] >= cand;
-        if (block_count(c, warp_sums[bit & 1]) >= K) thr = cand;
+        for (int s = 0; s < SLOTS; ++s) {
+            const bool in = i0 + s < nvis && (key[s] & tmask) == thr;
+            const uint32_t dg = in ? (key[s] >> shift) & 255u : 256u;
+            const uint32_t same = __match_any_sync(0xffffffffu, dg);
+            if (in && lane == __ffs(same) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(same));
+        }
+        __syncthreads();
+        if (tid < 32) {  // warp 0: lane l holds bins [8l, 8l + 8); scan from the top
+            uint32_t h[8], tot = 0u;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) { h[q] = hist[8 * tid + q]; tot += h[q]; }
+            uint32_t above = 0u;  // keys in the bins of the lanes above this one
+            for (int l = 31; l > 0; --l) {
+                const uint32_t v = __shfl_sync(0xffffffffu, tot, l);
+                if (l > tid) above += v;
+            }
+            for (int q = 7; q >= 0; --q) {
+                if (above < (uint32_t)need && (uint32_t)need <= above + h[q]) {
+                    sel_round[0] = 8 * tid + q;
+                    sel_round[1] = (int)above;
+                }
+                above += h[q];
+            }
+        }
+        __syncthreads();
+        thr |= (uint32_t)sel_round[0] << shift;
+        tmask |= 255u << shift;
+        need -= sel_round[1];
+        __syncthreads();  // hist and sel_round are rewritten by the next round
     }
     // ---- counts above and at the threshold, one scan of both (16-bit halves) ----
     int gt = 0, eq = 0;
@@ -248,6 +278,20 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         pos += take ? 1 : 0;
     }
     if (tid == kSelThreads - 1 && pos != K) set_status(a.status, LBCA_ERR_ARG);  // cannot happen: the select is exact
+}
+
+template <int SLOTS>
+cudaError_t launch_topk(const IndexerArgs& a, cudaStream_t s) {
+    const size_t smem = (size_t)kSelThreads * (SLOTS + 1) * sizeof(float);
+    static bool attr[64] = {};  // per device
+    const int dev_ = current_device();
+    if (dev_ < 0 || !attr[dev_]) {
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel<SLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev_ >= 0) attr[dev_] = true;
+    }
+    topk_kernel<SLOTS><<<a.B, kSelThreads, smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 template <int DI, int HI>
@@ -293,13 +337,12 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s) {
     }
     // the fewest register slots that hold every visible block of any sequence
     const int need = (a.max_blocks + kSelThreads - 1) / kSelThreads;
-    if (need <= 1) topk_kernel<1><<<a.B, kSelThreads, 0, s>>>(a);
-    else if (need <= 2) topk_kernel<2><<<a.B, kSelThreads, 0, s>>>(a);
-    else if (need <= 4) topk_kernel<4><<<a.B, kSelThreads, 0, s>>>(a);
-    else if (need <= 8) topk_kernel<8><<<a.B, kSelThreads, 0, s>>>(a);
-    else if (need <= 16) topk_kernel<16><<<a.B, kSelThreads, 0, s>>>(a);
-    else topk_kernel<kKeysPerThread><<<a.B, kSelThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    if (need <= 1) return launch_topk<1>(a, s);
+    if (need <= 2) return launch_topk<2>(a, s);
+    if (need <= 4) return launch_topk<4>(a, s);
+    if (need <= 8) return launch_topk<8>(a, s);
+    if (need <= 16) return launch_topk<16>(a, s);
+    return launch_topk<kKeysPerThread>(a, s);
 }
 
 }  // namespace lbca

@@ -208,9 +208,9 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         key[s] = i0 + s < nvis ? order_key(stage[tid * (SLOTS + 1) + s]) : 0u;  // 0: below every real key
     // ---- the k-th largest key, eight bits at a time ----
     // Round r histograms digit r (most significant first) of the keys that match
-    // the digits chosen so far; lanes of a warp holding the same digit add once
-    // (__match_any_sync), so keys that share their top bits do not serialise the
-    // shared-memory adds.  The digit whose bin holds the k-th largest of those
+    // the digits chosen so far; the lanes of a warp holding lane 0's digit add
+    // once (a ballot), so keys that share their top bits (most relevances do) do
+    // not serialise the shared-memory adds.  The digit whose bin holds the k-th largest of those
     // keys is kept, and k is reduced by the keys in the bins above it.
     uint32_t thr = 0u, tmask = 0u;
     int need = K;
@@ -224,19 +224,26 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const IndexerArgs a) 
         for (int s = 0; s < SLOTS; ++s) {
             const bool in = i0 + s < nvis && (key[s] & tmask) == thr;
             const uint32_t dg = in ? (key[s] >> shift) & 255u : 256u;
-            const uint32_t same = __match_any_sync(0xffffffffu, dg);
-            if (in && lane == __ffs(same) - 1) atomicAdd(&hist[dg], (uint32_t)__popc(same));
+            // the lanes that share lane 0's digit add once; the others one by one
+            const uint32_t d0 = __shfl_sync(0xffffffffu, dg, 0);
+            const uint32_t same = __ballot_sync(0xffffffffu, dg == d0);
+            if (lane == 0 && d0 != 256u) atomicAdd(&hist[d0], (uint32_t)__popc(same));
+            if (dg != d0 && in) atomicAdd(&hist[dg], 1u);
         }
         __syncthreads();
         if (tid < 32) {  // warp 0: lane l holds bins [8l, 8l + 8); scan from the top
             uint32_t h[8], tot = 0u;
 #pragma unroll
             for (int q = 0; q < 8; ++q) { h[q] = hist[8 * tid + q]; tot += h[q]; }
-            uint32_t above = 0u;  // keys in the bins of the lanes above this one
-            for (int l = 31; l > 0; --l) {
-                const uint32_t v = __shfl_sync(0xffffffffu, tot, l);
-                if (l > tid) above += v;
+            // keys in the bins of the lanes above this one: an inclusive suffix sum
+            // (log-step) minus this lane's own bins
+            uint32_t suf = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t y = __shfl_down_sync(0xffffffffu, suf, off);
+                if (tid + off < 32) suf += y;
             }
+            uint32_t above = suf - tot;
             for (int q = 7; q >= 0; --q) {
                 if (above < (uint32_t)need && (uint32_t)need <= above + h[q]) {
                     sel_round[0] = 8 * tid + q;

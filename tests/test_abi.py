@@ -233,3 +233,18 @@ def test_cache_struct_follows_field_changes(L):
     other = t(1, 2, 4, 32)
     c.pooled_k = other
     assert c.c().pooled_k == other.data_ptr()
+
+
+def test_f32_pool_exchange_wrappers_check_dtypes(L):
+    """The context-parallel exchange format is f32: the wrappers refuse other
+    dtypes before any call reaches the library."""
+    import torch
+    cfg = _cfg(L)
+    kv = torch.zeros(1, 64, 8, 128, dtype=torch.bfloat16)
+    bp = torch.zeros(64, 8 * 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        L.lbca_pool_f32(cfg, 0, kv, kv, bp, None, torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16))
+    q = torch.zeros(1, 16, 24, 128, dtype=torch.bfloat16)
+    pk = torch.zeros(1, 8, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        L.lbca_prefill_rows(cfg, q, 240, kv, kv, 192, pk, pk, None, None, None, torch.empty_like(q))

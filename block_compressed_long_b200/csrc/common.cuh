@@ -209,6 +209,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     return true;
 }
 
+// Rows [r, r + n) of an array of `rows` rows.  In the bounds-checked build
+// (LBCA_CHECKED) a range that leaves the array records LBCA_ERR_ARG on the
+// status word and is moved to the array's start, so the access stays inside
+// it (the result is then wrong, and flagged); otherwise r is returned as is.
+__device__ __forceinline__ long long checked_rows(long long r, long long n, long long rows, int32_t* status) {
+#ifdef LBCA_CHECKED
+    if (r < 0 || n < 0 || r + n > rows) {
+        set_status(status, LBCA_ERR_ARG);
+        return 0;
+    }
+#else
+    (void)n; (void)rows; (void)status;
+#endif
+    return r;
+}
+
 // The current device ordinal, or -1 (beyond 64 devices, or no device): kernel
 // attributes are set once per device, since a process may drive several.
 inline int current_device() {

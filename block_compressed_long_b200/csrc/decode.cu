@@ -154,20 +154,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeArgs a) {
         int e = e0, row = 0;
         if (e < P) {
             const int n = min(e1, P) - e;
-            bulk_g2s(kbuf, static_cast<const T*>(a.pooled_k) + (pool_head + e) * D, n * ROW, bar);
+            bulk_g2s(kbuf, static_cast<const T*>(a.pooled_k) + (pool_head + checked_rows(e, n, a.max_blocks, a.status)) * D, n * ROW, bar);
             if (!a.shared)
-                bulk_g2s(vbuf, static_cast<const T*>(a.pooled_v) + (pool_head + e) * D, n * ROW, bar);
+                bulk_g2s(vbuf, static_cast<const T*>(a.pooled_v) + (pool_head + checked_rows(e, n, a.max_blocks, a.status)) * D, n * ROW, bar);
             e += n;
             row += n;
         }
         while (e < e1) {
             const int slot = (s0 + (e - P)) % a.R;
             const int n = min(e1 - e, a.R - slot);
-            bulk_g2s(kbuf + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + slot) * D,
+            bulk_g2s(kbuf + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + checked_rows(slot, n, a.R, a.status)) * D,
                      n * ROW, bar);
             if (!a.shared)
                 bulk_g2s(vbuf + (size_t)row * D,
-                         static_cast<const T*>(a.ring_v) + (ring_head + slot) * D, n * ROW, bar);
+                         static_cast<const T*>(a.ring_v) + (ring_head + checked_rows(slot, n, a.R, a.status)) * D, n * ROW, bar);
             e += n;
             row += n;
         }

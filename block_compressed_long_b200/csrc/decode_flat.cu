@@ -253,19 +253,19 @@ __global__ void __launch_bounds__(kThreads, 3) decode_flat_kernel(const __grid_c
         int idx = j, row = 0;
         if (idx < c1 && idx < P) {
             const int cnt = min(c1, P) - idx;
-            bulk_g2s(kd, static_cast<const T*>(a.pooled_k) + (pool_head + idx) * D, cnt * ROW, &bars[buf]);
+            bulk_g2s(kd, static_cast<const T*>(a.pooled_k) + (pool_head + checked_rows(idx, cnt, a.max_blocks, a.status)) * D, cnt * ROW, &bars[buf]);
             if (!a.shared)
-                bulk_g2s(vd, static_cast<const T*>(a.pooled_v) + (pool_head + idx) * D, cnt * ROW, &bars[buf]);
+                bulk_g2s(vd, static_cast<const T*>(a.pooled_v) + (pool_head + checked_rows(idx, cnt, a.max_blocks, a.status)) * D, cnt * ROW, &bars[buf]);
             idx += cnt;
             row += cnt;
         }
         while (idx < c1) {
             const int slot = (s0 + (idx - P)) % a.R;
             const int cnt = min(c1 - idx, a.R - slot);
-            bulk_g2s(kd + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + slot) * D, cnt * ROW,
+            bulk_g2s(kd + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + checked_rows(slot, cnt, a.R, a.status)) * D, cnt * ROW,
                      &bars[buf]);
             if (!a.shared)
-                bulk_g2s(vd + (size_t)row * D, static_cast<const T*>(a.ring_v) + (ring_head + slot) * D,
+                bulk_g2s(vd + (size_t)row * D, static_cast<const T*>(a.ring_v) + (ring_head + checked_rows(slot, cnt, a.R, a.status)) * D,
                          cnt * ROW, &bars[buf]);
             idx += cnt;
             row += cnt;

@@ -416,9 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mqa_tc_kernel(const Decode
                         bytes = 0;  // zero row
                     }
                 }
-                src = pk + (pool_head + j) * D;
+                src = pk + (pool_head + checked_rows(j, 1, a.max_blocks, a.status)) * D;
             } else {
-                src = rk + (ring_head + (s0 + (idx - P)) % a.R) * D;
+                src = rk + (ring_head + checked_rows((s0 + (idx - P)) % a.R, 1, a.R, a.status)) * D;
             }
         }
         const uint32_t rbase = sE + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u;

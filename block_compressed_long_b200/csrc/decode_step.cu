@@ -166,19 +166,19 @@ __global__ void __launch_bounds__(kThreads) decode_step_kernel(const StepArgs a)
         int e = b0, row = 0;
         if (e < c1 && e < P) {
             const int n = min(c1, P) - e;
-            bulk_g2s(kd, static_cast<const T*>(a.pooled_k) + (pool_head + e) * D, n * ROW, &bars[st & 1]);
+            bulk_g2s(kd, static_cast<const T*>(a.pooled_k) + (pool_head + checked_rows(e, n, a.max_blocks, a.status)) * D, n * ROW, &bars[st & 1]);
             if (!a.shared)
-                bulk_g2s(vd, static_cast<const T*>(a.pooled_v) + (pool_head + e) * D, n * ROW, &bars[st & 1]);
+                bulk_g2s(vd, static_cast<const T*>(a.pooled_v) + (pool_head + checked_rows(e, n, a.max_blocks, a.status)) * D, n * ROW, &bars[st & 1]);
             e += n;
             row += n;
         }
         while (e < c1) {
             const int slot = (s0 + (e - P)) % a.R;
             const int n = min(c1 - e, a.R - slot);
-            bulk_g2s(kd + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + slot) * D, n * ROW,
+            bulk_g2s(kd + (size_t)row * D, static_cast<const T*>(a.ring_k) + (ring_head + checked_rows(slot, n, a.R, a.status)) * D, n * ROW,
                      &bars[st & 1]);
             if (!a.shared)
-                bulk_g2s(vd + (size_t)row * D, static_cast<const T*>(a.ring_v) + (ring_head + slot) * D, n * ROW,
+                bulk_g2s(vd + (size_t)row * D, static_cast<const T*>(a.ring_v) + (ring_head + checked_rows(slot, n, a.R, a.status)) * D, n * ROW,
                          &bars[st & 1]);
             e += n;
             row += n;

@@ -14,7 +14,9 @@ from dataclasses import dataclass
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbca.so")
+# LBCA_CHECKED=1 selects the bounds-checked build of the same library
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "liblbca_checked.so" if os.environ.get("LBCA_CHECKED") == "1" else "liblbca.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is not built; run `python -m block_compressed_long_b200.build` "
                       "(needs nvcc) -- there is no CPU fallback")

@@ -248,3 +248,14 @@ def test_f32_pool_exchange_wrappers_check_dtypes(L):
     pk = torch.zeros(1, 8, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         L.lbca_prefill_rows(cfg, q, 240, kv, kv, 192, pk, pk, None, None, None, torch.empty_like(q))
+
+
+def test_checked_variant_exports_the_same_symbols(L):
+    """The bounds-checked build (loaded with LBCA_CHECKED=1) is the same
+    library compiled with -DLBCA_CHECKED: every declared entry point is there."""
+    path = os.path.join(os.path.dirname(L._LIB_PATH), "liblbca_checked.so")
+    if not os.path.exists(path):
+        pytest.skip("the checked variant is built by build(); not present here")
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n

@@ -476,7 +476,9 @@ __global__ void __launch_bounds__(kTT, 2) row_pass_kernel(const BwdArgs a) {
     float* red = reinterpret_cast<float*>(Prow + RT);  // [kTT / 32]
 
     const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7, lane = tid & 31;
-    const int t0 = blockIdx.x * RT, h = blockIdx.y, b = blockIdx.z;
+    // later row tiles see more pooled entries: they are launched first, so the
+    // grid's last wave holds the short ones
+    const int t0 = (gridDim.x - 1 - blockIdx.x) * RT, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (a.Hq / a.G);
     const int nrow = min(RT, a.T - t0);
     for (int i = tid; i < RT * (D / 4); i += kTT) {
@@ -700,7 +702,7 @@ constexpr size_t entry_pass_smem() {
 // tile is seen by every later row, so its rows are cut into chunks of kRowChunk
 // row tiles, one CTA each, whose sums are added into the (zeroed) entry
 // gradients; a raw tile's few rows stay with one CTA, which stores its sums.
-constexpr int kRowChunk = 8;
+constexpr int kRowChunk = 4;
 template <int D>
 __global__ void __launch_bounds__(kTT, 1) entry_pass_kernel(const BwdArgs a) {
     constexpr int LD = D + 4, NC = D / 64;

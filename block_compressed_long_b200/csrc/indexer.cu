@@ -19,8 +19,9 @@
 //   128-byte-swizzled shared memory, so each key crosses HBM once.  Several
 //   CTAs per SM overlap one tile's copies with another's MMA and epilogue.
 //   Top-k: one CTA per sequence holds the relevances in registers as
-//   order-preserving 32-bit keys and finds the k-th largest one bit at a time
-//   (CTA-wide counts, no atomics), then writes the selected block indices in
+//   order-preserving 32-bit keys (staged through shared memory so the global
+//   reads are coalesced) and finds the k-th largest eight bits at a time (a
+//   256-bin histogram per round), then writes the selected block indices in
 //   increasing index order (equal relevances: lower index first) followed by
 //   -1 padding when fewer than k blocks are visible.
 #include <algorithm>

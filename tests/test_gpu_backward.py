@@ -50,7 +50,9 @@ def _run(L, w, inp, dout, gq=None, gkv=None):
     ("tiny_f32_prefill", dict(seq_len=16 * 6 + 9)),
     # more pooled entries than one entry tile and many row tiles, a ragged last row tile
     ("gqa_prefill_16k", dict(seq_len=16 * 40 + 7, n_win=48)),
-], ids=["gqa-m16", "gqa-m64", "hca", "shared-rope6", "tiny-f32", "gqa-multi-tile"])
+    # the tiled passes at head dim 64 with bf16 I/O and partial RoPE
+    ("gqa_prefill_16k", dict(seq_len=16 * 12 + 3, head_dim=64, rope_dims=32, n_win=40)),
+], ids=["gqa-m16", "gqa-m64", "hca", "shared-rope6", "tiny-f32", "gqa-multi-tile", "gqa-d64"])
 def test_backward_matches_oracle(L, name, kw):
     w = synth.scaled(W[name], **kw)
     inp = synth.make(w)

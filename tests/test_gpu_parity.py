@@ -224,6 +224,7 @@ def test_prefill_fp16_range_sets_status(L, where):
 @pytest.mark.parametrize("name,kw,world", [
     ("gqa_prefill_16k", dict(seq_len=16 * 40 + 7, n_win=48), 3),
     ("hca_mqa_decode_128k", dict(kind="prefill", seq_len=128 * 5 + 30, block_m=32, n_win=40, batch=2), 2),
+    ("tiny_f32_prefill", dict(seq_len=16 * 20 + 5, n_win=24), 3),
 ])
 def test_context_parallel_rows_equal_the_whole_prefill(L, name, kw, world):
     """The ranks' compute of a context-parallel prefill, run one after another

@@ -30,6 +30,9 @@ CASES = [
      20),
     # f32 I/O, 4 query heads on one shared entry, sink logit 0
     ("tiny_f32_prefill", dict(kind="decode", ctx=(0, 300), batch=100, n_kv_heads=1, n_q_heads=4), 18),
+    # the other head dims of the persistent kernel (bf16 D = 64 and 256), partial RoPE
+    ("ragged_gqa_decode_append", dict(ctx=(10, 1500), batch=16, head_dim=64, rope_dims=32), 20),
+    ("ragged_gqa_decode_append", dict(ctx=(10, 1200), batch=16, head_dim=256, rope_dims=64), 20),
 ]
 
 

@@ -98,7 +98,9 @@ class Config:
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # LBCA_ORACLE_LIB: another build of lbca_oracle.c (the pin-strength
+        # test loads copies with one planted mistake each)
+        lib = ctypes.CDLL(os.environ.get("LBCA_ORACLE_LIB") or build())
         dp = ctypes.POINTER(ctypes.c_double)
         lp = ctypes.POINTER(ctypes.c_long)
         lib.orc_visible_blocks.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int]

@@ -145,7 +145,7 @@ def test_pool_dual_is_a_convex_combination(orc):
 
 
 # ---------------------------------------------------------------- indexer ----
-def test_indexer_matches_brute_force_and_masks_incomplete_blocks(orc):
+def test_indexer_matches_brute_force(orc):
     rng = _rng(9)
     B, NB, HI, DI = 3, 20, 5, 8
     q, kx = rng.standard_normal((B, HI, DI)), rng.standard_normal((B, NB, DI))
@@ -155,7 +155,19 @@ def test_indexer_matches_brute_force_and_masks_incomplete_blocks(orc):
     for b in range(B):
         n = int(nvis[b])
         np.testing.assert_allclose(got[b, :n], brute.indexer(q[b], w[b], kx[b], n), rtol=0, atol=1e-12)
-        assert np.all(np.isneginf(got[b, n:]))
+
+
+def test_indexer_masks_the_blocks_a_query_cannot_see(orc):
+    """Entry j of a query that sees n complete blocks is finite for j < n and
+    -inf from n on (n = 0: every entry masked; n = NB: none)."""
+    rng = _rng(12)
+    B, NB, HI, DI = 4, 9, 3, 5
+    q, kx, w = rng.standard_normal((B, HI, DI)), rng.standard_normal((B, NB, DI)), rng.standard_normal((B, HI))
+    nvis = np.array([0, 1, 6, NB])
+    got = orc.indexer_scores(q, w, kx, nvis)
+    for b in range(B):
+        n = int(nvis[b])
+        assert np.all(np.isfinite(got[b, :n])) and np.all(np.isneginf(got[b, n:])), (b, n)
 
 
 def test_indexer_relu_closed_forms(orc):

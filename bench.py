@@ -645,8 +645,9 @@ POOL_CASES = {
 
 
 def pool_leg(label, reps=10, warm=3, baseline=True):
-    """lbca_pool of every complete block of a workload's raw K/V (or C), each
-    series once per call (HBM-bound: X and Z read once, entries written)."""
+    """Pooling of every complete block of a workload's raw K/V (or C): both
+    series of the GQA form in one lbca_pool_kv launch, the shared form's one
+    series by lbca_pool (HBM-bound: X and Z read once, entries written)."""
     import torch
 
     from block_compressed_long_b200 import lbca as L
@@ -667,6 +668,10 @@ def pool_leg(label, reps=10, warm=3, baseline=True):
         xb, zb, bpb = d(inp.csa["kb"]), d(inp.csa["zkb"]), d(inp.csa["bpos_kb"])
 
     def run():
+        if len(srcs) == 2:
+            (k, zk, bpk), (v, zv, bpv) = srcs
+            L.lbca_pool_kv(cfg, k, v, zk, zv, bpk, bpv, None, outs[0], outs[1])
+            return
         for s, (x, z, bp) in zip(series, srcs):
             if dual:
                 L.lbca_pool_dual(cfg, s, x, z, xb, zb, bp, bpb, None, outs[s])
@@ -683,7 +688,7 @@ def pool_leg(label, reps=10, warm=3, baseline=True):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                          "peak_source": src, "kernel": "pool_kernel" + (" (dual overlapped form)" if dual else ""),
                          "bytes_per_call": nbytes,
-                         "launches_per_call": len(srcs)},
+                         "launches_per_call": 1},
             "clocks": clocks}
     del srcs, outs
     if dual:

@@ -187,6 +187,18 @@ size_t lbca_prefill_workspace_bytes(const lbca_config* cfg, int32_t batch, int32
     return bytes;
 }
 
+// Fields common to every pooling call of blocks [pos0/m, pos0/m + T/m).
+static void pool_common(const lbca_config* cfg, int32_t batch, int32_t T, int32_t pos0, int32_t out_blocks,
+                        PoolArgs& a) {
+    a.dtype = cfg->dtype;
+    a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
+    a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
+    a.pos0 = pos0;
+    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
+    a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
+    a.state = nullptr; a.S = 1;
+}
+
 // One series pooled into `out` (the I/O dtype) or `out_f32` (f32 entries).
 static lbca_status pool_single(const lbca_config* cfg, int32_t series, const void* x, const void* z,
                                const void* b_pos, const void* gamma, int32_t batch, int32_t T, int32_t pos0,
@@ -202,19 +214,13 @@ static lbca_status pool_single(const lbca_config* cfg, int32_t series, const voi
         return LBCA_ERR_ALIGN;
     LBCA_TRY(check_device());
     PoolArgs a{};
-    a.dtype = cfg->dtype;
+    pool_common(cfg, batch, T, pos0, out_blocks, a);
     a.nser = 1;
     a.ser[0].x = x; a.ser[0].z = z; a.ser[0].bpos = b_pos; a.ser[0].gamma = gamma;
     // f32 I/O: the entries are f32 already
     a.ser[0].out = out ? out : (cfg->dtype == LBCA_F32 ? out_f32 : nullptr);
     a.ser[0].out_f32 = cfg->dtype == LBCA_F32 ? nullptr : out_f32;
     a.ser[0].key = series == LBCA_KEY; a.ser[0].state_series = 0;
-    a.out_blocks = out_blocks; a.blk_off = pos0 / cfg->block_m;
-    a.B = batch; a.T = T; a.G = cfg->n_kv_heads; a.D = cfg->head_dim; a.m = cfg->block_m;
-    a.pos0 = pos0;
-    a.rmsnorm = cfg->rmsnorm; a.rho = cfg->rope_dims;
-    a.rope_step = rope_step_of(cfg); a.eps = cfg->rms_eps;
-    a.state = nullptr; a.S = 1;
     return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -230,6 +236,31 @@ lbca_status lbca_pool_f32(const lbca_config* cfg, int32_t series, const void* x,
                           float* out, int32_t out_blocks, lbca_stream_t stream) {
     if (!out) return LBCA_ERR_ARG;
     return pool_single(cfg, series, x, z, b_pos, gamma, batch, T, pos0, nullptr, out, out_blocks, stream);
+}
+
+lbca_status lbca_pool_kv(const lbca_config* cfg, const void* k, const void* v, const void* zk, const void* zv,
+                         const void* b_pos_k, const void* b_pos_v, const void* gamma_kv, int32_t batch, int32_t T,
+                         int32_t pos0, void* pooled_k, void* pooled_v, int32_t out_blocks, lbca_stream_t stream) {
+    LBCA_TRY(check_cfg(cfg));
+    if (cfg->shared_kv) return LBCA_ERR_ARG;
+    if (!k || !v || !zk || !zv || !b_pos_k || !b_pos_v || !pooled_k || !pooled_v) return LBCA_ERR_ARG;
+    if (batch < 0 || T < 0 || pos0 < 0 || pos0 % cfg->block_m || out_blocks < 0) return LBCA_ERR_ARG;
+    if ((long long)pos0 / cfg->block_m + T / cfg->block_m > out_blocks) return LBCA_ERR_ARG;
+    if (!al16(k) || !al16(v) || !al16(zk) || !al16(zv) || !al16(b_pos_k) || !al16(b_pos_v) || !al16(pooled_k) ||
+        !al16(pooled_v) || !al16n(gamma_kv))
+        return LBCA_ERR_ALIGN;
+    LBCA_TRY(check_device());
+    PoolArgs a{};
+    pool_common(cfg, batch, T, pos0, out_blocks, a);
+    a.nser = 2;
+    for (int series = 0; series < 2; ++series) {
+        PoolSeries& sr = a.ser[series];
+        sr.x = series ? v : k; sr.z = series ? zv : zk; sr.bpos = series ? b_pos_v : b_pos_k;
+        sr.gamma = series ? nullptr : gamma_kv;
+        sr.out = series ? pooled_v : pooled_k;
+        sr.key = series == 0; sr.state_series = series;
+    }
+    return cuda_status(launch_pool(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lbca_status lbca_pool_dual(const lbca_config* cfg, int32_t series, const void* xa, const void* za, const void* xb,

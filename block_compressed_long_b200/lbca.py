@@ -33,7 +33,7 @@ ENTRY_POINTS = ("lbca_ring_slots", "lbca_pool_state_elems", "lbca_decode_workspa
                 "lbca_decode_step_workspace_bytes", "lbca_decode_step", "lbca_decode_step_launches",
                 "lbca_decode_step_form", "lbca_selftest_bounded_wait", "lbca_pool_dual", "lbca_decode_sparse",
                 "lbca_indexer_workspace_bytes", "lbca_indexer_topk", "lbca_prefill_backward_workspace_bytes",
-                "lbca_prefill_backward", "lbca_prefill_rows", "lbca_pool_f32")
+                "lbca_prefill_backward", "lbca_prefill_rows", "lbca_pool_f32", "lbca_pool_kv")
 
 
 class lbca_config(ctypes.Structure):
@@ -70,6 +70,8 @@ _lib.lbca_pool.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp,
 _lib.lbca_pool.restype = ctypes.c_int
 _lib.lbca_pool_f32.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp]
 _lib.lbca_pool_f32.restype = ctypes.c_int
+_lib.lbca_pool_kv.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp]
+_lib.lbca_pool_kv.restype = ctypes.c_int
 _lib.lbca_pool_dual.argtypes = [_CP, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp]
 _lib.lbca_pool_dual.restype = ctypes.c_int
 _lib.lbca_append.argtypes = [_CP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _KP, _vp, _vp]
@@ -228,6 +230,17 @@ def lbca_pool_f32(cfg, series, x, z, b_pos, gamma, out, pos0=0, out_blocks=None,
     ob = out.shape[2] if out_blocks is None else out_blocks
     _check("lbca_pool_f32", _lib.lbca_pool_f32(ctypes.byref(cfg), series, _ptr(x), _ptr(z), _ptr(b_pos), _ptr(gamma),
                                                B, T, pos0, _ptr(out), ob, _stream(stream)))
+
+
+def lbca_pool_kv(cfg, k, v, zk, zv, b_pos_k, b_pos_v, gamma_kv, pooled_k, pooled_v, pos0=0, out_blocks=None,
+                 stream=None):
+    """Both series of the GQA form in one launch: k, v, zk, zv [B, T, G, D];
+    pooled_k, pooled_v [B, G, out_blocks, D]."""
+    B, T = k.shape[0], k.shape[1]
+    ob = pooled_k.shape[2] if out_blocks is None else out_blocks
+    _check("lbca_pool_kv", _lib.lbca_pool_kv(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(zk), _ptr(zv), _ptr(b_pos_k),
+                                             _ptr(b_pos_v), _ptr(gamma_kv), B, T, pos0, _ptr(pooled_k),
+                                             _ptr(pooled_v), ob, _stream(stream)))
 
 
 def lbca_pool_dual(cfg, series, xa, za, xb, zb, b_pos_a, b_pos_b, gamma, out, out_blocks=None, stream=None):

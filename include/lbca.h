@@ -168,6 +168,20 @@ LBCA_API lbca_status lbca_pool(const lbca_config* cfg, int32_t series, const voi
                       int32_t pos0, void* out, int32_t out_blocks, lbca_stream_t stream);
 
 /*
+ * lbca_pool_kv -- lbca_pool of both series of the GQA form in one launch: the
+ * keys (k, zk, b_pos_k, gamma_kv: RMSNorm when enabled and RoPE at each block
+ * start) into pooled_k, the values (v, zv, b_pos_v, pooled as is) into
+ * pooled_v.  Each series' arguments mean what they mean in lbca_pool; the
+ * entries equal those of two lbca_pool calls bit for bit (HCA page, "What is
+ * implemented", Eqs 20-23; mSeek README, "How LBCA works", steps 2-3).
+ * Errors: as lbca_pool; LBCA_ERR_ARG also for the shared form (no value series).
+ */
+LBCA_API lbca_status lbca_pool_kv(const lbca_config* cfg, const void* k, const void* v, const void* zk,
+                         const void* zv, const void* b_pos_k, const void* b_pos_v,
+                         const void* gamma_kv, int32_t batch, int32_t T, int32_t pos0,
+                         void* pooled_k, void* pooled_v, int32_t out_blocks, lbca_stream_t stream);
+
+/*
  * lbca_pool_f32 -- lbca_pool with the entries written in f32 (out: device
  * [B, G, out_blocks, D] float), unrounded: the exchange format of a
  * context-parallel prefill, whose ranks all-gather their pooled entries and

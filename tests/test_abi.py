@@ -93,6 +93,17 @@ def test_pool_argument_checks(L):
     assert g(0, A, A, A, None, 1, 640, 0, A, 9, None) == L.LBCA_ERR_ARG            # out_blocks too small
     assert g(0, A, A, A, None, 1, 64, 0, A + 4, 1, None) == L.LBCA_ERR_ALIGN       # misaligned out
     assert g(0, A, A, A, None, 1, 64, 0, A, 1, None) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
+    # both series in one call: k, v, zk, zv, b_pos_k, b_pos_v, gamma, B, T, pos0, pooled_k, pooled_v, out_blocks
+    h = lambda *a: L._lib.lbca_pool_kv(ctypes.byref(cfg), *a)  # noqa: E731
+    assert h(A, None, A, A, A, A, None, 1, 64, 0, A, A, 1, None) == L.LBCA_ERR_ARG      # null v
+    assert h(A, A, A, A, A, A, None, 1, 64, 0, A, None, 1, None) == L.LBCA_ERR_ARG      # null pooled_v
+    assert h(A, A, A, A, A, A, None, 1, 64, 3, A, A, 8, None) == L.LBCA_ERR_ARG         # pos0 % m
+    assert h(A, A, A, A, A, A, None, 1, 640, 0, A, A, 9, None) == L.LBCA_ERR_ARG        # out_blocks too small
+    assert h(A, A, A, A, A + 8, A, None, 1, 64, 0, A, A, 1, None) == L.LBCA_ERR_ALIGN   # misaligned b_pos_k
+    assert h(A, A, A, A, A, A, None, 1, 64, 0, A, A + 4, 1, None) == L.LBCA_ERR_ALIGN   # misaligned pooled_v
+    assert L._lib.lbca_pool_kv(ctypes.byref(shared), A, A, A, A, A, A, None, 1, 64, 0, A, A, 1,
+                               None) == L.LBCA_ERR_ARG                                   # no value series
+    assert h(A, A, A, A, A, A, None, 1, 64, 0, A, A, 1, None) in (L.LBCA_ERR_CUDA, L.LBCA_ERR_UNSUPPORTED)
 
 
 def test_cache_and_decode_checks(L):

@@ -43,8 +43,10 @@ def test_pool_matches_oracle(L, name, kw, pos0_blocks):
     nb = T // m
     ob = pos0_blocks + nb + 2
     series = [(0, inp.k, inp.zk, inp.bpos_k)] + ([] if w.shared_kv else [(1, inp.v, inp.zv, inp.bpos_v)])
+    outs = []
     for s, x, z, bp in series:
         out = torch.full((B, w.n_kv_heads, ob, w.head_dim), 7.0, dtype=L.torch_dtype(cfg), device="cuda")
+        outs.append(out)
         L.lbca_pool(cfg, s, x.cuda(), z.cuda(), bp.cuda(), None, out, pos0=pos0_blocks * m)
         torch.cuda.synchronize()
         want = orc.pool(ocfg(w), s, f64(x), f64(z), f64(bp), None, pos0=pos0_blocks * m)  # [B, nb, G, D]
@@ -61,6 +63,12 @@ def test_pool_matches_oracle(L, name, kw, pos0_blocks):
         scale = max(float(np.abs(want).max()), 1e-30)
         assert np.abs(g32 - want).max() <= 1e-5 * scale, f"{name} series {s}: f32 entries"
         assert np.all(f64(o32[:, :, pos0_blocks + nb:]) == 7.0) and np.all(f64(o32[:, :, :pos0_blocks]) == 7.0)
+    if not w.shared_kv:  # both series in one launch: the same entries, bit for bit, and nothing else written
+        pk, pv = torch.full_like(outs[0], 7.0), torch.full_like(outs[1], 7.0)
+        L.lbca_pool_kv(cfg, inp.k.cuda(), inp.v.cuda(), inp.zk.cuda(), inp.zv.cuda(), inp.bpos_k.cuda(),
+                       inp.bpos_v.cuda(), None, pk, pv, pos0=pos0_blocks * m)
+        torch.cuda.synchronize()
+        assert torch.equal(pk, outs[0]) and torch.equal(pv, outs[1]), f"{name}: lbca_pool_kv"
 
 
 # ------------------------------------------------------------- prefill ----

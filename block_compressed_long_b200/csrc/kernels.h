@@ -49,8 +49,8 @@ struct PoolArgs {
     // sets LBCA_ERR_UNSUPPORTED (nullable)
     int32_t* status;
     // launch geometry (set by launch_pool): blocks per series and sequence,
-    // head slices, blocks per CTA
-    int nblk, gz, bpc;
+    // head slices
+    int nblk, gz;
     int dual;              // 1: every series is pooled in the dual overlapped form
 };
 cudaError_t launch_pool(const PoolArgs& a, cudaStream_t s);

@@ -185,11 +185,23 @@ def test_status_strings(L):
         assert L.lbca_status_string(s)
 
 
-def test_every_binding_wrapper_reaches_the_library(L):
+def test_every_binding_wrapper_reaches_the_library(L, monkeypatch):
     """Each Python wrapper marshals its arguments into the C entry point it
     names: called with host tensors (no GPU here) it must come back with a
-    library status, never with a ctypes arity or type error."""
+    library status, never with a ctypes arity or type error.  Every wrapper
+    of the binding is among the calls."""
+    import inspect
+    import re
+
     import torch
+    reached = set()
+    check = L._check
+
+    def record(fn, st):
+        reached.add(fn)
+        return check(fn, st)
+
+    monkeypatch.setattr(L, "_check", record)
     cfg = L.config(4, 2, 32, False, 4, 8, rope_dims=8)
     hca = L.config(64, 1, 256, True, 4, 8, rope_dims=8, rmsnorm=True)
     q = torch.zeros(1, 8, 4, 32)
@@ -209,6 +221,10 @@ def test_every_binding_wrapper_reaches_the_library(L):
     calls = [
         lambda: L.lbca_pool(cfg, 0, kv, kv, bp, None, torch.zeros(1, 2, 2, 32)),
         lambda: L.lbca_pool_dual(cfg, 0, kv, kv, kv, kv, bp, bp, None, torch.zeros(1, 2, 2, 32)),
+        lambda: L.lbca_pool_kv(cfg, kv, kv, kv, kv, bp, bp, None, torch.zeros(1, 2, 2, 32), torch.zeros(1, 2, 2, 32)),
+        lambda: L.lbca_pool_f32(cfg, 0, kv, kv, bp, None, torch.zeros(1, 2, 2, 32)),
+        lambda: L.lbca_prefill_rows(cfg, q, 0, kv, kv, 0, torch.zeros(1, 2, 2, 32), torch.zeros(1, 2, 2, 32), None,
+                                    None, None, torch.zeros_like(q)),
         lambda: L.lbca_append(cfg, tok, tok, tok, tok, bp, bp, None, cache, st),
         lambda: L.lbca_decode(cfg, q1, cache, None, None, None, torch.zeros_like(q1), ws, 8, st),
         lambda: L.lbca_decode_noalloc(cfg, q1, cache, None, None, None, torch.zeros_like(q1), 8, st),
@@ -226,6 +242,8 @@ def test_every_binding_wrapper_reaches_the_library(L):
     for i, call in enumerate(calls):
         with pytest.raises(L.LbcaError):
             call()
+    wrappers = set(re.findall(r'_check\("(\w+)"', inspect.getsource(L)))
+    assert wrappers == reached, sorted(wrappers ^ reached)
 
 
 def test_cache_struct_follows_field_changes(L):

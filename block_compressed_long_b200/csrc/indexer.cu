@@ -1,8 +1,8 @@
 // indexer.cu -- lightning-indexer relevance and top-k block selection (the
-// CSA form; CSA page, "What is implemented": low-rank indexer queries,
-// per-head ReLU-scored relevance against compressed indexer keys, learned
-// head weights, top-k selection restricted to causally visible blocks,
-// Eqs 13-17).
+// CSA form; CSA page, "What is implemented", Eqs 13-17: each indexer head
+// scores a compressed indexer key by the ReLU of its dot product with a
+// low-rank indexer query, learned per-head weights combine the heads, and the
+// k best of the blocks the query may causally see are kept).
 //
 // For one query per sequence with indexer heads q_h [HI, DI] and head
 // weights w_h, the relevance of complete block j is

@@ -1,8 +1,9 @@
 // pool.cu -- block pooling, raw-window fill and streaming append.
 //
-// Block pooling (HCA page, "What is implemented": single-series pooling of m
-// tokens per entry with content-dependent softmax weights plus a learnable
-// positional bias, Eqs 20-23; mSeek README, "How LBCA works", steps 2-3):
+// Block pooling (HCA page, "What is implemented", Eqs 20-23: one series, the
+// m tokens of a block folded into one entry by softmax weights computed from
+// their content plus a learned bias per position in the block; mSeek README,
+// "How LBCA works", steps 2-3):
 // per (block j, kv head g, channel c) the weights are softmax_i(Z + B_pos[i])
 // over the block's m positions and the entry is the weighted sum of X.  Key
 // entries are then finalised: RMSNorm (HCA form) and RoPE at the block-start

@@ -239,9 +239,10 @@ LBCA_API lbca_status lbca_append(const lbca_config* cfg, const void* k, const vo
 /*
  * lbca_decode -- attention of one query per sequence at its last position.
  * (mSeek README, "How LBCA works", step 4; HCA page, "What is implemented":
- * dense attention over all causally visible compressed entries plus the
- * sliding window, MQA shared KV, RMSNorm, partial RoPE, sink; CSA page,
- * "What is implemented": Eqs 18-19, Eq 27, the -i output rotation.)
+ * every compressed entry the query may causally see, attended densely with
+ * the raw window, one key/value entry shared by all query heads, RMSNorm,
+ * RoPE on part of the dims and a sink; CSA page, "What is implemented":
+ * Eqs 18-19, Eq 27, outputs turned back by -t.)
  *   q          device [B, Hq, D] queries; sequence b's query sits at position
  *              t = seq_lens[b] - 1 (call lbca_append for the token first)
  *   sink       device [Hq] f32 sink logits or NULL
@@ -443,10 +444,11 @@ LBCA_API lbca_status lbca_selftest_bounded_wait(int32_t arrive, uint64_t limit_n
 /*
  * lbca_decode_sparse -- core attention of the CSA form for one query per
  * sequence over the selected compressed entries plus the raw window (CSA page,
- * "What is implemented": shared-KV MQA core attention, Eqs 18-19, where the
- * selected compressed entries serve as both key and value, the sliding-window
- * branch of n_win uncompressed recent tokens, RMSNorm on queries and entries,
- * partial RoPE with the -i rotation of outputs, attention sink, Eq 27).
+ * "What is implemented", Eqs 18-19 and Eq 27: one key/value entry shared by
+ * all heads, each selected compressed entry used as key and as value, a
+ * window branch over the n_win most recent raw tokens, RMSNorm of queries and
+ * entries, RoPE on the last dims with the outputs turned back by -t, and a
+ * sink logit).
  *   q        device [B, Hq, D] queries at position t = seq_lens[b] - 1
  *   cache    pooled_k holds the finalised compressed entries (lbca_pool_dual,
  *            LBCA_KEY); ring_k the raw entries of (at least) the last n_win
@@ -470,10 +472,11 @@ LBCA_API lbca_status lbca_decode_sparse(const lbca_config* cfg, const void* q, c
 
 /*
  * lbca_indexer_topk -- lightning-indexer relevance and top-k block selection
- * for one query per sequence (the CSA form; CSA page, "What is implemented":
- * low-rank indexer queries, per-head ReLU-scored relevance against compressed
- * indexer keys, learned head weights, top-k selection restricted to causally
- * visible blocks, Eqs 13-17).
+ * for one query per sequence (the CSA form; CSA page, "What is implemented",
+ * Eqs 13-17: each indexer head scores a compressed indexer key by the ReLU of
+ * its dot product with a low-rank indexer query, learned per-head weights
+ * combine the heads, and the k best of the blocks the query may causally see
+ * are kept).
  *   q_idx      device [B, n_heads, head_dim] bf16 indexer queries
  *   w_idx      device [B, n_heads] f32 head weights
  *   k_idx      device [B, max_blocks, head_dim] bf16 compressed indexer keys

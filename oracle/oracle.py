@@ -18,9 +18,10 @@ Functions and the passages they follow:
   * ``Stream``    -- the same definition driven token by token, pooling each
                      block when it completes ("mSeek" README, repository
                      layout: generation through the LBCA cache).
-  * ``pool_dual``  -- CSA dual overlapped pooling: entry i pools its own block
-                     (a-series) and the preceding block (b-series) under one
-                     joint softmax (CSA page, "What is implemented", Eqs 9-12).
+  * ``pool_dual``  -- CSA dual overlapped pooling: entry i combines block i of
+                     the a-series with block i - 1 of the b-series, all 2m
+                     tokens weighted by a single softmax (CSA page, "What is
+                     implemented", Eqs 9-12).
   * ``indexer_scores`` / ``topk_blocks`` -- lightning-indexer relevance
                      sum_h w_h ReLU(q_h . k_j) over the complete blocks, and
                      the top-k of them (CSA page, "What is implemented",
